@@ -1,0 +1,453 @@
+#!/usr/bin/env python
+"""Benchmark of one sparse-MoE FFN layer forward on B200 (sm_100a).
+
+A step is one whole-layer forward (router, top-k, permutation, grouped
+SwiGLU experts + shared expert, combine) through the C-ABI on one synthetic
+token batch whose inputs and weights are already resident in HBM. The L2 is
+flushed (256 MB write) before every step, outside the step's CUDA events.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|prefill|...]
+                  [--impl reference]
+
+With N > 1 (launched by torch.distributed.run) every rank runs an independent
+replica of the layer on its own batch (tokens are independent: no data-path
+collective); timing is the max over ranks and `value` counts all ranks'
+tokens (weak scaling). `--impl reference` times the CPU oracle instead
+(rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "MoE-layer tokens/s (T=4096 prefill, T=32 decode) and % of roofline"
+L2_FLUSH_BYTES = 256 << 20
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def dist_init(world: int, backend: str):
+    import datetime
+
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+
+
+def reduce_max(value: float, device=None) -> float:
+    """Max of a scalar over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        if device is not None and str(device).startswith("cuda"):
+            dist.barrier(device_ids=[int(str(device).split(":")[1])])
+        else:
+            dist.barrier()
+
+
+def replica_config(cfg: workloads.MoEConfig, rank: int) -> workloads.MoEConfig:
+    """Rank r's replica: same layer weights, its own token batch."""
+    return cfg
+
+
+def replica_tokens_seed(cfg: workloads.MoEConfig, rank: int) -> int:
+    return rank  # step index offset for workloads.tokens(): every rank draws its own batch
+
+
+# ------------------------------------------------------------------ peaks, clocks
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=d["hbm_gbs"], bf16_tflops=d["bf16_tflops"],
+                    bf16_tflops_sustained=d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                    source="measured")
+    return dict(PEAKS_FALLBACK, source="fallback")
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,utilization.gpu,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"sgl_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.fh,
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9 and parts[1].isdigit():
+                    rows.append(parts)
+        try:
+            os.unlink(self.path)
+        except OSError:
+            pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        load = [r for r in rows if r[3].isdigit() and int(r[3]) > 0] or rows
+        reasons = set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for r in load:
+            for n, v in zip(names, r[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(int(r[1]) for r in load),
+                "sm_max_mhz": max(int(r[2]) for r in rows if r[2].isdigit()),
+                "reasons": sorted(reasons), "samples": len(load)}
+
+
+# ------------------------------------------------------------------ roofline arithmetic
+
+def algorithmic_work(cfg, T: int, touched: int):
+    """Bytes and FLOPs the layer must move / compute (intermediates not credited)."""
+    H, I, Is, K, E = cfg.H, cfg.I, cfg.I_shared, cfg.K, cfg.E
+    wb = 2  # bf16 weights
+    gu_bytes = touched * 2 * I * H * wb + 2 * Is * H * 2 + T * H * 2
+    dn_bytes = touched * H * I * wb + H * Is * 2
+    gu_flops = 2.0 * (T * K * 2 * I * H + T * 2 * Is * H)
+    dn_flops = 2.0 * (T * K * H * I + T * H * Is)
+    router_bytes = E * H * 4 + E * 4 + T * H * 2 + T * K * 8
+    layer_bytes = gu_bytes + dn_bytes + router_bytes - T * H * 2 + T * H * 2  # x counted once, y out
+    layer_flops = gu_flops + dn_flops
+    return dict(gateup=(gu_bytes, gu_flops), down=(dn_bytes, dn_flops),
+                layer=(layer_bytes, layer_flops), router_flops=2.0 * T * H * E)
+
+
+def roofline_entry(bytes_, flops, seconds, peaks, sustained=False):
+    tp = (peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]) * 1e12
+    bw = peaks["hbm_gbs"] * 1e9
+    t_mem, t_tc = bytes_ / bw, flops / tp
+    if t_mem >= t_tc:
+        ach = bytes_ / seconds / 1e9
+        return {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(ach / peaks["hbm_gbs"], 4)}
+    ach = flops / seconds / 1e12
+    pk = tp / 1e12
+    return {"bound": "tensor", "achieved": round(ach, 1), "peak": pk, "unit": "TFLOP/s",
+            "frac": round(ach / pk, 4)}
+
+
+# ------------------------------------------------------------------ GPU arm
+
+STAGES = ("route", "permute", "gateup", "down", "combine")
+KERNELS_PER_STEP = 8  # router 2, permutation 3, GEMM 2, combine 1
+
+
+def measure_gpu(cfg, steps, warmup, device, rank, with_e2e=True):
+    import torch
+
+    import sigmoid_group_limited_b200 as sgl
+
+    T = cfg.T
+    d = workloads.generate(replica_config(cfg, rank), device)
+    if rank:
+        d["x"] = workloads.tokens(cfg, T, replica_tokens_seed(cfg, rank), device)
+    W = sgl.make_weights(d["Wg"], d["Wu"], d["Wd"], d["Wg_s"], d["Wu_s"], d["Wd_s"])
+    ws = sgl.alloc_workspace(cfg, T, device)
+    y = torch.empty(T, cfg.H, dtype=torch.bfloat16, device=device)
+    idx = torch.empty(T, cfg.K, dtype=torch.int32, device=device)
+    w = torch.empty(T, cfg.K, dtype=torch.float32, device=device)
+    counts = torch.empty(cfg.E, dtype=torch.int32, device=device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def fwd(ev=None):
+        sgl.moe_layer_forward(cfg, d["x"], d["Wr"], d["bias"], W, y, ws, idx, w, counts,
+                              stream=stream, stage_events=ev)
+
+    for _ in range(warmup):
+        flush.zero_()
+        fwd()
+    torch.cuda.synchronize(device)
+    assert sgl.moe_read_error(cfg, T, ws) == 0
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+    barrier(device)
+    torch.cuda.synchronize(device)
+    t0 = time.perf_counter()
+    for i in range(steps):
+        flush.zero_()
+        fwd(evs[i])
+    torch.cuda.synchronize(device)
+    barrier(device)
+    wall = time.perf_counter() - t0
+    per_step = [evs[i][0].elapsed_time(evs[i][5]) for i in range(steps)]
+    stage_ms = {s: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(steps))
+                for j, s in enumerate(STAGES)}
+    dev_ms = sum(per_step)
+    assert sgl.moe_read_error(cfg, T, ws) == 0
+    touched = int((counts > 0).sum().item())
+    cnt = counts.cpu().numpy()
+    out = dict(device_ms_total=dev_ms, wall_s=wall, per_step_ms=per_step, stage_ms=stage_ms,
+               touched=touched, load_max=int(cnt.max()), load_mean=float(cnt.mean()),
+               d=d, launches=KERNELS_PER_STEP * steps)
+
+    if with_e2e:
+        # end to end through the public API: pinned host x -> device, forward, y -> pinned host
+        xh = d["x"].cpu().pin_memory()
+        yh = torch.empty(T, cfg.H, dtype=torch.bfloat16).pin_memory()
+        xd = torch.empty_like(d["x"])
+        e0 = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        e1 = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        for i in range(warmup):
+            xd.copy_(xh, non_blocking=True)
+            sgl.moe_layer_forward(cfg, xd, d["Wr"], d["bias"], W, y, ws, stream=stream)
+            yh.copy_(y, non_blocking=True)
+        torch.cuda.synchronize(device)
+        for i in range(steps):
+            flush.zero_()
+            e0[i].record(stream)
+            xd.copy_(xh, non_blocking=True)
+            sgl.moe_layer_forward(cfg, xd, d["Wr"], d["bias"], W, y, ws, stream=stream)
+            yh.copy_(y, non_blocking=True)
+            e1[i].record(stream)
+        torch.cuda.synchronize(device)
+        out["e2e_ms_total"] = sum(e0[i].elapsed_time(e1[i]) for i in range(steps))
+        out["e2e_h2d"] = T * cfg.H * 2
+        out["e2e_d2h"] = T * cfg.H * 2
+        assert torch.equal(yh.view(torch.int16), y.cpu().view(torch.int16))
+    del flush
+    return out
+
+
+# ------------------------------------------------------------------ oracle (CPU) arm
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_inputs(d):
+    """Host copies of the inputs (bytes as the GPU sees them)."""
+    import torch
+
+    def b16(t):
+        return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    return dict(x=b16(d["x"]), Wr=d["Wr"].cpu().numpy(), bias=d["bias"].cpu().numpy(),
+                Wg_s=b16(d["Wg_s"]), Wu_s=b16(d["Wu_s"]), Wd_s=b16(d["Wd_s"]),
+                experts=lambda e: (b16(d["Wg"][e]), b16(d["Wu"][e]), b16(d["Wd"][e])))
+
+
+def time_oracle(cfg, h, tokens):
+    """Oracle layer forward for `tokens` of the batch (routing covers the batch);
+    the touched experts' weights are fetched to host before the clock starts."""
+    import oracle
+    r = oracle.route(h["x"], h["Wr"], h["bias"], cfg.n_group, cfg.topk_group, cfg.K)
+    need = sorted(set(int(e) for e in r["idx"][tokens].reshape(-1)))
+    host = {e: h["experts"](e) for e in need}
+
+    def ew(e):
+        g, u, dd = host[e]
+        f = oracle.bf16_bits_to_f64
+        return f(g), f(u), f(dd)
+    t0 = time.perf_counter()
+    oracle.layer_forward(cfg, h["x"], h["Wr"], h["bias"], ew, h["Wg_s"], h["Wu_s"], h["Wd_s"],
+                         tokens=tokens)
+    return time.perf_counter() - t0
+
+
+def oracle_sample_tokens(cfg, step: int, n: int):
+    return np.array([(step * n + i) % cfg.T for i in range(n)])
+
+
+# ------------------------------------------------------------------ main
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="decode", choices=sorted(workloads.CONFIGS))
+    ap.add_argument("--also", default="prefill", help="second workload for the line ('' = none)")
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--oracle-tokens", type=int, default=8)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def config_block(cfg, world):
+    return {"workload": f"{cfg.name}: T={cfg.T} tokens per GPU, H={cfg.H}, E={cfg.E} experts "
+                        f"({cfg.n_group} groups keep {cfg.topk_group}, top-{cfg.K}), I={cfg.I}, "
+                        f"shared I={cfg.I_shared}",
+            "T": cfg.T, "H": cfg.H, "E": cfg.E, "n_group": cfg.n_group,
+            "topk_group": cfg.topk_group, "K": cfg.K, "I": cfg.I, "I_shared": cfg.I_shared,
+            "bias": cfg.bias_kind, "limits": [cfg.limit_routed, cfg.limit_shared],
+            "global_batch": cfg.T * world, "parallelism": f"replicas x{world} (tokens sharded, no collective)",
+            "l2": "flushed before every step (256 MB write, outside the step events)"}
+
+
+def run_reference(args, rank, world):
+    cfg = workloads.CONFIGS[args.workload]
+    if rank != 0:
+        return
+    import torch
+    dev = "cuda:0" if torch.cuda.is_available() else "cpu"
+    d = workloads.generate(cfg, dev)
+    h = oracle_inputs(d)
+    n = min(args.oracle_tokens, cfg.T)
+    for i in range(args.warmup):
+        time_oracle(cfg, h, oracle_sample_tokens(cfg, i, n))
+    ts = [time_oracle(cfg, h, oracle_sample_tokens(cfg, args.warmup + i, n)) for i in range(args.steps)]
+    tot = sum(ts)
+    value = n * args.steps / tot
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * tot / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_block(cfg, 1),
+            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": blas_threads(),
+                             "kind": "oracle",
+                             "sample": f"{n} tokens of the {cfg.T}-token batch per step (routing "
+                                       f"of the whole batch + their {cfg.K} experts and the shared "
+                                       f"expert, numpy float64)"},
+            "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_native(args, rank, world, local):
+    import torch
+    device = f"cuda:{local}"
+    torch.cuda.set_device(device)
+    peaks = load_peaks()
+    cfg = workloads.CONFIGS[args.workload]
+    with ClockSampler(local) as clk:
+        m = measure_gpu(cfg, args.steps, args.warmup, device, rank)
+        also = None
+        if args.also and args.also != args.workload:
+            acfg = workloads.CONFIGS[args.also]
+            also = (acfg, measure_gpu(acfg, args.steps, args.warmup, device, rank, with_e2e=False))
+    clocks = clk.summary()
+    dev_s = reduce_max(m["device_ms_total"], device) / 1e3
+    e2e_s = reduce_max(m["e2e_ms_total"], device) / 1e3
+    tokens = cfg.T * args.steps * world
+
+    def roof(cfg_, mm):
+        work = algorithmic_work(cfg_, cfg_.T, mm["touched"])
+        stage = max(("gateup", "down"), key=lambda s: mm["stage_ms"][s])
+        b, f = work[stage]
+        ent = roofline_entry(b, f, mm["stage_ms"][stage] / 1e3, peaks)
+        ent.update(kernel=f"moe_gemm<{'gate/up' if stage == 'gateup' else 'down'}>",
+                   traffic=None, peak_source=f"{peaks['source']} ({'HBM copy' if ent['bound'] == 'hbm' else 'cuBLAS bf16 burst'})",
+                   units_per_launch=f"{cfg_.T} tokens, {mm['touched']} routed experts + shared")
+        lb, lf = work["layer"]
+        t_roof = max(lb / (peaks["hbm_gbs"] * 1e9), lf / (peaks["bf16_tflops"] * 1e12))
+        step_s = statistics.mean(mm["per_step_ms"]) / 1e3
+        return ent, round(t_roof / step_s, 4)
+
+    ent, layer_frac = roof(cfg, m)
+    line = {"metric": METRIC, "value": round(tokens / dev_s, 1), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * dev_s / args.steps, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": config_block(cfg, world), "roofline": ent,
+            "layer_roofline_frac": layer_frac,
+            "stage_ms": {k: round(v, 4) for k, v in m["stage_ms"].items()},
+            "routing": {"experts_touched": m["touched"], "load_max": m["load_max"],
+                        "load_mean": round(m["load_mean"], 2)},
+            "e2e": {"value": round(tokens / e2e_s, 1), "unit": "tokens/s",
+                    "h2d_bytes_per_step": m["e2e_h2d"], "d2h_bytes_per_step": m["e2e_d2h"]},
+            "gpu_launches": m["launches"], "clocks": clocks}
+    if also is not None:
+        acfg, am = also
+        a_s = reduce_max(am["device_ms_total"], device) / 1e3
+        aent, afrac = roof(acfg, am)
+        line[acfg.name] = {"value": round(acfg.T * args.steps * world / a_s, 1), "unit": "tokens/s",
+                           "ms_per_step": round(1e3 * a_s / args.steps, 4), "roofline": aent,
+                           "layer_roofline_frac": afrac,
+                           "stage_ms": {k: round(v, 4) for k, v in am["stage_ms"].items()},
+                           "routing": {"experts_touched": am["touched"], "load_max": am["load_max"],
+                                       "load_mean": round(am["load_mean"], 2)},
+                           "config": config_block(acfg, world)}
+        line["gpu_launches"] += am["launches"]
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        h = oracle_inputs(m["d"])
+        n = min(args.oracle_tokens, cfg.T)
+        t = time_oracle(cfg, h, oracle_sample_tokens(cfg, 0, n))
+        line["cpu_baseline"] = {"value": round(n / t, 3), "unit": "tokens/s", "cores": blas_threads(),
+                                "kind": "oracle",
+                                "sample": f"{n} of the {cfg.T} tokens (routing of the whole batch, "
+                                          f"their experts and the shared expert; numpy float64)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_env()
+    if args.gpus != world and world > 1:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    dist_init(world, "nccl")
+    try:
+        run_native(args, rank, world, local)
+    finally:
+        import torch.distributed as dist
+        if dist.is_available() and dist.is_initialized():
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

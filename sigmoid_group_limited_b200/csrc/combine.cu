@@ -1,0 +1,67 @@
+// combine.cu - stage 9: weighted combine back to token order.
+//
+// Every token's output is the sum of its K routed-expert contributions
+// (already multiplied by their combine weights) plus the shared expert's
+// output (page "Ling-3.0-flash-VL MoE sparse routing", sec. 2 and sec. 4).
+// The sum runs in fp32 in slot order k = 0..K-1, then adds the shared row,
+// and is rounded once to bf16 (nearest even). 16-byte loads and stores; each
+// thread owns 8 consecutive features of one token.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "internal.h"
+
+namespace sgl {
+namespace {
+
+__device__ __forceinline__ void add8(float* acc, const uint4 v) {
+  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    acc[2 * i] += __uint_as_float(u[i] << 16);
+    acc[2 * i + 1] += __uint_as_float(u[i] & 0xFFFF0000u);
+  }
+}
+
+__global__ void __launch_bounds__(256) combine_kernel(int T, int H, int K, int with_shared,
+                                                      const uint16_t* __restrict__ y_slot,
+                                                      uint16_t* __restrict__ y) {
+  const int chunks = H / 8;
+  const long long total = static_cast<long long>(T) * chunks;
+  const uint4* src = reinterpret_cast<const uint4*>(y_slot);
+  uint4* dst = reinterpret_cast<uint4*>(y);
+  const long long TKrows = static_cast<long long>(T) * K;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long t = i / chunks;
+    const int c = static_cast<int>(i - t * chunks);
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+    for (int k = 0; k < K; ++k) add8(acc, src[(t * K + k) * chunks + c]);
+    if (with_shared) add8(acc, src[(TKrows + t) * chunks + c]);
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(acc[2 * q]));
+      const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(acc[2 * q + 1]));
+      o[q] = lo | (hi << 16);
+    }
+    dst[i] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const moe_cfg& c, int T, const uint16_t* y_slot, int with_shared,
+                           uint16_t* y, cudaStream_t s) {
+  const long long total = static_cast<long long>(T) * (c.H / 8);
+  const int threads = 256;
+  long long blocks = (total + threads - 1) / threads;
+  const long long cap = static_cast<long long>(num_sms()) * 8;
+  if (blocks > cap) blocks = cap;
+  combine_kernel<<<static_cast<int>(blocks), threads, 0, s>>>(T, c.H, c.K, with_shared, y_slot, y);
+  return cudaGetLastError();
+}
+
+}  // namespace sgl

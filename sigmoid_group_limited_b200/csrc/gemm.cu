@@ -1,0 +1,450 @@
+// gemm.cu - stages 7 and 8: the grouped SwiGLU expert FFN and the shared
+// expert, as two persistent tcgen05 GEMM kernels.
+//
+// Page "Ling-3.0-flash-VL MoE sparse routing" (lqnn.cn/news/282163): sec. 2
+// (an expert is a gate / up / down SwiGLU FFN, hidden 2560, intermediate 768;
+// one shared expert sees every token) and sec. 4 (SwiGLU limit +-4 on routed
+// experts, +-5/+-7 on the shared expert). The limit clamps gate and up to
+// [-L, L] before silu(gate) * up.
+//
+// Both kernels compute D = W_tile * X_tile^T with the weights as the MMA's
+// 128-row A operand and a tile of BN tokens as its N (the tokens of one
+// expert are few, so the weights fill the 128-row side):
+//   gate/up: D_g, D_u [128 features x BN tokens] over K = H, epilogue
+//            h = bf16(silu(clamp(D_g)) * clamp(D_u)), stored in permuted row
+//            order; the token rows are gathered from x with TMA gather4.
+//   down:    D [128 features x BN rows] over K = I, epilogue
+//            y_slot[j] = bf16(w_j * D) written to the slot's flat index j.
+// Work items (expert, row tile, output tile) come from a device-built list;
+// each CTA walks the list with a grid stride. Warp roles per CTA:
+//   warp 0  TMA producer (one lane), warp 1  MMA issuer (one lane) and TMEM
+//   owner, warps 2..5  epilogue (TMEM lanes 32*(warp%4) ...).
+// Pipelines: STAGES shared-memory stages (full/empty mbarriers) and two TMEM
+// accumulators (tmem_full/tmem_empty) so the epilogue of one item overlaps
+// the main loop of the next. Every wait is bounded (ptx.cuh).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace sgl {
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kSmemBudget = 200 * 1024;
+
+struct GemmParams {
+  int T, K, E, H, I, Is;
+  int has_shared;
+  float lim_r, lim_s;  // <= 0: no limit
+  const int32_t* perm;
+  const float* w;
+  uint16_t* h_r;  // [T*K, I] permuted rows
+  uint16_t* h_s;  // [T, Is]
+  uint16_t* y_slot;
+  const WorkItem* items;
+  const int32_t* nitems;  // device count of valid items
+  int max_items;
+  int32_t* err;
+};
+
+__host__ __device__ constexpr int pow2_at_least(int v) {
+  int p = 32;
+  while (p < v) p <<= 1;
+  return p;
+}
+
+template <int MODE, int BN>
+struct Cfg {
+  static constexpr int NA = MODE == 0 ? 2 : 1;       // weight tiles per stage (gate+up or down)
+  static constexpr int A_BYTES = kTileN * 128;       // 128 rows x 64 bf16
+  static constexpr int B_BYTES = BN * 128;           // BN rows x 64 bf16
+  static constexpr int STAGE_BYTES = NA * A_BYTES + B_BYTES;
+  static constexpr int STAGES_RAW = kSmemBudget / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+  static constexpr int ACC_COLS = NA * BN;           // fp32 columns per accumulator
+  static constexpr int TMEM_COLS = pow2_at_least(2 * ACC_COLS);
+  static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/ +
+                             BN * 4 /*token rows*/;
+};
+
+__device__ __forceinline__ float clampL(float v, float L) {
+  return L > 0.f ? fminf(fmaxf(v, -L), L) : v;
+}
+
+__device__ __forceinline__ uint16_t f2bf(float v) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
+
+// Same validity rule in every role, so all roles skip the same items.
+__device__ __forceinline__ bool item_ok(const GemmParams& p, const WorkItem& it, int mode,
+                                        int bn) {
+  const bool sh = it.e == p.E;
+  if (it.e < 0 || it.e > p.E || (sh && !p.has_shared)) return false;
+  if (it.nrows <= 0 || it.nrows > bn || it.row0 < 0) return false;
+  const int rows = sh ? p.T : p.T * p.K;
+  if (it.row0 + it.nrows > rows) return false;
+  const int nt = mode == 0 ? (sh ? p.Is : p.I) : p.H;
+  if (it.ntile < 0 || it.ntile * kTileN >= nt) return false;
+  return true;
+}
+
+template <int MODE, int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+    moe_gemm(const __grid_constant__ GemmParams p, const __grid_constant__ CUtensorMap tA0,
+             const __grid_constant__ CUtensorMap tA1, const __grid_constant__ CUtensorMap tS0,
+             const __grid_constant__ CUtensorMap tS1, const __grid_constant__ CUtensorMap tB0,
+             const __grid_constant__ CUtensorMap tB1) {
+  using C = Cfg<MODE, BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* tfull = empty + C::STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* tok = reinterpret_cast<int*>(smem + C::STAGES * C::STAGE_BYTES + 256);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tA0);
+    prefetch_tmap(&tB0);
+    if (p.has_shared) prefetch_tmap(&tS0);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int n_items = min(*p.nitems, p.max_items);
+  const int KB_r = (MODE == 0 ? p.H : p.I) / 64;
+  const int KB_s = (MODE == 0 ? p.H : p.Is) / 64;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    const uint64_t pol_w = policy_evict_first();
+    const uint64_t pol_x = policy_evict_last();
+    int stage = 0;
+    uint32_t phase = 0;
+    bool live = true;
+    for (int item = blockIdx.x; item < n_items && live; item += gridDim.x) {
+      const WorkItem it = p.items[item];
+      if (!item_ok(p, it, MODE, BN)) {
+        if (lane == 0) atomicExch(p.err, MOE_DEVERR_SCHEDULE);
+        continue;
+      }
+      const bool sh = it.e == p.E;
+      if (MODE == 0) {
+        for (int r = lane; r < BN; r += 32) {
+          const int row = it.row0 + min(r, it.nrows - 1);
+          int t = sh ? row : p.perm[row] / p.K;
+          t = min(max(t, 0), p.T - 1);
+          tok[r] = t;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) {
+        const int nkb = sh ? KB_s : KB_r;
+        const int arow = sh ? it.ntile * kTileN
+                            : it.e * (MODE == 0 ? p.I : p.H) + it.ntile * kTileN;
+        const CUtensorMap* mA0 = sh ? &tS0 : &tA0;
+        const CUtensorMap* mA1 = sh ? &tS1 : &tA1;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) {
+            live = false;
+            break;
+          }
+          uint8_t* sA = smem + stage * C::STAGE_BYTES;
+          uint8_t* sB = sA + C::NA * C::A_BYTES;
+          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+          tma_load_2d(sA, mA0, &full[stage], kb * 64, arow, pol_w);
+          if (MODE == 0) tma_load_2d(sA + C::A_BYTES, mA1, &full[stage], kb * 64, arow, pol_w);
+          if (MODE == 0) {
+#pragma unroll 4
+            for (int q = 0; q < BN / 4; ++q)
+              tma_gather4(sB + q * 512, &tB0, &full[stage], kb * 64, tok[4 * q], tok[4 * q + 1],
+                          tok[4 * q + 2], tok[4 * q + 3], pol_x);
+          } else {
+            tma_load_2d(sB, sh ? &tB1 : &tB0, &full[stage], kb * 64, it.row0, pol_x);
+          }
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      live = __shfl_sync(0xffffffffu, live ? 1 : 0, 0) != 0;
+      __syncwarp();
+    }
+    // drain: every stage must be released by its MMA commit before teardown
+    if (lane == 0 && live) {
+      for (int i = 0; i < C::STAGES; ++i) {
+        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) break;
+        if (++stage == C::STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(kTileN, BN);
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool live = true;
+      for (int item = blockIdx.x; item < n_items && live; item += gridDim.x) {
+        const WorkItem it = p.items[item];
+        if (!item_ok(p, it, MODE, BN)) continue;
+        const int nkb = it.e == p.E ? KB_s : KB_r;
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) break;
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + acc * C::ACC_COLS;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) {
+            live = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t b0 = a0 + C::NA * C::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t bd = sdesc_k128(b0 + kk * 32);
+            const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
+            umma_bf16(d0, sdesc_k128(a0 + kk * 32), bd, idesc, accum);
+            if (MODE == 0) umma_bf16(d0 + BN, sdesc_k128(a0 + C::A_BYTES + kk * 32), bd, idesc, accum);
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!live) break;
+        umma_commit(&tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1;
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;                  // TMEM lane quarter of this warp
+    const int orow = q * 32 + lane;          // output feature within the tile
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+      const WorkItem it = p.items[item];
+      if (!item_ok(p, it, MODE, BN)) continue;
+      const bool sh = it.e == p.E;
+      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * C::ACC_COLS;
+      const int nfeat = it.ntile * kTileN + orow;
+      if (MODE == 0) {
+        const int ncols = sh ? p.Is : p.I;
+        const bool ok = nfeat < ncols;
+        const float L = sh ? p.lim_s : p.lim_r;
+        uint16_t* hout = sh ? p.h_s : p.h_r;
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+          float gv[16], uv[16];
+          tmem_ld16(taddr + c0, gv);
+          tmem_ld16(taddr + BN + c0, uv);
+          tmem_ld_wait();
+          if (ok) {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const int r = c0 + c;
+              if (r < it.nrows) {
+                const float g = clampL(gv[c], L), u = clampL(uv[c], L);
+                const float hval = (g / (1.0f + expf(-g))) * u;
+                hout[static_cast<size_t>(it.row0 + r) * ncols + nfeat] = f2bf(hval);
+              }
+            }
+          }
+        }
+      } else {
+        const bool ok = nfeat < p.H;
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+          float ov[16];
+          tmem_ld16(taddr + c0, ov);
+          tmem_ld_wait();
+          if (ok) {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const int r = c0 + c;
+              if (r < it.nrows) {
+                const int row = it.row0 + r;
+                int j;
+                float wt;
+                if (sh) {
+                  j = p.T * p.K + row;
+                  wt = 1.0f;
+                } else {
+                  j = p.perm[row];
+                  if (j < 0 || j >= p.T * p.K) {  // a bad permutation: report, never store
+                    atomicExch(p.err, MOE_DEVERR_SCHEDULE);
+                    continue;
+                  }
+                  wt = p.w[j];
+                }
+                p.y_slot[static_cast<size_t>(j) * p.H + nfeat] = f2bf(wt * ov[c]);
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  }
+  return fn;
+}
+
+// bf16 row-major [rows, cols] matrix, box = box_rows x 64 columns, 128B swizzle.
+bool map_bf16(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr || ptr == nullptr || rows == 0) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+GemmParams make_params(const GemmArgs& a, int mode) {
+  const moe_cfg& c = *a.cfg;
+  GemmParams p;
+  p.T = a.T;
+  p.K = c.K;
+  p.E = c.E;
+  p.H = c.H;
+  p.I = c.I;
+  p.Is = c.I_shared;
+  p.has_shared = (c.I_shared > 0 && a.W->Wg_s != nullptr) ? 1 : 0;
+  p.lim_r = (c.limit_routed > 0.f && isfinite(c.limit_routed)) ? c.limit_routed : 0.f;
+  p.lim_s = (c.limit_shared > 0.f && isfinite(c.limit_shared)) ? c.limit_shared : 0.f;
+  p.perm = a.perm;
+  p.w = a.w;
+  p.h_r = a.h_r;
+  p.h_s = a.h_s;
+  p.y_slot = a.y_slot;
+  p.items = mode == 0 ? a.items_gu : a.items_dn;
+  p.nitems = a.nitems + mode;
+  p.max_items = mode == 0 ? a.max_items_gu : a.max_items_dn;
+  p.err = a.err;
+  return p;
+}
+
+template <int MODE, int BN>
+cudaError_t launch_mode(const GemmArgs& a, cudaStream_t s) {
+  using C = Cfg<MODE, BN>;
+  const moe_cfg& c = *a.cfg;
+  GemmParams p = make_params(a, MODE);
+  CUtensorMap tA0, tA1, tS0, tS1, tB0, tB1;
+  const int T = a.T, TK = a.T * c.K;
+  bool ok = true;
+  if (MODE == 0) {
+    ok &= map_bf16(&tA0, a.W->Wg, static_cast<uint64_t>(c.E) * c.I, c.H, kTileN);
+    ok &= map_bf16(&tA1, a.W->Wu, static_cast<uint64_t>(c.E) * c.I, c.H, kTileN);
+    ok &= map_bf16(&tB0, a.x, T, c.H, 1);
+    tB1 = tB0;
+    if (p.has_shared) {
+      ok &= map_bf16(&tS0, a.W->Wg_s, c.I_shared, c.H, kTileN);
+      ok &= map_bf16(&tS1, a.W->Wu_s, c.I_shared, c.H, kTileN);
+    } else {
+      tS0 = tA0;
+      tS1 = tA1;
+    }
+  } else {
+    ok &= map_bf16(&tA0, a.W->Wd, static_cast<uint64_t>(c.E) * c.H, c.I, kTileN);
+    tA1 = tA0;
+    ok &= map_bf16(&tB0, a.h_r, TK, c.I, BN);
+    if (p.has_shared) {
+      ok &= map_bf16(&tS0, a.W->Wd_s, c.H, c.I_shared, kTileN);
+      ok &= map_bf16(&tB1, a.h_s, T, c.I_shared, BN);
+    } else {
+      tS0 = tA0;
+      tB1 = tB0;
+    }
+    tS1 = tS0;
+  }
+  if (!ok) return cudaErrorInvalidValue;
+  auto kern = moe_gemm<MODE, BN>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  const int max_items = p.max_items;
+  const int grid = max(1, min(num_sms(), max_items));
+  kern<<<grid, kThreads, C::SMEM, s>>>(p, tA0, tA1, tS0, tS1, tB0, tB1);
+  return cudaGetLastError();
+}
+
+template <int MODE>
+cudaError_t launch_bn(const GemmArgs& a, cudaStream_t s) {
+  switch (a.bn) {
+    case 16: return launch_mode<MODE, 16>(a, s);
+    case 32: return launch_mode<MODE, 32>(a, s);
+    case 64: return launch_mode<MODE, 64>(a, s);
+    case 128: return launch_mode<MODE, 128>(a, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_gateup(const GemmArgs& a, cudaStream_t s) { return launch_bn<0>(a, s); }
+cudaError_t launch_gemm_down(const GemmArgs& a, cudaStream_t s) { return launch_bn<1>(a, s); }
+
+}  // namespace sgl

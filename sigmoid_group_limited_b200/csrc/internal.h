@@ -1,0 +1,86 @@
+// internal.h - host-side declarations shared by the library's translation
+// units: workspace layout, GEMM work items and kernel launchers.
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace sgl {
+
+// One GEMM work item: expert `e` (e == E: the shared expert), rows
+// [row0, row0 + nrows) of that expert's row range, output tile `ntile`
+// (128 output features). Rows are positions in the permuted row space for
+// routed experts (offsets[e] + m*BN) and token ids for the shared expert.
+struct WorkItem {
+  int32_t e;
+  int32_t row0;
+  int32_t nrows;
+  int32_t ntile;
+};
+
+constexpr int kPermTile = 2048;   // (token, slot) entries per permutation tile
+constexpr int kTileN = 128;       // output features per GEMM tile (MMA M)
+
+// Token-tile width (MMA N) for a batch: small for decode, wide for prefill.
+inline int choose_bn(int T, int K, int E) {
+  const double avg = static_cast<double>(T) * K / E;
+  if (avg <= 12.0) return 16;
+  if (avg <= 24.0) return 32;
+  if (avg <= 48.0) return 64;
+  return 128;
+}
+
+inline int cdiv(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
+__host__ __device__ inline int cdiv_dev(int a, int b) { return (a + b - 1) / b; }
+
+struct WsLayout {
+  size_t z, tile_hist, idx, w, counts, offsets, perm, inv_perm, items_gu, items_dn, nitems, h_r,
+      h_s, y_slot, err, total;
+  int n_ptiles, bn, max_items_gu, max_items_dn;
+};
+
+WsLayout ws_layout(const moe_cfg& c, int T);
+
+// Launchers (return cudaGetLastError()).
+cudaError_t launch_router(const moe_cfg& c, int T, const uint16_t* x, const float* Wr,
+                          const float* bias, float* z, int32_t* idx, float* w, cudaStream_t s);
+
+cudaError_t launch_permute(const moe_cfg& c, int T, const int32_t* idx, int32_t* tile_hist,
+                           int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv_perm,
+                           int32_t* err, const WsLayout& L, WorkItem* items_gu, WorkItem* items_dn,
+                           int32_t* nitems, cudaStream_t s);
+
+cudaError_t launch_schedule(const moe_cfg& c, int T, const int32_t* offsets, const WsLayout& L,
+                            WorkItem* items_gu, WorkItem* items_dn, int32_t* nitems,
+                            cudaStream_t s);
+
+struct GemmArgs {
+  const moe_cfg* cfg;
+  int T;
+  const uint16_t* x;
+  const int32_t* perm;
+  const float* w;
+  const moe_weights* W;
+  uint16_t* h_r;
+  uint16_t* h_s;
+  uint16_t* y_slot;
+  const WorkItem* items_gu;
+  const WorkItem* items_dn;
+  const int32_t* nitems;
+  int32_t* err;
+  int bn;
+  int max_items_gu;
+  int max_items_dn;
+};
+
+cudaError_t launch_gemm_gateup(const GemmArgs& a, cudaStream_t s);
+cudaError_t launch_gemm_down(const GemmArgs& a, cudaStream_t s);
+
+cudaError_t launch_combine(const moe_cfg& c, int T, const uint16_t* y_slot, int with_shared,
+                           uint16_t* y, cudaStream_t s);
+
+int num_sms();
+
+}  // namespace sgl

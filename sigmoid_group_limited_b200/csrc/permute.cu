@@ -1,0 +1,314 @@
+// permute.cu - stage 6: group the T*K (token, slot) pairs by expert.
+//
+// Each token selects K experts (page "Ling-3.0-flash-VL MoE sparse routing",
+// sec. 3 step 2); the expert FFNs then run on the rows routed to them. The
+// order is a stable counting sort of the flat slot index j = t*K + k by
+// expert id, so it is deterministic and equal to the oracle's.
+//
+// Three kernels over tiles of kPermTile flat entries:
+//   perm_hist    per-tile expert histogram (shared-memory atomics; counts do
+//                not depend on their order),
+//   perm_scan    one CTA: per-expert totals, exclusive offsets, per-(expert,
+//                tile) bases, and the GEMM work lists,
+//   perm_scatter per tile: stable ranks from warp match/ballot in flat order,
+//                then perm / inv_perm.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "internal.h"
+
+namespace sgl {
+namespace {
+
+constexpr int kMaxE = 1024;
+constexpr int kScatterWarps = 8;
+
+__global__ void __launch_bounds__(256) perm_hist(int TK, int E, int n_ptiles,
+                                                 const int32_t* __restrict__ idx,
+                                                 int32_t* __restrict__ tile_cnt,  // [E][n_ptiles]
+                                                 int32_t* __restrict__ err) {
+  __shared__ int hist[kMaxE];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int base = blockIdx.x * kPermTile;
+  const int n = min(kPermTile, TK - base);
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const int e = idx[base + i];
+    if (e < 0 || e >= E) {
+      atomicExch(err, MOE_DEVERR_EXPERT_ID);
+      continue;
+    }
+    atomicAdd(&hist[e], 1);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    tile_cnt[static_cast<size_t>(e) * n_ptiles + blockIdx.x] = hist[e];
+}
+
+// Block-wide exclusive scan of up to 2 values per thread (1024 threads).
+// Returns the exclusive prefix of this thread's first value; *total gets the sum.
+__device__ int block_exscan2(int v0, int v1, int* scratch /*32*/, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int v = v0 + v1;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) scratch[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = blockDim.x >> 5;
+    int s = lane < nw ? scratch[lane] : 0;
+    int si = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, si, o);
+      if (lane >= o) si += y;
+    }
+    if (lane < nw) scratch[lane] = si - s;
+    if (lane == 31) scratch[32] = si;
+  }
+  __syncthreads();
+  const int ex = scratch[warp] + incl - v;
+  *total = scratch[32];
+  __syncthreads();
+  return ex;
+}
+
+struct SchedArgs {
+  int T, K, E, H, I, Is, has_shared, bn;
+  int max_gu, max_dn;
+  WorkItem* items_gu;
+  WorkItem* items_dn;
+  int32_t* nitems;
+};
+
+// Work lists for the two grouped GEMMs from per-expert row counts. Expert e
+// (e == E: the shared expert, whose rows are the T tokens) gets
+// ceil(rows/bn) row tiles times its output tiles; within an expert the row
+// tile varies fastest so that neighbouring CTAs share a weight tile in L2.
+// Needs blockDim.x == 1024 and counts/offsets in shared memory.
+__device__ void build_schedule(const SchedArgs& a, const int* cnt, const int* off, int* scratch) {
+  const int nslots = a.E + (a.has_shared ? 1 : 0);
+  const int nt_gu_r = cdiv_dev(a.I, kTileN), nt_gu_s = cdiv_dev(a.Is, kTileN);
+  const int nt_dn = cdiv_dev(a.H, kTileN);
+  int ngu[2] = {0, 0}, ndn[2] = {0, 0}, nm[2] = {0, 0};
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const int e = 2 * threadIdx.x + q;
+    if (e < nslots) {
+      const bool sh = e == a.E;
+      const int rows = sh ? a.T : cnt[e];
+      nm[q] = (rows + a.bn - 1) / a.bn;
+      ngu[q] = nm[q] * (sh ? nt_gu_s : nt_gu_r);
+      ndn[q] = nm[q] * nt_dn;
+    }
+  }
+  int tot_gu, tot_dn;
+  const int base_gu = block_exscan2(ngu[0], ngu[1], scratch, &tot_gu);
+  const int base_dn = block_exscan2(ndn[0], ndn[1], scratch, &tot_dn);
+  int bg = base_gu, bd = base_dn;
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const int e = 2 * threadIdx.x + q;
+    if (e < nslots && nm[q] > 0) {
+      const bool sh = e == a.E;
+      const int rows = sh ? a.T : cnt[e];
+      const int r0 = sh ? 0 : off[e];
+      const int ntg = sh ? nt_gu_s : nt_gu_r;
+      for (int n = 0; n < ntg; ++n)
+        for (int m = 0; m < nm[q]; ++m) {
+          const int i = bg + n * nm[q] + m;
+          if (i < a.max_gu)
+            a.items_gu[i] = WorkItem{e, r0 + m * a.bn, min(a.bn, rows - m * a.bn), n};
+        }
+      for (int n = 0; n < nt_dn; ++n)
+        for (int m = 0; m < nm[q]; ++m) {
+          const int i = bd + n * nm[q] + m;
+          if (i < a.max_dn)
+            a.items_dn[i] = WorkItem{e, r0 + m * a.bn, min(a.bn, rows - m * a.bn), n};
+        }
+    }
+    bg += ngu[q];
+    bd += ndn[q];
+  }
+  if (threadIdx.x == 0) {
+    a.nitems[0] = min(tot_gu, a.max_gu);
+    a.nitems[1] = min(tot_dn, a.max_dn);
+  }
+}
+
+__global__ void __launch_bounds__(1024) perm_scan(int E, int n_ptiles,
+                                                  const int32_t* __restrict__ tile_cnt,
+                                                  int32_t* __restrict__ tile_base,
+                                                  int32_t* __restrict__ counts,
+                                                  int32_t* __restrict__ offsets, SchedArgs sa,
+                                                  int build) {
+  __shared__ int cnt[kMaxE + 1];
+  __shared__ int off[kMaxE + 1];
+  __shared__ int scratch[33];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  // per-expert totals: one warp per expert, lanes over tiles
+  for (int e = warp; e < E; e += nw) {
+    int s = 0;
+    for (int t = lane; t < n_ptiles; t += 32) s += tile_cnt[static_cast<size_t>(e) * n_ptiles + t];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) cnt[e] = s;
+  }
+  __syncthreads();
+  int total;
+  const int e0 = 2 * threadIdx.x;
+  const int c0 = e0 < E ? cnt[e0] : 0, c1 = e0 + 1 < E ? cnt[e0 + 1] : 0;
+  const int ex = block_exscan2(c0, c1, scratch, &total);
+  if (e0 < E) off[e0] = ex;
+  if (e0 + 1 < E) off[e0 + 1] = ex + c0;
+  if (threadIdx.x == 0) off[E] = total;
+  __syncthreads();
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) {
+    offsets[e] = off[e];
+    if (e < E) counts[e] = cnt[e];
+  }
+  // per-(expert, tile) exclusive bases: one warp per expert, warp scan over tiles
+  for (int e = warp; e < E; e += nw) {
+    int carry = off[e];
+    for (int t0 = 0; t0 < n_ptiles; t0 += 32) {
+      const int t = t0 + lane;
+      const int v = t < n_ptiles ? tile_cnt[static_cast<size_t>(e) * n_ptiles + t] : 0;
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (t < n_ptiles) tile_base[static_cast<size_t>(e) * n_ptiles + t] = carry + incl - v;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+  }
+  if (build) build_schedule(sa, cnt, off, scratch);
+}
+
+__global__ void __launch_bounds__(1024) schedule_only(const int32_t* __restrict__ offsets,
+                                                      SchedArgs sa) {
+  __shared__ int cnt[kMaxE + 1];
+  __shared__ int off[kMaxE + 1];
+  __shared__ int scratch[33];
+  for (int e = threadIdx.x; e < sa.E; e += blockDim.x) {
+    off[e] = offsets[e];
+    cnt[e] = offsets[e + 1] - offsets[e];
+  }
+  __syncthreads();
+  build_schedule(sa, cnt, off, scratch);
+}
+
+__global__ void __launch_bounds__(kScatterWarps * 32) perm_scatter(
+    int TK, int E, int n_ptiles, const int32_t* __restrict__ idx,
+    const int32_t* __restrict__ tile_base, int32_t* __restrict__ perm,
+    int32_t* __restrict__ inv_perm, int32_t* __restrict__ err) {
+  __shared__ int whist[kScatterWarps][kMaxE];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < kScatterWarps * E; i += blockDim.x) whist[i / E][i % E] = 0;
+  __syncthreads();
+  const int tbase = blockIdx.x * kPermTile;
+  const int n = min(kPermTile, TK - tbase);
+  constexpr int chunk = kPermTile / kScatterWarps;
+  const int c0 = warp * chunk, c1 = min(c0 + chunk, n);
+  const unsigned lt = (1u << lane) - 1u;
+  // pass 1: this warp's per-expert counts (its chunk is contiguous in flat order)
+  for (int r = c0; r < c1; r += 32) {
+    const int i = r + lane;
+    int e = -1;
+    if (i < c1) {
+      e = idx[tbase + i];
+      if (e < 0 || e >= E) e = -1;
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && (peers & lt) == 0) whist[warp][e] += __popc(peers);
+  }
+  __syncthreads();
+  // exclusive scan over warps, seeded with the tile's base for each expert
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = tile_base[static_cast<size_t>(e) * n_ptiles + blockIdx.x];
+#pragma unroll
+    for (int w = 0; w < kScatterWarps; ++w) {
+      const int v = whist[w][e];
+      whist[w][e] = run;
+      run += v;
+    }
+  }
+  __syncthreads();
+  // pass 2: stable positions
+  for (int r = c0; r < c1; r += 32) {
+    const int i = r + lane;
+    int e = -1;
+    if (i < c1) {
+      e = idx[tbase + i];
+      if (e < 0 || e >= E) e = -1;
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    int pos = -1;
+    if (e >= 0) pos = whist[warp][e] + __popc(peers & lt);
+    __syncwarp();
+    if (e >= 0 && (peers & lt) == 0) whist[warp][e] += __popc(peers);
+    __syncwarp();
+    if (i < c1) {
+      const int j = tbase + i;
+      if (e >= 0 && (pos < 0 || pos >= TK)) {  // cannot happen for consistent counts
+        atomicExch(err, MOE_DEVERR_SCHEDULE);
+        pos = -1;
+        e = -1;
+      }
+      if (e >= 0) perm[pos] = j;
+      if (inv_perm) inv_perm[j] = pos;
+    }
+  }
+}
+
+SchedArgs make_sched(const moe_cfg& c, int T, const WsLayout& L, WorkItem* gu, WorkItem* dn,
+                     int32_t* nitems) {
+  SchedArgs a;
+  a.T = T;
+  a.K = c.K;
+  a.E = c.E;
+  a.H = c.H;
+  a.I = c.I;
+  a.Is = c.I_shared;
+  a.has_shared = c.I_shared > 0;
+  a.bn = L.bn;
+  a.max_gu = L.max_items_gu;
+  a.max_dn = L.max_items_dn;
+  a.items_gu = gu;
+  a.items_dn = dn;
+  a.nitems = nitems;
+  return a;
+}
+
+}  // namespace
+
+cudaError_t launch_permute(const moe_cfg& c, int T, const int32_t* idx, int32_t* tile_cnt,
+                           int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv_perm,
+                           int32_t* err, const WsLayout& L, WorkItem* items_gu,
+                           WorkItem* items_dn, int32_t* nitems, cudaStream_t s) {
+  const int TK = T * c.K;
+  const int np = L.n_ptiles;
+  int32_t* tile_base = tile_cnt + static_cast<size_t>(c.E) * np;
+  perm_hist<<<np, 256, 0, s>>>(TK, c.E, np, idx, tile_cnt, err);
+  SchedArgs sa = make_sched(c, T, L, items_gu, items_dn, nitems);
+  perm_scan<<<1, 1024, 0, s>>>(c.E, np, tile_cnt, tile_base, counts, offsets, sa,
+                               items_gu != nullptr ? 1 : 0);
+  perm_scatter<<<np, kScatterWarps * 32, 0, s>>>(TK, c.E, np, idx, tile_base, perm, inv_perm,
+                                                 err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_schedule(const moe_cfg& c, int T, const int32_t* offsets, const WsLayout& L,
+                            WorkItem* items_gu, WorkItem* items_dn, int32_t* nitems,
+                            cudaStream_t s) {
+  SchedArgs sa = make_sched(c, T, L, items_gu, items_dn, nitems);
+  schedule_only<<<1, 1024, 0, s>>>(offsets, sa);
+  return cudaGetLastError();
+}
+
+}  // namespace sgl

@@ -1,0 +1,81 @@
+"""The C-ABI library without a GPU: it loads, exports every function that
+include/moe.h declares, sizes workspaces, and rejects bad arguments on the
+host (before any launch)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sigmoid_group_limited_b200 as sgl
+import workloads
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    return set(re.findall(r"MOE_API\s+[\w\s\*]*?\b(moe_\w+)\s*\(", src))
+
+
+def test_library_exports_every_declared_function():
+    L = sgl.lib()
+    decl = _declared()
+    assert decl == set(sgl.C_FUNCTIONS)
+    for name in decl:
+        assert hasattr(L, name), name
+    assert "sm_100a" in sgl.version()
+
+
+def test_status_strings():
+    L = sgl.lib()
+    for code, name in sgl.STATUS.items():
+        assert L.moe_status_string(code).decode().startswith(name)
+
+
+def test_workspace_size_full_configs():
+    for name in ("decode", "prefill", "zipf"):
+        cfg = workloads.CONFIGS[name]
+        n = sgl.workspace_size(cfg, cfg.T)
+        # dominated by y_slot: (T*K + T) rows of H bf16, plus h (T*K rows of I bf16)
+        lower = (cfg.T * cfg.K + cfg.T) * cfg.H * 2 + cfg.T * cfg.K * cfg.I * 2
+        assert lower <= n <= lower * 1.5 + (64 << 20)
+
+
+@pytest.mark.parametrize("field,value", [("H", 100), ("E", 48), ("n_group", 3), ("topk_group", 9),
+                                         ("K", 0), ("K", 33), ("I", 96), ("I_shared", -64),
+                                         ("wfmt", 7), ("scale", float("nan"))])
+def test_bad_config_rejected(field, value):
+    cfg = workloads.CONFIGS["decode"].with_(**{field: value})
+    c = sgl.make_cfg(cfg)
+    assert sgl.lib().moe_workspace_size(ctypes.byref(c), 32) == 0
+    st = sgl.lib().moe_route(ctypes.byref(c), 32, 16, 16, None, 16, 16, 16, 1 << 30, None)
+    assert st == -1
+
+
+def test_bad_token_count_rejected():
+    c = sgl.make_cfg(workloads.CONFIGS["decode"])
+    for T in (0, -1, (1 << 20) + 1):
+        assert sgl.lib().moe_workspace_size(ctypes.byref(c), T) == 0
+        assert sgl.lib().moe_permute(ctypes.byref(c), T, 16, 16, 16, 16, 16, 16, 1 << 30, None) == -1
+
+
+def test_null_misaligned_and_small_workspace_rejected_before_launch():
+    L = sgl.lib()
+    cfg = workloads.CONFIGS["decode"]
+    c = sgl.make_cfg(cfg)
+    need = sgl.workspace_size(cfg, 32)
+    A = 1 << 20  # fake, aligned "device" addresses: never dereferenced on these paths
+    assert L.moe_route(ctypes.byref(c), 32, None, A, None, A, A, A, need, None) == -2
+    assert L.moe_route(ctypes.byref(c), 32, A + 2, A, None, A, A, A, need, None) == -3
+    assert L.moe_route(ctypes.byref(c), 32, A, A, None, A, A, A, need - 1, None) == -4
+    assert L.moe_route(ctypes.byref(c), 32, A, A, None, A, None, A, need, None) == -2
+    assert L.moe_route(ctypes.byref(c), 32, A, A, None, A, A, None, need, None) == -4
+    w = sgl.moe_weights(A, A, A, None, None, None, A, A, None)   # shared Wd missing
+    assert L.moe_layer_forward(ctypes.byref(c), 32, A, A, None, ctypes.byref(w), A, None, None,
+                               None, A, need, None, None) == -2
+    w = sgl.moe_weights(A, A + 8, A, None, None, None, A, A, A)
+    assert L.moe_layer_forward(ctypes.byref(c), 32, A, A, None, ctypes.byref(w), A, None, None,
+                               None, A, need, None, None) == -3
+    assert L.moe_combine(ctypes.byref(c), 32, None, 1, A, None) == -2
+    assert L.moe_grouped_swiglu(ctypes.byref(c), 32, A, A, A, A, None, A, A, need, None) == -2

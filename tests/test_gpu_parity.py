@@ -1,0 +1,203 @@
+"""GPU parity: the CUDA path (through the C-ABI) against the CPU oracle on the
+same seeded inputs.
+
+Bars: routing indices bit-exact except listed near-tie tokens (oracle margin
+< 1e-6 between the 4th/5th group or the Kth/(K+1)th candidate); combine
+weights within 1e-6; permutation bit-exact; layer output max |err| <=
+2e-2 * RMS(oracle output) (bf16 weights). Full-size configs compare every
+token's routing and sampled tokens' outputs (the oracle runs those one by one).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sigmoid_group_limited_b200 as sgl
+import workloads
+from helpers import (DeviceExperts, bits, check_routing, check_y, host_inputs, near_tie_tokens,
+                     run_layer, run_staged)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _oracle_layer(cfg, d, tokens=None):
+    h = host_inputs(d)
+    return oracle.layer_forward(cfg, h["x"], h["Wr"], h["bias"], DeviceExperts(d), h["Wg_s"],
+                                h["Wu_s"], h["Wd_s"], tokens=tokens)
+
+
+def _full_check(cfg, d, tokens=None):
+    """Whole layer on the GPU vs the oracle; returns the oracle result."""
+    g = run_layer(cfg, d)
+    ref = _oracle_layer(cfg, d, tokens)
+    near = check_routing(ref, g["idx"].cpu().numpy(), g["w"].cpu().numpy())
+    counts = np.bincount(g["idx"].cpu().numpy().reshape(-1), minlength=cfg.E)
+    assert np.array_equal(g["counts"].cpu().numpy(), counts)
+    tok = ref["tokens"]
+    keep = ~np.isin(tok, near)
+    check_y(bits(g["y"])[tok[keep]], ref["y"][keep])
+    return g, ref, near
+
+
+# ------------------------------------------------------------------ small configs
+
+TINY = workloads.CONFIGS["tiny"]
+
+
+@pytest.mark.parametrize("T", [64, 1, 7, 33, 300, 600])
+def test_tiny_layer(T):
+    cfg = TINY
+    d = workloads.generate(cfg, DEV, T=T)
+    _full_check(cfg, d)
+
+
+@pytest.mark.parametrize("variant", [
+    dict(limit_routed=0.5, limit_shared=0.7),           # clamps that bite
+    dict(n_group=1, topk_group=1),                      # plain top-k
+    dict(K=1),                                          # argmax routing
+    dict(topk_group=4),                                 # all groups kept
+    dict(I_shared=0),                                   # no shared expert
+    dict(I=128, I_shared=192),                          # several output tiles, different sizes
+    dict(renorm=False),
+    dict(bias_kind="zero"),
+    dict(bias_kind="zipf"),
+])
+def test_tiny_variants(variant):
+    cfg = TINY.with_(**variant)
+    d = workloads.generate(cfg, DEV, T=200)
+    if cfg.I_shared == 0:
+        d.update(Wg_s=None, Wu_s=None, Wd_s=None)
+        g = run_layer(cfg, d)
+        h = host_inputs({**d, "Wg_s": torch.zeros(1, dtype=torch.bfloat16),
+                         "Wu_s": torch.zeros(1, dtype=torch.bfloat16),
+                         "Wd_s": torch.zeros(1, dtype=torch.bfloat16)})
+        # oracle with a zero shared expert (contributes exactly 0)
+        z = np.zeros((64, cfg.H), np.uint16)
+        ref = oracle.layer_forward(cfg.with_(I_shared=64), h["x"], h["Wr"], h["bias"],
+                                   DeviceExperts(d), z, z, z.T.copy())
+        check_routing(ref, g["idx"].cpu().numpy(), g["w"].cpu().numpy())
+        keep = ~np.isin(np.arange(200), near_tie_tokens(ref))
+        check_y(bits(g["y"])[keep], ref["y"][keep])
+    else:
+        _full_check(cfg, d)
+
+
+def test_tiny_staged_with_oracle_routing_and_y_slot():
+    cfg = TINY.with_(limit_routed=1.0, limit_shared=2.0)
+    d = workloads.generate(cfg, DEV, T=64)
+    ref = _oracle_layer(cfg, d)
+    idx = torch.from_numpy(ref["idx"]).to(DEV)
+    w = torch.from_numpy(ref["w"]).to(DEV)
+    g = run_staged(cfg, d, idx, w)
+    # permutation bit-exact against the oracle's stable counting sort
+    assert np.array_equal(g["counts"].cpu().numpy(), ref["counts"])
+    assert np.array_equal(g["offsets"].cpu().numpy(), ref["offsets"])
+    assert np.array_equal(g["perm"].cpu().numpy(), ref["perm"])
+    assert np.array_equal(g["inv"].cpu().numpy(), ref["inv_perm"])
+    ys = oracle.bf16_bits_to_f64(bits(g["y_slot"]))
+    T, K = 64, cfg.K
+    routed = ys[:T * K].reshape(T, K, cfg.H)
+    rs = ref["y_slot"].astype(np.float64)
+    assert np.abs(routed - rs).max() <= 1e-2 * np.sqrt((rs ** 2).mean())
+    sh = ys[T * K:]
+    ro = ref["y_shared"].astype(np.float64)
+    assert np.abs(sh - ro).max() <= 1e-2 * np.sqrt((ro ** 2).mean())
+    check_y(bits(g["y"]), ref["y"])
+
+
+def test_tiny_identical_experts_closed_form():
+    """All routed experts equal: y = bf16(2.5 FFN(x) + shared(x)) whatever the routing."""
+    cfg = TINY
+    d = workloads.generate(cfg, DEV, T=64)
+    for k in ("Wg", "Wu", "Wd"):
+        d[k] = d[k][:1].expand_as(d[k]).contiguous()
+    g = run_layer(cfg, d)
+    f = oracle.bf16_bits_to_f64
+    x = f(bits(d["x"]))
+    o, _ = oracle.swiglu_expert(x, f(bits(d["Wg"][0])), f(bits(d["Wu"][0])), f(bits(d["Wd"][0])))
+    osh, _ = oracle.swiglu_expert(x, f(bits(d["Wg_s"])), f(bits(d["Wu_s"])), f(bits(d["Wd_s"])))
+    expect = oracle.f32_to_bf16_bits((2.5 * o.astype(np.float64) + osh).astype(np.float32))
+    check_y(bits(g["y"]), expect)
+
+
+def test_deterministic_bits():
+    cfg = TINY
+    d = workloads.generate(cfg, DEV, T=300)
+    a = run_layer(cfg, d)
+    b = run_layer(cfg, d)
+    assert torch.equal(a["y"].view(torch.int16), b["y"].view(torch.int16))
+    assert torch.equal(a["idx"], b["idx"])
+
+
+# ------------------------------------------------------------------ permutation alone
+
+@pytest.mark.parametrize("T,skew", [(1, False), (32, False), (300, False), (4096, False),
+                                    (16384, False), (4096, True), (2049, True)])
+def test_permute_bit_exact(T, skew):
+    cfg = workloads.CONFIGS["prefill"]
+    g = torch.Generator().manual_seed(T)
+    if skew:
+        idx = torch.full((T, cfg.K), 7, dtype=torch.int32)
+        idx[:, 1:] = torch.randint(0, 3, (T, cfg.K - 1), generator=g, dtype=torch.int32)
+    else:
+        idx = torch.randint(0, cfg.E, (T, cfg.K), generator=g, dtype=torch.int32)
+    ws = sgl.alloc_workspace(cfg, T)
+    out = [torch.empty(n, dtype=torch.int32, device=DEV)
+           for n in (cfg.E, cfg.E + 1, T * cfg.K, T * cfg.K)]
+    sgl.moe_permute(cfg, T, idx.to(DEV), *out, ws)
+    torch.cuda.synchronize()
+    ref = oracle.permute(idx.numpy(), cfg.E)
+    for a, b in zip(out, ref):
+        assert np.array_equal(a.cpu().numpy(), b)
+    assert sgl.moe_read_error(cfg, T, ws) == 0
+
+
+def test_permute_bad_id_sets_error_word():
+    cfg = workloads.CONFIGS["prefill"]
+    T = 40
+    idx = torch.randint(0, cfg.E, (T, cfg.K), dtype=torch.int32)
+    idx[3, 2] = cfg.E + 5
+    idx[9, 0] = -1
+    ws = sgl.alloc_workspace(cfg, T)
+    out = [torch.empty(n, dtype=torch.int32, device=DEV)
+           for n in (cfg.E, cfg.E + 1, T * cfg.K, T * cfg.K)]
+    sgl.moe_permute(cfg, T, idx.to(DEV), *out, ws)
+    torch.cuda.synchronize()
+    assert sgl.moe_read_error(cfg, T, ws) == 1
+    assert out[0].sum().item() == T * cfg.K - 2       # bad slots are dropped
+    assert sgl.moe_read_error(cfg, T, ws) == 0        # reading clears the word
+
+
+# ------------------------------------------------------------------ full size
+
+def _sample(T, n, seed):
+    rng = np.random.default_rng(seed)
+    s = set(range(min(4, T))) | {T - 1} | set(rng.choice(T, size=min(n, T), replace=False).tolist())
+    return np.array(sorted(s))
+
+
+@pytest.mark.slow
+def test_decode_full_size():
+    cfg = workloads.CONFIGS["decode"]
+    d = workloads.generate(cfg, DEV)
+    _full_check(cfg, d)          # every one of the 32 tokens
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["prefill", "prefill_bias0", "zipf"])
+def test_full_size_sampled(name):
+    cfg = workloads.CONFIGS[name]
+    d = workloads.generate(cfg, DEV)
+    tok = _sample(cfg.T, 12, cfg.seed)
+    g, ref, near = _full_check(cfg, d, tokens=tok)
+    # permutation of the GPU's own routing, bit-exact, on every slot
+    st = run_staged(cfg, d, g["idx"], g["w"])
+    p_ref = oracle.permute(g["idx"].cpu().numpy(), cfg.E)
+    assert np.array_equal(st["perm"].cpu().numpy(), p_ref[2])
+    assert np.array_equal(st["offsets"].cpu().numpy(), p_ref[1])
+    # staged path with the oracle's own routing covers the near-tie tokens too
+    st2 = run_staged(cfg, d, torch.from_numpy(ref["idx"]).to(DEV), torch.from_numpy(ref["w"]).to(DEV))
+    check_y(bits(st2["y"])[tok], ref["y"])
+    del d
+    torch.cuda.empty_cache()
