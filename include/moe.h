@@ -29,7 +29,9 @@
  *    launched (host-side validation) or a launch failed (MOE_ERR_CUDA).
  *  - Kernels that detect bad data (an expert id out of range, a wait that
  *    timed out) set an error word inside the workspace instead of trapping;
- *    read it with moe_read_error().
+ *    read it with moe_read_error(). moe_route, moe_permute and
+ *    moe_layer_forward clear the word when they start; moe_grouped_swiglu
+ *    and moe_combine only add to it.
  *  - bf16 tensors are raw bfloat16 (uint16) arrays; all matrices are
  *    row-major with the reduction (K) dimension contiguous: Wr [E,H] fp32,
  *    Wg/Wu [E,I,H], Wd [E,H,I], Wg_s/Wu_s [I_s,H], Wd_s [H,I_s].
@@ -126,7 +128,7 @@ MOE_API moe_status moe_permute(const moe_cfg* cfg, int32_t T, const int32_t* idx
 /* Stage 7 (and 8 when shared weights are given): grouped SwiGLU experts on
  * tcgen05 tensor cores (page 3 sec. 2 and sec. 4).
  * in: x [T,H] bf16, perm and offsets from moe_permute, w [T,K] fp32;
- * out: y_slot [(T*K + T), H] bf16 where row j = t*K + k holds
+ * out: y_slot [(T*K + T), H] fp32 where row j = t*K + k holds
  *      w[t,k] * Expert_{idx[t,k]}(x_t) and row T*K + t holds the shared
  *      expert's output for token t (left untouched without shared weights).
  * All device. */
@@ -137,7 +139,8 @@ MOE_API moe_status moe_grouped_swiglu(const moe_cfg* cfg, int32_t T, const void*
 /* Stage 9, weighted combine back to token order:
  * y[t] = bf16( (sum over k = 0..K-1 of y_slot[t*K+k]) + y_slot[T*K+t] ),
  * summed in fp32 in slot order; the shared row is added only when
- * with_shared != 0. y_slot as produced by moe_grouped_swiglu; y [T,H] bf16. */
+ * with_shared != 0. y_slot (fp32) as produced by moe_grouped_swiglu;
+ * y [T,H] bf16, rounded once (nearest even). */
 MOE_API moe_status moe_combine(const moe_cfg* cfg, int32_t T, const void* y_slot, int32_t with_shared,
                        void* y, void* stream);
 

@@ -266,8 +266,9 @@ def layer_forward(cfg, x_bits: np.ndarray, Wr: np.ndarray, bias: np.ndarray,
     limit_shared. With `tokens` given, routing still covers all rows of x but
     the expert stages run only for those tokens (sampled outputs of a large
     batch). Returns a dict with the routing results, permutation, h of the
-    shared expert, y_slot [n,K,H] fp32 and y bf16 bits [n,H] for the
-    evaluated tokens (in the order of `tokens`)."""
+    shared expert, y_slot [n,K,H] fp32, the fp32 output before its final
+    rounding y_f32 [n,H] and y bf16 bits [n,H] for the evaluated tokens (in
+    the order of `tokens`)."""
     r = route(x_bits, Wr, bias, cfg.n_group, cfg.topk_group, cfg.K, cfg.scale, cfg.renorm)
     counts, offsets, perm, inv_perm = permute(r["idx"], cfg.E)
     T = x_bits.shape[0]
@@ -291,5 +292,5 @@ def layer_forward(cfg, x_bits: np.ndarray, Wr: np.ndarray, bias: np.ndarray,
     y = f32_to_bf16_bits(acc)
     out = dict(r)
     out.update(counts=counts, offsets=offsets, perm=perm, inv_perm=inv_perm,
-               tokens=tok, y_slot=y_slot, y_shared=o_sh, h_shared=h_sh, y=y)
+               tokens=tok, y_slot=y_slot, y_shared=o_sh, h_shared=h_sh, y_f32=acc, y=y)
     return out

@@ -47,6 +47,7 @@ WsLayout ws_layout(const moe_cfg& c, int T) {
   L.err = take(16);
   L.nitems = take(16);
   L.z = take(static_cast<size_t>(T) * c.E * 4);
+  L.unc = take(static_cast<size_t>(T) * 4);
   L.tile_hist = take(static_cast<size_t>(2) * c.E * L.n_ptiles * 4);
   L.idx = take(TK * 4);
   L.w = take(TK * 4);
@@ -58,7 +59,7 @@ WsLayout ws_layout(const moe_cfg& c, int T) {
   L.items_dn = take(static_cast<size_t>(L.max_items_dn) * sizeof(WorkItem));
   L.h_r = take(TK * c.I * 2);
   L.h_s = take(static_cast<size_t>(T) * (c.I_shared > 0 ? c.I_shared : 0) * 2);
-  L.y_slot = take((TK + T) * c.H * 2);
+  L.y_slot = take((TK + T) * c.H * 4);
   L.total = o;
   return L;
 }
@@ -143,7 +144,7 @@ moe_status moe_route(const moe_cfg* cfg, int32_t T, const void* x, const float* 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(at<int32_t>(ws, L.err), 0, 16, s) != cudaSuccess) return MOE_ERR_CUDA;
   return cu(launch_router(*cfg, T, static_cast<const uint16_t*>(x), Wr, bias, at<float>(ws, L.z),
-                          idx, w, s));
+                          idx, w, at<int32_t>(ws, L.unc), at<int32_t>(ws, L.err) + 1, s));
 }
 
 moe_status moe_permute(const moe_cfg* cfg, int32_t T, const int32_t* idx, int32_t* counts,
@@ -158,6 +159,7 @@ moe_status moe_permute(const moe_cfg* cfg, int32_t T, const int32_t* idx, int32_
   moe_status st = device_ok();
   if (st != MOE_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(at<int32_t>(ws, L.err), 0, 16, s) != cudaSuccess) return MOE_ERR_CUDA;
   return cu(launch_permute(*cfg, T, idx, at<int32_t>(ws, L.tile_hist), counts, offsets, perm,
                            inv_perm, at<int32_t>(ws, L.err), L, nullptr, nullptr,
                            at<int32_t>(ws, L.nitems), s));
@@ -190,7 +192,7 @@ moe_status moe_grouped_swiglu(const moe_cfg* cfg, int32_t T, const void* x, cons
   a.W = W;
   a.h_r = at<uint16_t>(ws, L.h_r);
   a.h_s = at<uint16_t>(ws, L.h_s);
-  a.y_slot = static_cast<uint16_t*>(y_slot);
+  a.y_slot = static_cast<float*>(y_slot);
   a.items_gu = gu;
   a.items_dn = dn;
   a.nitems = nitems;
@@ -209,7 +211,7 @@ moe_status moe_combine(const moe_cfg* cfg, int32_t T, const void* y_slot, int32_
   if (!al16(y_slot) || !al16(y)) return MOE_ERR_ALIGN;
   moe_status st = device_ok();
   if (st != MOE_OK) return st;
-  return cu(launch_combine(*cfg, T, static_cast<const uint16_t*>(y_slot), with_shared ? 1 : 0,
+  return cu(launch_combine(*cfg, T, static_cast<const float*>(y_slot), with_shared ? 1 : 0,
                            static_cast<uint16_t*>(y), static_cast<cudaStream_t>(stream)));
 }
 
@@ -242,12 +244,12 @@ moe_status moe_layer_forward(const moe_cfg* cfg, int32_t T, const void* x, const
   WorkItem* gu = at<WorkItem>(ws, L.items_gu);
   WorkItem* dn = at<WorkItem>(ws, L.items_dn);
   int32_t* nitems = at<int32_t>(ws, L.nitems);
-  uint16_t* y_slot = at<uint16_t>(ws, L.y_slot);
+  float* y_slot = at<float>(ws, L.y_slot);
   cudaError_t e;
   rec(0);
   if (cudaMemsetAsync(err, 0, 16, s) != cudaSuccess) return MOE_ERR_CUDA;
   if ((e = launch_router(*cfg, T, static_cast<const uint16_t*>(x), Wr, bias, at<float>(ws, L.z),
-                         idx, w, s)) != cudaSuccess)
+                         idx, w, at<int32_t>(ws, L.unc), err + 1, s)) != cudaSuccess)
     return MOE_ERR_CUDA;
   rec(1);
   if ((e = launch_permute(*cfg, T, idx, at<int32_t>(ws, L.tile_hist), counts, offsets, perm,

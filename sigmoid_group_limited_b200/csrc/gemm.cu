@@ -14,7 +14,7 @@
 //            h = bf16(silu(clamp(D_g)) * clamp(D_u)), stored in permuted row
 //            order; the token rows are gathered from x with TMA gather4.
 //   down:    D [128 features x BN rows] over K = I, epilogue
-//            y_slot[j] = bf16(w_j * D) written to the slot's flat index j.
+//            y_slot[j] = w_j * D (fp32) written to the slot's flat index j.
 // Work items (expert, row tile, output tile) come from a device-built list;
 // each CTA walks the list with a grid stride. Warp roles per CTA:
 //   warp 0  TMA producer (one lane), warp 1  MMA issuer (one lane) and TMEM
@@ -45,7 +45,7 @@ struct GemmParams {
   const float* w;
   uint16_t* h_r;  // [T*K, I] permuted rows
   uint16_t* h_s;  // [T, Is]
-  uint16_t* y_slot;
+  float* y_slot;   // [(T*K + T), H] fp32
   const WorkItem* items;
   const int32_t* nitems;  // device count of valid items
   int max_items;
@@ -311,7 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   }
                   wt = p.w[j];
                 }
-                p.y_slot[static_cast<size_t>(j) * p.H + nfeat] = f2bf(wt * ov[c]);
+                p.y_slot[static_cast<size_t>(j) * p.H + nfeat] = wt * ov[c];
               }
             }
           }

@@ -36,7 +36,7 @@ inline int cdiv(long long a, long long b) { return static_cast<int>((a + b - 1) 
 __host__ __device__ inline int cdiv_dev(int a, int b) { return (a + b - 1) / b; }
 
 struct WsLayout {
-  size_t z, tile_hist, idx, w, counts, offsets, perm, inv_perm, items_gu, items_dn, nitems, h_r,
+  size_t z, unc, tile_hist, idx, w, counts, offsets, perm, inv_perm, items_gu, items_dn, nitems, h_r,
       h_s, y_slot, err, total;
   int n_ptiles, bn, max_items_gu, max_items_dn;
 };
@@ -44,8 +44,11 @@ struct WsLayout {
 WsLayout ws_layout(const moe_cfg& c, int T);
 
 // Launchers (return cudaGetLastError()).
+// Routing. unc [T] / unc_n: scratch list (and its count, zeroed by the
+// caller) of tokens whose fp32 decision is re-derived from exact logits.
 cudaError_t launch_router(const moe_cfg& c, int T, const uint16_t* x, const float* Wr,
-                          const float* bias, float* z, int32_t* idx, float* w, cudaStream_t s);
+                          const float* bias, float* z, int32_t* idx, float* w, int32_t* unc,
+                          int32_t* unc_n, cudaStream_t s);
 
 cudaError_t launch_permute(const moe_cfg& c, int T, const int32_t* idx, int32_t* tile_hist,
                            int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv_perm,
@@ -65,7 +68,7 @@ struct GemmArgs {
   const moe_weights* W;
   uint16_t* h_r;
   uint16_t* h_s;
-  uint16_t* y_slot;
+  float* y_slot;
   const WorkItem* items_gu;
   const WorkItem* items_dn;
   const int32_t* nitems;
@@ -78,7 +81,7 @@ struct GemmArgs {
 cudaError_t launch_gemm_gateup(const GemmArgs& a, cudaStream_t s);
 cudaError_t launch_gemm_down(const GemmArgs& a, cudaStream_t s);
 
-cudaError_t launch_combine(const moe_cfg& c, int T, const uint16_t* y_slot, int with_shared,
+cudaError_t launch_combine(const moe_cfg& c, int T, const float* y_slot, int with_shared,
                            uint16_t* y, cudaStream_t s);
 
 int num_sms();

@@ -15,64 +15,74 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <algorithm>
+
 #include "internal.h"
 
 namespace sgl {
 namespace {
 
-__device__ __forceinline__ float bf16_to_f32(uint16_t b) {
-  return __uint_as_float(static_cast<uint32_t>(b) << 16);
-}
-
 // ---------------------------------------------------------------------------
-// Logits for small batches (T <= 32): one warp per expert. The tokens sit in
-// shared memory as bf16; each lane holds a strided slice of the expert's
-// fp32 router row in registers and accumulates lane partial sums in fp32,
-// finished by a butterfly sum across the warp.
+// Exact logits for a list of rows: one warp per expert, the expert's fp32
+// router row held in registers (a strided slice per lane), up to 32 token
+// rows staged in shared memory as bf16. Every product bf16 * fp32 is exact
+// in float64 and the sum of 2560 of them is accumulated in float64, so the
+// single final rounding to fp32 gives the same logit as an exact dot
+// product. Used for whole decode batches and to re-derive the logits of the
+// tokens whose fp32 routing decision was too close to call.
 // ---------------------------------------------------------------------------
 constexpr int kSmallT = 32;
 constexpr int kRowRegs = 24;  // float4 per lane: H <= 24 * 128 = 3072
+constexpr int kRowWarps = 4;
 
-__global__ void __launch_bounds__(256) router_logits_small(int T, int H, int E,
-                                                           const uint16_t* __restrict__ x,
-                                                           const float* __restrict__ Wr,
-                                                           float* __restrict__ z) {
-  extern __shared__ __align__(16) uint16_t xs[];  // [T][H]
-  const int tid = threadIdx.x;
-  {
-    const int n16 = T * H / 8;  // 16-byte chunks
-    const uint4* src = reinterpret_cast<const uint4*>(x);
-    uint4* dst = reinterpret_cast<uint4*>(xs);
-    for (int i = tid; i < n16; i += blockDim.x) dst[i] = src[i];
-  }
-  __syncthreads();
-  const int warp = tid >> 5, lane = tid & 31;
-  const int e = blockIdx.x * 8 + warp;
-  if (e >= E) return;
-  const float* row = Wr + static_cast<size_t>(e) * H;
+__global__ void __launch_bounds__(kRowWarps * 32) router_logits_exact(
+    int T, int H, int E, const uint16_t* __restrict__ x, const float* __restrict__ Wr,
+    float* __restrict__ z, const int32_t* __restrict__ list, const int32_t* __restrict__ list_n) {
+  extern __shared__ __align__(16) uint16_t xs[];  // [kSmallT][H]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int e = blockIdx.x * kRowWarps + warp;
+  const bool have = e < E;
+  const int n = list ? min(*list_n, T) : T;
   float4 wv[kRowRegs];
 #pragma unroll
   for (int j = 0; j < kRowRegs; ++j) {
     const int k = 4 * lane + 128 * j;
-    wv[j] = (k < H) ? *reinterpret_cast<const float4*>(row + k) : make_float4(0.f, 0.f, 0.f, 0.f);
+    wv[j] = (have && k < H) ? *reinterpret_cast<const float4*>(Wr + static_cast<size_t>(e) * H + k)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  for (int t = 0; t < T; ++t) {
-    const uint16_t* xr = xs + t * H;
-    float acc = 0.f;
+  const int c16 = H / 8;  // 16-byte chunks per row
+  for (int c0 = 0; c0 < n; c0 += kSmallT) {
+    const int nc = min(kSmallT, n - c0);
+    __syncthreads();
+    for (int i = tid; i < nc * c16; i += blockDim.x) {
+      const int r = i / c16, c = i - r * c16;
+      const int t = list ? list[c0 + r] : c0 + r;
+      reinterpret_cast<uint4*>(xs)[r * c16 + c] =
+          reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H)[c];
+    }
+    __syncthreads();
+    if (!have) continue;
+    for (int r = 0; r < nc; ++r) {
+      const uint16_t* xr = xs + r * H;
+      double acc = 0.0;
 #pragma unroll
-    for (int j = 0; j < kRowRegs; ++j) {
-      const int k = 4 * lane + 128 * j;
-      if (k < H) {
-        const uint2 p = *reinterpret_cast<const uint2*>(xr + k);
-        acc = fmaf(wv[j].x, __uint_as_float(p.x << 16), acc);
-        acc = fmaf(wv[j].y, __uint_as_float(p.x & 0xFFFF0000u), acc);
-        acc = fmaf(wv[j].z, __uint_as_float(p.y << 16), acc);
-        acc = fmaf(wv[j].w, __uint_as_float(p.y & 0xFFFF0000u), acc);
+      for (int j = 0; j < kRowRegs; ++j) {
+        const int k = 4 * lane + 128 * j;
+        if (k < H) {
+          const uint2 p = *reinterpret_cast<const uint2*>(xr + k);
+          acc = fma(static_cast<double>(wv[j].x), static_cast<double>(__uint_as_float(p.x << 16)), acc);
+          acc = fma(static_cast<double>(wv[j].y), static_cast<double>(__uint_as_float(p.x & 0xFFFF0000u)), acc);
+          acc = fma(static_cast<double>(wv[j].z), static_cast<double>(__uint_as_float(p.y << 16)), acc);
+          acc = fma(static_cast<double>(wv[j].w), static_cast<double>(__uint_as_float(p.y & 0xFFFF0000u)), acc);
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (lane == 0) {
+        const int t = list ? list[c0 + r] : c0 + r;
+        z[static_cast<size_t>(t) * E + e] = static_cast<float>(acc);
       }
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) z[static_cast<size_t>(t) * E + e] = acc;
   }
 }
 
@@ -167,6 +177,13 @@ __global__ void __launch_bounds__(256) router_logits_tiled(int T, int H, int E,
 // Scores and group-limited top-k: one warp per token. Lane l holds experts
 // e = l + 32*j. Scores use a float64 sigmoid rounded to fp32; the weights are
 // computed in float64 from the fp32 scores and rounded once.
+//
+// Certification: with tau > 0 the kernel also measures its own decision
+// margins (the topk_group-th minus the next group score, and every gap
+// between neighbours in the ranking of the K+1 best candidates, since slot
+// order is rank order) and appends the token to `unc` when one is below tau;
+// those tokens get exact logits and a second pass (list mode) before anything
+// downstream reads idx / w.
 // ---------------------------------------------------------------------------
 template <int NV>
 __global__ void __launch_bounds__(256) router_topk(int T, int E, int n_group, int topk_group,
@@ -174,162 +191,221 @@ __global__ void __launch_bounds__(256) router_topk(int T, int E, int n_group, in
                                                    const float* __restrict__ z,
                                                    const float* __restrict__ bias,
                                                    int32_t* __restrict__ idx,
-                                                   float* __restrict__ wout) {
+                                                   float* __restrict__ wout, float tau,
+                                                   int32_t* __restrict__ unc,
+                                                   int32_t* __restrict__ unc_n,
+                                                   const int32_t* __restrict__ list,
+                                                   const int32_t* __restrict__ list_n) {
   const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (t >= T) return;
+  const int wpb = blockDim.x >> 5;
+  const int n = list ? min(*list_n, T) : T;
   const int per = E / n_group;
-  const float* zr = z + static_cast<size_t>(t) * E;
-  float s[NV], b[NV];
-  int g[NV];
+  for (int q = blockIdx.x * wpb + (threadIdx.x >> 5); q < n; q += gridDim.x * wpb) {
+    const int t = list ? list[q] : q;
+    const float* zr = z + static_cast<size_t>(t) * E;
+    float s[NV], b[NV];
+    int g[NV];
 #pragma unroll
-  for (int j = 0; j < NV; ++j) {
-    const int e = lane + 32 * j;
-    if (e < E) {
-      const float zz = zr[e];
-      s[j] = static_cast<float>(1.0 / (1.0 + exp(-static_cast<double>(zz))));
-      b[j] = s[j] + (bias ? bias[e] : 0.f);
-      g[j] = e / per;
-    } else {
-      s[j] = 0.f;
-      b[j] = -INFINITY;
-      g[j] = -1;
+    for (int j = 0; j < NV; ++j) {
+      const int e = lane + 32 * j;
+      if (e < E) {
+        const float zz = zr[e];
+        s[j] = static_cast<float>(1.0 / (1.0 + exp(-static_cast<double>(zz))));
+        b[j] = s[j] + (bias ? bias[e] : 0.f);
+        g[j] = e / per;
+      } else {
+        s[j] = 0.f;
+        b[j] = -INFINITY;
+        g[j] = -1;
+      }
     }
-  }
-  // group score (max of b) held by lane g
-  float my_gscore = -INFINITY;
-  for (int gg = 0; gg < n_group; ++gg) {
-    float m = -INFINITY;
+    // group score (max of b) held by lane g
+    float my_gscore = -INFINITY;
+    for (int gg = 0; gg < n_group; ++gg) {
+      float m = -INFINITY;
 #pragma unroll
-    for (int j = 0; j < NV; ++j)
-      if (g[j] == gg && b[j] > m) m = b[j];
+      for (int j = 0; j < NV; ++j)
+        if (g[j] == gg && b[j] > m) m = b[j];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float other = __shfl_xor_sync(0xffffffffu, m, o);
-      m = other > m ? other : m;
+      for (int o = 16; o > 0; o >>= 1) {
+        const float other = __shfl_xor_sync(0xffffffffu, m, o);
+        m = other > m ? other : m;
+      }
+      if (lane == gg) my_gscore = m;
     }
-    if (lane == gg) my_gscore = m;
-  }
-  // keep topk_group groups: repeated argmax over lanes < n_group, ties -> lower lane
-  bool my_kept = false;
-  {
-    float v = lane < n_group ? my_gscore : -INFINITY;
-    bool avail = lane < n_group;
-    for (int r = 0; r < topk_group; ++r) {
-      float bv = avail ? v : -INFINITY;
-      int bi = avail ? lane : 0x7fffffff;
+    // keep topk_group groups: repeated argmax over lanes < n_group, ties -> lower lane;
+    // one more round (when a group is left) gives the group margin
+    bool my_kept = false;
+    float last_kept = 0.f, gmargin = INFINITY;
+    {
+      bool avail = lane < n_group;
+      const int rounds = topk_group < n_group ? topk_group + 1 : topk_group;
+      for (int r = 0; r < rounds; ++r) {
+        float bv = avail ? my_gscore : -INFINITY;
+        int bi = avail ? lane : 0x7fffffff;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+          const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+          if (ov > bv || (ov == bv && oi < bi)) {
+            bv = ov;
+            bi = oi;
+          }
+        }
+        if (r < topk_group) {
+          if (lane == bi) {
+            my_kept = true;
+            avail = false;
+          }
+          last_kept = bv;
+        } else {
+          gmargin = last_kept - bv;
+        }
+      }
+    }
+    uint32_t cand = 0;
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      const int src = g[j] < 0 ? 0 : g[j];
+      const bool k = __shfl_sync(0xffffffffu, my_kept ? 1 : 0, src) != 0;
+      if (k && g[j] >= 0) cand |= 1u << j;
+    }
+    // K rounds of warp argmax over candidates (ties -> lower expert id), plus
+    // one more for the expert margin
+    int my_e = -1;
+    float my_s = 0.f, last_b = 0.f, emargin = INFINITY;
+    for (int k = 0; k <= K; ++k) {
+      float bv = -INFINITY;
+      int be = 0x7fffffff;
+#pragma unroll
+      for (int j = 0; j < NV; ++j) {
+        if ((cand >> j) & 1u) {
+          if (b[j] > bv || be == 0x7fffffff) {
+            bv = b[j];
+            be = lane + 32 * j;
+          }
+        }
+      }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
         const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (ov > bv || (ov == bv && oi < bi)) {
+        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+        if (ov > bv || (ov == bv && oe < be)) {
           bv = ov;
-          bi = oi;
+          be = oe;
         }
       }
-      if (lane == bi) {
-        my_kept = true;
-        avail = false;
-      }
-    }
-  }
-  uint32_t cand = 0;
+      // every adjacent gap of the ranking counts: slot order is rank order
+      if (k > 0 && be != 0x7fffffff) emargin = fminf(emargin, last_b - bv);
+      if (k == K) break;
+      // owner lane removes the winner and publishes its unbiased score
+      const int owner = be & 31, jw = be >> 5;
+      float sw = 0.f;
 #pragma unroll
-  for (int j = 0; j < NV; ++j) {
-    const int src = g[j] < 0 ? 0 : g[j];
-    const bool k = __shfl_sync(0xffffffffu, my_kept ? 1 : 0, src) != 0;
-    if (k && g[j] >= 0) cand |= 1u << j;
-  }
-  // K rounds of warp argmax over candidates (ties -> lower expert id)
-  int my_e = -1;
-  float my_s = 0.f;
-  for (int k = 0; k < K; ++k) {
-    float bv = -INFINITY;
-    int be = 0x7fffffff;
-#pragma unroll
-    for (int j = 0; j < NV; ++j) {
-      if ((cand >> j) & 1u) {
-        if (b[j] > bv || be == 0x7fffffff) {
-          bv = b[j];
-          be = lane + 32 * j;
+      for (int j = 0; j < NV; ++j)
+        if (j == jw && lane == owner) {
+          sw = s[j];
+          cand &= ~(1u << j);
         }
+      sw = __shfl_sync(0xffffffffu, sw, owner);
+      if (lane == k) {
+        my_e = be;
+        my_s = sw;
       }
+      last_b = bv;
     }
+    double den;
+    {
+      double v = (lane < K) ? static_cast<double>(my_s) : 0.0;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      if (ov > bv || (ov == bv && oe < be)) {
-        bv = ov;
-        be = oe;
-      }
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      den = v;  // exact: a sum of K <= 32 fp32 values of similar magnitude
     }
-    // owner lane removes the winner and publishes its unbiased score
-    const int owner = be & 31, jw = be >> 5;
-    float sw = 0.f;
-#pragma unroll
-    for (int j = 0; j < NV; ++j)
-      if (j == jw && lane == owner) {
-        sw = s[j];
-        cand &= ~(1u << j);
-      }
-    sw = __shfl_sync(0xffffffffu, sw, owner);
-    if (lane == k) {
-      my_e = be;
-      my_s = sw;
+    if (lane < K) {
+      const double sk = static_cast<double>(my_s);
+      const double wv = renorm ? static_cast<double>(scale) * (sk / den)
+                               : static_cast<double>(scale) * sk;
+      idx[static_cast<size_t>(t) * K + lane] = my_e;
+      wout[static_cast<size_t>(t) * K + lane] = static_cast<float>(wv);
     }
-  }
-  double den = 0.0;
-  {
-    double v = (lane < K) ? static_cast<double>(my_s) : 0.0;
+    if (tau > 0.f) {
+      // the fp32 logit error grows with the logits' magnitude: scale the margin
+      float zz = 0.f;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    den = v;  // exact: a sum of K <= 32 fp32 values of similar magnitude
-  }
-  if (lane < K) {
-    const double sk = static_cast<double>(my_s);
-    const double wv = renorm ? static_cast<double>(scale) * (sk / den)
-                             : static_cast<double>(scale) * sk;
-    idx[static_cast<size_t>(t) * K + lane] = my_e;
-    wout[static_cast<size_t>(t) * K + lane] = static_cast<float>(wv);
+      for (int j = 0; j < NV; ++j)
+        if (lane + 32 * j < E) zz = fmaf(zr[lane + 32 * j], zr[lane + 32 * j], zz);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) zz += __shfl_xor_sync(0xffffffffu, zz, o);
+      const float tau_t = tau * fmaxf(1.f, sqrtf(zz / E));
+      if (lane == 0 && (gmargin < tau_t || emargin < tau_t)) unc[atomicAdd(unc_n, 1)] = t;
+    }
   }
 }
 
 template <int NV>
 cudaError_t launch_topk(const moe_cfg& c, int T, const float* z, const float* bias, int32_t* idx,
-                        float* w, cudaStream_t s) {
+                        float* w, float tau, int32_t* unc, int32_t* unc_n, const int32_t* list,
+                        cudaStream_t s) {
   const int warps = 8;
-  router_topk<NV><<<cdiv(T, warps), warps * 32, 0, s>>>(T, c.E, c.n_group, c.topk_group, c.K,
-                                                        c.scale, c.renorm, z, bias, idx, w);
+  int grid = cdiv(T, warps);
+  if (list) grid = std::min(grid, num_sms() * 4);
+  router_topk<NV><<<grid, warps * 32, 0, s>>>(T, c.E, c.n_group, c.topk_group, c.K, c.scale,
+                                              c.renorm, z, bias, idx, w, tau, unc, unc_n, list,
+                                              list ? unc_n : nullptr);
+  return cudaGetLastError();
+}
+
+cudaError_t topk_dispatch(const moe_cfg& c, int T, const float* z, const float* bias,
+                          int32_t* idx, float* w, float tau, int32_t* unc, int32_t* unc_n,
+                          const int32_t* list, cudaStream_t s) {
+  const int nv = cdiv(c.E, 32);
+  if (nv <= 1) return launch_topk<1>(c, T, z, bias, idx, w, tau, unc, unc_n, list, s);
+  if (nv <= 2) return launch_topk<2>(c, T, z, bias, idx, w, tau, unc, unc_n, list, s);
+  if (nv <= 4) return launch_topk<4>(c, T, z, bias, idx, w, tau, unc, unc_n, list, s);
+  if (nv <= 8) return launch_topk<8>(c, T, z, bias, idx, w, tau, unc, unc_n, list, s);
+  if (nv <= 16) return launch_topk<16>(c, T, z, bias, idx, w, tau, unc, unc_n, list, s);
+  return launch_topk<32>(c, T, z, bias, idx, w, tau, unc, unc_n, list, s);
+}
+
+cudaError_t launch_exact(const moe_cfg& c, int T, const uint16_t* x, const float* Wr, float* z,
+                         const int32_t* list, const int32_t* list_n, cudaStream_t s) {
+  const size_t smem = static_cast<size_t>(kSmallT) * c.H * sizeof(uint16_t);
+  cudaError_t e = cudaFuncSetAttribute(router_logits_exact,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  router_logits_exact<<<cdiv(c.E, kRowWarps), kRowWarps * 32, smem, s>>>(T, c.H, c.E, x, Wr, z,
+                                                                        list, list_n);
   return cudaGetLastError();
 }
 
 }  // namespace
 
+// Margin (on biased scores, per unit of logit RMS) below which an fp32
+// decision is re-derived from exact logits. A 2560-term fp32 dot product of
+// N(0,1) activations and N(0, 1/2560) router weights has a rounding error of
+// about 1.2e-6 (one standard deviation), i.e. 3e-7 on a sigmoid score; the
+// largest of millions of such errors stays below ~2e-6, a tenth of this.
+constexpr float kCertifyMargin = 1.0f / 32768.0f;
+
 cudaError_t launch_router(const moe_cfg& c, int T, const uint16_t* x, const float* Wr,
-                          const float* bias, float* z, int32_t* idx, float* w, cudaStream_t s) {
-  if (T <= kSmallT && c.H <= kRowRegs * 128) {
-    const size_t smem = static_cast<size_t>(T) * c.H * sizeof(uint16_t);
-    static bool attr_set = false;
-    if (!attr_set) {
-      cudaFuncSetAttribute(router_logits_small, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           kSmallT * kRowRegs * 128 * 2);
-      attr_set = true;
-    }
-    router_logits_small<<<cdiv(c.E, 8), 256, smem, s>>>(T, c.H, c.E, x, Wr, z);
-  } else {
-    dim3 grid(cdiv(T, kRT), cdiv(c.E, kRE));
-    router_logits_tiled<<<grid, 256, 0, s>>>(T, c.H, c.E, x, Wr, z);
+                          const float* bias, float* z, int32_t* idx, float* w, int32_t* unc,
+                          int32_t* unc_n, cudaStream_t s) {
+  cudaError_t e;
+  if (c.H > kRowRegs * 128) return cudaErrorInvalidValue;
+  if (T <= kSmallT) {
+    // small batch: exact logits for every token, one selection pass
+    if ((e = launch_exact(c, T, x, Wr, z, nullptr, nullptr, s)) != cudaSuccess) return e;
+    return topk_dispatch(c, T, z, bias, idx, w, 0.f, nullptr, nullptr, nullptr, s);
   }
-  cudaError_t err = cudaGetLastError();
-  if (err != cudaSuccess) return err;
-  const int nv = cdiv(c.E, 32);
-  if (nv <= 1) return launch_topk<1>(c, T, z, bias, idx, w, s);
-  if (nv <= 2) return launch_topk<2>(c, T, z, bias, idx, w, s);
-  if (nv <= 4) return launch_topk<4>(c, T, z, bias, idx, w, s);
-  if (nv <= 8) return launch_topk<8>(c, T, z, bias, idx, w, s);
-  if (nv <= 16) return launch_topk<16>(c, T, z, bias, idx, w, s);
-  return launch_topk<32>(c, T, z, bias, idx, w, s);
+  dim3 grid(cdiv(T, kRT), cdiv(c.E, kRE));
+  router_logits_tiled<<<grid, 256, 0, s>>>(T, c.H, c.E, x, Wr, z);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = topk_dispatch(c, T, z, bias, idx, w, kCertifyMargin, unc, unc_n, nullptr, s)) !=
+      cudaSuccess)
+    return e;
+  if ((e = launch_exact(c, T, x, Wr, z, unc, unc_n, s)) != cudaSuccess) return e;
+  return topk_dispatch(c, T, z, bias, idx, w, 0.f, nullptr, unc_n, unc, s);
 }
 
 }  // namespace sgl

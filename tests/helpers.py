@@ -63,7 +63,7 @@ def run_staged(cfg, d, idx: torch.Tensor, w: torch.Tensor):
     offsets = torch.empty(cfg.E + 1, dtype=torch.int32, device=dev)
     perm = torch.empty(T * cfg.K, dtype=torch.int32, device=dev)
     inv = torch.empty(T * cfg.K, dtype=torch.int32, device=dev)
-    y_slot = torch.zeros(T * cfg.K + T, cfg.H, dtype=torch.bfloat16, device=dev)
+    y_slot = torch.zeros(T * cfg.K + T, cfg.H, dtype=torch.float32, device=dev)
     y = torch.empty(T, cfg.H, dtype=torch.bfloat16, device=dev)
     sgl.moe_permute(cfg, T, idx, counts, offsets, perm, inv, ws)
     sgl.moe_grouped_swiglu(cfg, T, d["x"], perm, offsets, w, weights(d), y_slot, ws)
@@ -90,11 +90,21 @@ def check_routing(ref, idx_gpu: np.ndarray, w_gpu: np.ndarray):
     return near
 
 
-def check_y(y_gpu_bits: np.ndarray, y_ref_bits: np.ndarray, tol: float = Y_TOL_BF16):
+def check_y(y_gpu_bits: np.ndarray, y_ref_f32: np.ndarray, y_ref_bits: np.ndarray = None,
+            tol: float = Y_TOL_BF16):
+    """Layer output bar: max |y_gpu - y_oracle| <= tol * RMS(y_oracle), measured
+    against the oracle's fp32 result before its final bf16 rounding.
+
+    Why not against the oracle's bf16 result: one bf16 ulp is 2^-5 * RMS for
+    |y| in [4, 8) * RMS, above the tolerance, and two correct results that
+    straddle a rounding boundary differ by one ulp. The GPU's own rounding
+    costs at most half an ulp (<= 2^-6 * RMS below 8 * RMS), which leaves
+    room for the other legitimate differences (fp32 accumulation order, and
+    h values whose bf16 rounding flips because of it)."""
     g = oracle.bf16_bits_to_f64(y_gpu_bits)
-    r = oracle.bf16_bits_to_f64(y_ref_bits)
+    r = np.asarray(y_ref_f32, dtype=np.float64)
     rms = np.sqrt(np.mean(r * r))
-    err = np.abs(g - r).max()
     assert np.all(np.isfinite(g)), "non-finite output"
+    err = np.abs(g - r).max()
     assert err <= tol * rms, f"max |y err| {err:.4g} > {tol} * rms {rms:.4g}"
     return err / rms

@@ -37,8 +37,8 @@ def test_workspace_size_full_configs():
     for name in ("decode", "prefill", "zipf"):
         cfg = workloads.CONFIGS[name]
         n = sgl.workspace_size(cfg, cfg.T)
-        # dominated by y_slot: (T*K + T) rows of H bf16, plus h (T*K rows of I bf16)
-        lower = (cfg.T * cfg.K + cfg.T) * cfg.H * 2 + cfg.T * cfg.K * cfg.I * 2
+        # dominated by y_slot: (T*K + T) rows of H fp32, plus h (T*K rows of I bf16)
+        lower = (cfg.T * cfg.K + cfg.T) * cfg.H * 4 + cfg.T * cfg.K * cfg.I * 2
         assert lower <= n <= lower * 1.5 + (64 << 20)
 
 

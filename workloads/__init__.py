@@ -104,6 +104,8 @@ def _bf16(shape, var, g, device, chunk_rows=0) -> torch.Tensor:
     out = torch.empty(shape, dtype=torch.bfloat16, device=device)
     std = math.sqrt(var)
     rows = shape[0]
+    if out.numel() == 0:
+        return out
     step = chunk_rows if chunk_rows > 0 else rows
     for r0 in range(0, rows, step):
         r1 = min(rows, r0 + step)
@@ -177,7 +179,7 @@ def generate(cfg: MoEConfig, device="cpu", T: Optional[int] = None) -> Dict[str,
         raise ValueError("unknown weight format")
     out["Wg_s"] = _bf16((Is, H), 1.0 / H, _gen(device, s + 6), device)
     out["Wu_s"] = _bf16((Is, H), 1.0 / H, _gen(device, s + 7), device)
-    out["Wd_s"] = _bf16((H, Is), 1.0 / Is, _gen(device, s + 8), device)
+    out["Wd_s"] = _bf16((H, Is), 1.0 / max(Is, 1), _gen(device, s + 8), device)
     return out
 
 
