@@ -125,6 +125,26 @@ MOE_API moe_status moe_permute(const moe_cfg* cfg, int32_t T, const int32_t* idx
                        int32_t* offsets, int32_t* perm, int32_t* inv_perm, void* ws,
                        size_t ws_bytes, void* stream);
 
+/* moe_permute without a workspace, for callers that cannot allocate device
+ * memory: code that runs where cudaMalloc is not allowed or not available
+ * (inside a region being captured into a CUDA graph, a plugin whose host
+ * framework owns all device memory and hands out no workspace, a real-time
+ * loop that must not allocate). The pages describe no such call; it exists
+ * only for those callers. Same inputs, outputs and results as moe_permute
+ * (all device pointers, owned by the caller).
+ * Scratch: a fixed array inside the library, 256.25 KiB per device, held by
+ * every GPU that loads the library until the process exits. Limits:
+ * T*K <= 65536 and E <= 1024, else MOE_ERR_WORKSPACE and nothing runs.
+ * The first call on a device looks the array's address up (once per
+ * device, with that device current): make that first call before any
+ * stream capture. All calls share the array, so calls that overlap on the
+ * GPU (other streams, other threads) race: serialise them. Expert ids
+ * outside [0,E) are dropped as in moe_permute; there is no error word to
+ * read back. Allocates nothing (no cudaMalloc, no cudaFree). */
+MOE_API moe_status moe_permute_static(const moe_cfg* cfg, int32_t T, const int32_t* idx,
+                                      int32_t* counts, int32_t* offsets, int32_t* perm,
+                                      int32_t* inv_perm, void* stream);
+
 /* Stage 7 (and 8 when shared weights are given): grouped SwiGLU experts on
  * tcgen05 tensor cores (page 3 sec. 2 and sec. 4).
  * in: x [T,H] bf16, perm and offsets from moe_permute, w [T,K] fp32;

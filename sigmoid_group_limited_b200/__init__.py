@@ -29,7 +29,8 @@ STATUS = {0: "MOE_OK", -1: "MOE_ERR_CFG", -2: "MOE_ERR_NULL", -3: "MOE_ERR_ALIGN
 DEVERR = {0: "none", 1: "expert id out of range", 2: "pipeline wait timed out",
           3: "work item out of range"}
 
-C_FUNCTIONS = ("moe_workspace_size", "moe_route", "moe_permute", "moe_grouped_swiglu",
+C_FUNCTIONS = ("moe_workspace_size", "moe_route", "moe_permute", "moe_permute_static",
+               "moe_grouped_swiglu",
                "moe_combine", "moe_layer_forward", "moe_read_error", "moe_status_string",
                "moe_version")
 
@@ -72,6 +73,7 @@ def lib() -> ctypes.CDLL:
     L.moe_workspace_size.restype = sz
     L.moe_route.argtypes = [cp, i32, vp, vp, vp, vp, vp, vp, sz, vp]
     L.moe_permute.argtypes = [cp, i32, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.moe_permute_static.argtypes = [cp, i32, vp, vp, vp, vp, vp, vp]
     L.moe_grouped_swiglu.argtypes = [cp, i32, vp, vp, vp, vp, wp, vp, vp, sz, vp]
     L.moe_combine.argtypes = [cp, i32, vp, i32, vp, vp]
     L.moe_layer_forward.argtypes = [cp, i32, vp, vp, vp, wp, vp, vp, vp, vp, vp, sz, vp, vp]
@@ -79,7 +81,7 @@ def lib() -> ctypes.CDLL:
     L.moe_status_string.argtypes = [i32]
     L.moe_status_string.restype = ctypes.c_char_p
     L.moe_version.restype = ctypes.c_char_p
-    for f in ("moe_route", "moe_permute", "moe_grouped_swiglu", "moe_combine",
+    for f in ("moe_route", "moe_permute", "moe_permute_static", "moe_grouped_swiglu", "moe_combine",
               "moe_layer_forward", "moe_read_error"):
         getattr(L, f).restype = i32
     _lib = L
@@ -142,6 +144,14 @@ def moe_permute(cfg, T, idx, counts, offsets, perm, inv_perm, ws, stream=None):
     c = make_cfg(cfg)
     _check(lib().moe_permute(ctypes.byref(c), int(T), _p(idx), _p(counts), _p(offsets), _p(perm),
                              _p(inv_perm), _p(ws), ws.numel(), _stream(stream)), "moe_permute")
+
+
+def moe_permute_static(cfg, T, idx, counts, offsets, perm, inv_perm, stream=None):
+    """moe_permute without a workspace (scratch in a fixed array inside the
+    library; T*K <= 65536). For callers that cannot allocate device memory."""
+    c = make_cfg(cfg)
+    _check(lib().moe_permute_static(ctypes.byref(c), int(T), _p(idx), _p(counts), _p(offsets),
+                                    _p(perm), _p(inv_perm), _stream(stream)), "moe_permute_static")
 
 
 def moe_grouped_swiglu(cfg, T, x, perm, offsets, w, weights: moe_weights, y_slot, ws, stream=None):

@@ -165,6 +165,20 @@ moe_status moe_permute(const moe_cfg* cfg, int32_t T, const int32_t* idx, int32_
                            at<int32_t>(ws, L.nitems), s));
 }
 
+moe_status moe_permute_static(const moe_cfg* cfg, int32_t T, const int32_t* idx, int32_t* counts,
+                              int32_t* offsets, int32_t* perm, int32_t* inv_perm, void* stream) {
+  if (!cfg_ok(cfg) || !T_ok(T)) return MOE_ERR_CFG;
+  if (!idx || !counts || !offsets || !perm) return MOE_ERR_NULL;
+  if (!al16(idx) || !al16(counts) || !al16(offsets) || !al16(perm) || (inv_perm && !al16(inv_perm)))
+    return MOE_ERR_ALIGN;
+  if (static_cast<long long>(T) * cfg->K > kStaticMaxSlots || cfg->E > kStaticMaxExperts)
+    return MOE_ERR_WORKSPACE;
+  moe_status st = device_ok();
+  if (st != MOE_OK) return st;
+  return cu(launch_permute_static(*cfg, T, idx, counts, offsets, perm, inv_perm,
+                                  static_cast<cudaStream_t>(stream)));
+}
+
 moe_status moe_grouped_swiglu(const moe_cfg* cfg, int32_t T, const void* x, const int32_t* perm,
                               const int32_t* offsets, const float* w, const moe_weights* W,
                               void* y_slot, void* ws, size_t ws_bytes, void* stream) {

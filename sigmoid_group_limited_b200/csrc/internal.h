@@ -55,6 +55,15 @@ cudaError_t launch_permute(const moe_cfg& c, int T, const int32_t* idx, int32_t*
                            int32_t* err, const WsLayout& L, WorkItem* items_gu, WorkItem* items_dn,
                            int32_t* nitems, cudaStream_t s);
 
+// Allocation-free permutation (moe_permute_static): scratch in a fixed
+// device array; needs T*K <= kStaticMaxSlots and E <= kStaticMaxExperts.
+constexpr int kStaticMaxSlots = 65536;
+constexpr int kStaticMaxExperts = 1024;
+constexpr int kMaxDevices = 64;
+cudaError_t launch_permute_static(const moe_cfg& c, int T, const int32_t* idx, int32_t* counts,
+                                  int32_t* offsets, int32_t* perm, int32_t* inv_perm,
+                                  cudaStream_t s);
+
 cudaError_t launch_schedule(const moe_cfg& c, int T, const int32_t* offsets, const WsLayout& L,
                             WorkItem* items_gu, WorkItem* items_dn, int32_t* nitems,
                             cudaStream_t s);

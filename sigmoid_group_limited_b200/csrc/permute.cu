@@ -15,6 +15,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "internal.h"
 
 namespace sgl {
@@ -298,6 +300,57 @@ cudaError_t launch_permute(const moe_cfg& c, int T, const int32_t* idx, int32_t*
   SchedArgs sa = make_sched(c, T, L, items_gu, items_dn, nitems);
   perm_scan<<<1, 1024, 0, s>>>(c.E, np, tile_cnt, tile_base, counts, offsets, sa,
                                items_gu != nullptr ? 1 : 0);
+  perm_scatter<<<np, kScatterWarps * 32, 0, s>>>(TK, c.E, np, idx, tile_base, perm, inv_perm,
+                                                 err);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Scratch for moe_permute_static, for callers that cannot allocate device
+// memory: the per-(expert, tile) counts and bases of the three kernels above
+// plus an error word, in one file-scope device array of fixed size. Every
+// device that loads the library holds it until the process exits.
+// Layout (int32): [0] error word, [1..63] unused, [64, 64 + E*n_tiles)
+// counts, then E*n_tiles bases.
+// ---------------------------------------------------------------------------
+constexpr int kStaticScratchHead = 64;
+constexpr int kStaticScratchInts =
+    kStaticScratchHead + 2 * kStaticMaxExperts * (kStaticMaxSlots / kPermTile);
+static __device__ __align__(256) int32_t g_permute_scratch[kStaticScratchInts];
+
+// Device address of g_permute_scratch on the current device, looked up once
+// per device (with that device current) and cached; nullptr on failure.
+static int32_t* static_scratch_address() {
+  static std::mutex mu;
+  static int32_t* addr[kMaxDevices] = {};
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<int32_t*>(p);
+  }
+  return addr[dev];
+}
+
+cudaError_t launch_permute_static(const moe_cfg& c, int T, const int32_t* idx, int32_t* counts,
+                                  int32_t* offsets, int32_t* perm, int32_t* inv_perm,
+                                  cudaStream_t s) {
+  const int TK = T * c.K;
+  const int np = cdiv(TK, kPermTile);
+  int32_t* base = static_scratch_address();
+  if (base == nullptr) return cudaErrorInvalidSymbol;
+  int32_t* err = base;
+  int32_t* tile_cnt = base + kStaticScratchHead;
+  int32_t* tile_base = tile_cnt + static_cast<size_t>(c.E) * np;
+  // the error word must start at zero; the tile arrays are fully written
+  cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int32_t), s);
+  if (e != cudaSuccess) return e;
+  perm_hist<<<np, 256, 0, s>>>(TK, c.E, np, idx, tile_cnt, err);
+  SchedArgs sa{};
+  sa.nitems = base + 1;
+  perm_scan<<<1, 1024, 0, s>>>(c.E, np, tile_cnt, tile_base, counts, offsets, sa, 0);
   perm_scatter<<<np, kScatterWarps * 32, 0, s>>>(TK, c.E, np, idx, tile_base, perm, inv_perm,
                                                  err);
   return cudaGetLastError();
