@@ -187,7 +187,13 @@ def roofline_entry(bytes_, flops, seconds, peaks, sustained=False):
 # ------------------------------------------------------------------ GPU arm
 
 STAGES = ("route", "permute", "gateup", "down", "combine")
-KERNELS_PER_STEP = 8  # router 2, permutation 3, GEMM 2, combine 1
+
+
+def kernels_per_step(cfg) -> int:
+    """Library kernels launched by one moe_layer_forward: router 4 (logits,
+    certified top-k, exact re-derivation, exact top-k), permutation 1 when
+    all T*K slots fit one 2048-entry tile else 3, grouped GEMMs 2, combine 1."""
+    return 4 + (1 if cfg.T * cfg.K <= 2048 else 3) + 2 + 1
 
 
 def measure_gpu(cfg, steps, warmup, device, rank, with_e2e=True):
@@ -227,16 +233,44 @@ def measure_gpu(cfg, steps, warmup, device, rank, with_e2e=True):
     torch.cuda.synchronize(device)
     barrier(device)
     wall = time.perf_counter() - t0
-    per_step = [evs[i][0].elapsed_time(evs[i][5]) for i in range(steps)]
+    per_step_plain = [evs[i][0].elapsed_time(evs[i][5]) for i in range(steps)]
     stage_ms = {s: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(steps))
                 for j, s in enumerate(STAGES)}
+    assert sgl.moe_read_error(cfg, T, ws) == 0
+
+    # the same forward captured once into a CUDA graph and replayed per step
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(device)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side, capture_error_mode="thread_local"):
+            sgl.moe_layer_forward(cfg, d["x"], d["Wr"], d["bias"], W, y, ws, idx, w, counts,
+                                  stream=side)
+    stream.wait_stream(side)
+    for _ in range(warmup):
+        flush.zero_()
+        graph.replay()
+    g0 = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    g1 = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    barrier(device)
+    torch.cuda.synchronize(device)
+    for i in range(steps):
+        flush.zero_()
+        g0[i].record(stream)
+        graph.replay()
+        g1[i].record(stream)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    per_step = [g0[i].elapsed_time(g1[i]) for i in range(steps)]
     dev_ms = sum(per_step)
     assert sgl.moe_read_error(cfg, T, ws) == 0
+    del graph
     touched = int((counts > 0).sum().item())
     cnt = counts.cpu().numpy()
-    out = dict(device_ms_total=dev_ms, wall_s=wall, per_step_ms=per_step, stage_ms=stage_ms,
+    out = dict(device_ms_total=dev_ms, plain_ms_total=sum(per_step_plain), wall_s=wall,
+               per_step_ms=per_step, stage_ms=stage_ms,
                touched=touched, load_max=int(cnt.max()), load_mean=float(cnt.mean()),
-               d=d, launches=KERNELS_PER_STEP * steps)
+               d=d, launches=kernels_per_step(cfg) * 2 * steps)
 
     if with_e2e:
         # end to end through the public API: pinned host x -> device, forward, y -> pinned host
@@ -259,6 +293,7 @@ def measure_gpu(cfg, steps, warmup, device, rank, with_e2e=True):
             e1[i].record(stream)
         torch.cuda.synchronize(device)
         out["e2e_ms_total"] = sum(e0[i].elapsed_time(e1[i]) for i in range(steps))
+        out["launches"] += kernels_per_step(cfg) * steps
         out["e2e_h2d"] = T * cfg.H * 2
         out["e2e_d2h"] = T * cfg.H * 2
         assert torch.equal(yh.view(torch.int16), y.cpu().view(torch.int16))
@@ -379,6 +414,7 @@ def run_native(args, rank, world, local):
             also = (acfg, measure_gpu(acfg, args.steps, args.warmup, device, rank, with_e2e=False))
     clocks = clk.summary()
     dev_s = reduce_max(m["device_ms_total"], device) / 1e3
+    plain_s = reduce_max(m["plain_ms_total"], device) / 1e3
     e2e_s = reduce_max(m["e2e_ms_total"], device) / 1e3
     tokens = cfg.T * args.steps * world
 
@@ -400,6 +436,9 @@ def run_native(args, rank, world, local):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(1e3 * dev_s / args.steps, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "timing": "CUDA-event time of K graph replays of moe_layer_forward (one capture of "
+                      "the C-ABI call); value_no_graph: the same K steps as plain C-ABI calls",
+            "value_no_graph": round(tokens / plain_s, 1),
             "config": config_block(cfg, world), "roofline": ent,
             "layer_roofline_frac": layer_frac,
             "stage_ms": {k: round(v, 4) for k, v in m["stage_ms"].items()},
@@ -412,7 +451,9 @@ def run_native(args, rank, world, local):
         acfg, am = also
         a_s = reduce_max(am["device_ms_total"], device) / 1e3
         aent, afrac = roof(acfg, am)
+        ap_s = reduce_max(am["plain_ms_total"], device) / 1e3
         line[acfg.name] = {"value": round(acfg.T * args.steps * world / a_s, 1), "unit": "tokens/s",
+                           "value_no_graph": round(acfg.T * args.steps * world / ap_s, 1),
                            "ms_per_step": round(1e3 * a_s / args.steps, 4), "roofline": aent,
                            "layer_roofline_frac": afrac,
                            "stage_ms": {k: round(v, 4) for k, v in am["stage_ms"].items()},

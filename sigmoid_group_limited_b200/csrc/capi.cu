@@ -144,7 +144,8 @@ moe_status moe_route(const moe_cfg* cfg, int32_t T, const void* x, const float* 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(at<int32_t>(ws, L.err), 0, 16, s) != cudaSuccess) return MOE_ERR_CUDA;
   return cu(launch_router(*cfg, T, static_cast<const uint16_t*>(x), Wr, bias, at<float>(ws, L.z),
-                          idx, w, at<int32_t>(ws, L.unc), at<int32_t>(ws, L.err) + 1, s));
+                          idx, w, at<int32_t>(ws, L.unc), at<int32_t>(ws, L.err) + 1,
+                          at<int32_t>(ws, L.err), s));
 }
 
 moe_status moe_permute(const moe_cfg* cfg, int32_t T, const int32_t* idx, int32_t* counts,
@@ -263,7 +264,7 @@ moe_status moe_layer_forward(const moe_cfg* cfg, int32_t T, const void* x, const
   rec(0);
   if (cudaMemsetAsync(err, 0, 16, s) != cudaSuccess) return MOE_ERR_CUDA;
   if ((e = launch_router(*cfg, T, static_cast<const uint16_t*>(x), Wr, bias, at<float>(ws, L.z),
-                         idx, w, at<int32_t>(ws, L.unc), err + 1, s)) != cudaSuccess)
+                         idx, w, at<int32_t>(ws, L.unc), err + 1, err, s)) != cudaSuccess)
     return MOE_ERR_CUDA;
   rec(1);
   if ((e = launch_permute(*cfg, T, idx, at<int32_t>(ws, L.tile_hist), counts, offsets, perm,

@@ -34,11 +34,14 @@
 namespace sgl {
 namespace {
 
-constexpr int kThreads = 192;
+// Warps: 0 weight TMA, 1 MMA, 2..5 epilogue; gate/up adds 6..9 token gatherers.
+constexpr int kGatherWarps = 4;
+__host__ __device__ constexpr int threads_for(int mode) { return mode == 0 ? 320 : 192; }
 constexpr int kSmemBudget = 200 * 1024;
 
 struct GemmParams {
   int T, K, E, H, I, Is;
+  const uint16_t* x;  // [T, H] tokens (gate/up operand)
   int has_shared;
   float lim_r, lim_s;  // <= 0: no limit
   const int32_t* perm;
@@ -69,8 +72,11 @@ struct Cfg {
   static constexpr int ACC_COLS = NA * BN;           // fp32 columns per accumulator
   static constexpr int TMEM_COLS = pow2_at_least(2 * ACC_COLS);
   static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/ +
-                             BN * 4 /*token rows*/;
+                             BN * 4 /*token rows*/ + BN * 8 /*row metadata*/;
 };
+
+// Named barrier 1 over the four epilogue warps (128 threads).
+__device__ __forceinline__ void epilogue_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 __device__ __forceinline__ float clampL(float v, float L) {
   return L > 0.f ? fminf(fmaxf(v, -L), L) : v;
@@ -94,7 +100,7 @@ __device__ __forceinline__ bool item_ok(const GemmParams& p, const WorkItem& it,
 }
 
 template <int MODE, int BN>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(threads_for(MODE), 1)
     moe_gemm(const __grid_constant__ GemmParams p, const __grid_constant__ CUtensorMap tA0,
              const __grid_constant__ CUtensorMap tA1, const __grid_constant__ CUtensorMap tS0,
              const __grid_constant__ CUtensorMap tS1, const __grid_constant__ CUtensorMap tB0,
@@ -110,11 +116,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* tok = reinterpret_cast<int*>(smem + C::STAGES * C::STAGE_BYTES + 256);
+  int* meta_j = tok + BN;                                       // down: slot of each row
+  float* meta_w = reinterpret_cast<float*>(meta_j + BN);        // down: its routing weight
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&full[s], 1);
+      // gate/up: the weight TMA arrival plus one arrival per token-gatherer thread
+      mbar_init(&full[s], MODE == 0 ? 1 + kGatherWarps * 32 : 1);
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -153,15 +162,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         continue;
       }
       const bool sh = it.e == p.E;
-      if (MODE == 0) {
-        for (int r = lane; r < BN; r += 32) {
-          const int row = it.row0 + min(r, it.nrows - 1);
-          int t = sh ? row : p.perm[row] / p.K;
-          t = min(max(t, 0), p.T - 1);
-          tok[r] = t;
-        }
-      }
-      __syncwarp();
       if (lane == 0) {
         const int nkb = sh ? KB_s : KB_r;
         const int arow = sh ? it.ntile * kTileN
@@ -175,15 +175,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           uint8_t* sA = smem + stage * C::STAGE_BYTES;
           uint8_t* sB = sA + C::NA * C::A_BYTES;
-          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
-          tma_load_2d(sA, mA0, &full[stage], kb * 64, arow, pol_w);
-          if (MODE == 0) tma_load_2d(sA + C::A_BYTES, mA1, &full[stage], kb * 64, arow, pol_w);
           if (MODE == 0) {
-#pragma unroll 4
-            for (int q = 0; q < BN / 4; ++q)
-              tma_gather4(sB + q * 512, &tB0, &full[stage], kb * 64, tok[4 * q], tok[4 * q + 1],
-                          tok[4 * q + 2], tok[4 * q + 3], pol_x);
+            // weights only; the token rows come from the gatherer warps
+            mbar_arrive_expect_tx(&full[stage], C::NA * C::A_BYTES);
+            tma_load_2d(sA, mA0, &full[stage], kb * 64, arow, pol_w);
+            tma_load_2d(sA + C::A_BYTES, mA1, &full[stage], kb * 64, arow, pol_w);
           } else {
+            mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+            tma_load_2d(sA, mA0, &full[stage], kb * 64, arow, pol_w);
             tma_load_2d(sB, sh ? &tB1 : &tB0, &full[stage], kb * 64, it.row0, pol_x);
           }
           if (++stage == C::STAGES) {
@@ -248,6 +247,66 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
+  } else if (MODE == 0 && warp >= 6) {
+    // ------------------------------------------------------------ token gatherers
+    // Thread g copies 16-byte chunk (g % 8) of rows g/8, g/8 + 16, ... of the
+    // stage's BN x 64 token tile, straight into the 128-byte-swizzled layout
+    // (chunk c of row r lands at chunk c ^ (r % 8)). A stage's copies are
+    // retired two stages later: wait for the group, make it visible to the
+    // tensor cores (proxy fence), then arrive on the stage's full barrier.
+    constexpr int kRowsPerThread = BN / 16;
+    constexpr int kLag = 2;
+    const int g = tid - 6 * 32;
+    const int chunk = g & 7, rbase = g >> 3;
+    const uint64_t pol_x = policy_evict_last();
+    int stage = 0;
+    uint32_t phase = 0;
+    int pend0 = -1, pend1 = -1;  // stages issued two and one steps ago, not yet retired
+    bool live = true;
+    for (int item = blockIdx.x; item < n_items && live; item += gridDim.x) {
+      const WorkItem it = p.items[item];
+      if (!item_ok(p, it, MODE, BN)) continue;
+      const bool sh = it.e == p.E;
+      const int nkb = sh ? KB_s : KB_r;
+      const uint16_t* src[kRowsPerThread];
+#pragma unroll
+      for (int i = 0; i < kRowsPerThread; ++i) {
+        const int row = it.row0 + min(rbase + 16 * i, it.nrows - 1);
+        int t = sh ? row : p.perm[row] / p.K;
+        t = min(max(t, 0), p.T - 1);
+        src[i] = p.x + static_cast<size_t>(t) * p.H + chunk * 8;
+      }
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) {
+          live = false;
+          break;
+        }
+        uint8_t* sB = smem + stage * C::STAGE_BYTES + C::NA * C::A_BYTES;
+#pragma unroll
+        for (int i = 0; i < kRowsPerThread; ++i) {
+          const int r = rbase + 16 * i;
+          cp_async16(sB + r * 128 + ((chunk ^ (r & 7)) << 4), src[i] + kb * 64, pol_x);
+        }
+        cp_async_commit();
+        if (pend0 >= 0) {
+          cp_async_wait<kLag>();  // all but the two newest groups have landed
+          fence_proxy_async_smem();
+          mbar_arrive(&full[pend0]);
+        }
+        pend0 = pend1;
+        pend1 = stage;
+        if (++stage == C::STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+    cp_async_wait<0>();  // nothing may still be landing in shared memory at exit
+    fence_proxy_async_smem();
+    if (live) {
+      if (pend0 >= 0) mbar_arrive(&full[pend0]);
+      if (pend1 >= 0) mbar_arrive(&full[pend1]);
+    }
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                  // TMEM lane quarter of this warp
@@ -258,6 +317,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       const WorkItem it = p.items[item];
       if (!item_ok(p, it, MODE, BN)) continue;
       const bool sh = it.e == p.E;
+      if (MODE == 1) {
+        // destination slot and routing weight of every row of the item, loaded
+        // while the item's MMAs run (the store loop then touches no metadata in
+        // global memory)
+        epilogue_bar();  // all four warps are done with the previous item's rows
+        if (orow < BN) {
+          int j = -1;
+          float wt = 0.f;
+          if (orow < it.nrows) {
+            const int row = it.row0 + orow;
+            if (sh) {
+              j = p.T * p.K + row;
+              wt = 1.0f;
+            } else {
+              j = p.perm[row];
+              if (j < 0 || j >= p.T * p.K) {  // a bad permutation: report, never store
+                atomicExch(p.err, MOE_DEVERR_SCHEDULE);
+                j = -1;
+              } else {
+                wt = p.w[j];
+              }
+            }
+          }
+          meta_j[orow] = j;
+          meta_w[orow] = wt;
+        }
+        epilogue_bar();
+      }
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * C::ACC_COLS;
@@ -295,24 +382,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (ok) {
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
-              const int r = c0 + c;
-              if (r < it.nrows) {
-                const int row = it.row0 + r;
-                int j;
-                float wt;
-                if (sh) {
-                  j = p.T * p.K + row;
-                  wt = 1.0f;
-                } else {
-                  j = p.perm[row];
-                  if (j < 0 || j >= p.T * p.K) {  // a bad permutation: report, never store
-                    atomicExch(p.err, MOE_DEVERR_SCHEDULE);
-                    continue;
-                  }
-                  wt = p.w[j];
-                }
-                p.y_slot[static_cast<size_t>(j) * p.H + nfeat] = wt * ov[c];
-              }
+              const int j = meta_j[c0 + c];
+              if (j >= 0) p.y_slot[static_cast<size_t>(j) * p.H + nfeat] = meta_w[c0 + c] * ov[c];
             }
           }
         }
@@ -377,6 +448,7 @@ GemmParams make_params(const GemmArgs& a, int mode) {
   p.lim_r = (c.limit_routed > 0.f && isfinite(c.limit_routed)) ? c.limit_routed : 0.f;
   p.lim_s = (c.limit_shared > 0.f && isfinite(c.limit_shared)) ? c.limit_shared : 0.f;
   p.perm = a.perm;
+  p.x = a.x;
   p.w = a.w;
   p.h_r = a.h_r;
   p.h_s = a.h_s;
@@ -427,7 +499,7 @@ cudaError_t launch_mode(const GemmArgs& a, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   const int max_items = p.max_items;
   const int grid = max(1, min(num_sms(), max_items));
-  kern<<<grid, kThreads, C::SMEM, s>>>(p, tA0, tA1, tS0, tS1, tB0, tB1);
+  kern<<<grid, threads_for(MODE), C::SMEM, s>>>(p, tA0, tA1, tS0, tS1, tB0, tB1);
   return cudaGetLastError();
 }
 

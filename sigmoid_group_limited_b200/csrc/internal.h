@@ -48,7 +48,7 @@ WsLayout ws_layout(const moe_cfg& c, int T);
 // caller) of tokens whose fp32 decision is re-derived from exact logits.
 cudaError_t launch_router(const moe_cfg& c, int T, const uint16_t* x, const float* Wr,
                           const float* bias, float* z, int32_t* idx, float* w, int32_t* unc,
-                          int32_t* unc_n, cudaStream_t s);
+                          int32_t* unc_n, int32_t* err, cudaStream_t s);
 
 cudaError_t launch_permute(const moe_cfg& c, int T, const int32_t* idx, int32_t* tile_hist,
                            int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv_perm,

@@ -268,6 +268,95 @@ __global__ void __launch_bounds__(kScatterWarps * 32) perm_scatter(
   }
 }
 
+// The whole permutation in one CTA when all T*K entries fit one tile (decode
+// batches): per-warp histograms of contiguous chunks, per-expert totals and
+// their exclusive scan, per-warp bases, stable positions, and optionally the
+// GEMM work lists, with no round trip through global memory in between.
+__global__ void __launch_bounds__(1024) perm_single(int TK, int E, const int32_t* __restrict__ idx,
+                                                    int32_t* __restrict__ counts,
+                                                    int32_t* __restrict__ offsets,
+                                                    int32_t* __restrict__ perm,
+                                                    int32_t* __restrict__ inv_perm,
+                                                    int32_t* __restrict__ err, SchedArgs sa,
+                                                    int build) {
+  extern __shared__ int whist[];  // [32 warps][E]
+  __shared__ int cnt[kMaxE + 1];
+  __shared__ int off[kMaxE + 1];
+  __shared__ int scratch[33];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int i = tid; i < 32 * E; i += blockDim.x) whist[i] = 0;
+  __syncthreads();
+  const int chunk = ((cdiv_dev(TK, 32) + 31) / 32) * 32;
+  const int c0 = warp * chunk, c1 = min(c0 + chunk, TK);
+  const unsigned lt = (1u << lane) - 1u;
+  int* wh = whist + warp * E;
+  for (int r = c0; r < c1; r += 32) {
+    const int i = r + lane;
+    int e = -1;
+    if (i < c1) {
+      e = idx[i];
+      if (e < 0 || e >= E) {
+        atomicExch(err, MOE_DEVERR_EXPERT_ID);
+        e = -1;
+      }
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && (peers & lt) == 0) wh[e] += __popc(peers);
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x) {
+    int tot = 0;
+    for (int w = 0; w < 32; ++w) tot += whist[w * E + e];
+    cnt[e] = tot;
+  }
+  __syncthreads();
+  int total;
+  const int e0 = 2 * tid;
+  const int v0 = e0 < E ? cnt[e0] : 0, v1 = e0 + 1 < E ? cnt[e0 + 1] : 0;
+  const int ex = block_exscan2(v0, v1, scratch, &total);
+  if (e0 < E) off[e0] = ex;
+  if (e0 + 1 < E) off[e0 + 1] = ex + v0;
+  if (tid == 0) off[E] = total;
+  __syncthreads();
+  for (int e = tid; e <= E; e += blockDim.x) {
+    offsets[e] = off[e];
+    if (e < E) counts[e] = cnt[e];
+  }
+  for (int e = tid; e < E; e += blockDim.x) {
+    int run = off[e];
+    for (int w = 0; w < 32; ++w) {
+      const int v = whist[w * E + e];
+      whist[w * E + e] = run;
+      run += v;
+    }
+  }
+  __syncthreads();
+  for (int r = c0; r < c1; r += 32) {
+    const int i = r + lane;
+    int e = -1;
+    if (i < c1) {
+      e = idx[i];
+      if (e < 0 || e >= E) e = -1;
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    int pos = -1;
+    if (e >= 0) pos = wh[e] + __popc(peers & lt);
+    __syncwarp();
+    if (e >= 0 && (peers & lt) == 0) wh[e] += __popc(peers);
+    __syncwarp();
+    if (i < c1) {
+      if (e >= 0 && (pos < 0 || pos >= TK)) {
+        atomicExch(err, MOE_DEVERR_SCHEDULE);
+        e = -1;
+        pos = -1;
+      }
+      if (e >= 0) perm[pos] = i;
+      if (inv_perm) inv_perm[i] = pos;
+    }
+  }
+  if (build) build_schedule(sa, cnt, off, scratch);
+}
+
 SchedArgs make_sched(const moe_cfg& c, int T, const WsLayout& L, WorkItem* gu, WorkItem* dn,
                      int32_t* nitems) {
   SchedArgs a;
@@ -295,9 +384,18 @@ cudaError_t launch_permute(const moe_cfg& c, int T, const int32_t* idx, int32_t*
                            WorkItem* items_dn, int32_t* nitems, cudaStream_t s) {
   const int TK = T * c.K;
   const int np = L.n_ptiles;
+  SchedArgs sa = make_sched(c, T, L, items_gu, items_dn, nitems);
+  if (np == 1) {
+    const int smem = 32 * c.E * static_cast<int>(sizeof(int));
+    cudaError_t e = cudaFuncSetAttribute(perm_single, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         smem);
+    if (e != cudaSuccess) return e;
+    perm_single<<<1, 1024, smem, s>>>(TK, c.E, idx, counts, offsets, perm, inv_perm, err, sa,
+                                      items_gu != nullptr ? 1 : 0);
+    return cudaGetLastError();
+  }
   int32_t* tile_base = tile_cnt + static_cast<size_t>(c.E) * np;
   perm_hist<<<np, 256, 0, s>>>(TK, c.E, np, idx, tile_cnt, err);
-  SchedArgs sa = make_sched(c, T, L, items_gu, items_dn, nitems);
   perm_scan<<<1, 1024, 0, s>>>(c.E, np, tile_cnt, tile_base, counts, offsets, sa,
                                items_gu != nullptr ? 1 : 0);
   perm_scatter<<<np, kScatterWarps * 32, 0, s>>>(TK, c.E, np, idx, tile_base, perm, inv_perm,

@@ -16,33 +16,63 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <type_traits>
 
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace sgl {
 namespace {
 
 // ---------------------------------------------------------------------------
-// Exact logits for a list of rows: one warp per expert, the expert's fp32
-// router row held in registers (a strided slice per lane), up to 32 token
-// rows staged in shared memory as bf16. Every product bf16 * fp32 is exact
-// in float64 and the sum of 2560 of them is accumulated in float64, so the
-// single final rounding to fp32 gives the same logit as an exact dot
-// product. Used for whole decode batches and to re-derive the logits of the
-// tokens whose fp32 routing decision was too close to call.
+// Logits for a set of rows, one warp per expert: the expert's fp32 router row
+// is held in registers (a strided slice per lane) and up to 32 token rows are
+// staged in shared memory as bf16; ILP tokens are accumulated at once.
+//  EXACT = false: fp32 FMA accumulation (the pages' fp32 router), for small
+//                 batches;
+//  EXACT = true:  every product bf16 * fp32 is exact in float64 and the sum
+//                 of H of them is accumulated in float64, so the one final
+//                 rounding to fp32 gives the logit of an exact dot product.
+//                 Used for the tokens whose fp32 decision was too close.
+// With `list`, the rows are list[0 .. *list_n) instead of 0 .. T-1.
 // ---------------------------------------------------------------------------
 constexpr int kSmallT = 32;
 constexpr int kRowRegs = 24;  // float4 per lane: H <= 24 * 128 = 3072
-constexpr int kRowWarps = 4;
+constexpr int kRowWarps = 4;  // experts per CTA
+constexpr int kTokSplit = 2;  // warps per expert (they split the token rows)
 
-__global__ void __launch_bounds__(kRowWarps * 32) router_logits_exact(
+// bf16 bits -> float64 by field arithmetic (no conversion instruction):
+// sign, exponent rebiased from 127 to 1023, 7 mantissa bits on top.
+__device__ __forceinline__ double bf16_bits_to_double(uint32_t b) {
+  const uint32_t ex = (b >> 7) & 0xFFu;
+  if (ex == 0u || ex == 0xFFu) return static_cast<double>(__uint_as_float(b << 16));
+  const unsigned long long bits = (static_cast<unsigned long long>(b & 0x8000u) << 48) |
+                                  (static_cast<unsigned long long>(ex + 896u) << 52) |
+                                  (static_cast<unsigned long long>(b & 0x7Fu) << 45);
+  return __longlong_as_double(static_cast<long long>(bits));
+}
+
+template <bool EXACT, int ILP>
+__global__ void __launch_bounds__(kRowWarps * kTokSplit * 32) router_logits_rows(
     int T, int H, int E, const uint16_t* __restrict__ x, const float* __restrict__ Wr,
-    float* __restrict__ z, const int32_t* __restrict__ list, const int32_t* __restrict__ list_n) {
-  extern __shared__ __align__(16) uint16_t xs[];  // [kSmallT][H]
+    float* __restrict__ z, const int32_t* __restrict__ list, const int32_t* __restrict__ list_n,
+    int32_t* __restrict__ err) {
+  using Acc = typename std::conditional<EXACT, double, float>::type;
+  extern __shared__ __align__(128) uint16_t xs[];  // [kSmallT][H]
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int e = blockIdx.x * kRowWarps + warp;
+  const int e = blockIdx.x * kRowWarps + (warp % kRowWarps);
+  const int split = warp / kRowWarps;  // this warp takes token groups split, split+kTokSplit, ...
   const bool have = e < E;
   const int n = list ? min(*list_n, T) : T;
+  if (n <= 0) return;
+  if (tid == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  uint32_t phase = 0;
   float4 wv[kRowRegs];
 #pragma unroll
   for (int j = 0; j < kRowRegs; ++j) {
@@ -50,37 +80,69 @@ __global__ void __launch_bounds__(kRowWarps * 32) router_logits_exact(
     wv[j] = (have && k < H) ? *reinterpret_cast<const float4*>(Wr + static_cast<size_t>(e) * H + k)
                             : make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  const int c16 = H / 8;  // 16-byte chunks per row
+  const uint32_t row_bytes = static_cast<uint32_t>(H) * 2;
   for (int c0 = 0; c0 < n; c0 += kSmallT) {
     const int nc = min(kSmallT, n - c0);
-    __syncthreads();
-    for (int i = tid; i < nc * c16; i += blockDim.x) {
-      const int r = i / c16, c = i - r * c16;
-      const int t = list ? list[c0 + r] : c0 + r;
-      reinterpret_cast<uint4*>(xs)[r * c16 + c] =
-          reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H)[c];
+    __syncthreads();  // everyone is done with the previous chunk
+    if (tid == 0) {
+      // one bulk copy per token row, all in flight at once
+      fence_proxy_async_smem();
+      mbar_arrive_expect_tx(&bar, row_bytes * nc);
+      for (int r = 0; r < nc; ++r) {
+        const int t = list ? list[c0 + r] : c0 + r;
+        bulk_load(xs + r * H, x + static_cast<size_t>(t) * H, row_bytes, &bar);
+      }
     }
-    __syncthreads();
+    mbar_wait(&bar, phase, &abort_flag, err, MOE_DEVERR_TIMEOUT);
+    phase ^= 1;
     if (!have) continue;
-    for (int r = 0; r < nc; ++r) {
-      const uint16_t* xr = xs + r * H;
-      double acc = 0.0;
+    for (int r0 = split * ILP; r0 < nc; r0 += ILP * kTokSplit) {
+      Acc acc[ILP];
+#pragma unroll
+      for (int q = 0; q < ILP; ++q) acc[q] = Acc(0);
 #pragma unroll
       for (int j = 0; j < kRowRegs; ++j) {
         const int k = 4 * lane + 128 * j;
         if (k < H) {
-          const uint2 p = *reinterpret_cast<const uint2*>(xr + k);
-          acc = fma(static_cast<double>(wv[j].x), static_cast<double>(__uint_as_float(p.x << 16)), acc);
-          acc = fma(static_cast<double>(wv[j].y), static_cast<double>(__uint_as_float(p.x & 0xFFFF0000u)), acc);
-          acc = fma(static_cast<double>(wv[j].z), static_cast<double>(__uint_as_float(p.y << 16)), acc);
-          acc = fma(static_cast<double>(wv[j].w), static_cast<double>(__uint_as_float(p.y & 0xFFFF0000u)), acc);
+          Acc w0, w1, w2, w3;
+          if (EXACT) {
+            w0 = static_cast<Acc>(wv[j].x); w1 = static_cast<Acc>(wv[j].y);
+            w2 = static_cast<Acc>(wv[j].z); w3 = static_cast<Acc>(wv[j].w);
+          } else {
+            w0 = wv[j].x; w1 = wv[j].y; w2 = wv[j].z; w3 = wv[j].w;
+          }
+#pragma unroll
+          for (int q = 0; q < ILP; ++q) {
+            const int r = min(r0 + q, nc - 1);
+            const uint2 p = *reinterpret_cast<const uint2*>(xs + r * H + k);
+            if (EXACT) {
+              acc[q] = fma(w0, static_cast<Acc>(bf16_bits_to_double(p.x & 0xFFFFu)), acc[q]);
+              acc[q] = fma(w1, static_cast<Acc>(bf16_bits_to_double(p.x >> 16)), acc[q]);
+              acc[q] = fma(w2, static_cast<Acc>(bf16_bits_to_double(p.y & 0xFFFFu)), acc[q]);
+              acc[q] = fma(w3, static_cast<Acc>(bf16_bits_to_double(p.y >> 16)), acc[q]);
+            } else {
+              acc[q] = fmaf(w0, __uint_as_float(p.x << 16), acc[q]);
+              acc[q] = fmaf(w1, __uint_as_float(p.x & 0xFFFF0000u), acc[q]);
+              acc[q] = fmaf(w2, __uint_as_float(p.y << 16), acc[q]);
+              acc[q] = fmaf(w3, __uint_as_float(p.y & 0xFFFF0000u), acc[q]);
+            }
+          }
         }
       }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (lane == 0) {
-        const int t = list ? list[c0 + r] : c0 + r;
-        z[static_cast<size_t>(t) * E + e] = static_cast<float>(acc);
+      for (int q = 0; q < ILP; ++q) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc[q] += __shfl_xor_sync(0xffffffffu, acc[q], o);
+      }
+      if (lane < ILP) {
+        Acc v = acc[0];
+#pragma unroll
+        for (int q = 1; q < ILP; ++q)
+          if (lane == q) v = acc[q];
+        if (r0 + lane < nc) {
+          const int t = list ? list[c0 + r0 + lane] : c0 + r0 + lane;
+          z[static_cast<size_t>(t) * E + e] = static_cast<float>(v);
+        }
       }
     }
   }
@@ -175,17 +237,22 @@ __global__ void __launch_bounds__(256) router_logits_tiled(int T, int H, int E,
 
 // ---------------------------------------------------------------------------
 // Scores and group-limited top-k: one warp per token. Lane l holds experts
-// e = l + 32*j. Scores use a float64 sigmoid rounded to fp32; the weights are
-// computed in float64 from the fp32 scores and rounded once.
+// e = l + 32*j. The combine weights are computed in float64 from the fp32
+// scores and rounded once.
 //
-// Certification: with tau > 0 the kernel also measures its own decision
-// margins (the topk_group-th minus the next group score, and every gap
-// between neighbours in the ranking of the K+1 best candidates, since slot
-// order is rank order) and appends the token to `unc` when one is below tau;
-// those tokens get exact logits and a second pass (list mode) before anything
-// downstream reads idx / w.
+// Two modes:
+//  certified (tau > 0): scores from an fp32 sigmoid of the fp32 logits; the
+//    kernel also measures its own decision margins (the topk_group-th minus
+//    the next group score, and every gap between neighbours in the ranking
+//    of the K+1 best candidates, since slot order is rank order) and appends
+//    the token to `unc` when one is below tau (scaled by the token's logit
+//    RMS); those tokens get exact logits and a second, exact pass.
+//  exact (tau == 0): scores from a float64 sigmoid rounded to fp32 (the
+//    reference definition), over the tokens in `list`.
+// GJ > 0: every group spans GJ whole register slots (E/n_group a multiple of
+// 32), so group maxima are reduced in registers, all groups at once.
 // ---------------------------------------------------------------------------
-template <int NV>
+template <int NV, int GJ>
 __global__ void __launch_bounds__(256) router_topk(int T, int E, int n_group, int topk_group,
                                                    int K, float scale, int renorm,
                                                    const float* __restrict__ z,
@@ -204,41 +271,69 @@ __global__ void __launch_bounds__(256) router_topk(int T, int E, int n_group, in
     const int t = list ? list[q] : q;
     const float* zr = z + static_cast<size_t>(t) * E;
     float s[NV], b[NV];
-    int g[NV];
+    float zz = 0.f;
 #pragma unroll
     for (int j = 0; j < NV; ++j) {
       const int e = lane + 32 * j;
       if (e < E) {
-        const float zz = zr[e];
-        s[j] = static_cast<float>(1.0 / (1.0 + exp(-static_cast<double>(zz))));
+        const float zv = zr[e];
+        zz = fmaf(zv, zv, zz);
+        s[j] = tau > 0.f ? 1.0f / (1.0f + expf(-zv))
+                         : static_cast<float>(1.0 / (1.0 + exp(-static_cast<double>(zv))));
         b[j] = s[j] + (bias ? bias[e] : 0.f);
-        g[j] = e / per;
       } else {
         s[j] = 0.f;
         b[j] = -INFINITY;
-        g[j] = -1;
       }
     }
-    // group score (max of b) held by lane g
-    float my_gscore = -INFINITY;
-    for (int gg = 0; gg < n_group; ++gg) {
-      float m = -INFINITY;
+    // ---- groups: keep topk_group by their max b (ties -> lower group)
+    uint32_t kept_groups = 0;  // bit g set when group g is kept
+    float gmargin = INFINITY;
+    if (GJ > 0) {
+      constexpr int G = GJ > 0 ? NV / GJ : 1;
+      float gs[G];
 #pragma unroll
-      for (int j = 0; j < NV; ++j)
-        if (g[j] == gg && b[j] > m) m = b[j];
+      for (int g = 0; g < G; ++g) {
+        float m = b[g * GJ];
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float other = __shfl_xor_sync(0xffffffffu, m, o);
-        m = other > m ? other : m;
+        for (int i = 1; i < GJ; ++i) m = fmaxf(m, b[g * GJ + i]);
+        gs[g] = m;
       }
-      if (lane == gg) my_gscore = m;
-    }
-    // keep topk_group groups: repeated argmax over lanes < n_group, ties -> lower lane;
-    // one more round (when a group is left) gives the group margin
-    bool my_kept = false;
-    float last_kept = 0.f, gmargin = INFINITY;
-    {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int g = 0; g < G; ++g) gs[g] = fmaxf(gs[g], __shfl_xor_sync(0xffffffffu, gs[g], o));
+      float last = 0.f;
+      for (int r = 0; r <= topk_group && r < G; ++r) {
+        float bv = -INFINITY;
+        int bi = -1;
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+          if (!((kept_groups >> g) & 1u) && (bi < 0 || gs[g] > bv)) {
+            bv = gs[g];
+            bi = g;
+          }
+        if (r < topk_group) {
+          kept_groups |= 1u << bi;
+          last = bv;
+        } else {
+          gmargin = last - bv;
+        }
+      }
+    } else {
+      // generic: group g's score is held by lane g
+      float my_gscore = -INFINITY;
+      for (int gg = 0; gg < n_group; ++gg) {
+        float m = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < NV; ++j)
+          if (lane + 32 * j < E && (lane + 32 * j) / per == gg && b[j] > m) m = b[j];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == gg) my_gscore = m;
+      }
       bool avail = lane < n_group;
+      float last = 0.f;
       const int rounds = topk_group < n_group ? topk_group + 1 : topk_group;
       for (int r = 0; r < rounds; ++r) {
         float bv = avail ? my_gscore : -INFINITY;
@@ -253,25 +348,23 @@ __global__ void __launch_bounds__(256) router_topk(int T, int E, int n_group, in
           }
         }
         if (r < topk_group) {
-          if (lane == bi) {
-            my_kept = true;
-            avail = false;
-          }
-          last_kept = bv;
+          if (lane == bi) avail = false;
+          kept_groups |= 1u << bi;
+          last = bv;
         } else {
-          gmargin = last_kept - bv;
+          gmargin = last - bv;
         }
       }
     }
     uint32_t cand = 0;
 #pragma unroll
     for (int j = 0; j < NV; ++j) {
-      const int src = g[j] < 0 ? 0 : g[j];
-      const bool k = __shfl_sync(0xffffffffu, my_kept ? 1 : 0, src) != 0;
-      if (k && g[j] >= 0) cand |= 1u << j;
+      const int e = lane + 32 * j;
+      const int g = GJ > 0 ? j / (GJ > 0 ? GJ : 1) : e / per;
+      if (e < E && ((kept_groups >> g) & 1u)) cand |= 1u << j;
     }
-    // K rounds of warp argmax over candidates (ties -> lower expert id), plus
-    // one more for the expert margin
+    // ---- K rounds of warp argmax over candidates (ties -> lower expert id),
+    // plus one more for the last gap of the ranking
     int my_e = -1;
     float my_s = 0.f, last_b = 0.f, emargin = INFINITY;
     for (int k = 0; k <= K; ++k) {
@@ -279,11 +372,9 @@ __global__ void __launch_bounds__(256) router_topk(int T, int E, int n_group, in
       int be = 0x7fffffff;
 #pragma unroll
       for (int j = 0; j < NV; ++j) {
-        if ((cand >> j) & 1u) {
-          if (b[j] > bv || be == 0x7fffffff) {
-            bv = b[j];
-            be = lane + 32 * j;
-          }
+        if (((cand >> j) & 1u) && (be == 0x7fffffff || b[j] > bv)) {
+          bv = b[j];
+          be = lane + 32 * j;
         }
       }
 #pragma unroll
@@ -295,7 +386,6 @@ __global__ void __launch_bounds__(256) router_topk(int T, int E, int n_group, in
           be = oe;
         }
       }
-      // every adjacent gap of the ranking counts: slot order is rank order
       if (k > 0 && be != 0x7fffffff) emargin = fminf(emargin, last_b - bv);
       if (k == K) break;
       // owner lane removes the winner and publishes its unbiased score
@@ -330,10 +420,6 @@ __global__ void __launch_bounds__(256) router_topk(int T, int E, int n_group, in
     }
     if (tau > 0.f) {
       // the fp32 logit error grows with the logits' magnitude: scale the margin
-      float zz = 0.f;
-#pragma unroll
-      for (int j = 0; j < NV; ++j)
-        if (lane + 32 * j < E) zz = fmaf(zr[lane + 32 * j], zr[lane + 32 * j], zz);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) zz += __shfl_xor_sync(0xffffffffu, zz, o);
       const float tau_t = tau * fmaxf(1.f, sqrtf(zz / E));
@@ -342,16 +428,17 @@ __global__ void __launch_bounds__(256) router_topk(int T, int E, int n_group, in
   }
 }
 
-template <int NV>
+template <int NV, int GJ>
 cudaError_t launch_topk(const moe_cfg& c, int T, const float* z, const float* bias, int32_t* idx,
                         float* w, float tau, int32_t* unc, int32_t* unc_n, const int32_t* list,
                         cudaStream_t s) {
-  const int warps = 8;
+  // small batches: one token per CTA, so every token's warp has an SM to itself
+  const int warps = T <= 4 * num_sms() ? 1 : 8;
   int grid = cdiv(T, warps);
   if (list) grid = std::min(grid, num_sms() * 4);
-  router_topk<NV><<<grid, warps * 32, 0, s>>>(T, c.E, c.n_group, c.topk_group, c.K, c.scale,
-                                              c.renorm, z, bias, idx, w, tau, unc, unc_n, list,
-                                              list ? unc_n : nullptr);
+  router_topk<NV, GJ><<<grid, warps * 32, 0, s>>>(T, c.E, c.n_group, c.topk_group, c.K, c.scale,
+                                                  c.renorm, z, bias, idx, w, tau, unc, unc_n,
+                                                  list, list ? unc_n : nullptr);
   return cudaGetLastError();
 }
 
@@ -359,23 +446,37 @@ cudaError_t topk_dispatch(const moe_cfg& c, int T, const float* z, const float* 
                           int32_t* idx, float* w, float tau, int32_t* unc, int32_t* unc_n,
                           const int32_t* list, cudaStream_t s) {
   const int nv = cdiv(c.E, 32);
-  if (nv <= 1) return launch_topk<1>(c, T, z, bias, idx, w, tau, unc, unc_n, list, s);
-  if (nv <= 2) return launch_topk<2>(c, T, z, bias, idx, w, tau, unc, unc_n, list, s);
-  if (nv <= 4) return launch_topk<4>(c, T, z, bias, idx, w, tau, unc, unc_n, list, s);
-  if (nv <= 8) return launch_topk<8>(c, T, z, bias, idx, w, tau, unc, unc_n, list, s);
-  if (nv <= 16) return launch_topk<16>(c, T, z, bias, idx, w, tau, unc, unc_n, list, s);
-  return launch_topk<32>(c, T, z, bias, idx, w, tau, unc, unc_n, list, s);
+  const int per = c.E / c.n_group;
+#define SGL_TOPK(NV_)                                                                    \
+  if (nv <= NV_) {                                                                       \
+    if (c.E == NV_ * 32 && per % 32 == 0 && per / 32 == 2 && NV_ >= 2)                   \
+      return launch_topk<NV_, (NV_ >= 2 ? 2 : 1)>(c, T, z, bias, idx, w, tau, unc, unc_n, \
+                                                  list, s);                              \
+    if (c.E == NV_ * 32 && per % 32 == 0 && per / 32 == 1)                               \
+      return launch_topk<NV_, 1>(c, T, z, bias, idx, w, tau, unc, unc_n, list, s);       \
+    return launch_topk<NV_, 0>(c, T, z, bias, idx, w, tau, unc, unc_n, list, s);         \
+  }
+  SGL_TOPK(1)
+  SGL_TOPK(2)
+  SGL_TOPK(4)
+  SGL_TOPK(8)
+  SGL_TOPK(16)
+  SGL_TOPK(32)
+#undef SGL_TOPK
+  return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_exact(const moe_cfg& c, int T, const uint16_t* x, const float* Wr, float* z,
-                         const int32_t* list, const int32_t* list_n, cudaStream_t s) {
+template <bool EXACT, int ILP>
+cudaError_t launch_rows(const moe_cfg& c, int T, const uint16_t* x, const float* Wr, float* z,
+                        const int32_t* list, const int32_t* list_n, int32_t* err, cudaStream_t s) {
   const size_t smem = static_cast<size_t>(kSmallT) * c.H * sizeof(uint16_t);
-  cudaError_t e = cudaFuncSetAttribute(router_logits_exact,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  auto kern = router_logits_rows<EXACT, ILP>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  router_logits_exact<<<cdiv(c.E, kRowWarps), kRowWarps * 32, smem, s>>>(T, c.H, c.E, x, Wr, z,
-                                                                        list, list_n);
+  kern<<<cdiv(c.E, kRowWarps), kRowWarps * kTokSplit * 32, smem, s>>>(T, c.H, c.E, x, Wr, z, list,
+                                                                      list_n,
+                                                          err);
   return cudaGetLastError();
 }
 
@@ -390,21 +491,21 @@ constexpr float kCertifyMargin = 1.0f / 32768.0f;
 
 cudaError_t launch_router(const moe_cfg& c, int T, const uint16_t* x, const float* Wr,
                           const float* bias, float* z, int32_t* idx, float* w, int32_t* unc,
-                          int32_t* unc_n, cudaStream_t s) {
+                          int32_t* unc_n, int32_t* err, cudaStream_t s) {
   cudaError_t e;
   if (c.H > kRowRegs * 128) return cudaErrorInvalidValue;
   if (T <= kSmallT) {
-    // small batch: exact logits for every token, one selection pass
-    if ((e = launch_exact(c, T, x, Wr, z, nullptr, nullptr, s)) != cudaSuccess) return e;
-    return topk_dispatch(c, T, z, bias, idx, w, 0.f, nullptr, nullptr, nullptr, s);
+    e = launch_rows<false, 4>(c, T, x, Wr, z, nullptr, nullptr, err, s);
+  } else {
+    dim3 grid(cdiv(T, kRT), cdiv(c.E, kRE));
+    router_logits_tiled<<<grid, 256, 0, s>>>(T, c.H, c.E, x, Wr, z);
+    e = cudaGetLastError();
   }
-  dim3 grid(cdiv(T, kRT), cdiv(c.E, kRE));
-  router_logits_tiled<<<grid, 256, 0, s>>>(T, c.H, c.E, x, Wr, z);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (e != cudaSuccess) return e;
   if ((e = topk_dispatch(c, T, z, bias, idx, w, kCertifyMargin, unc, unc_n, nullptr, s)) !=
       cudaSuccess)
     return e;
-  if ((e = launch_exact(c, T, x, Wr, z, unc, unc_n, s)) != cudaSuccess) return e;
+  if ((e = launch_rows<true, 8>(c, T, x, Wr, z, unc, unc_n, err, s)) != cudaSuccess) return e;
   return topk_dispatch(c, T, z, bias, idx, w, 0.f, nullptr, unc_n, unc, s);
 }
 
