@@ -5,7 +5,9 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "internal.h"
 
@@ -22,6 +24,20 @@ int num_sms() {
     cache[dev] = v > 0 ? v : 1;
   }
   return cache[dev];
+}
+
+cudaError_t ensure_dyn_smem(const void* func, int bytes) {
+  static std::mutex mu;
+  static std::map<std::pair<int, const void*>, int> granted;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  int& have = granted[std::make_pair(dev, func)];
+  if (have >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) have = bytes;
+  return e;
 }
 
 static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -55,8 +71,8 @@ WsLayout ws_layout(const moe_cfg& c, int T) {
   L.offsets = take(static_cast<size_t>(c.E + 1) * 4);
   L.perm = take(TK * 4);
   L.inv_perm = take(TK * 4);
-  L.items_gu = take(static_cast<size_t>(L.max_items_gu) * sizeof(WorkItem));
-  L.items_dn = take(static_cast<size_t>(L.max_items_dn) * sizeof(WorkItem));
+  L.gu_start = take(static_cast<size_t>(c.E + 2) * 4);
+  L.dn_start = take(static_cast<size_t>(c.E + 2) * 4);
   L.h_r = take(TK * c.I * 2);
   L.h_s = take(static_cast<size_t>(T) * (c.I_shared > 0 ? c.I_shared : 0) * 2);
   L.y_slot = take((TK + T) * c.H * 4);
@@ -193,8 +209,8 @@ moe_status moe_grouped_swiglu(const moe_cfg* cfg, int32_t T, const void* x, cons
   st = device_ok();
   if (st != MOE_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  WorkItem* gu = at<WorkItem>(ws, L.items_gu);
-  WorkItem* dn = at<WorkItem>(ws, L.items_dn);
+  int32_t* gu = at<int32_t>(ws, L.gu_start);
+  int32_t* dn = at<int32_t>(ws, L.dn_start);
   int32_t* nitems = at<int32_t>(ws, L.nitems);
   cudaError_t e = launch_schedule(*cfg, T, offsets, L, gu, dn, nitems, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
@@ -208,8 +224,9 @@ moe_status moe_grouped_swiglu(const moe_cfg* cfg, int32_t T, const void* x, cons
   a.h_r = at<uint16_t>(ws, L.h_r);
   a.h_s = at<uint16_t>(ws, L.h_s);
   a.y_slot = static_cast<float*>(y_slot);
-  a.items_gu = gu;
-  a.items_dn = dn;
+  a.offsets = offsets;
+  a.gu_start = gu;
+  a.dn_start = dn;
   a.nitems = nitems;
   a.err = at<int32_t>(ws, L.err);
   a.bn = L.bn;
@@ -256,8 +273,8 @@ moe_status moe_layer_forward(const moe_cfg* cfg, int32_t T, const void* x, const
   int32_t* offsets = at<int32_t>(ws, L.offsets);
   int32_t* perm = at<int32_t>(ws, L.perm);
   int32_t* err = at<int32_t>(ws, L.err);
-  WorkItem* gu = at<WorkItem>(ws, L.items_gu);
-  WorkItem* dn = at<WorkItem>(ws, L.items_dn);
+  int32_t* gu = at<int32_t>(ws, L.gu_start);
+  int32_t* dn = at<int32_t>(ws, L.dn_start);
   int32_t* nitems = at<int32_t>(ws, L.nitems);
   float* y_slot = at<float>(ws, L.y_slot);
   cudaError_t e;
@@ -281,8 +298,9 @@ moe_status moe_layer_forward(const moe_cfg* cfg, int32_t T, const void* x, const
   a.h_r = at<uint16_t>(ws, L.h_r);
   a.h_s = at<uint16_t>(ws, L.h_s);
   a.y_slot = y_slot;
-  a.items_gu = gu;
-  a.items_dn = dn;
+  a.offsets = offsets;
+  a.gu_start = gu;
+  a.dn_start = dn;
   a.nitems = nitems;
   a.err = err;
   a.bn = L.bn;

@@ -49,8 +49,9 @@ struct GemmParams {
   uint16_t* h_r;  // [T*K, I] permuted rows
   uint16_t* h_s;  // [T, Is]
   float* y_slot;   // [(T*K + T), H] fp32
-  const WorkItem* items;
-  const int32_t* nitems;  // device count of valid items
+  const int32_t* offsets;  // [E+1] routed row offsets
+  const int32_t* start;    // [E+2] first work item of each slot (slot E: shared expert)
+  const int32_t* nitems;   // device count of valid items
   int max_items;
   int32_t* err;
 };
@@ -99,6 +100,31 @@ __device__ __forceinline__ bool item_ok(const GemmParams& p, const WorkItem& it,
   return true;
 }
 
+// Work item `i` from the per-slot item prefix sums (staged in shared memory):
+// the slot is the last one whose first item is <= i; within a slot the row
+// tile varies fastest, so neighbouring CTAs share a weight tile in L2.
+__device__ __forceinline__ WorkItem decode_item(int i, const int* s_start, const int* s_off,
+                                                int nslots, int E, int T, int bn, int mode,
+                                                int nt_r, int nt_s) {
+  int lo = 0, hi = nslots;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (s_start[mid] <= i) lo = mid;
+    else hi = mid;
+  }
+  const int e = lo;
+  const bool sh = e == E;
+  const int rows = sh ? T : s_off[e + 1] - s_off[e];
+  const int r0 = sh ? 0 : s_off[e];
+  const int nm = max(1, (rows + bn - 1) / bn);
+  const int local = i - s_start[e];
+  const int n = local / nm, m = local - n * nm;
+  (void)mode;
+  (void)nt_r;
+  (void)nt_s;
+  return WorkItem{e, r0 + m * bn, min(bn, rows - m * bn), n};
+}
+
 template <int MODE, int BN>
 __global__ void __launch_bounds__(threads_for(MODE), 1)
     moe_gemm(const __grid_constant__ GemmParams p, const __grid_constant__ CUtensorMap tA0,
@@ -118,6 +144,8 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
   int* tok = reinterpret_cast<int*>(smem + C::STAGES * C::STAGE_BYTES + 256);
   int* meta_j = tok + BN;                                       // down: slot of each row
   float* meta_w = reinterpret_cast<float*>(meta_j + BN);        // down: its routing weight
+  int* s_start = reinterpret_cast<int*>(meta_w + BN);           // [E+2] item starts
+  int* s_off = s_start + (p.E + 2);                             // [E+1] row offsets
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
@@ -140,10 +168,16 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
+  for (int i = threadIdx.x; i < p.E + 2; i += blockDim.x) s_start[i] = p.start[i];
+  for (int i = threadIdx.x; i < p.E + 1; i += blockDim.x) s_off[i] = p.offsets[i];
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  const int nslots = p.E + (p.has_shared ? 1 : 0);
+  auto item_at = [&](int i) {
+    return decode_item(i, s_start, s_off, nslots, p.E, p.T, BN, MODE, 0, 0);
+  };
   const int n_items = min(*p.nitems, p.max_items);
   const int KB_r = (MODE == 0 ? p.H : p.I) / 64;
   const int KB_s = (MODE == 0 ? p.H : p.Is) / 64;
@@ -156,7 +190,7 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
     uint32_t phase = 0;
     bool live = true;
     for (int item = blockIdx.x; item < n_items && live; item += gridDim.x) {
-      const WorkItem it = p.items[item];
+      const WorkItem it = item_at(item);
       if (!item_ok(p, it, MODE, BN)) {
         if (lane == 0) atomicExch(p.err, MOE_DEVERR_SCHEDULE);
         continue;
@@ -213,7 +247,7 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
       uint32_t phase = 0, acc_phase = 0;
       bool live = true;
       for (int item = blockIdx.x; item < n_items && live; item += gridDim.x) {
-        const WorkItem it = p.items[item];
+        const WorkItem it = item_at(item);
         if (!item_ok(p, it, MODE, BN)) continue;
         const int nkb = it.e == p.E ? KB_s : KB_r;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) break;
@@ -264,7 +298,7 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
     int pend0 = -1, pend1 = -1;  // stages issued two and one steps ago, not yet retired
     bool live = true;
     for (int item = blockIdx.x; item < n_items && live; item += gridDim.x) {
-      const WorkItem it = p.items[item];
+      const WorkItem it = item_at(item);
       if (!item_ok(p, it, MODE, BN)) continue;
       const bool sh = it.e == p.E;
       const int nkb = sh ? KB_s : KB_r;
@@ -314,7 +348,7 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-      const WorkItem it = p.items[item];
+      const WorkItem it = item_at(item);
       if (!item_ok(p, it, MODE, BN)) continue;
       const bool sh = it.e == p.E;
       if (MODE == 1) {
@@ -453,7 +487,8 @@ GemmParams make_params(const GemmArgs& a, int mode) {
   p.h_r = a.h_r;
   p.h_s = a.h_s;
   p.y_slot = a.y_slot;
-  p.items = mode == 0 ? a.items_gu : a.items_dn;
+  p.offsets = a.offsets;
+  p.start = mode == 0 ? a.gu_start : a.dn_start;
   p.nitems = a.nitems + mode;
   p.max_items = mode == 0 ? a.max_items_gu : a.max_items_dn;
   p.err = a.err;
@@ -495,11 +530,13 @@ cudaError_t launch_mode(const GemmArgs& a, cudaStream_t s) {
   }
   if (!ok) return cudaErrorInvalidValue;
   auto kern = moe_gemm<MODE, BN>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  const int smem = C::SMEM + (2 * c.E + 3) * static_cast<int>(sizeof(int));
+  cudaError_t e = ensure_dyn_smem(reinterpret_cast<const void*>(kern),
+                                  C::SMEM + (2 * 1024 + 3) * static_cast<int>(sizeof(int)));
   if (e != cudaSuccess) return e;
   const int max_items = p.max_items;
   const int grid = max(1, min(num_sms(), max_items));
-  kern<<<grid, threads_for(MODE), C::SMEM, s>>>(p, tA0, tA1, tS0, tS1, tB0, tB1);
+  kern<<<grid, threads_for(MODE), smem, s>>>(p, tA0, tA1, tS0, tS1, tB0, tB1);
   return cudaGetLastError();
 }
 

@@ -13,6 +13,8 @@ namespace sgl {
 // [row0, row0 + nrows) of that expert's row range, output tile `ntile`
 // (128 output features). Rows are positions in the permuted row space for
 // routed experts (offsets[e] + m*BN) and token ids for the shared expert.
+// Items are not stored: the GEMM kernels decode an item index from the
+// per-slot item prefix sums (gu_start / dn_start) and the row offsets.
 struct WorkItem {
   int32_t e;
   int32_t row0;
@@ -36,7 +38,7 @@ inline int cdiv(long long a, long long b) { return static_cast<int>((a + b - 1) 
 __host__ __device__ inline int cdiv_dev(int a, int b) { return (a + b - 1) / b; }
 
 struct WsLayout {
-  size_t z, unc, tile_hist, idx, w, counts, offsets, perm, inv_perm, items_gu, items_dn, nitems, h_r,
+  size_t z, unc, tile_hist, idx, w, counts, offsets, perm, inv_perm, gu_start, dn_start, nitems, h_r,
       h_s, y_slot, err, total;
   int n_ptiles, bn, max_items_gu, max_items_dn;
 };
@@ -52,7 +54,7 @@ cudaError_t launch_router(const moe_cfg& c, int T, const uint16_t* x, const floa
 
 cudaError_t launch_permute(const moe_cfg& c, int T, const int32_t* idx, int32_t* tile_hist,
                            int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv_perm,
-                           int32_t* err, const WsLayout& L, WorkItem* items_gu, WorkItem* items_dn,
+                           int32_t* err, const WsLayout& L, int32_t* gu_start, int32_t* dn_start,
                            int32_t* nitems, cudaStream_t s);
 
 // Allocation-free permutation (moe_permute_static): scratch in a fixed
@@ -65,7 +67,7 @@ cudaError_t launch_permute_static(const moe_cfg& c, int T, const int32_t* idx, i
                                   cudaStream_t s);
 
 cudaError_t launch_schedule(const moe_cfg& c, int T, const int32_t* offsets, const WsLayout& L,
-                            WorkItem* items_gu, WorkItem* items_dn, int32_t* nitems,
+                            int32_t* gu_start, int32_t* dn_start, int32_t* nitems,
                             cudaStream_t s);
 
 struct GemmArgs {
@@ -78,8 +80,9 @@ struct GemmArgs {
   uint16_t* h_r;
   uint16_t* h_s;
   float* y_slot;
-  const WorkItem* items_gu;
-  const WorkItem* items_dn;
+  const int32_t* offsets;   // [E+1] routed row offsets
+  const int32_t* gu_start;  // [E+2] item prefix sums, gate/up
+  const int32_t* dn_start;  // [E+2] item prefix sums, down
   const int32_t* nitems;
   int32_t* err;
   int bn;
@@ -94,5 +97,9 @@ cudaError_t launch_combine(const moe_cfg& c, int T, const float* y_slot, int wit
                            uint16_t* y, cudaStream_t s);
 
 int num_sms();
+
+// Raises `func`'s dynamic shared-memory limit to at least `bytes`, once per
+// device (later calls with a size already granted cost a table lookup).
+cudaError_t ensure_dyn_smem(const void* func, int bytes);
 
 }  // namespace sgl

@@ -81,64 +81,47 @@ __device__ int block_exscan2(int v0, int v1, int* scratch /*32*/, int* total) {
 
 struct SchedArgs {
   int T, K, E, H, I, Is, has_shared, bn;
-  int max_gu, max_dn;
-  WorkItem* items_gu;
-  WorkItem* items_dn;
-  int32_t* nitems;
+  int32_t* gu_start;  // [E+2] first gate/up work item of slot e (e == E: shared expert)
+  int32_t* dn_start;  // [E+2] first down work item of slot e
+  int32_t* nitems;    // [2] totals
 };
 
-// Work lists for the two grouped GEMMs from per-expert row counts. Expert e
-// (e == E: the shared expert, whose rows are the T tokens) gets
-// ceil(rows/bn) row tiles times its output tiles; within an expert the row
-// tile varies fastest so that neighbouring CTAs share a weight tile in L2.
-// Needs blockDim.x == 1024 and counts/offsets in shared memory.
-__device__ void build_schedule(const SchedArgs& a, const int* cnt, const int* off, int* scratch) {
+// Work lists of the two grouped GEMMs, as prefix sums of per-slot item counts.
+// Slot e (e == E: the shared expert, whose rows are the T tokens) has
+// ceil(rows/bn) row tiles times its output tiles; the GEMM kernels decode an
+// item index back to (slot, row tile, output tile) with a binary search over
+// these starts. Needs blockDim.x == 1024 and counts in shared memory.
+__device__ void build_schedule(const SchedArgs& a, const int* cnt, int* scratch) {
   const int nslots = a.E + (a.has_shared ? 1 : 0);
   const int nt_gu_r = cdiv_dev(a.I, kTileN), nt_gu_s = cdiv_dev(a.Is, kTileN);
   const int nt_dn = cdiv_dev(a.H, kTileN);
-  int ngu[2] = {0, 0}, ndn[2] = {0, 0}, nm[2] = {0, 0};
+  int ngu[2] = {0, 0}, ndn[2] = {0, 0};
 #pragma unroll
   for (int q = 0; q < 2; ++q) {
     const int e = 2 * threadIdx.x + q;
     if (e < nslots) {
       const bool sh = e == a.E;
       const int rows = sh ? a.T : cnt[e];
-      nm[q] = (rows + a.bn - 1) / a.bn;
-      ngu[q] = nm[q] * (sh ? nt_gu_s : nt_gu_r);
-      ndn[q] = nm[q] * nt_dn;
+      const int nm = (rows + a.bn - 1) / a.bn;
+      ngu[q] = nm * (sh ? nt_gu_s : nt_gu_r);
+      ndn[q] = nm * nt_dn;
     }
   }
   int tot_gu, tot_dn;
   const int base_gu = block_exscan2(ngu[0], ngu[1], scratch, &tot_gu);
   const int base_dn = block_exscan2(ndn[0], ndn[1], scratch, &tot_dn);
-  int bg = base_gu, bd = base_dn;
 #pragma unroll
   for (int q = 0; q < 2; ++q) {
     const int e = 2 * threadIdx.x + q;
-    if (e < nslots && nm[q] > 0) {
-      const bool sh = e == a.E;
-      const int rows = sh ? a.T : cnt[e];
-      const int r0 = sh ? 0 : off[e];
-      const int ntg = sh ? nt_gu_s : nt_gu_r;
-      for (int n = 0; n < ntg; ++n)
-        for (int m = 0; m < nm[q]; ++m) {
-          const int i = bg + n * nm[q] + m;
-          if (i < a.max_gu)
-            a.items_gu[i] = WorkItem{e, r0 + m * a.bn, min(a.bn, rows - m * a.bn), n};
-        }
-      for (int n = 0; n < nt_dn; ++n)
-        for (int m = 0; m < nm[q]; ++m) {
-          const int i = bd + n * nm[q] + m;
-          if (i < a.max_dn)
-            a.items_dn[i] = WorkItem{e, r0 + m * a.bn, min(a.bn, rows - m * a.bn), n};
-        }
+    if (e <= a.E + 1) {
+      const bool real = e < nslots;
+      a.gu_start[e] = real ? base_gu + (q ? ngu[0] : 0) : tot_gu;
+      a.dn_start[e] = real ? base_dn + (q ? ndn[0] : 0) : tot_dn;
     }
-    bg += ngu[q];
-    bd += ndn[q];
   }
   if (threadIdx.x == 0) {
-    a.nitems[0] = min(tot_gu, a.max_gu);
-    a.nitems[1] = min(tot_dn, a.max_dn);
+    a.nitems[0] = tot_gu;
+    a.nitems[1] = tot_dn;
   }
 }
 
@@ -189,20 +172,16 @@ __global__ void __launch_bounds__(1024) perm_scan(int E, int n_ptiles,
       carry += __shfl_sync(0xffffffffu, incl, 31);
     }
   }
-  if (build) build_schedule(sa, cnt, off, scratch);
+  if (build) build_schedule(sa, cnt, scratch);
 }
 
 __global__ void __launch_bounds__(1024) schedule_only(const int32_t* __restrict__ offsets,
                                                       SchedArgs sa) {
   __shared__ int cnt[kMaxE + 1];
-  __shared__ int off[kMaxE + 1];
   __shared__ int scratch[33];
-  for (int e = threadIdx.x; e < sa.E; e += blockDim.x) {
-    off[e] = offsets[e];
-    cnt[e] = offsets[e + 1] - offsets[e];
-  }
+  for (int e = threadIdx.x; e < sa.E; e += blockDim.x) cnt[e] = offsets[e + 1] - offsets[e];
   __syncthreads();
-  build_schedule(sa, cnt, off, scratch);
+  build_schedule(sa, cnt, scratch);
 }
 
 __global__ void __launch_bounds__(kScatterWarps * 32) perm_scatter(
@@ -354,11 +333,11 @@ __global__ void __launch_bounds__(1024) perm_single(int TK, int E, const int32_t
       if (inv_perm) inv_perm[i] = pos;
     }
   }
-  if (build) build_schedule(sa, cnt, off, scratch);
+  if (build) build_schedule(sa, cnt, scratch);
 }
 
-SchedArgs make_sched(const moe_cfg& c, int T, const WsLayout& L, WorkItem* gu, WorkItem* dn,
-                     int32_t* nitems) {
+SchedArgs make_sched(const moe_cfg& c, int T, const WsLayout& L, int32_t* gu_start,
+                     int32_t* dn_start, int32_t* nitems) {
   SchedArgs a;
   a.T = T;
   a.K = c.K;
@@ -368,10 +347,8 @@ SchedArgs make_sched(const moe_cfg& c, int T, const WsLayout& L, WorkItem* gu, W
   a.Is = c.I_shared;
   a.has_shared = c.I_shared > 0;
   a.bn = L.bn;
-  a.max_gu = L.max_items_gu;
-  a.max_dn = L.max_items_dn;
-  a.items_gu = gu;
-  a.items_dn = dn;
+  a.gu_start = gu_start;
+  a.dn_start = dn_start;
   a.nitems = nitems;
   return a;
 }
@@ -380,24 +357,24 @@ SchedArgs make_sched(const moe_cfg& c, int T, const WsLayout& L, WorkItem* gu, W
 
 cudaError_t launch_permute(const moe_cfg& c, int T, const int32_t* idx, int32_t* tile_cnt,
                            int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv_perm,
-                           int32_t* err, const WsLayout& L, WorkItem* items_gu,
-                           WorkItem* items_dn, int32_t* nitems, cudaStream_t s) {
+                           int32_t* err, const WsLayout& L, int32_t* gu_start,
+                           int32_t* dn_start, int32_t* nitems, cudaStream_t s) {
   const int TK = T * c.K;
   const int np = L.n_ptiles;
-  SchedArgs sa = make_sched(c, T, L, items_gu, items_dn, nitems);
+  SchedArgs sa = make_sched(c, T, L, gu_start, dn_start, nitems);
   if (np == 1) {
     const int smem = 32 * c.E * static_cast<int>(sizeof(int));
-    cudaError_t e = cudaFuncSetAttribute(perm_single, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         smem);
+    cudaError_t e = ensure_dyn_smem(reinterpret_cast<const void*>(perm_single),
+                                    32 * kMaxE * static_cast<int>(sizeof(int)));
     if (e != cudaSuccess) return e;
     perm_single<<<1, 1024, smem, s>>>(TK, c.E, idx, counts, offsets, perm, inv_perm, err, sa,
-                                      items_gu != nullptr ? 1 : 0);
+                                      gu_start != nullptr ? 1 : 0);
     return cudaGetLastError();
   }
   int32_t* tile_base = tile_cnt + static_cast<size_t>(c.E) * np;
   perm_hist<<<np, 256, 0, s>>>(TK, c.E, np, idx, tile_cnt, err);
   perm_scan<<<1, 1024, 0, s>>>(c.E, np, tile_cnt, tile_base, counts, offsets, sa,
-                               items_gu != nullptr ? 1 : 0);
+                               gu_start != nullptr ? 1 : 0);
   perm_scatter<<<np, kScatterWarps * 32, 0, s>>>(TK, c.E, np, idx, tile_base, perm, inv_perm,
                                                  err);
   return cudaGetLastError();
@@ -455,9 +432,9 @@ cudaError_t launch_permute_static(const moe_cfg& c, int T, const int32_t* idx, i
 }
 
 cudaError_t launch_schedule(const moe_cfg& c, int T, const int32_t* offsets, const WsLayout& L,
-                            WorkItem* items_gu, WorkItem* items_dn, int32_t* nitems,
+                            int32_t* gu_start, int32_t* dn_start, int32_t* nitems,
                             cudaStream_t s) {
-  SchedArgs sa = make_sched(c, T, L, items_gu, items_dn, nitems);
+  SchedArgs sa = make_sched(c, T, L, gu_start, dn_start, nitems);
   schedule_only<<<1, 1024, 0, s>>>(offsets, sa);
   return cudaGetLastError();
 }

@@ -38,6 +38,7 @@ namespace {
 // ---------------------------------------------------------------------------
 constexpr int kSmallT = 32;
 constexpr int kRowRegs = 24;  // float4 per lane: H <= 24 * 128 = 3072
+constexpr int kMaxExperts = 1024;
 constexpr int kRowWarps = 4;  // experts per CTA
 constexpr int kTokSplit = 2;  // warps per expert (they split the token rows)
 
@@ -74,11 +75,16 @@ __global__ void __launch_bounds__(kRowWarps * kTokSplit * 32) router_logits_rows
   }
   uint32_t phase = 0;
   float4 wv[kRowRegs];
+  {
+    // unconditional loads from clamped addresses (all in flight together),
+    // then zero the slots past the row's end
+    const float* row = Wr + static_cast<size_t>(have ? e : 0) * H;
 #pragma unroll
-  for (int j = 0; j < kRowRegs; ++j) {
-    const int k = 4 * lane + 128 * j;
-    wv[j] = (have && k < H) ? *reinterpret_cast<const float4*>(Wr + static_cast<size_t>(e) * H + k)
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < kRowRegs; ++j)
+      wv[j] = *reinterpret_cast<const float4*>(row + min(4 * lane + 128 * j, H - 4));
+#pragma unroll
+    for (int j = 0; j < kRowRegs; ++j)
+      if (4 * lane + 128 * j >= H) wv[j] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
   const uint32_t row_bytes = static_cast<uint32_t>(H) * 2;
   for (int c0 = 0; c0 < n; c0 += kSmallT) {
@@ -270,21 +276,22 @@ __global__ void __launch_bounds__(256) router_topk(int T, int E, int n_group, in
   for (int q = blockIdx.x * wpb + (threadIdx.x >> 5); q < n; q += gridDim.x * wpb) {
     const int t = list ? list[q] : q;
     const float* zr = z + static_cast<size_t>(t) * E;
-    float s[NV], b[NV];
+    float s[NV], b[NV], zv[NV], bv0[NV];
+    // all loads first, from clamped (always valid) addresses, so they are in
+    // flight together; lanes past E are masked afterwards
+#pragma unroll
+    for (int j = 0; j < NV; ++j) zv[j] = zr[min(lane + 32 * j, E - 1)];
+#pragma unroll
+    for (int j = 0; j < NV; ++j) bv0[j] = bias ? bias[min(lane + 32 * j, E - 1)] : 0.f;
     float zz = 0.f;
 #pragma unroll
     for (int j = 0; j < NV; ++j) {
-      const int e = lane + 32 * j;
-      if (e < E) {
-        const float zv = zr[e];
-        zz = fmaf(zv, zv, zz);
-        s[j] = tau > 0.f ? 1.0f / (1.0f + expf(-zv))
-                         : static_cast<float>(1.0 / (1.0 + exp(-static_cast<double>(zv))));
-        b[j] = s[j] + (bias ? bias[e] : 0.f);
-      } else {
-        s[j] = 0.f;
-        b[j] = -INFINITY;
-      }
+      const bool in = lane + 32 * j < E;
+      if (in) zz = fmaf(zv[j], zv[j], zz);
+      s[j] = tau > 0.f ? 1.0f / (1.0f + expf(-zv[j]))
+                       : static_cast<float>(1.0 / (1.0 + exp(-static_cast<double>(zv[j]))));
+      b[j] = in ? s[j] + bv0[j] : -INFINITY;
+      if (!in) s[j] = 0.f;
     }
     // ---- groups: keep topk_group by their max b (ties -> lower group)
     uint32_t kept_groups = 0;  // bit g set when group g is kept
@@ -428,6 +435,340 @@ __global__ void __launch_bounds__(256) router_topk(int T, int E, int n_group, in
   }
 }
 
+// ---------------------------------------------------------------------------
+// Exact re-derivation of a close fp32 decision, one CTA per listed token.
+// With every fp32 biased score within eps = tau_t / 2 of its exact value:
+//  1. only groups whose fp32 score is within 2 eps of the (topk_group+1)-th
+//     can be kept, and a group's exact maximum comes from its experts within
+//     2 eps of its fp32 maximum: those experts get exact scores, and the kept
+//     groups are chosen from the exact maxima;
+//  2. among the kept groups' experts only those within 2 eps of the (K+1)-th
+//     fp32 candidate can be in the exact top K+1: they get exact scores and
+//     the K best are taken from them.
+// An exact score is the float64 dot product of the bf16 token row with the
+// fp32 router row (every product exact in float64), rounded once to fp32,
+// then the float64 sigmoid rounded to fp32, plus the bias in fp32: the same
+// arithmetic as the reference definition.
+// ---------------------------------------------------------------------------
+constexpr int kRefineThreads = 128;
+
+template <int NV>
+__device__ __forceinline__ void load_scores(const float* zr, const float* bias, int E, int lane,
+                                            float* b, float* zz_out) {
+  float zv[NV], bv0[NV];
+#pragma unroll
+  for (int j = 0; j < NV; ++j) zv[j] = zr[min(lane + 32 * j, E - 1)];
+#pragma unroll
+  for (int j = 0; j < NV; ++j) bv0[j] = bias ? bias[min(lane + 32 * j, E - 1)] : 0.f;
+  float zz = 0.f;
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    const bool in = lane + 32 * j < E;
+    if (in) zz = fmaf(zv[j], zv[j], zz);
+    b[j] = in ? 1.0f / (1.0f + expf(-zv[j])) + bv0[j] : -INFINITY;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) zz += __shfl_xor_sync(0xffffffffu, zz, o);
+  *zz_out = zz;
+}
+
+template <int NV>
+__global__ void __launch_bounds__(kRefineThreads) router_refine(
+    int T, int H, int E, int n_group, int topk_group, int K, float scale, int renorm,
+    float tau, const uint16_t* __restrict__ x, const float* __restrict__ Wr,
+    const float* __restrict__ z, const float* __restrict__ bias, int32_t* __restrict__ idx,
+    float* __restrict__ wout, const int32_t* __restrict__ list,
+    const int32_t* __restrict__ list_n) {
+  __shared__ __align__(16) uint16_t xs[kRowRegs * 128];
+  __shared__ int need[kMaxExperts];
+  __shared__ float bex[kMaxExperts], sex[kMaxExperts];
+  __shared__ uint32_t done[kMaxExperts / 32];
+  __shared__ float gsc[32];
+  __shared__ int kept_mask_s, n_need;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n = min(*list_n, T);
+  const int per = E / n_group;
+  for (int q = blockIdx.x; q < n; q += gridDim.x) {
+    const int t = list[q];
+    __syncthreads();  // smem of the previous token is no longer in use
+    for (int i = tid; i < H / 8; i += blockDim.x)
+      reinterpret_cast<uint4*>(xs)[i] = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H)[i];
+    for (int i = tid; i < (E + 31) / 32; i += blockDim.x) done[i] = 0u;
+    if (tid == 0) n_need = 0;
+    __syncthreads();
+
+    // ---- warp 0: fp32 scores, group scores, the experts that decide group maxima
+    float b[NV];
+    float tau_t = 0.f, gth = -INFINITY;
+    if (warp == 0) {
+      float zz;
+      load_scores<NV>(z + static_cast<size_t>(t) * E, bias, E, lane, b, &zz);
+      tau_t = tau * fmaxf(1.f, sqrtf(zz / E));
+      for (int g = 0; g < n_group; ++g) {
+        float m = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < NV; ++j)
+          if ((lane + 32 * j) / per == g && b[j] > m) m = b[j];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) gsc[g] = m;
+      }
+      __syncwarp();
+      // (topk_group+1)-th largest fp32 group score
+      if (topk_group < n_group) {
+        uint32_t taken = 0;
+        for (int r = 0; r <= topk_group; ++r) {
+          int bi = -1;
+          for (int g = 0; g < n_group; ++g)
+            if (!((taken >> g) & 1u) && (bi < 0 || gsc[g] > gsc[bi])) bi = g;
+          taken |= 1u << bi;
+          gth = gsc[bi];
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < NV; ++j) {
+        const int e = lane + 32 * j;
+        bool nd = false;
+        if (e < E) {
+          const float gs = gsc[e / per];
+          nd = gs >= gth - tau_t && b[j] >= gs - tau_t;
+        }
+        const unsigned bal = __ballot_sync(0xffffffffu, nd);
+        const int base = n_need;
+        __syncwarp();
+        if (nd) need[base + __popc(bal & ((1u << lane) - 1u))] = e;
+        __syncwarp();
+        if (lane == 0) n_need = base + __popc(bal);
+        __syncwarp();
+      }
+    }
+    __syncthreads();
+
+    // ---- exact scores for the listed experts: one warp per expert
+    for (int round = 0; round < 2; ++round) {
+      const int nn = n_need;
+      for (int i = warp; i < nn; i += blockDim.x / 32) {
+        const int e = need[i];
+        const float* row = Wr + static_cast<size_t>(e) * H;
+        float4 wv[kRowRegs];
+#pragma unroll
+        for (int j = 0; j < kRowRegs; ++j)
+          wv[j] = *reinterpret_cast<const float4*>(row + min(4 * lane + 128 * j, H - 4));
+        double acc = 0.0;
+#pragma unroll
+        for (int j = 0; j < kRowRegs; ++j) {
+          const int k = 4 * lane + 128 * j;
+          if (k < H) {
+            const uint2 p = *reinterpret_cast<const uint2*>(xs + k);
+            acc = fma(static_cast<double>(wv[j].x), bf16_bits_to_double(p.x & 0xFFFFu), acc);
+            acc = fma(static_cast<double>(wv[j].y), bf16_bits_to_double(p.x >> 16), acc);
+            acc = fma(static_cast<double>(wv[j].z), bf16_bits_to_double(p.y & 0xFFFFu), acc);
+            acc = fma(static_cast<double>(wv[j].w), bf16_bits_to_double(p.y >> 16), acc);
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) {
+          const float zf = static_cast<float>(acc);
+          const float sf = static_cast<float>(1.0 / (1.0 + exp(-static_cast<double>(zf))));
+          sex[e] = sf;
+          bex[e] = sf + (bias ? bias[e] : 0.f);
+          atomicOr(&done[e >> 5], 1u << (e & 31));
+        }
+      }
+      __syncthreads();
+      if (round == 1) break;
+      // ---- warp 0: kept groups from exact maxima, then the candidates near the cut
+      if (warp == 0) {
+        // exact maximum of every group that can be kept
+        float gex = -INFINITY;  // lane g holds group g's exact maximum
+        for (int g = 0; g < n_group; ++g) {
+          float m = -INFINITY;
+          if (gsc[g] >= gth - tau_t) {
+            for (int i = lane; i < nn; i += 32) {
+              const int e = need[i];
+              if (e / per == g) m = fmaxf(m, bex[e]);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+          }
+          if (lane == g) gex = m;
+        }
+        uint32_t kept = 0;
+        for (int r = 0; r < topk_group; ++r) {
+          float bv = lane < n_group && !((kept >> lane) & 1u) ? gex : -INFINITY;
+          int bi = lane < n_group && !((kept >> lane) & 1u) ? lane : 0x7fffffff;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            if (ov > bv || (ov == bv && oi < bi)) {
+              bv = ov;
+              bi = oi;
+            }
+          }
+          kept |= 1u << bi;
+        }
+        // (K+1)-th largest fp32 score among the kept groups' experts
+        uint32_t cand = 0;
+#pragma unroll
+        for (int j = 0; j < NV; ++j) {
+          const int e = lane + 32 * j;
+          if (e < E && ((kept >> (e / per)) & 1u)) cand |= 1u << j;
+        }
+        float bth = -INFINITY;
+        {
+          uint32_t c2 = cand;
+          for (int k = 0; k <= K; ++k) {
+            float bv = -INFINITY;
+            int be = 0x7fffffff;
+#pragma unroll
+            for (int j = 0; j < NV; ++j)
+              if (((c2 >> j) & 1u) && (be == 0x7fffffff || b[j] > bv)) {
+                bv = b[j];
+                be = lane + 32 * j;
+              }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+              const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+              const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+              if (ov > bv || (ov == bv && oe < be)) {
+                bv = ov;
+                be = oe;
+              }
+            }
+            if (be == 0x7fffffff) break;
+            bth = bv;
+            if ((be & 31) == lane) c2 &= ~(1u << (be >> 5));
+          }
+        }
+        if (lane == 0) {
+          kept_mask_s = static_cast<int>(kept);
+          n_need = 0;
+        }
+        __syncwarp();
+        // the final pool C (kept-group experts within 2 eps of the cut) goes to
+        // need[]; the ones without an exact score yet are computed next round
+#pragma unroll
+        for (int j = 0; j < NV; ++j) {
+          const int e = lane + 32 * j;
+          const bool inC = ((cand >> j) & 1u) && b[j] >= bth - tau_t;
+          const unsigned bal = __ballot_sync(0xffffffffu, inC);
+          const int base = n_need;
+          __syncwarp();
+          if (inC) need[base + __popc(bal & ((1u << lane) - 1u))] = e;
+          __syncwarp();
+          if (lane == 0) n_need = base + __popc(bal);
+          __syncwarp();
+        }
+      }
+      __syncthreads();
+      // skip experts that already have an exact score (compact the list in place)
+      if (warp == 0) {
+        const int nc = n_need;
+        int m = 0;
+        for (int i0 = 0; i0 < nc; i0 += 32) {
+          const int i = i0 + lane;
+          const int e = i < nc ? need[i] : 0;
+          const bool todo = i < nc && !((done[e >> 5] >> (e & 31)) & 1u);
+          const unsigned bal = __ballot_sync(0xffffffffu, todo);
+          __syncwarp();
+          // stash the full pool behind the to-do list: pool in bex-free slots is
+          // rebuilt below from `done` and the kept groups, so only the to-do part
+          // needs to stay in need[]
+          if (todo) need[m + __popc(bal & ((1u << lane) - 1u))] = e;
+          m += __popc(bal);
+          __syncwarp();
+        }
+        if (lane == 0) n_need = m;
+      }
+      __syncthreads();
+    }
+
+    // ---- warp 0: final top K over the pool, from exact scores
+    if (warp == 0) {
+      const uint32_t kept = static_cast<uint32_t>(kept_mask_s);
+      // recompute the pool membership (same rule as above) from registers
+      uint32_t cand = 0;
+#pragma unroll
+      for (int j = 0; j < NV; ++j) {
+        const int e = lane + 32 * j;
+        if (e < E && ((kept >> (e / per)) & 1u)) cand |= 1u << j;
+      }
+      float bth = -INFINITY;
+      {
+        uint32_t c2 = cand;
+        for (int k = 0; k <= K; ++k) {
+          float bv = -INFINITY;
+          int be = 0x7fffffff;
+#pragma unroll
+          for (int j = 0; j < NV; ++j)
+            if (((c2 >> j) & 1u) && (be == 0x7fffffff || b[j] > bv)) {
+              bv = b[j];
+              be = lane + 32 * j;
+            }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+            if (ov > bv || (ov == bv && oe < be)) {
+              bv = ov;
+              be = oe;
+            }
+          }
+          if (be == 0x7fffffff) break;
+          bth = bv;
+          if ((be & 31) == lane) c2 &= ~(1u << (be >> 5));
+        }
+      }
+      uint32_t pool = 0;
+#pragma unroll
+      for (int j = 0; j < NV; ++j)
+        if (((cand >> j) & 1u) && b[j] >= bth - tau_t) pool |= 1u << j;
+      int my_e = -1;
+      float my_s = 0.f;
+      for (int k = 0; k < K; ++k) {
+        float bv = -INFINITY;
+        int be = 0x7fffffff;
+#pragma unroll
+        for (int j = 0; j < NV; ++j) {
+          if ((pool >> j) & 1u) {
+            const float v = bex[lane + 32 * j];
+            if (be == 0x7fffffff || v > bv) {
+              bv = v;
+              be = lane + 32 * j;
+            }
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+          const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+          if (ov > bv || (ov == bv && oe < be)) {
+            bv = ov;
+            be = oe;
+          }
+        }
+        if ((be & 31) == lane) pool &= ~(1u << (be >> 5));
+        if (lane == k) {
+          my_e = be;
+          my_s = sex[be];
+        }
+      }
+      double v = (lane < K) ? static_cast<double>(my_s) : 0.0;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane < K) {
+        const double sk = static_cast<double>(my_s);
+        const double wv = renorm ? static_cast<double>(scale) * (sk / v)
+                                 : static_cast<double>(scale) * sk;
+        idx[static_cast<size_t>(t) * K + lane] = my_e;
+        wout[static_cast<size_t>(t) * K + lane] = static_cast<float>(wv);
+      }
+    }
+  }
+}
+
 template <int NV, int GJ>
 cudaError_t launch_topk(const moe_cfg& c, int T, const float* z, const float* bias, int32_t* idx,
                         float* w, float tau, int32_t* unc, int32_t* unc_n, const int32_t* list,
@@ -466,13 +807,36 @@ cudaError_t topk_dispatch(const moe_cfg& c, int T, const float* z, const float* 
   return cudaErrorInvalidValue;
 }
 
+template <int NV>
+cudaError_t launch_refine_nv(const moe_cfg& c, int T, const uint16_t* x, const float* Wr,
+                             const float* z, const float* bias, int32_t* idx, float* w, float tau,
+                             const int32_t* list, const int32_t* list_n, cudaStream_t s) {
+  const int grid = std::max(1, std::min(T, num_sms() * 4));
+  router_refine<NV><<<grid, kRefineThreads, 0, s>>>(T, c.H, c.E, c.n_group, c.topk_group, c.K,
+                                                    c.scale, c.renorm, tau, x, Wr, z, bias, idx,
+                                                    w, list, list_n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_refine(const moe_cfg& c, int T, const uint16_t* x, const float* Wr,
+                          const float* z, const float* bias, int32_t* idx, float* w, float tau,
+                          const int32_t* list, const int32_t* list_n, cudaStream_t s) {
+  const int nv = cdiv(c.E, 32);
+  if (nv <= 1) return launch_refine_nv<1>(c, T, x, Wr, z, bias, idx, w, tau, list, list_n, s);
+  if (nv <= 2) return launch_refine_nv<2>(c, T, x, Wr, z, bias, idx, w, tau, list, list_n, s);
+  if (nv <= 4) return launch_refine_nv<4>(c, T, x, Wr, z, bias, idx, w, tau, list, list_n, s);
+  if (nv <= 8) return launch_refine_nv<8>(c, T, x, Wr, z, bias, idx, w, tau, list, list_n, s);
+  if (nv <= 16) return launch_refine_nv<16>(c, T, x, Wr, z, bias, idx, w, tau, list, list_n, s);
+  return launch_refine_nv<32>(c, T, x, Wr, z, bias, idx, w, tau, list, list_n, s);
+}
+
 template <bool EXACT, int ILP>
 cudaError_t launch_rows(const moe_cfg& c, int T, const uint16_t* x, const float* Wr, float* z,
                         const int32_t* list, const int32_t* list_n, int32_t* err, cudaStream_t s) {
   const size_t smem = static_cast<size_t>(kSmallT) * c.H * sizeof(uint16_t);
   auto kern = router_logits_rows<EXACT, ILP>;
-  cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  cudaError_t e = ensure_dyn_smem(reinterpret_cast<const void*>(kern),
+                                  kSmallT * kRowRegs * 128 * static_cast<int>(sizeof(uint16_t)));
   if (e != cudaSuccess) return e;
   kern<<<cdiv(c.E, kRowWarps), kRowWarps * kTokSplit * 32, smem, s>>>(T, c.H, c.E, x, Wr, z, list,
                                                                       list_n,
@@ -505,8 +869,8 @@ cudaError_t launch_router(const moe_cfg& c, int T, const uint16_t* x, const floa
   if ((e = topk_dispatch(c, T, z, bias, idx, w, kCertifyMargin, unc, unc_n, nullptr, s)) !=
       cudaSuccess)
     return e;
-  if ((e = launch_rows<true, 8>(c, T, x, Wr, z, unc, unc_n, err, s)) != cudaSuccess) return e;
-  return topk_dispatch(c, T, z, bias, idx, w, 0.f, nullptr, unc_n, unc, s);
+  (void)err;
+  return launch_refine(c, T, x, Wr, z, bias, idx, w, kCertifyMargin, unc, unc_n, s);
 }
 
 }  // namespace sgl
