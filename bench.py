@@ -158,7 +158,8 @@ class ClockSampler:
 def algorithmic_work(cfg, T: int, touched: int):
     """Bytes and FLOPs the layer must move / compute (intermediates not credited)."""
     H, I, Is, K, E = cfg.H, cfg.I, cfg.I_shared, cfg.K, cfg.E
-    wb = 2  # bf16 weights
+    # bytes per routed weight: bf16, or MXFP4 (half a byte + one scale byte per 32)
+    wb = 2 if cfg.wfmt == workloads.MOE_W_BF16 else 0.5 + 1.0 / 32
     gu_bytes = touched * 2 * I * H * wb + 2 * Is * H * 2 + T * H * 2
     dn_bytes = touched * H * I * wb + H * Is * 2
     gu_flops = 2.0 * (T * K * 2 * I * H + T * 2 * Is * H)
@@ -205,7 +206,11 @@ def measure_gpu(cfg, steps, warmup, device, rank, with_e2e=True):
     d = workloads.generate(replica_config(cfg, rank), device)
     if rank:
         d["x"] = workloads.tokens(cfg, T, replica_tokens_seed(cfg, rank), device)
-    W = sgl.make_weights(d["Wg"], d["Wu"], d["Wd"], d["Wg_s"], d["Wu_s"], d["Wd_s"])
+    if "Wg_q" in d:
+        W = sgl.make_weights(d["Wg_q"], d["Wu_q"], d["Wd_q"], d["Wg_s"], d["Wu_s"], d["Wd_s"],
+                             d["Wg_sc"], d["Wu_sc"], d["Wd_sc"])
+    else:
+        W = sgl.make_weights(d["Wg"], d["Wu"], d["Wd"], d["Wg_s"], d["Wu_s"], d["Wd_s"])
     ws = sgl.alloc_workspace(cfg, T, device)
     y = torch.empty(T, cfg.H, dtype=torch.bfloat16, device=device)
     idx = torch.empty(T, cfg.K, dtype=torch.int32, device=device)
@@ -318,9 +323,22 @@ def oracle_inputs(d):
 
     def b16(t):
         return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    if "Wg_q" in d:
+        import oracle
+
+        def experts(e):
+            q = lambda k: d[k][e].cpu().numpy()  # noqa: E731
+            return (oracle.mxfp4_dequantize(q("Wg_q"), q("Wg_sc")),
+                    oracle.mxfp4_dequantize(q("Wu_q"), q("Wu_sc")),
+                    oracle.mxfp4_dequantize(q("Wd_q"), q("Wd_sc")))
+        fmt = "mxfp4"
+    else:
+        def experts(e):
+            return b16(d["Wg"][e]), b16(d["Wu"][e]), b16(d["Wd"][e])
+        fmt = "bf16"
     return dict(x=b16(d["x"]), Wr=d["Wr"].cpu().numpy(), bias=d["bias"].cpu().numpy(),
                 Wg_s=b16(d["Wg_s"]), Wu_s=b16(d["Wu_s"]), Wd_s=b16(d["Wd_s"]),
-                experts=lambda e: (b16(d["Wg"][e]), b16(d["Wu"][e]), b16(d["Wd"][e])))
+                experts=experts, fmt=fmt)
 
 
 def time_oracle(cfg, h, tokens):
@@ -333,6 +351,8 @@ def time_oracle(cfg, h, tokens):
 
     def ew(e):
         g, u, dd = host[e]
+        if h["fmt"] == "mxfp4":
+            return g, u, dd
         f = oracle.bf16_bits_to_f64
         return f(g), f(u), f(dd)
     t0 = time.perf_counter()

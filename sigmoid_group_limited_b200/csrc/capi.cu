@@ -76,6 +76,16 @@ WsLayout ws_layout(const moe_cfg& c, int T) {
   L.h_r = take(TK * c.I * 2);
   L.h_s = take(static_cast<size_t>(T) * (c.I_shared > 0 ? c.I_shared : 0) * 2);
   L.y_slot = take((TK + T) * c.H * 4);
+  if (c.wfmt == MOE_W_MXFP4) {
+    L.max_touched = static_cast<int>(TK < static_cast<size_t>(c.E) ? TK : c.E);
+    const size_t mat = static_cast<size_t>(L.max_touched) * c.I * c.H * 2;
+    L.slot_of = take(static_cast<size_t>(c.E) * 4);
+    L.touched = take(static_cast<size_t>(c.E) * 4);
+    L.ntouched = take(16);
+    L.wq_g = take(mat);
+    L.wq_u = take(mat);
+    L.wq_d = take(mat);
+  }
   L.total = o;
   return L;
 }
@@ -130,7 +140,10 @@ moe_status cu(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; 
 moe_status check_weights(const moe_cfg* c, const moe_weights* W) {
   if (W == nullptr || W->Wg == nullptr || W->Wu == nullptr || W->Wd == nullptr) return MOE_ERR_NULL;
   if (!al16(W->Wg) || !al16(W->Wu) || !al16(W->Wd)) return MOE_ERR_ALIGN;
-  if (c->wfmt == MOE_W_MXFP4) return MOE_ERR_UNSUPPORTED;
+  if (c->wfmt == MOE_W_MXFP4) {
+    if (!W->Wg_scale || !W->Wu_scale || !W->Wd_scale) return MOE_ERR_NULL;
+    if (!al16(W->Wg_scale) || !al16(W->Wu_scale) || !al16(W->Wd_scale)) return MOE_ERR_ALIGN;
+  }
   if (c->I_shared > 0) {
     if (W->Wg_s == nullptr || W->Wu_s == nullptr || W->Wd_s == nullptr) return MOE_ERR_NULL;
     if (!al16(W->Wg_s) || !al16(W->Wu_s) || !al16(W->Wd_s)) return MOE_ERR_ALIGN;
@@ -214,6 +227,7 @@ moe_status moe_grouped_swiglu(const moe_cfg* cfg, int32_t T, const void* x, cons
   int32_t* nitems = at<int32_t>(ws, L.nitems);
   cudaError_t e = launch_schedule(*cfg, T, offsets, L, gu, dn, nitems, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
+  const int32_t* a_offsets = offsets;
   GemmArgs a;
   a.cfg = cfg;
   a.T = T;
@@ -221,6 +235,23 @@ moe_status moe_grouped_swiglu(const moe_cfg* cfg, int32_t T, const void* x, cons
   a.perm = perm;
   a.w = w;
   a.W = W;
+  a.Wg = W->Wg;
+  a.Wu = W->Wu;
+  a.Wd = W->Wd;
+  a.wslot = nullptr;
+  a.wrows = cfg->E;
+  if (cfg->wfmt == MOE_W_MXFP4) {
+    if (launch_mxfp4_expand(*cfg, a_offsets, W, at<int32_t>(ws, L.slot_of),
+                            at<int32_t>(ws, L.touched), at<int32_t>(ws, L.ntouched),
+                            at<uint16_t>(ws, L.wq_g), at<uint16_t>(ws, L.wq_u),
+                            at<uint16_t>(ws, L.wq_d), s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    a.Wg = at<uint16_t>(ws, L.wq_g);
+    a.Wu = at<uint16_t>(ws, L.wq_u);
+    a.Wd = at<uint16_t>(ws, L.wq_d);
+    a.wslot = at<int32_t>(ws, L.slot_of);
+    a.wrows = L.max_touched;
+  }
   a.h_r = at<uint16_t>(ws, L.h_r);
   a.h_s = at<uint16_t>(ws, L.h_s);
   a.y_slot = static_cast<float*>(y_slot);
@@ -288,6 +319,7 @@ moe_status moe_layer_forward(const moe_cfg* cfg, int32_t T, const void* x, const
                           at<int32_t>(ws, L.inv_perm), err, L, gu, dn, nitems, s)) != cudaSuccess)
     return MOE_ERR_CUDA;
   rec(2);
+  const int32_t* a_offsets = offsets;
   GemmArgs a;
   a.cfg = cfg;
   a.T = T;
@@ -295,6 +327,23 @@ moe_status moe_layer_forward(const moe_cfg* cfg, int32_t T, const void* x, const
   a.perm = perm;
   a.w = w;
   a.W = W;
+  a.Wg = W->Wg;
+  a.Wu = W->Wu;
+  a.Wd = W->Wd;
+  a.wslot = nullptr;
+  a.wrows = cfg->E;
+  if (cfg->wfmt == MOE_W_MXFP4) {
+    if (launch_mxfp4_expand(*cfg, a_offsets, W, at<int32_t>(ws, L.slot_of),
+                            at<int32_t>(ws, L.touched), at<int32_t>(ws, L.ntouched),
+                            at<uint16_t>(ws, L.wq_g), at<uint16_t>(ws, L.wq_u),
+                            at<uint16_t>(ws, L.wq_d), s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    a.Wg = at<uint16_t>(ws, L.wq_g);
+    a.Wu = at<uint16_t>(ws, L.wq_u);
+    a.Wd = at<uint16_t>(ws, L.wq_d);
+    a.wslot = at<int32_t>(ws, L.slot_of);
+    a.wrows = L.max_touched;
+  }
   a.h_r = at<uint16_t>(ws, L.h_r);
   a.h_s = at<uint16_t>(ws, L.h_s);
   a.y_slot = y_slot;

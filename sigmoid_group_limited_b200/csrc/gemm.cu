@@ -50,6 +50,7 @@ struct GemmParams {
   uint16_t* h_s;  // [T, Is]
   float* y_slot;   // [(T*K + T), H] fp32
   const int32_t* offsets;  // [E+1] routed row offsets
+  const int32_t* wslot;    // nullable: weight row block of expert e
   const int32_t* start;    // [E+2] first work item of each slot (slot E: shared expert)
   const int32_t* nitems;   // device count of valid items
   int max_items;
@@ -198,8 +199,9 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
       const bool sh = it.e == p.E;
       if (lane == 0) {
         const int nkb = sh ? KB_s : KB_r;
+        const int wblk = p.wslot ? p.wslot[it.e] : it.e;
         const int arow = sh ? it.ntile * kTileN
-                            : it.e * (MODE == 0 ? p.I : p.H) + it.ntile * kTileN;
+                            : wblk * (MODE == 0 ? p.I : p.H) + it.ntile * kTileN;
         const CUtensorMap* mA0 = sh ? &tS0 : &tA0;
         const CUtensorMap* mA1 = sh ? &tS1 : &tA1;
         for (int kb = 0; kb < nkb; ++kb) {
@@ -488,6 +490,7 @@ GemmParams make_params(const GemmArgs& a, int mode) {
   p.h_s = a.h_s;
   p.y_slot = a.y_slot;
   p.offsets = a.offsets;
+  p.wslot = a.wslot;
   p.start = mode == 0 ? a.gu_start : a.dn_start;
   p.nitems = a.nitems + mode;
   p.max_items = mode == 0 ? a.max_items_gu : a.max_items_dn;
@@ -504,8 +507,8 @@ cudaError_t launch_mode(const GemmArgs& a, cudaStream_t s) {
   const int T = a.T, TK = a.T * c.K;
   bool ok = true;
   if (MODE == 0) {
-    ok &= map_bf16(&tA0, a.W->Wg, static_cast<uint64_t>(c.E) * c.I, c.H, kTileN);
-    ok &= map_bf16(&tA1, a.W->Wu, static_cast<uint64_t>(c.E) * c.I, c.H, kTileN);
+    ok &= map_bf16(&tA0, a.Wg, static_cast<uint64_t>(a.wrows) * c.I, c.H, kTileN);
+    ok &= map_bf16(&tA1, a.Wu, static_cast<uint64_t>(a.wrows) * c.I, c.H, kTileN);
     ok &= map_bf16(&tB0, a.x, T, c.H, 1);
     tB1 = tB0;
     if (p.has_shared) {
@@ -516,7 +519,7 @@ cudaError_t launch_mode(const GemmArgs& a, cudaStream_t s) {
       tS1 = tA1;
     }
   } else {
-    ok &= map_bf16(&tA0, a.W->Wd, static_cast<uint64_t>(c.E) * c.H, c.I, kTileN);
+    ok &= map_bf16(&tA0, a.Wd, static_cast<uint64_t>(a.wrows) * c.H, c.I, kTileN);
     tA1 = tA0;
     ok &= map_bf16(&tB0, a.h_r, TK, c.I, BN);
     if (p.has_shared) {

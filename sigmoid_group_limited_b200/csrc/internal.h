@@ -40,6 +40,9 @@ __host__ __device__ inline int cdiv_dev(int a, int b) { return (a + b - 1) / b; 
 struct WsLayout {
   size_t z, unc, tile_hist, idx, w, counts, offsets, perm, inv_perm, gu_start, dn_start, nitems, h_r,
       h_s, y_slot, err, total;
+  // MXFP4 routed weights only: touched-expert slots and their bf16 copies
+  size_t slot_of, touched, ntouched, wq_g, wq_u, wq_d;
+  int max_touched;
   int n_ptiles, bn, max_items_gu, max_items_dn;
 };
 
@@ -77,6 +80,11 @@ struct GemmArgs {
   const int32_t* perm;
   const float* w;
   const moe_weights* W;
+  const void* Wg;            // routed weights the GEMMs read (bf16), expert- or slot-major
+  const void* Wu;
+  const void* Wd;
+  const int32_t* wslot;      // nullable: row block of expert e is wslot[e] instead of e
+  int wrows;                 // row blocks in Wg/Wu/Wd (E, or the slot capacity)
   uint16_t* h_r;
   uint16_t* h_s;
   float* y_slot;
@@ -92,6 +100,11 @@ struct GemmArgs {
 
 cudaError_t launch_gemm_gateup(const GemmArgs& a, cudaStream_t s);
 cudaError_t launch_gemm_down(const GemmArgs& a, cudaStream_t s);
+
+// MXFP4: list the touched experts and dequantise each once into bf16 slots.
+cudaError_t launch_mxfp4_expand(const moe_cfg& c, const int32_t* offsets, const moe_weights* W,
+                                int32_t* slot_of, int32_t* touched, int32_t* ntouched,
+                                uint16_t* gout, uint16_t* uout, uint16_t* dout, cudaStream_t s);
 
 cudaError_t launch_combine(const moe_cfg& c, int T, const float* y_slot, int with_shared,
                            uint16_t* y, cudaStream_t s);

@@ -35,7 +35,29 @@ class DeviceExperts:
         return f(bits(self.d["Wg"][e])), f(bits(self.d["Wu"][e])), f(bits(self.d["Wd"][e]))
 
 
+class DeviceExpertsMXFP4:
+    """Oracle accessor for MXFP4 routed weights: host copies of one expert's
+    packed codes and scales, dequantised by the oracle."""
+
+    def __init__(self, d):
+        self.d = d
+
+    def __call__(self, e: int):
+        d = self.d
+        q = lambda k: d[k][e].cpu().numpy()  # noqa: E731
+        return (oracle.mxfp4_dequantize(q("Wg_q"), q("Wg_sc")),
+                oracle.mxfp4_dequantize(q("Wu_q"), q("Wu_sc")),
+                oracle.mxfp4_dequantize(q("Wd_q"), q("Wd_sc")))
+
+
+def experts_of(d):
+    return DeviceExpertsMXFP4(d) if "Wg_q" in d else DeviceExperts(d)
+
+
 def weights(d):
+    if "Wg_q" in d:
+        return sgl.make_weights(d["Wg_q"], d["Wu_q"], d["Wd_q"], d.get("Wg_s"), d.get("Wu_s"),
+                                d.get("Wd_s"), d["Wg_sc"], d["Wu_sc"], d["Wd_sc"])
     return sgl.make_weights(d["Wg"], d["Wu"], d["Wd"], d.get("Wg_s"), d.get("Wu_s"), d.get("Wd_s"))
 
 

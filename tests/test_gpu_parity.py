@@ -14,8 +14,8 @@ import torch
 import oracle
 import sigmoid_group_limited_b200 as sgl
 import workloads
-from helpers import (DeviceExperts, bits, check_routing, check_y, host_inputs, near_tie_tokens,
-                     run_layer, run_staged)
+from helpers import (DeviceExperts, bits, check_routing, check_y, experts_of, host_inputs,
+                     near_tie_tokens, run_layer, run_staged)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -23,8 +23,12 @@ DEV = "cuda"
 
 def _oracle_layer(cfg, d, tokens=None):
     h = host_inputs(d)
-    return oracle.layer_forward(cfg, h["x"], h["Wr"], h["bias"], DeviceExperts(d), h["Wg_s"],
+    return oracle.layer_forward(cfg, h["x"], h["Wr"], h["bias"], experts_of(d), h["Wg_s"],
                                 h["Wu_s"], h["Wd_s"], tokens=tokens)
+
+
+def _tol(cfg):
+    return 5e-2 if cfg.wfmt == workloads.MOE_W_MXFP4 else 2e-2
 
 
 def _full_check(cfg, d, tokens=None):
@@ -36,7 +40,7 @@ def _full_check(cfg, d, tokens=None):
     assert np.array_equal(g["counts"].cpu().numpy(), counts)
     tok = ref["tokens"]
     keep = ~np.isin(tok, near)
-    check_y(bits(g["y"])[tok[keep]], ref["y_f32"][keep], ref["y"][keep])
+    check_y(bits(g["y"])[tok[keep]], ref["y_f32"][keep], ref["y"][keep], tol=_tol(cfg))
     return g, ref, near
 
 
@@ -185,7 +189,7 @@ def test_decode_full_size():
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("name", ["prefill", "prefill_bias0", "zipf"])
+@pytest.mark.parametrize("name", ["prefill", "prefill_bias0", "zipf", "mxfp4"])
 def test_full_size_sampled(name):
     cfg = workloads.CONFIGS[name]
     d = workloads.generate(cfg, DEV)
@@ -198,7 +202,7 @@ def test_full_size_sampled(name):
     assert np.array_equal(st["offsets"].cpu().numpy(), p_ref[1])
     # staged path with the oracle's own routing covers the near-tie tokens too
     st2 = run_staged(cfg, d, torch.from_numpy(ref["idx"]).to(DEV), torch.from_numpy(ref["w"]).to(DEV))
-    check_y(bits(st2["y"])[tok], ref["y_f32"], ref["y"])
+    check_y(bits(st2["y"])[tok], ref["y_f32"], ref["y"], tol=_tol(cfg))
     del d
     torch.cuda.empty_cache()
 
@@ -236,3 +240,14 @@ def test_route_full_size_every_token(T):
     ref = oracle.route(bits(x), Wr.cpu().numpy(), bias.cpu().numpy(), cfg.n_group, cfg.topk_group, cfg.K)
     near = check_routing(ref, idx.cpu().numpy(), w.cpu().numpy())
     assert len(near) <= max(2, T // 500)
+
+
+@pytest.mark.parametrize("T,variant", [(64, {}), (300, dict(limit_routed=0.5, limit_shared=0.7)),
+                                       (7, dict(I=128, I_shared=192))])
+def test_tiny_mxfp4(T, variant):
+    """Routed weights as MXFP4 codes + e8m0 scales; the oracle dequantises the
+    same bytes (the bar for this format is 5e-2 x RMS)."""
+    cfg = TINY.with_(wfmt=workloads.MOE_W_MXFP4, **variant)
+    d = workloads.generate(cfg, DEV, T=T)
+    assert "Wg" not in d and d["Wg_q"].dtype == torch.uint8
+    _full_check(cfg, d)
