@@ -76,6 +76,7 @@ WsLayout ws_layout(const moe_cfg& c, int T) {
   L.h_r = take(TK * c.I * 2);
   L.h_s = take(static_cast<size_t>(T) * (c.I_shared > 0 ? c.I_shared : 0) * 2);
   L.y_slot = take((TK + T) * c.H * 4);
+  L.wr_split = T > 32 ? take(static_cast<size_t>(3) * c.E * c.H * 2) : 0;
   if (c.wfmt == MOE_W_MXFP4) {
     L.max_touched = static_cast<int>(TK < static_cast<size_t>(c.E) ? TK : c.E);
     const size_t mat = static_cast<size_t>(L.max_touched) * c.I * c.H * 2;
@@ -174,7 +175,8 @@ moe_status moe_route(const moe_cfg* cfg, int32_t T, const void* x, const float* 
   if (cudaMemsetAsync(at<int32_t>(ws, L.err), 0, 16, s) != cudaSuccess) return MOE_ERR_CUDA;
   return cu(launch_router(*cfg, T, static_cast<const uint16_t*>(x), Wr, bias, at<float>(ws, L.z),
                           idx, w, at<int32_t>(ws, L.unc), at<int32_t>(ws, L.err) + 1,
-                          at<int32_t>(ws, L.err), s));
+                          at<int32_t>(ws, L.err), T > 32 ? at<uint16_t>(ws, L.wr_split) : nullptr,
+                          s));
 }
 
 moe_status moe_permute(const moe_cfg* cfg, int32_t T, const int32_t* idx, int32_t* counts,
@@ -312,7 +314,8 @@ moe_status moe_layer_forward(const moe_cfg* cfg, int32_t T, const void* x, const
   rec(0);
   if (cudaMemsetAsync(err, 0, 16, s) != cudaSuccess) return MOE_ERR_CUDA;
   if ((e = launch_router(*cfg, T, static_cast<const uint16_t*>(x), Wr, bias, at<float>(ws, L.z),
-                         idx, w, at<int32_t>(ws, L.unc), err + 1, err, s)) != cudaSuccess)
+                         idx, w, at<int32_t>(ws, L.unc), err + 1, err,
+                         T > 32 ? at<uint16_t>(ws, L.wr_split) : nullptr, s)) != cudaSuccess)
     return MOE_ERR_CUDA;
   rec(1);
   if ((e = launch_permute(*cfg, T, idx, at<int32_t>(ws, L.tile_hist), counts, offsets, perm,

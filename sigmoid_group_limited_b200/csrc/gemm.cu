@@ -27,6 +27,9 @@
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
+#include <string.h>
+
+#include <algorithm>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -48,6 +51,7 @@ struct GemmParams {
   const float* w;
   uint16_t* h_r;  // [T*K, I] permuted rows
   uint16_t* h_s;  // [T, Is]
+  float* z;       // router mode: logits [T, E]
   float* y_slot;   // [(T*K + T), H] fp32
   const int32_t* offsets;  // [E+1] routed row offsets
   const int32_t* wslot;    // nullable: weight row block of expert e
@@ -65,14 +69,18 @@ __host__ __device__ constexpr int pow2_at_least(int v) {
 
 template <int MODE, int BN>
 struct Cfg {
-  static constexpr int NA = MODE == 0 ? 2 : 1;       // weight tiles per stage (gate+up or down)
+  // weight tiles per stage: gate + up (0), down (1), router hi + mid + lo (2)
+  static constexpr int NA = MODE == 0 ? 2 : (MODE == 2 ? 3 : 1);
   static constexpr int A_BYTES = kTileN * 128;       // 128 rows x 64 bf16
   static constexpr int B_BYTES = BN * 128;           // BN rows x 64 bf16
   static constexpr int STAGE_BYTES = NA * A_BYTES + B_BYTES;
   static constexpr int STAGES_RAW = kSmemBudget / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
-  static constexpr int ACC_COLS = NA * BN;           // fp32 columns per accumulator
-  static constexpr int TMEM_COLS = pow2_at_least(2 * ACC_COLS);
+  // fp32 columns per accumulator buffer: gate and up side by side (0), one (1, 2)
+  static constexpr int ACC_COLS = (MODE == 0 ? 2 : 1) * BN;
+  // router mode: two hi-term chunk buffers + the mid and lo accumulators
+  static constexpr int TMEM_COLS = pow2_at_least(MODE == 2 ? 4 * BN : 2 * ACC_COLS);
+  static_assert(TMEM_COLS <= 512, "two accumulator buffers must fit the 512 TMEM columns");
   static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/ +
                              BN * 4 /*token rows*/ + BN * 8 /*row metadata*/;
 };
@@ -91,6 +99,9 @@ __device__ __forceinline__ uint16_t f2bf(float v) {
 // Same validity rule in every role, so all roles skip the same items.
 __device__ __forceinline__ bool item_ok(const GemmParams& p, const WorkItem& it, int mode,
                                         int bn) {
+  if (mode == 2)
+    return it.e == 0 && it.nrows > 0 && it.nrows <= bn && it.row0 >= 0 &&
+           it.row0 + it.nrows <= p.T && it.ntile >= 0 && it.ntile * kTileN < p.E;
   const bool sh = it.e == p.E;
   if (it.e < 0 || it.e > p.E || (sh && !p.has_shared)) return false;
   if (it.nrows <= 0 || it.nrows > bn || it.row0 < 0) return false;
@@ -140,7 +151,9 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
   uint64_t* empty = full + C::STAGES;
   uint64_t* tfull = empty + C::STAGES;
   uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint64_t* hfull = tempty + 2;   // router mode: hi-term chunk buffers
+  uint64_t* hempty = hfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(hempty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* tok = reinterpret_cast<int*>(smem + C::STAGES * C::STAGE_BYTES + 256);
   int* meta_j = tok + BN;                                       // down: slot of each row
@@ -158,6 +171,8 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], 4);
+      mbar_init(&hfull[a], 1);
+      mbar_init(&hempty[a], 4);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -169,19 +184,26 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
-  for (int i = threadIdx.x; i < p.E + 2; i += blockDim.x) s_start[i] = p.start[i];
-  for (int i = threadIdx.x; i < p.E + 1; i += blockDim.x) s_off[i] = p.offsets[i];
+  if (MODE != 2) {
+    for (int i = threadIdx.x; i < p.E + 2; i += blockDim.x) s_start[i] = p.start[i];
+    for (int i = threadIdx.x; i < p.E + 1; i += blockDim.x) s_off[i] = p.offsets[i];
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int nslots = p.E + (p.has_shared ? 1 : 0);
   auto item_at = [&](int i) {
+    if (MODE == 2) {  // router: output tile n of 128 experts x token tile m
+      const int nm = (p.T + BN - 1) / BN;
+      const int n = i / nm, m = i - n * nm;
+      return WorkItem{0, m * BN, min(BN, p.T - m * BN), n};
+    }
     return decode_item(i, s_start, s_off, nslots, p.E, p.T, BN, MODE, 0, 0);
   };
-  const int n_items = min(*p.nitems, p.max_items);
-  const int KB_r = (MODE == 0 ? p.H : p.I) / 64;
-  const int KB_s = (MODE == 0 ? p.H : p.Is) / 64;
+  const int n_items = p.nitems ? min(*p.nitems, p.max_items) : p.max_items;
+  const int KB_r = (MODE == 1 ? p.I : p.H) / 64;
+  const int KB_s = (MODE == 1 ? p.Is : p.H) / 64;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -199,9 +221,9 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
       const bool sh = it.e == p.E;
       if (lane == 0) {
         const int nkb = sh ? KB_s : KB_r;
-        const int wblk = p.wslot ? p.wslot[it.e] : it.e;
-        const int arow = sh ? it.ntile * kTileN
-                            : wblk * (MODE == 0 ? p.I : p.H) + it.ntile * kTileN;
+        const int wblk = (MODE != 2 && p.wslot) ? p.wslot[it.e] : it.e;
+        const int arow = (sh || MODE == 2) ? it.ntile * kTileN
+                                           : wblk * (MODE == 0 ? p.I : p.H) + it.ntile * kTileN;
         const CUtensorMap* mA0 = sh ? &tS0 : &tA0;
         const CUtensorMap* mA1 = sh ? &tS1 : &tA1;
         for (int kb = 0; kb < nkb; ++kb) {
@@ -216,6 +238,13 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
             mbar_arrive_expect_tx(&full[stage], C::NA * C::A_BYTES);
             tma_load_2d(sA, mA0, &full[stage], kb * 64, arow, pol_w);
             tma_load_2d(sA + C::A_BYTES, mA1, &full[stage], kb * 64, arow, pol_w);
+          } else if (MODE == 2) {
+            // router: the three bf16 terms of the fp32 router rows, and the tokens
+            mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+            tma_load_2d(sA, &tA0, &full[stage], kb * 64, arow, pol_x);
+            tma_load_2d(sA + C::A_BYTES, &tA1, &full[stage], kb * 64, arow, pol_x);
+            tma_load_2d(sA + 2 * C::A_BYTES, &tS0, &full[stage], kb * 64, arow, pol_x);
+            tma_load_2d(sB, &tB0, &full[stage], kb * 64, it.row0, pol_w);
           } else {
             mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
             tma_load_2d(sA, mA0, &full[stage], kb * 64, arow, pol_w);
@@ -243,7 +272,53 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && MODE == 2) {
+      // Router: the hi term goes into a fresh chunk accumulator per 64-wide
+      // k-block (double-buffered; the epilogue adds the chunks in fp32
+      // registers), mid and lo accumulate over the whole K in their own
+      // buffers. Short accumulations keep the tensor cores' fp32 rounding small.
+      constexpr uint32_t idesc = idesc_bf16(kTileN, BN);
+      int stage = 0, ck = 0;
+      uint32_t phase = 0, tph = 0;
+      bool live = true;
+      const uint32_t d_mid = tmem_base + 2 * BN, d_lo = tmem_base + 3 * BN;
+      for (int item = blockIdx.x; item < n_items && live; item += gridDim.x) {
+        const WorkItem it = item_at(item);
+        if (!item_ok(p, it, MODE, BN)) continue;
+        if (!mbar_wait(&tempty[0], tph ^ 1, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) break;
+        tc_fence_after();
+        for (int kb = 0; kb < KB_r; ++kb, ++ck) {
+          const int hb = ck & 1;
+          const uint32_t hph = (ck >> 1) & 1;
+          if (!mbar_wait(&hempty[hb], hph ^ 1, abort_flag, p.err, MOE_DEVERR_TIMEOUT) ||
+              !mbar_wait(&full[stage], phase, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) {
+            live = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t b0 = a0 + C::NA * C::A_BYTES;
+          const uint32_t d_hi = tmem_base + hb * BN;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t bd = sdesc_k128(b0 + kk * 32);
+            const uint32_t acc_all = (kb | kk) != 0 ? 1u : 0u;
+            umma_bf16(d_hi, sdesc_k128(a0 + kk * 32), bd, idesc, kk != 0 ? 1u : 0u);
+            umma_bf16(d_mid, sdesc_k128(a0 + C::A_BYTES + kk * 32), bd, idesc, acc_all);
+            umma_bf16(d_lo, sdesc_k128(a0 + 2 * C::A_BYTES + kk * 32), bd, idesc, acc_all);
+          }
+          umma_commit(&empty[stage]);
+          umma_commit(&hfull[hb]);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!live) break;
+        umma_commit(&tfull[0]);
+        tph ^= 1;
+      }
+    } else if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(kTileN, BN);
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
@@ -269,6 +344,10 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
             const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
             umma_bf16(d0, sdesc_k128(a0 + kk * 32), bd, idesc, accum);
             if (MODE == 0) umma_bf16(d0 + BN, sdesc_k128(a0 + C::A_BYTES + kk * 32), bd, idesc, accum);
+            if (MODE == 2) {  // x * (hi + mid + lo): every product exact, one fp32 accumulator
+              umma_bf16(d0, sdesc_k128(a0 + C::A_BYTES + kk * 32), bd, idesc, 1u);
+              umma_bf16(d0, sdesc_k128(a0 + 2 * C::A_BYTES + kk * 32), bd, idesc, 1u);
+            }
           }
           umma_commit(&empty[stage]);
           if (++stage == C::STAGES) {
@@ -349,7 +428,65 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
     const int orow = q * 32 + lane;          // output feature within the tile
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+    if (MODE == 2) {
+      // router: z = sum over k-blocks of the hi chunks (fp32, in order) + mid + lo
+      int ck = 0;
+      uint32_t tph = 0;
+      const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+      for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+        const WorkItem it = item_at(item);
+        if (!item_ok(p, it, MODE, BN)) continue;
+        float sum[BN];
+#pragma unroll
+        for (int c = 0; c < BN; ++c) sum[c] = 0.f;
+        bool live = true;
+        for (int kb = 0; kb < KB_r; ++kb, ++ck) {
+          const int hb = ck & 1;
+          if (!mbar_wait(&hfull[hb], (ck >> 1) & 1, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) {
+            live = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int c0 = 0; c0 < BN; c0 += 32) {
+            float v0[16], v1[16];
+            tmem_ld16(lane_base + hb * BN + c0, v0);
+            tmem_ld16(lane_base + hb * BN + c0 + 16, v1);
+            tmem_ld_wait();
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              sum[c0 + c] += v0[c];
+              sum[c0 + 16 + c] += v1[c];
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&hempty[hb]);
+        }
+        if (!live || !mbar_wait(&tfull[0], tph, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+          float vm[16], vl[16];
+          tmem_ld16(lane_base + 2 * BN + c0, vm);
+          tmem_ld16(lane_base + 3 * BN + c0, vl);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < 16; ++c) sum[c0 + c] += vm[c] + vl[c];
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[0]);
+        tph ^= 1;
+        const int e = it.ntile * kTileN + orow;
+        if (e < p.E) {
+#pragma unroll
+          for (int c = 0; c < BN; ++c)
+            if (c < it.nrows) p.z[static_cast<size_t>(it.row0 + c) * p.E + e] = sum[c];
+        }
+      }
+    }
+    for (int item = blockIdx.x; item < (MODE == 2 ? 0 : n_items); item += gridDim.x) {
       const WorkItem it = item_at(item);
       if (!item_ok(p, it, MODE, BN)) continue;
       const bool sh = it.e == p.E;
@@ -542,6 +679,43 @@ cudaError_t launch_mode(const GemmArgs& a, cudaStream_t s) {
   kern<<<grid, threads_for(MODE), smem, s>>>(p, tA0, tA1, tS0, tS1, tB0, tB1);
   return cudaGetLastError();
 }
+
+}  // namespace
+
+// Router logits on the tensor cores: z[T,E] = x [T,H] . (hi + mid + lo)^T with
+// the fp32 router matrix split into three bf16 terms (exact for normal values).
+cudaError_t launch_router_gemm(const moe_cfg& c, int T, const uint16_t* x, const uint16_t* w_hi,
+                               const uint16_t* w_mid, const uint16_t* w_lo, float* z,
+                               int32_t* err, cudaStream_t s) {
+  constexpr int BN = 128;
+  using C = Cfg<2, BN>;
+  GemmParams p;
+  memset(&p, 0, sizeof(p));
+  p.T = T;
+  p.K = c.K;
+  p.E = c.E;
+  p.H = c.H;
+  p.I = c.I;
+  p.Is = c.I_shared;
+  p.x = x;
+  p.z = z;
+  p.err = err;
+  p.nitems = nullptr;
+  p.max_items = cdiv(c.E, kTileN) * cdiv(T, BN);
+  CUtensorMap tA0, tA1, tS0, tB0;
+  bool ok = map_bf16(&tA0, w_hi, c.E, c.H, kTileN) && map_bf16(&tA1, w_mid, c.E, c.H, kTileN) &&
+            map_bf16(&tS0, w_lo, c.E, c.H, kTileN) && map_bf16(&tB0, x, T, c.H, BN);
+  if (!ok) return cudaErrorInvalidValue;
+  auto kern = moe_gemm<2, BN>;
+  const int smem = C::SMEM + (2 * 1024 + 3) * static_cast<int>(sizeof(int));
+  cudaError_t e = ensure_dyn_smem(reinterpret_cast<const void*>(kern), smem);
+  if (e != cudaSuccess) return e;
+  const int grid = std::max(1, std::min(num_sms(), p.max_items));
+  kern<<<grid, threads_for(2), smem, s>>>(p, tA0, tA1, tS0, tS0, tB0, tB0);
+  return cudaGetLastError();
+}
+
+namespace {
 
 template <int MODE>
 cudaError_t launch_bn(const GemmArgs& a, cudaStream_t s) {

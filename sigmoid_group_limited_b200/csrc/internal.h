@@ -42,6 +42,7 @@ struct WsLayout {
       h_s, y_slot, err, total;
   // MXFP4 routed weights only: touched-expert slots and their bf16 copies
   size_t slot_of, touched, ntouched, wq_g, wq_u, wq_d;
+  size_t wr_split;  // router matrix as three bf16 terms (batches above 32 tokens)
   int max_touched;
   int n_ptiles, bn, max_items_gu, max_items_dn;
 };
@@ -51,9 +52,12 @@ WsLayout ws_layout(const moe_cfg& c, int T);
 // Launchers (return cudaGetLastError()).
 // Routing. unc [T] / unc_n: scratch list (and its count, zeroed by the
 // caller) of tokens whose fp32 decision is re-derived from exact logits.
+// wr_split: scratch for the router matrix as three bf16 terms [3][E][H]
+// (tensor-core logits for batches above 32 tokens), or nullptr for the fp32
+// SIMT logits.
 cudaError_t launch_router(const moe_cfg& c, int T, const uint16_t* x, const float* Wr,
                           const float* bias, float* z, int32_t* idx, float* w, int32_t* unc,
-                          int32_t* unc_n, int32_t* err, cudaStream_t s);
+                          int32_t* unc_n, int32_t* err, uint16_t* wr_split, cudaStream_t s);
 
 cudaError_t launch_permute(const moe_cfg& c, int T, const int32_t* idx, int32_t* tile_hist,
                            int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv_perm,
@@ -99,6 +103,9 @@ struct GemmArgs {
 };
 
 cudaError_t launch_gemm_gateup(const GemmArgs& a, cudaStream_t s);
+cudaError_t launch_router_gemm(const moe_cfg& c, int T, const uint16_t* x, const uint16_t* w_hi,
+                               const uint16_t* w_mid, const uint16_t* w_lo, float* z,
+                               int32_t* err, cudaStream_t s);
 cudaError_t launch_gemm_down(const GemmArgs& a, cudaStream_t s);
 
 // MXFP4: list the touched experts and dequantise each once into bf16 slots.

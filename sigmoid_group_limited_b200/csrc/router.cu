@@ -11,6 +11,7 @@
 //                  renormalised to sum to 1 and scaled by 2.5.
 // Readings: the group score and the candidate ranking use the biased score;
 // the weights use the unbiased one; ties go to the lower index.
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -807,6 +808,28 @@ cudaError_t topk_dispatch(const moe_cfg& c, int T, const float* z, const float* 
   return cudaErrorInvalidValue;
 }
 
+// The fp32 router matrix as three bf16 terms, w = hi + mid + lo: hi is w
+// rounded to bf16, mid the rounded remainder, lo the rounded rest; for normal
+// values the three 8-bit significands cover all 24 bits of w, so a bf16 token
+// times each term is exact in fp32 and the tensor cores can form the fp32
+// router product.
+__global__ void __launch_bounds__(256) split_router(long long n, const float* __restrict__ w,
+                                                    uint16_t* __restrict__ hi,
+                                                    uint16_t* __restrict__ mid,
+                                                    uint16_t* __restrict__ lo) {
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const float v = w[i];
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    const float r1 = v - __bfloat162float(h);
+    const __nv_bfloat16 m = __float2bfloat16_rn(r1);
+    const float r2 = r1 - __bfloat162float(m);
+    hi[i] = __bfloat16_as_ushort(h);
+    mid[i] = __bfloat16_as_ushort(m);
+    lo[i] = __bfloat16_as_ushort(__float2bfloat16_rn(r2));
+  }
+}
+
 template <int NV>
 cudaError_t launch_refine_nv(const moe_cfg& c, int T, const uint16_t* x, const float* Wr,
                              const float* z, const float* bias, int32_t* idx, float* w, float tau,
@@ -855,11 +878,20 @@ constexpr float kCertifyMargin = 1.0f / 32768.0f;
 
 cudaError_t launch_router(const moe_cfg& c, int T, const uint16_t* x, const float* Wr,
                           const float* bias, float* z, int32_t* idx, float* w, int32_t* unc,
-                          int32_t* unc_n, int32_t* err, cudaStream_t s) {
+                          int32_t* unc_n, int32_t* err, uint16_t* wr_split, cudaStream_t s) {
   cudaError_t e;
   if (c.H > kRowRegs * 128) return cudaErrorInvalidValue;
   if (T <= kSmallT) {
     e = launch_rows<false, 4>(c, T, x, Wr, z, nullptr, nullptr, err, s);
+  } else if (wr_split != nullptr) {
+    // tensor cores: split the router matrix, then one bf16 x 3 GEMM into z
+    const long long n = static_cast<long long>(c.E) * c.H;
+    uint16_t* hi = wr_split;
+    uint16_t* mid = hi + n;
+    uint16_t* lo = mid + n;
+    split_router<<<num_sms() * 4, 256, 0, s>>>(n, Wr, hi, mid, lo);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    e = launch_router_gemm(c, T, x, hi, mid, lo, z, err, s);
   } else {
     dim3 grid(cdiv(T, kRT), cdiv(c.E, kRE));
     router_logits_tiled<<<grid, 256, 0, s>>>(T, c.H, c.E, x, Wr, z);
