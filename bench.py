@@ -191,10 +191,13 @@ STAGES = ("route", "permute", "gateup", "down", "combine")
 
 
 def kernels_per_step(cfg) -> int:
-    """Library kernels launched by one moe_layer_forward: router 4 (logits,
-    certified top-k, exact re-derivation, exact top-k), permutation 1 when
-    all T*K slots fit one 2048-entry tile else 3, grouped GEMMs 2, combine 1."""
-    return 4 + (1 if cfg.T * cfg.K <= 2048 else 3) + 2 + 1
+    """Library kernels launched by one moe_layer_forward: router 3 (logits,
+    certified top-k, exact re-derivation; the logits take 2 kernels, split and
+    tensor-core GEMM, above 32 tokens), permutation 1 when all T*K slots fit
+    one 2048-entry tile else 3, the fused expert FFN 1, combine 1; MXFP4 adds
+    2 (touched-expert list, dequantisation)."""
+    n = (3 if cfg.T <= 32 else 4) + (1 if cfg.T * cfg.K <= 2048 else 3) + 1 + 1
+    return n + (2 if cfg.wfmt == workloads.MOE_W_MXFP4 else 0)
 
 
 def measure_gpu(cfg, steps, warmup, device, rank, with_e2e=True):
@@ -241,6 +244,7 @@ def measure_gpu(cfg, steps, warmup, device, rank, with_e2e=True):
     per_step_plain = [evs[i][0].elapsed_time(evs[i][5]) for i in range(steps)]
     stage_ms = {s: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(steps))
                 for j, s in enumerate(STAGES)}
+    stage_ms["ffn"] = stage_ms.pop("gateup") + stage_ms.pop("down")
     assert sgl.moe_read_error(cfg, T, ws) == 0
 
     # the same forward captured once into a CUDA graph and replayed per step
@@ -440,11 +444,13 @@ def run_native(args, rank, world, local):
 
     def roof(cfg_, mm):
         work = algorithmic_work(cfg_, cfg_.T, mm["touched"])
-        stage = max(("gateup", "down"), key=lambda s: mm["stage_ms"][s])
-        b, f = work[stage]
-        ent = roofline_entry(b, f, mm["stage_ms"][stage] / 1e3, peaks)
-        ent.update(kernel=f"moe_gemm<{'gate/up' if stage == 'gateup' else 'down'}>",
-                   traffic=None, peak_source=f"{peaks['source']} ({'HBM copy' if ent['bound'] == 'hbm' else 'cuBLAS bf16 burst'})",
+        # the dominant kernel is the fused expert FFN (gate/up and down in one launch)
+        b = work["gateup"][0] + work["down"][0]
+        f = work["gateup"][1] + work["down"][1]
+        t_ffn = (mm["stage_ms"]["ffn"]) / 1e3
+        ent = roofline_entry(b, f, t_ffn, peaks)
+        ent.update(kernel="moe_ffn_fused (gate/up + down)", traffic=None,
+                   peak_source=f"{peaks['source']} ({'HBM copy' if ent['bound'] == 'hbm' else 'cuBLAS bf16 burst'})",
                    units_per_launch=f"{cfg_.T} tokens, {mm['touched']} routed experts + shared")
         lb, lf = work["layer"]
         t_roof = max(lb / (peaks["hbm_gbs"] * 1e9), lf / (peaks["bf16_tflops"] * 1e12))

@@ -73,6 +73,7 @@ WsLayout ws_layout(const moe_cfg& c, int T) {
   L.inv_perm = take(TK * 4);
   L.gu_start = take(static_cast<size_t>(c.E + 2) * 4);
   L.dn_start = take(static_cast<size_t>(c.E + 2) * 4);
+  L.ready = take(static_cast<size_t>(L.max_items_gu) * 4);
   L.h_r = take(TK * c.I * 2);
   L.h_s = take(static_cast<size_t>(T) * (c.I_shared > 0 ? c.I_shared : 0) * 2);
   L.y_slot = take((TK + T) * c.H * 4);
@@ -193,7 +194,7 @@ moe_status moe_permute(const moe_cfg* cfg, int32_t T, const int32_t* idx, int32_
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(at<int32_t>(ws, L.err), 0, 16, s) != cudaSuccess) return MOE_ERR_CUDA;
   return cu(launch_permute(*cfg, T, idx, at<int32_t>(ws, L.tile_hist), counts, offsets, perm,
-                           inv_perm, at<int32_t>(ws, L.err), L, nullptr, nullptr,
+                           inv_perm, at<int32_t>(ws, L.err), L, nullptr, nullptr, nullptr,
                            at<int32_t>(ws, L.nitems), s));
 }
 
@@ -227,7 +228,7 @@ moe_status moe_grouped_swiglu(const moe_cfg* cfg, int32_t T, const void* x, cons
   int32_t* gu = at<int32_t>(ws, L.gu_start);
   int32_t* dn = at<int32_t>(ws, L.dn_start);
   int32_t* nitems = at<int32_t>(ws, L.nitems);
-  cudaError_t e = launch_schedule(*cfg, T, offsets, L, gu, dn, nitems, s);
+  cudaError_t e = launch_schedule(*cfg, T, offsets, L, gu, dn, at<int32_t>(ws, L.ready), nitems, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   const int32_t* a_offsets = offsets;
   GemmArgs a;
@@ -260,13 +261,13 @@ moe_status moe_grouped_swiglu(const moe_cfg* cfg, int32_t T, const void* x, cons
   a.offsets = offsets;
   a.gu_start = gu;
   a.dn_start = dn;
+  a.ready = at<int32_t>(ws, L.ready);
   a.nitems = nitems;
   a.err = at<int32_t>(ws, L.err);
   a.bn = L.bn;
   a.max_items_gu = L.max_items_gu;
   a.max_items_dn = L.max_items_dn;
-  if ((e = launch_gemm_gateup(a, s)) != cudaSuccess) return MOE_ERR_CUDA;
-  return cu(launch_gemm_down(a, s));
+  return cu(launch_ffn_fused(a, s));
 }
 
 moe_status moe_combine(const moe_cfg* cfg, int32_t T, const void* y_slot, int32_t with_shared,
@@ -319,7 +320,8 @@ moe_status moe_layer_forward(const moe_cfg* cfg, int32_t T, const void* x, const
     return MOE_ERR_CUDA;
   rec(1);
   if ((e = launch_permute(*cfg, T, idx, at<int32_t>(ws, L.tile_hist), counts, offsets, perm,
-                          at<int32_t>(ws, L.inv_perm), err, L, gu, dn, nitems, s)) != cudaSuccess)
+                          at<int32_t>(ws, L.inv_perm), err, L, gu, dn, at<int32_t>(ws, L.ready),
+                          nitems, s)) != cudaSuccess)
     return MOE_ERR_CUDA;
   rec(2);
   const int32_t* a_offsets = offsets;
@@ -353,14 +355,14 @@ moe_status moe_layer_forward(const moe_cfg* cfg, int32_t T, const void* x, const
   a.offsets = offsets;
   a.gu_start = gu;
   a.dn_start = dn;
+  a.ready = at<int32_t>(ws, L.ready);
   a.nitems = nitems;
   a.err = err;
   a.bn = L.bn;
   a.max_items_gu = L.max_items_gu;
   a.max_items_dn = L.max_items_dn;
-  if ((e = launch_gemm_gateup(a, s)) != cudaSuccess) return MOE_ERR_CUDA;
+  if ((e = launch_ffn_fused(a, s)) != cudaSuccess) return MOE_ERR_CUDA;
   rec(3);
-  if ((e = launch_gemm_down(a, s)) != cudaSuccess) return MOE_ERR_CUDA;
   rec(4);
   if ((e = launch_combine(*cfg, T, y_slot, cfg->I_shared > 0 ? 1 : 0, static_cast<uint16_t*>(y),
                           s)) != cudaSuccess)

@@ -576,6 +576,443 @@ __global__ void __launch_bounds__(threads_for(MODE), 1)
   }
 }
 
+// ===========================================================================
+// Fused expert FFN: gate/up and down in one persistent, cooperative launch.
+// Item space: [0, Ngu) gate/up items, then [Ngu, Ngu + Ndn) down items, both
+// decoded from their per-slot prefix sums. Items are claimed dynamically: a
+// CTA's producer takes the next index from a global counter and hands it to
+// the CTA's other roles through a small shared-memory queue. Indices are
+// claimed in increasing order, so every gate/up item is claimed before any
+// down item.
+// A down item (slot e, row tile m) reads h rows written by the gate/up
+// epilogues of other CTAs: those epilogues count finished output tiles per
+// (e, m) in ready[] (stores, proxy fence, CTA barrier, threadfence, atomic);
+// the producer waits with an acquire load until all of the slot's output tiles
+// are in. Gate/up items never wait, and the cooperative launch keeps every CTA
+// resident, so every waited-for item is owned by a running CTA that does it
+// first. Waits are bounded like every other wait here.
+// ===========================================================================
+constexpr int kFusedThreads = 320;
+
+struct FusedParams {
+  GemmParams g;
+  const int32_t* gu_start;  // [E+2]
+  const int32_t* dn_start;  // [E+2]
+  int32_t* ready;           // [max_gu] finished gate/up output tiles per (slot, row tile)
+  int32_t* counter;         // next unclaimed item (zeroed by the schedule builder)
+  int max_gu, max_dn;
+};
+constexpr int kQueue = 4;  // items a CTA's producer may run ahead of its slowest role
+
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+__device__ __forceinline__ int ld_acquire(const int32_t* a) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
+  return v;
+}
+
+// Bounded wait until *addr >= need (acquire). Same abort protocol as mbar_wait.
+__device__ __forceinline__ bool wait_count(const int32_t* addr, int need, volatile int* abort_flag,
+                                           int* err) {
+  const long long t0 = clock64();
+  while (ld_acquire(addr) < need) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitLimitCycles) {
+      *abort_flag = 1;
+      atomicExch(err, MOE_DEVERR_TIMEOUT);
+      return false;
+    }
+    __nanosleep(100);
+  }
+  return true;
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kFusedThreads, 1)
+    moe_ffn_fused(const __grid_constant__ FusedParams fp, const __grid_constant__ CUtensorMap tWg,
+                  const __grid_constant__ CUtensorMap tWu, const __grid_constant__ CUtensorMap tWgS,
+                  const __grid_constant__ CUtensorMap tWuS, const __grid_constant__ CUtensorMap tWd,
+                  const __grid_constant__ CUtensorMap tWdS, const __grid_constant__ CUtensorMap tH,
+                  const __grid_constant__ CUtensorMap tHs) {
+  using C = Cfg<0, BN>;  // stage = gate + up tiles + token tile (down uses one A tile)
+  const GemmParams& p = fp.g;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* tfull = empty + C::STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* qfull = tempty + 2;   // item queue: producer -> the other roles
+  uint64_t* qempty = qfull + kQueue;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qempty + kQueue);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* qitem = reinterpret_cast<volatile int*>(tmem_slot + 2);  // [kQueue]
+  int* meta_j = reinterpret_cast<int*>(smem + C::STAGES * C::STAGE_BYTES + 256);
+  float* meta_w = reinterpret_cast<float*>(meta_j + BN);
+  int* s_gu = reinterpret_cast<int*>(meta_w + BN);  // [E+2]
+  int* s_dn = s_gu + (p.E + 2);                      // [E+2]
+  int* s_off = s_dn + (p.E + 2);                     // [E+1]
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1 + kGatherWarps);  // weight TMA + one arrival per gatherer warp
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);
+    }
+    for (int q = 0; q < kQueue; ++q) {
+      mbar_init(&qfull[q], 1);
+      mbar_init(&qempty[q], 1 + 4 + kGatherWarps);  // MMA lane, epilogue and gatherer warps
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tWg);
+    prefetch_tmap(&tWd);
+    prefetch_tmap(&tH);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  for (int i = tid; i < p.E + 2; i += blockDim.x) {
+    s_gu[i] = fp.gu_start[i];
+    s_dn[i] = fp.dn_start[i];
+  }
+  for (int i = tid; i < p.E + 1; i += blockDim.x) s_off[i] = p.offsets[i];
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int nslots = p.E + (p.has_shared ? 1 : 0);
+  const int n_gu = min(p.nitems[0], fp.max_gu);
+  const int n_dn = min(p.nitems[1], fp.max_dn);
+  const int n_all = n_gu + n_dn;
+  // item i -> (is gate/up, work item)
+  auto item_at = [&](int i, bool& gu) {
+    gu = i < n_gu;
+    return gu ? decode_item(i, s_gu, s_off, nslots, p.E, p.T, BN, 0, 0, 0)
+              : decode_item(i - n_gu, s_dn, s_off, nslots, p.E, p.T, BN, 1, 0, 0);
+  };
+  // ready[] index of (slot, row tile) of an item
+  auto ready_idx = [&](const WorkItem& it) {
+    const int r0 = it.e == p.E ? 0 : s_off[it.e];
+    return s_gu[it.e] + (it.row0 - r0) / BN;
+  };
+  // next item index from the queue (every role reads every entry once);
+  // -1 ends the walk. One arrival per warp (lane 0) frees the entry.
+  // whole_warp: every lane of the calling warp takes part (else lane 0 alone)
+  auto next_item = [&](int n, int& item, bool whole_warp) -> bool {
+    const int q = n % kQueue;
+    if (!mbar_wait(&qfull[q], (n / kQueue) & 1, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) return false;
+    item = qitem[q];
+    if (whole_warp) __syncwarp();
+    if (lane == 0) mbar_arrive(&qempty[q]);
+    return item >= 0;
+  };
+  const int KB_gu = p.H / 64;
+  const int KB_dn_r = p.I / 64, KB_dn_s = p.Is / 64;
+  auto nkb_of = [&](bool gu, bool sh) { return gu ? KB_gu : (sh ? KB_dn_s : KB_dn_r); };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ weight / h TMA
+    const uint64_t pol_w = policy_evict_first();
+    const uint64_t pol_h = policy_evict_last();
+    int stage = 0;
+    uint32_t phase = 0;
+    bool live = true;
+    for (int n = 0; live; ++n) {
+      // claim the next item (dynamic: whoever is free takes it) and queue it
+      int item = -1;
+      if (lane == 0) {
+        const int q = n % kQueue;
+        if (!mbar_wait(&qempty[q], ((n / kQueue) & 1) ^ 1, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) {
+          live = false;
+        } else {
+          item = atomicAdd(fp.counter, 1);
+          if (item >= n_all) item = -1;
+          qitem[q] = item;
+          mbar_arrive(&qfull[q]);
+        }
+      }
+      item = __shfl_sync(0xffffffffu, item, 0);
+      live = __shfl_sync(0xffffffffu, live ? 1 : 0, 0) != 0;
+      if (!live || item < 0) break;
+      bool gu;
+      const WorkItem it = item_at(item, gu);
+      if (!item_ok(p, it, gu ? 0 : 1, BN)) {
+        if (lane == 0) atomicExch(p.err, MOE_DEVERR_SCHEDULE);
+        continue;
+      }
+      const bool sh = it.e == p.E;
+      if (lane == 0) {
+        if (!gu) {
+          // every gate/up output tile of this (slot, row tile) must be in h
+          const int need = cdiv_dev(sh ? p.Is : p.I, kTileN);
+          if (!wait_count(fp.ready + ready_idx(it), need, abort_flag, p.err)) live = false;
+          fence_proxy_async_global();
+        }
+        const int wblk = p.wslot ? p.wslot[it.e] : it.e;
+        const int nkb = nkb_of(gu, sh);
+        for (int kb = 0; kb < nkb && live; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) {
+            live = false;
+            break;
+          }
+          uint8_t* sA = smem + stage * C::STAGE_BYTES;
+          uint8_t* sB = sA + C::NA * C::A_BYTES;
+          if (gu) {
+            const int arow = sh ? it.ntile * kTileN : wblk * p.I + it.ntile * kTileN;
+            mbar_arrive_expect_tx(&full[stage], 2 * C::A_BYTES);
+            tma_load_2d(sA, sh ? &tWgS : &tWg, &full[stage], kb * 64, arow, pol_w);
+            tma_load_2d(sA + C::A_BYTES, sh ? &tWuS : &tWu, &full[stage], kb * 64, arow, pol_w);
+          } else {
+            const int arow = sh ? it.ntile * kTileN : wblk * p.H + it.ntile * kTileN;
+            mbar_arrive_expect_tx(&full[stage], C::A_BYTES + C::B_BYTES);
+            tma_load_2d(sA, sh ? &tWdS : &tWd, &full[stage], kb * 64, arow, pol_w);
+            tma_load_2d(sB, sh ? &tHs : &tH, &full[stage], kb * 64, it.row0, pol_h);
+          }
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      live = __shfl_sync(0xffffffffu, live ? 1 : 0, 0) != 0;
+      __syncwarp();
+    }
+    if (lane == 0 && live) {
+      for (int i = 0; i < C::STAGES; ++i) {
+        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) break;
+        if (++stage == C::STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(kTileN, BN);
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool live = true;
+      for (int n = 0; live; ++n) {
+        int item;
+        if (!next_item(n, item, false)) break;
+        bool gu;
+        const WorkItem it = item_at(item, gu);
+        if (!item_ok(p, it, gu ? 0 : 1, BN)) continue;
+        const int nkb = nkb_of(gu, it.e == p.E);
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) break;
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + acc * C::ACC_COLS;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) {
+            live = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t b0 = a0 + C::NA * C::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t bd = sdesc_k128(b0 + kk * 32);
+            const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
+            umma_bf16(d0, sdesc_k128(a0 + kk * 32), bd, idesc, accum);
+            if (gu) umma_bf16(d0 + BN, sdesc_k128(a0 + C::A_BYTES + kk * 32), bd, idesc, accum);
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!live) break;
+        umma_commit(&tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1;
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 6) {
+    // ------------------------------------------------------------ token gatherers
+    // gate/up items: copy the routed token rows into the swizzled stage layout
+    // (as in the separate gate/up kernel); down items: nothing to copy, but the
+    // stage sequence and the full-barrier arrivals stay the same (an empty
+    // copy group completes at once).
+    constexpr int kRowsPerThread = BN / 16;
+    constexpr int kLag = 2;
+    const int g = tid - 6 * 32;
+    const int chunk = g & 7, rbase = g >> 3;
+    const uint64_t pol_x = policy_evict_last();
+    int stage = 0;
+    uint32_t phase = 0;
+    int pend0 = -1, pend1 = -1;
+    bool live = true;
+    for (int n = 0; live; ++n) {
+      int item;
+      if (!next_item(n, item, true)) break;
+      bool gu;
+      const WorkItem it = item_at(item, gu);
+      if (!item_ok(p, it, gu ? 0 : 1, BN)) continue;
+      const bool sh = it.e == p.E;
+      const int nkb = nkb_of(gu, sh);
+      const uint16_t* src[kRowsPerThread];
+#pragma unroll
+      for (int i = 0; i < kRowsPerThread; ++i) {
+        const int row = it.row0 + min(rbase + 16 * i, it.nrows - 1);
+        int t = 0;
+        if (gu) t = sh ? row : p.perm[row] / p.K;
+        t = min(max(t, 0), p.T - 1);
+        src[i] = p.x + static_cast<size_t>(t) * p.H + chunk * 8;
+      }
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) {
+          live = false;
+          break;
+        }
+        if (gu) {
+          uint8_t* sB = smem + stage * C::STAGE_BYTES + C::NA * C::A_BYTES;
+#pragma unroll
+          for (int i = 0; i < kRowsPerThread; ++i) {
+            const int r = rbase + 16 * i;
+            cp_async16(sB + r * 128 + ((chunk ^ (r & 7)) << 4), src[i] + kb * 64, pol_x);
+          }
+        }
+        cp_async_commit();
+        if (pend0 >= 0) {
+          cp_async_wait<kLag>();      // this lane's copies for stage pend0 have landed
+          fence_proxy_async_smem();   // ... and are visible to the tensor cores
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&full[pend0]);
+        }
+        pend0 = pend1;
+        pend1 = stage;
+        if (++stage == C::STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+    cp_async_wait<0>();
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (live && lane == 0) {
+      if (pend0 >= 0) mbar_arrive(&full[pend0]);
+      if (pend1 >= 0) mbar_arrive(&full[pend1]);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    const int orow = q * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int n = 0;; ++n) {
+      int item;
+      if (!next_item(n, item, true)) break;
+      bool gu;
+      const WorkItem it = item_at(item, gu);
+      if (!item_ok(p, it, gu ? 0 : 1, BN)) continue;
+      const bool sh = it.e == p.E;
+      if (!gu) {
+        epilogue_bar();
+        if (orow < BN) {
+          int j = -1;
+          float wt = 0.f;
+          if (orow < it.nrows) {
+            const int row = it.row0 + orow;
+            if (sh) {
+              j = p.T * p.K + row;
+              wt = 1.0f;
+            } else {
+              j = p.perm[row];
+              if (j < 0 || j >= p.T * p.K) {
+                atomicExch(p.err, MOE_DEVERR_SCHEDULE);
+                j = -1;
+              } else {
+                wt = p.w[j];
+              }
+            }
+          }
+          meta_j[orow] = j;
+          meta_w[orow] = wt;
+        }
+        epilogue_bar();
+      }
+      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * C::ACC_COLS;
+      const int nfeat = it.ntile * kTileN + orow;
+      if (gu) {
+        const int ncols = sh ? p.Is : p.I;
+        const bool ok = nfeat < ncols;
+        const float L = sh ? p.lim_s : p.lim_r;
+        uint16_t* hout = sh ? p.h_s : p.h_r;
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+          float gv[16], uv[16];
+          tmem_ld16(taddr + c0, gv);
+          tmem_ld16(taddr + BN + c0, uv);
+          tmem_ld_wait();
+          if (ok) {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const int r = c0 + c;
+              if (r < it.nrows) {
+                const float gg = clampL(gv[c], L), uu = clampL(uv[c], L);
+                hout[static_cast<size_t>(it.row0 + r) * ncols + nfeat] =
+                    f2bf((gg / (1.0f + expf(-gg))) * uu);
+              }
+            }
+          }
+        }
+      } else {
+        const bool ok = nfeat < p.H;
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+          float ov[16];
+          tmem_ld16(taddr + c0, ov);
+          tmem_ld_wait();
+          if (ok) {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const int j = meta_j[c0 + c];
+              if (j >= 0) p.y_slot[static_cast<size_t>(j) * p.H + nfeat] = meta_w[c0 + c] * ov[c];
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1;
+      if (gu) {
+        // publish this output tile of h: stores -> async proxy -> CTA -> GPU
+        fence_proxy_async_global();
+        epilogue_bar();
+        if (warp == 2 && lane == 0) {
+          __threadfence();
+          atomicAdd(fp.ready + ready_idx(it), 1);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
 // ------------------------------------------------------------------ host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -717,6 +1154,57 @@ cudaError_t launch_router_gemm(const moe_cfg& c, int T, const uint16_t* x, const
 
 namespace {
 
+template <int BN>
+cudaError_t launch_fused_bn(const GemmArgs& a, cudaStream_t s) {
+  using C = Cfg<0, BN>;
+  const moe_cfg& c = *a.cfg;
+  FusedParams fp;
+  memset(&fp, 0, sizeof(fp));
+  fp.g = make_params(a, 0);
+  fp.gu_start = a.gu_start;
+  fp.dn_start = a.dn_start;
+  fp.ready = a.ready;
+  fp.counter = const_cast<int32_t*>(a.nitems) + 2;
+  fp.max_gu = a.max_items_gu;
+  fp.max_dn = a.max_items_dn;
+  const int T = a.T, TK = a.T * c.K;
+  CUtensorMap tWg, tWu, tWgS, tWuS, tWd, tWdS, tH, tHs;
+  bool ok = map_bf16(&tWg, a.Wg, static_cast<uint64_t>(a.wrows) * c.I, c.H, kTileN) &&
+            map_bf16(&tWu, a.Wu, static_cast<uint64_t>(a.wrows) * c.I, c.H, kTileN) &&
+            map_bf16(&tWd, a.Wd, static_cast<uint64_t>(a.wrows) * c.H, c.I, kTileN) &&
+            map_bf16(&tH, a.h_r, TK, c.I, BN);
+  if (fp.g.has_shared) {
+    ok = ok && map_bf16(&tWgS, a.W->Wg_s, c.I_shared, c.H, kTileN) &&
+         map_bf16(&tWuS, a.W->Wu_s, c.I_shared, c.H, kTileN) &&
+         map_bf16(&tWdS, a.W->Wd_s, c.H, c.I_shared, kTileN) &&
+         map_bf16(&tHs, a.h_s, T, c.I_shared, BN);
+  } else {
+    tWgS = tWg;
+    tWuS = tWu;
+    tWdS = tWd;
+    tHs = tH;
+  }
+  if (!ok) return cudaErrorInvalidValue;
+  auto kern = moe_ffn_fused<BN>;
+  const int smem_max = C::SMEM + (3 * 1024 + 5) * static_cast<int>(sizeof(int));
+  const int smem = C::SMEM + (3 * c.E + 5) * static_cast<int>(sizeof(int));
+  cudaError_t e = ensure_dyn_smem(reinterpret_cast<const void*>(kern), smem_max);
+  if (e != cudaSuccess) return e;
+  // one CTA per SM, all resident at once (down items wait on other CTAs)
+  cudaLaunchConfig_t lc;
+  memset(&lc, 0, sizeof(lc));
+  lc.gridDim = dim3(num_sms());
+  lc.blockDim = dim3(kFusedThreads);
+  lc.dynamicSmemBytes = smem;
+  lc.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  return cudaLaunchKernelEx(&lc, kern, fp, tWg, tWu, tWgS, tWuS, tWd, tWdS, tH, tHs);
+}
+
 template <int MODE>
 cudaError_t launch_bn(const GemmArgs& a, cudaStream_t s) {
   switch (a.bn) {
@@ -731,6 +1219,15 @@ cudaError_t launch_bn(const GemmArgs& a, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_gemm_gateup(const GemmArgs& a, cudaStream_t s) { return launch_bn<0>(a, s); }
+cudaError_t launch_ffn_fused(const GemmArgs& a, cudaStream_t s) {
+  switch (a.bn) {
+    case 16: return launch_fused_bn<16>(a, s);
+    case 32: return launch_fused_bn<32>(a, s);
+    case 64: return launch_fused_bn<64>(a, s);
+    case 128: return launch_fused_bn<128>(a, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
 cudaError_t launch_gemm_down(const GemmArgs& a, cudaStream_t s) { return launch_bn<1>(a, s); }
 
 }  // namespace sgl

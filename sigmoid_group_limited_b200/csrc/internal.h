@@ -38,7 +38,7 @@ inline int cdiv(long long a, long long b) { return static_cast<int>((a + b - 1) 
 __host__ __device__ inline int cdiv_dev(int a, int b) { return (a + b - 1) / b; }
 
 struct WsLayout {
-  size_t z, unc, tile_hist, idx, w, counts, offsets, perm, inv_perm, gu_start, dn_start, nitems, h_r,
+  size_t z, unc, tile_hist, idx, w, counts, offsets, perm, inv_perm, gu_start, dn_start, ready, nitems, h_r,
       h_s, y_slot, err, total;
   // MXFP4 routed weights only: touched-expert slots and their bf16 copies
   size_t slot_of, touched, ntouched, wq_g, wq_u, wq_d;
@@ -62,7 +62,7 @@ cudaError_t launch_router(const moe_cfg& c, int T, const uint16_t* x, const floa
 cudaError_t launch_permute(const moe_cfg& c, int T, const int32_t* idx, int32_t* tile_hist,
                            int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv_perm,
                            int32_t* err, const WsLayout& L, int32_t* gu_start, int32_t* dn_start,
-                           int32_t* nitems, cudaStream_t s);
+                           int32_t* ready, int32_t* nitems, cudaStream_t s);
 
 // Allocation-free permutation (moe_permute_static): scratch in a fixed
 // device array; needs T*K <= kStaticMaxSlots and E <= kStaticMaxExperts.
@@ -74,8 +74,8 @@ cudaError_t launch_permute_static(const moe_cfg& c, int T, const int32_t* idx, i
                                   cudaStream_t s);
 
 cudaError_t launch_schedule(const moe_cfg& c, int T, const int32_t* offsets, const WsLayout& L,
-                            int32_t* gu_start, int32_t* dn_start, int32_t* nitems,
-                            cudaStream_t s);
+                            int32_t* gu_start, int32_t* dn_start, int32_t* ready,
+                            int32_t* nitems, cudaStream_t s);
 
 struct GemmArgs {
   const moe_cfg* cfg;
@@ -95,6 +95,7 @@ struct GemmArgs {
   const int32_t* offsets;   // [E+1] routed row offsets
   const int32_t* gu_start;  // [E+2] item prefix sums, gate/up
   const int32_t* dn_start;  // [E+2] item prefix sums, down
+  int32_t* ready;           // [max_items_gu] per (slot, row tile) finished gate/up tiles
   const int32_t* nitems;
   int32_t* err;
   int bn;
@@ -103,6 +104,9 @@ struct GemmArgs {
 };
 
 cudaError_t launch_gemm_gateup(const GemmArgs& a, cudaStream_t s);
+// gate/up and down in one cooperative persistent launch (counters in a.ready,
+// zeroed by the schedule builder)
+cudaError_t launch_ffn_fused(const GemmArgs& a, cudaStream_t s);
 cudaError_t launch_router_gemm(const moe_cfg& c, int T, const uint16_t* x, const uint16_t* w_hi,
                                const uint16_t* w_mid, const uint16_t* w_lo, float* z,
                                int32_t* err, cudaStream_t s);

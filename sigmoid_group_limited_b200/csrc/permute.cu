@@ -83,6 +83,7 @@ struct SchedArgs {
   int T, K, E, H, I, Is, has_shared, bn;
   int32_t* gu_start;  // [E+2] first gate/up work item of slot e (e == E: shared expert)
   int32_t* dn_start;  // [E+2] first down work item of slot e
+  int32_t* ready;     // nullable: [gate/up items] zeroed for the fused FFN's row-tile counters
   int32_t* nitems;    // [2] totals
 };
 
@@ -119,9 +120,23 @@ __device__ void build_schedule(const SchedArgs& a, const int* cnt, int* scratch)
       a.dn_start[e] = real ? base_dn + (q ? ndn[0] : 0) : tot_dn;
     }
   }
+  if (a.ready) {
+    // one counter per (slot, row tile): the slot's first nm gate/up item indices
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int e = 2 * threadIdx.x + q;
+      if (e < nslots) {
+        const int ntg = e == a.E ? nt_gu_s : nt_gu_r;
+        const int nm = ntg > 0 ? (q ? ngu[1] : ngu[0]) / ntg : 0;
+        const int b0 = base_gu + (q ? ngu[0] : 0);
+        for (int m = 0; m < nm; ++m) a.ready[b0 + m] = 0;
+      }
+    }
+  }
   if (threadIdx.x == 0) {
     a.nitems[0] = tot_gu;
     a.nitems[1] = tot_dn;
+    a.nitems[2] = 0;  // the fused FFN's item counter
   }
 }
 
@@ -337,7 +352,7 @@ __global__ void __launch_bounds__(1024) perm_single(int TK, int E, const int32_t
 }
 
 SchedArgs make_sched(const moe_cfg& c, int T, const WsLayout& L, int32_t* gu_start,
-                     int32_t* dn_start, int32_t* nitems) {
+                     int32_t* dn_start, int32_t* ready, int32_t* nitems) {
   SchedArgs a;
   a.T = T;
   a.K = c.K;
@@ -349,6 +364,7 @@ SchedArgs make_sched(const moe_cfg& c, int T, const WsLayout& L, int32_t* gu_sta
   a.bn = L.bn;
   a.gu_start = gu_start;
   a.dn_start = dn_start;
+  a.ready = ready;
   a.nitems = nitems;
   return a;
 }
@@ -358,10 +374,10 @@ SchedArgs make_sched(const moe_cfg& c, int T, const WsLayout& L, int32_t* gu_sta
 cudaError_t launch_permute(const moe_cfg& c, int T, const int32_t* idx, int32_t* tile_cnt,
                            int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv_perm,
                            int32_t* err, const WsLayout& L, int32_t* gu_start,
-                           int32_t* dn_start, int32_t* nitems, cudaStream_t s) {
+                           int32_t* dn_start, int32_t* ready, int32_t* nitems, cudaStream_t s) {
   const int TK = T * c.K;
   const int np = L.n_ptiles;
-  SchedArgs sa = make_sched(c, T, L, gu_start, dn_start, nitems);
+  SchedArgs sa = make_sched(c, T, L, gu_start, dn_start, ready, nitems);
   if (np == 1) {
     const int smem = 32 * c.E * static_cast<int>(sizeof(int));
     cudaError_t e = ensure_dyn_smem(reinterpret_cast<const void*>(perm_single),
@@ -425,6 +441,7 @@ cudaError_t launch_permute_static(const moe_cfg& c, int T, const int32_t* idx, i
   perm_hist<<<np, 256, 0, s>>>(TK, c.E, np, idx, tile_cnt, err);
   SchedArgs sa{};
   sa.nitems = base + 1;
+  sa.ready = nullptr;
   perm_scan<<<1, 1024, 0, s>>>(c.E, np, tile_cnt, tile_base, counts, offsets, sa, 0);
   perm_scatter<<<np, kScatterWarps * 32, 0, s>>>(TK, c.E, np, idx, tile_base, perm, inv_perm,
                                                  err);
@@ -432,9 +449,9 @@ cudaError_t launch_permute_static(const moe_cfg& c, int T, const int32_t* idx, i
 }
 
 cudaError_t launch_schedule(const moe_cfg& c, int T, const int32_t* offsets, const WsLayout& L,
-                            int32_t* gu_start, int32_t* dn_start, int32_t* nitems,
-                            cudaStream_t s) {
-  SchedArgs sa = make_sched(c, T, L, gu_start, dn_start, nitems);
+                            int32_t* gu_start, int32_t* dn_start, int32_t* ready,
+                            int32_t* nitems, cudaStream_t s) {
+  SchedArgs sa = make_sched(c, T, L, gu_start, dn_start, ready, nitems);
   schedule_only<<<1, 1024, 0, s>>>(offsets, sa);
   return cudaGetLastError();
 }
