@@ -449,7 +449,7 @@ def run_native(args, rank, world, local):
         f = work["gateup"][1] + work["down"][1]
         t_ffn = (mm["stage_ms"]["ffn"]) / 1e3
         ent = roofline_entry(b, f, t_ffn, peaks)
-        ent.update(kernel="moe_ffn_fused (gate/up + down)", traffic=None,
+        ent.update(kernel="moe_ffn (gate/up + down)", traffic=None,
                    peak_source=f"{peaks['source']} ({'HBM copy' if ent['bound'] == 'hbm' else 'cuBLAS bf16 burst'})",
                    units_per_launch=f"{cfg_.T} tokens, {mm['touched']} routed experts + shared")
         lb, lf = work["layer"]

@@ -48,7 +48,7 @@ WsLayout ws_layout(const moe_cfg& c, int T) {
   const size_t TK = static_cast<size_t>(T) * c.K;
   L.n_ptiles = cdiv(static_cast<long long>(TK), kPermTile);
   L.bn = choose_bn(T, c.K, c.E);
-  const int rt_gu = cdiv(c.I, kTileN), st_gu = cdiv(c.I_shared, kTileN), nt_dn = cdiv(c.H, kTileN);
+  const int rt_gu = cdiv(c.I, kTileN), st_gu = cdiv(c.I_shared, kTileN), nt_dn = cdiv(c.H, kDownTile);
   const long long mt_r = cdiv(static_cast<long long>(TK), L.bn) +
                          (static_cast<long long>(TK) < c.E ? static_cast<long long>(TK) : c.E);
   const long long mt_s = c.I_shared > 0 ? cdiv(T, L.bn) : 0;
@@ -101,7 +101,7 @@ namespace {
 bool cfg_ok(const moe_cfg* c) {
   if (c == nullptr) return false;
   if (c->H <= 0 || c->H % 64 != 0 || c->H > 16384) return false;
-  if (c->E <= 0 || c->E % 32 != 0 || c->E > 1024) return false;
+  if (c->E <= 0 || c->E % 32 != 0 || c->E > kMaxExpertsCfg) return false;
   if (c->n_group <= 0 || c->n_group > 32 || c->E % c->n_group != 0) return false;
   if (c->topk_group <= 0 || c->topk_group > c->n_group) return false;
   if (c->K <= 0 || c->K > 32 || c->K > c->topk_group * (c->E / c->n_group)) return false;
@@ -267,7 +267,7 @@ moe_status moe_grouped_swiglu(const moe_cfg* cfg, int32_t T, const void* x, cons
   a.bn = L.bn;
   a.max_items_gu = L.max_items_gu;
   a.max_items_dn = L.max_items_dn;
-  return cu(launch_ffn_fused(a, s));
+  return cu(launch_ffn(a, s));
 }
 
 moe_status moe_combine(const moe_cfg* cfg, int32_t T, const void* y_slot, int32_t with_shared,
@@ -361,7 +361,7 @@ moe_status moe_layer_forward(const moe_cfg* cfg, int32_t T, const void* x, const
   a.bn = L.bn;
   a.max_items_gu = L.max_items_gu;
   a.max_items_dn = L.max_items_dn;
-  if ((e = launch_ffn_fused(a, s)) != cudaSuccess) return MOE_ERR_CUDA;
+  if ((e = launch_ffn(a, s)) != cudaSuccess) return MOE_ERR_CUDA;
   rec(3);
   rec(4);
   if ((e = launch_combine(*cfg, T, y_slot, cfg->I_shared > 0 ? 1 : 0, static_cast<uint16_t*>(y),

@@ -1,6 +1,7 @@
 // internal.h - host-side declarations shared by the library's translation
 // units: workspace layout, GEMM work items and kernel launchers.
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -9,9 +10,10 @@
 
 namespace sgl {
 
-// One GEMM work item: expert `e` (e == E: the shared expert), rows
+// One expert-FFN work item: expert `e` (e == E: the shared expert), rows
 // [row0, row0 + nrows) of that expert's row range, output tile `ntile`
-// (128 output features). Rows are positions in the permuted row space for
+// (kTileN intermediate features for gate/up, kDownTile hidden features for
+// down). Rows are positions in the permuted row space for
 // routed experts (offsets[e] + m*BN) and token ids for the shared expert.
 // Items are not stored: the GEMM kernels decode an item index from the
 // per-slot item prefix sums (gu_start / dn_start) and the row offsets.
@@ -24,6 +26,8 @@ struct WorkItem {
 
 constexpr int kPermTile = 2048;   // (token, slot) entries per permutation tile
 constexpr int kTileN = 128;       // output features per GEMM tile (MMA M)
+constexpr int kDownTile = 256;    // hidden features per down item (two MMA tiles)
+constexpr int kMaxExpertsCfg = 1024;  // largest E a configuration may have
 
 // Token-tile width (MMA N) for a batch: small for decode, wide for prefill.
 inline int choose_bn(int T, int K, int E) {
@@ -103,14 +107,12 @@ struct GemmArgs {
   int max_items_dn;
 };
 
-cudaError_t launch_gemm_gateup(const GemmArgs& a, cudaStream_t s);
-// gate/up and down in one cooperative persistent launch (counters in a.ready,
-// zeroed by the schedule builder)
-cudaError_t launch_ffn_fused(const GemmArgs& a, cudaStream_t s);
+// The expert FFN: gate/up and down in one cooperative persistent launch
+// (counters in a.ready and a.nitems[2], zeroed by the schedule builder).
+cudaError_t launch_ffn(const GemmArgs& a, cudaStream_t s);
 cudaError_t launch_router_gemm(const moe_cfg& c, int T, const uint16_t* x, const uint16_t* w_hi,
                                const uint16_t* w_mid, const uint16_t* w_lo, float* z,
                                int32_t* err, cudaStream_t s);
-cudaError_t launch_gemm_down(const GemmArgs& a, cudaStream_t s);
 
 // MXFP4: list the touched experts and dequantise each once into bf16 slots.
 cudaError_t launch_mxfp4_expand(const moe_cfg& c, const int32_t* offsets, const moe_weights* W,
@@ -121,6 +123,10 @@ cudaError_t launch_combine(const moe_cfg& c, int T, const float* y_slot, int wit
                            uint16_t* y, cudaStream_t s);
 
 int num_sms();
+
+// Tensor map of a bf16 row-major [rows, cols] matrix for TMA: box of
+// box_rows x 64 columns, 128-byte swizzle. False if it cannot be encoded.
+bool map_bf16(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows);
 
 // Raises `func`'s dynamic shared-memory limit to at least `bytes`, once per
 // device (later calls with a size already granted cost a table lookup).

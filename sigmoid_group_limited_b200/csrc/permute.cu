@@ -95,7 +95,7 @@ struct SchedArgs {
 __device__ void build_schedule(const SchedArgs& a, const int* cnt, int* scratch) {
   const int nslots = a.E + (a.has_shared ? 1 : 0);
   const int nt_gu_r = cdiv_dev(a.I, kTileN), nt_gu_s = cdiv_dev(a.Is, kTileN);
-  const int nt_dn = cdiv_dev(a.H, kTileN);
+  const int nt_dn = cdiv_dev(a.H, kDownTile);
   int ngu[2] = {0, 0}, ndn[2] = {0, 0};
 #pragma unroll
   for (int q = 0; q < 2; ++q) {
