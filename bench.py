@@ -381,7 +381,20 @@ def parse():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--oracle-tokens", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override the workload's T (small profiling cases)")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="override the workload's E (small profiling cases; E %% n_group == 0)")
     return ap.parse_args()
+
+
+def workload_cfg(args):
+    cfg = workloads.CONFIGS[args.workload]
+    if args.tokens > 0:
+        cfg = cfg.with_(T=args.tokens)
+    if args.experts > 0:
+        cfg = cfg.with_(E=args.experts)
+    return cfg
 
 
 def config_block(cfg, world):
@@ -396,7 +409,7 @@ def config_block(cfg, world):
 
 
 def run_reference(args, rank, world):
-    cfg = workloads.CONFIGS[args.workload]
+    cfg = workload_cfg(args)
     if rank != 0:
         return
     import torch
@@ -429,7 +442,7 @@ def run_native(args, rank, world, local):
     device = f"cuda:{local}"
     torch.cuda.set_device(device)
     peaks = load_peaks()
-    cfg = workloads.CONFIGS[args.workload]
+    cfg = workload_cfg(args)
     with ClockSampler(local) as clk:
         m = measure_gpu(cfg, args.steps, args.warmup, device, rank)
         also = None

@@ -60,7 +60,7 @@ WsLayout ws_layout(const moe_cfg& c, int T) {
     o = align_up(o + bytes, 256);
     return at;
   };
-  L.err = take(16);
+  L.err = take(kCtrlBytes);
   L.nitems = take(16);
   L.z = take(static_cast<size_t>(T) * c.E * 4);
   L.unc = take(static_cast<size_t>(T) * 4);
@@ -78,6 +78,7 @@ WsLayout ws_layout(const moe_cfg& c, int T) {
   L.h_s = take(static_cast<size_t>(T) * (c.I_shared > 0 ? c.I_shared : 0) * 2);
   L.y_slot = take((TK + T) * c.H * 4);
   L.wr_split = T > 32 ? take(static_cast<size_t>(3) * c.E * c.H * 2) : 0;
+  L.zpart = T <= 32 ? take(static_cast<size_t>(cdiv(c.H, 128)) * T * c.E * 4) : 0;
   if (c.wfmt == MOE_W_MXFP4) {
     L.max_touched = static_cast<int>(TK < static_cast<size_t>(c.E) ? TK : c.E);
     const size_t mat = static_cast<size_t>(L.max_touched) * c.I * c.H * 2;
@@ -173,11 +174,12 @@ moe_status moe_route(const moe_cfg* cfg, int32_t T, const void* x, const float* 
   moe_status st = device_ok();
   if (st != MOE_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(at<int32_t>(ws, L.err), 0, 16, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemsetAsync(at<int32_t>(ws, L.err), 0, kCtrlBytes, s) != cudaSuccess) return MOE_ERR_CUDA;
   return cu(launch_router(*cfg, T, static_cast<const uint16_t*>(x), Wr, bias, at<float>(ws, L.z),
                           idx, w, at<int32_t>(ws, L.unc), at<int32_t>(ws, L.err) + 1,
                           at<int32_t>(ws, L.err), T > 32 ? at<uint16_t>(ws, L.wr_split) : nullptr,
-                          s));
+                          T <= 32 ? at<float>(ws, L.zpart) : nullptr,
+                          at<int32_t>(ws, L.err) + kCtrlSplitCnt, s));
 }
 
 moe_status moe_permute(const moe_cfg* cfg, int32_t T, const int32_t* idx, int32_t* counts,
@@ -313,10 +315,12 @@ moe_status moe_layer_forward(const moe_cfg* cfg, int32_t T, const void* x, const
   float* y_slot = at<float>(ws, L.y_slot);
   cudaError_t e;
   rec(0);
-  if (cudaMemsetAsync(err, 0, 16, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemsetAsync(err, 0, kCtrlBytes, s) != cudaSuccess) return MOE_ERR_CUDA;
   if ((e = launch_router(*cfg, T, static_cast<const uint16_t*>(x), Wr, bias, at<float>(ws, L.z),
                          idx, w, at<int32_t>(ws, L.unc), err + 1, err,
-                         T > 32 ? at<uint16_t>(ws, L.wr_split) : nullptr, s)) != cudaSuccess)
+                         T > 32 ? at<uint16_t>(ws, L.wr_split) : nullptr,
+                         T <= 32 ? at<float>(ws, L.zpart) : nullptr, err + kCtrlSplitCnt, s)) !=
+      cudaSuccess)
     return MOE_ERR_CUDA;
   rec(1);
   if ((e = launch_permute(*cfg, T, idx, at<int32_t>(ws, L.tile_hist), counts, offsets, perm,

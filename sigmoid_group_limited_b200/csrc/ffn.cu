@@ -70,7 +70,11 @@ struct Cfg {
   static constexpr int STAGES_RAW = kSmemBudget / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
   static constexpr int ACC_COLS = 2 * BN;       // two fp32 accumulators side by side
-  static constexpr int TMEM_COLS = 2 * ACC_COLS < 32 ? 32 : 2 * ACC_COLS;
+  // accumulator buffers: two (the epilogue of one item overlaps the MMAs of
+  // the next) while they fit the 512 TMEM columns, else one
+  static constexpr int NACC = 2 * ACC_COLS <= 512 ? 2 : 1;
+  static constexpr int TMEM_COLS = NACC * ACC_COLS < 32 ? 32 : NACC * ACC_COLS;
+  static constexpr int H_BOX = BN < 64 ? BN : 64;  // rows per TMA box of h
   static_assert((TMEM_COLS & (TMEM_COLS - 1)) == 0 && TMEM_COLS <= 512, "TMEM allocation");
   static constexpr int CTRL_BYTES = 512;        // barriers, queue, flags
   // + the per-slot item starts and row offsets, (3E + 5) ints, added at launch
@@ -262,6 +266,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
   auto two_halves = [&](const WorkItem& it, bool gu) {
     return gu || it.ntile * kDownTile + kTileN < p.H;
   };
+  auto mma_n = [&](const WorkItem& it) { return (min(it.nrows, BN) + 15) & ~15; };
   // queue entry n: wait for it, read it, release it (one arrival per warp)
   auto next_item = [&](int n, int& item, bool whole_warp) -> bool {
     const int q = n % kQueue;
@@ -339,7 +344,8 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
         const int arow0 = gu ? (sh ? 0 : wblk * p.I) + it.ntile * kTileN
                              : (sh ? 0 : wblk * p.H) + it.ntile * kDownTile;
         const int arow1 = gu ? arow0 : arow0 + kTileN;
-        const uint32_t bytes = (two ? 2 : 1) * C::A_BYTES + (gu ? 0 : C::B_BYTES);
+        const int nhbox = gu ? 0 : (mma_n(it) + C::H_BOX - 1) / C::H_BOX;
+        const uint32_t bytes = (two ? 2 : 1) * C::A_BYTES + nhbox * C::H_BOX * 128;
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) {
             live = false;
@@ -349,8 +355,9 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
           mbar_arrive_expect_tx(&full[stage], bytes);
           tma_load_2d(sA, mA0, &full[stage], kb * 64, arow0, pol_w);
           if (two) tma_load_2d(sA + C::A_BYTES, mA1, &full[stage], kb * 64, arow1, pol_w);
-          if (!gu)
-            tma_load_2d(sA + 2 * C::A_BYTES, sh ? &tHs : &tH, &full[stage], kb * 64, it.row0, pol_h);
+          for (int hb = 0; hb < nhbox; ++hb)
+            tma_load_2d(sA + 2 * C::A_BYTES + hb * C::H_BOX * 128, sh ? &tHs : &tH, &full[stage],
+                        kb * 64, it.row0 + hb * C::H_BOX, pol_h);
           *prog = n * kProgStride + kb + 1;
           if (++stage == C::STAGES) {
             stage = 0;
@@ -371,7 +378,6 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16(kTileN, BN);
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool live = true;
@@ -383,6 +389,8 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
         if (!item_ok(p, it, gu, BN)) continue;
         const int nkb = nkb_of(gu, it.e == p.E);
         const bool two = two_halves(it, gu);
+        // MMA N = the item's rows rounded up to 16 (the B rows past it are never read)
+        const uint32_t idesc = idesc_bf16(kTileN, mma_n(it));
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) break;
         tc_fence_after();
         const uint32_t d0 = tmem_base + acc * C::ACC_COLS;
@@ -409,8 +417,10 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
         }
         if (!live) break;
         umma_commit(&tfull[acc]);
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1;
+        if (++acc == C::NACC) {
+          acc = 0;
+          acc_phase ^= 1;
+        }
       }
     }
     __syncwarp();
@@ -419,18 +429,21 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
     // Gate/up items: thread g copies 16-byte chunk (g % 8) of rows g/8,
     // g/8 + 16, ... of the stage's BN x 64 token tile straight into the
     // 128-byte-swizzled layout (chunk c of row r lands at c ^ (r % 8)). A
-    // stage's copies retire two stages later: wait for the group, make it
+    // stage's copies retire kLag stages later: wait for the group, make it
     // visible to the tensor cores (proxy fence), then one arrival per warp on
     // the stage's full barrier. Down items copy nothing, but keep the stage
     // sequence and the arrivals (an empty copy group completes at once).
     constexpr int kRowsPerThread = BN / 16;
-    constexpr int kLag = 2;
+    // stages a gatherer keeps in flight before retiring the oldest: two, but
+    // one when the ring has only three stages (else the MMA would never run
+    // ahead of the gatherers)
+    constexpr int kLag = C::STAGES >= 4 ? 2 : 1;
     const int g = tid - 6 * 32;
     const int chunk = g & 7, rbase = g >> 3;
     const uint64_t pol_x = policy_evict_last();
     int stage = 0;
     uint32_t phase = 0;
-    int pend0 = -1, pend1 = -1;  // stages issued two and one steps ago, not yet retired
+    int pend[2] = {-1, -1};  // stages issued and not yet retired, oldest first (kLag used)
     bool live = true;
     for (int n = 0; live; ++n) {
       int item;
@@ -440,6 +453,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
       if (!item_ok(p, it, gu, BN)) continue;
       const bool sh = it.e == p.E;
       const int nkb = nkb_of(gu, sh);
+      const int nb = mma_n(it);  // B rows the MMA reads
       const uint16_t* src[kRowsPerThread];
 #pragma unroll
       for (int i = 0; i < kRowsPerThread; ++i) {
@@ -459,18 +473,22 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
 #pragma unroll
           for (int i = 0; i < kRowsPerThread; ++i) {
             const int r = rbase + 16 * i;
-            cp_async16(sB + r * 128 + ((chunk ^ (r & 7)) << 4), src[i] + kb * 64, pol_x);
+            if (r < nb) cp_async16(sB + r * 128 + ((chunk ^ (r & 7)) << 4), src[i] + kb * 64, pol_x);
           }
         }
         cp_async_commit();
-        if (pend0 >= 0) {
-          cp_async_wait<kLag>();      // this lane's copies for stage pend0 have landed
+        if (pend[0] >= 0) {
+          cp_async_wait<kLag>();      // this lane's copies for the oldest pending stage landed
           fence_proxy_async_smem();   // ... and are visible to the tensor cores
           __syncwarp();
-          if (lane == 0) mbar_arrive(&full[pend0]);
+          if (lane == 0) mbar_arrive(&full[pend[0]]);
         }
-        pend0 = pend1;
-        pend1 = stage;
+        if (kLag == 2) {
+          pend[0] = pend[1];
+          pend[1] = stage;
+        } else {
+          pend[0] = stage;
+        }
         if (++stage == C::STAGES) {
           stage = 0;
           phase ^= 1;
@@ -481,8 +499,8 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
     fence_proxy_async_smem();
     __syncwarp();
     if (live && lane == 0) {
-      if (pend0 >= 0) mbar_arrive(&full[pend0]);
-      if (pend1 >= 0) mbar_arrive(&full[pend1]);
+      if (pend[0] >= 0) mbar_arrive(&full[pend[0]]);
+      if (kLag == 2 && pend[1] >= 0) mbar_arrive(&full[pend[1]]);
     }
   } else {
     // ------------------------------------------------------------ epilogue
@@ -501,11 +519,11 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
         // destination slot and routing weight of every row, staged while the
         // item's MMAs run (the store loop then touches no metadata in global)
         epilogue_bar();  // all four warps are done with the previous item's rows
-        if (orow < BN) {
+        for (int rr = orow; rr < BN; rr += 4 * 32) {
           int j = -1;
           float wt = 0.f;
-          if (orow < it.nrows) {
-            const int row = it.row0 + orow;
+          if (rr < it.nrows) {
+            const int row = it.row0 + rr;
             if (sh) {
               j = p.T * p.K + row;
               wt = 1.0f;
@@ -519,8 +537,8 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
               }
             }
           }
-          meta_j[orow] = j;
-          meta_w[orow] = wt;
+          meta_j[rr] = j;
+          meta_w[rr] = wt;
         }
         epilogue_bar();
       }
@@ -533,8 +551,9 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
         const bool ok = nfeat < ncols;
         const float L = sh ? p.lim_s : p.lim_r;
         uint16_t* hout = sh ? p.h_s : p.h_r;
+        const int ncol = mma_n(it);
 #pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += 16) {
+        for (int c0 = 0; c0 < ncol; c0 += 16) {
           float gv[16], uv[16];
           tmem_ld16(taddr + c0, gv);
           tmem_ld16(taddr + BN + c0, uv);
@@ -552,12 +571,13 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
           }
         }
       } else {
+        const int ncol = mma_n(it);
 #pragma unroll 1
         for (int half = 0; half < 2; ++half) {
           const int nfeat = it.ntile * kDownTile + half * kTileN + orow;
           const bool ok = nfeat < p.H;
 #pragma unroll 1
-          for (int c0 = 0; c0 < BN; c0 += 16) {
+          for (int c0 = 0; c0 < ncol; c0 += 16) {
             float ov[16];
             tmem_ld16(taddr + half * BN + c0, ov);
             tmem_ld_wait();
@@ -574,8 +594,10 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1;
+      if (++acc == C::NACC) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
       if (gu) {
         // publish this output tile of h: stores -> async proxy -> CTA -> GPU
         fence_proxy_async_global();
@@ -632,12 +654,12 @@ cudaError_t launch_bn(const GemmArgs& a, cudaStream_t s) {
   bool ok = map_bf16(&tWg, a.Wg, static_cast<uint64_t>(a.wrows) * c.I, c.H, kTileN) &&
             map_bf16(&tWu, a.Wu, static_cast<uint64_t>(a.wrows) * c.I, c.H, kTileN) &&
             map_bf16(&tWd, a.Wd, static_cast<uint64_t>(a.wrows) * c.H, c.I, kTileN) &&
-            map_bf16(&tH, a.h_r, TK, c.I, BN);
+            map_bf16(&tH, a.h_r, TK, c.I, C::H_BOX);
   if (p.has_shared) {
     ok = ok && map_bf16(&tWgS, a.W->Wg_s, c.I_shared, c.H, kTileN) &&
          map_bf16(&tWuS, a.W->Wu_s, c.I_shared, c.H, kTileN) &&
          map_bf16(&tWdS, a.W->Wd_s, c.H, c.I_shared, kTileN) &&
-         map_bf16(&tHs, a.h_s, T, c.I_shared, BN);
+         map_bf16(&tHs, a.h_s, T, c.I_shared, C::H_BOX);
   } else {
     tWgS = tWg;
     tWuS = tWu;

@@ -26,22 +26,22 @@ namespace sgl {
 namespace {
 
 // ---------------------------------------------------------------------------
-// Logits for a set of rows, one warp per expert: the expert's fp32 router row
-// is held in registers (a strided slice per lane) and up to 32 token rows are
-// staged in shared memory as bf16; ILP tokens are accumulated at once.
-//  EXACT = false: fp32 FMA accumulation (the pages' fp32 router), for small
-//                 batches;
-//  EXACT = true:  every product bf16 * fp32 is exact in float64 and the sum
-//                 of H of them is accumulated in float64, so the one final
-//                 rounding to fp32 gives the logit of an exact dot product.
-//                 Used for the tokens whose fp32 decision was too close.
-// With `list`, the rows are list[0 .. *list_n) instead of 0 .. T-1.
+// Logits for small batches (T <= 32), split over K: CTA (s, eb) forms the
+// partial dot products of all tokens with experts [32 eb, 32 eb + 32) over
+// hidden columns [128 s, 128 s + 128), in fp32, and writes them to
+// zpart[s][t][e]. Lane t
+// of every warp holds token t's 128 columns in registers, the 32 router rows
+// of the block sit in shared memory and are read as broadcasts, and warp w
+// accumulates experts 4w .. 4w+3 of the block: no cross-lane reduction.
+// block_cnt[eb] counts the finished CTAs of expert block eb (zeroed by the
+// caller); the last one writes z[t][e] = sum over s of zpart[s][t][e].
 // ---------------------------------------------------------------------------
 constexpr int kSmallT = 32;
-constexpr int kRowRegs = 24;  // float4 per lane: H <= 24 * 128 = 3072
+constexpr int kRowRegs = 24;  // float4 per lane in router_refine: H <= 24 * 128 = 3072
 constexpr int kMaxExperts = 1024;
-constexpr int kRowWarps = 4;  // experts per CTA
-constexpr int kTokSplit = 2;  // warps per expert (they split the token rows)
+constexpr int kSplitH = 128;  // hidden columns per partial
+constexpr int kSplitE = 32;   // experts per CTA
+constexpr int kMaxSplit = kRowRegs * 128 / kSplitH;  // H <= 3072
 
 // bf16 bits -> float64 by field arithmetic (no conversion instruction):
 // sign, exponent rebiased from 127 to 1023, 7 mantissa bits on top.
@@ -54,211 +54,121 @@ __device__ __forceinline__ double bf16_bits_to_double(uint32_t b) {
   return __longlong_as_double(static_cast<long long>(bits));
 }
 
-template <bool EXACT, int ILP>
-__global__ void __launch_bounds__(kRowWarps * kTokSplit * 32) router_logits_rows(
-    int T, int H, int E, const uint16_t* __restrict__ x, const float* __restrict__ Wr,
-    float* __restrict__ z, const int32_t* __restrict__ list, const int32_t* __restrict__ list_n,
-    int32_t* __restrict__ err) {
-  using Acc = typename std::conditional<EXACT, double, float>::type;
-  extern __shared__ __align__(128) uint16_t xs[];  // [kSmallT][H]
-  __shared__ __align__(8) uint64_t bar;
-  __shared__ int abort_flag;
+__global__ void __launch_bounds__(256) router_logits_splitk(int T, int H, int E,
+                                                           const uint16_t* __restrict__ x,
+                                                           const float* __restrict__ Wr,
+                                                           float* __restrict__ zpart,
+                                                           int32_t* __restrict__ block_cnt,
+                                                           float* __restrict__ z) {
+  __shared__ __align__(16) float ws[kSplitE][kSplitH];
+  // token rows of the chunk, padded by 16 bytes so that 8 lanes reading the
+  // same column of 8 rows hit 8 different bank groups
+  constexpr int kXRow = kSplitH + 8;  // bf16 elements
+  __shared__ __align__(16) uint16_t xs[kSmallT][kXRow];
+  __shared__ float out[kSmallT][kSplitE + 1];
+  __shared__ int is_last;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int e = blockIdx.x * kRowWarps + (warp % kRowWarps);
-  const int split = warp / kRowWarps;  // this warp takes token groups split, split+kTokSplit, ...
-  const bool have = e < E;
-  const int n = list ? min(*list_n, T) : T;
-  if (n <= 0) return;
-  if (tid == 0) {
-    mbar_init(&bar, 1);
-    abort_flag = 0;
-    fence_mbar_init();
+  const int s = blockIdx.x, e0 = blockIdx.y * kSplitE;
+  const int k0 = s * kSplitH, kn = min(kSplitH, H - k0);  // kn is a multiple of 64
+  // the block's router rows and the batch's token columns, all copies in
+  // flight at once (16-byte cp.async); zeros past the ends
+  const uint64_t pol = policy_evict_first();
+#pragma unroll
+  for (int it = 0; it < kSplitE * kSplitH / 4 / 256; ++it) {
+    const int i = tid + 256 * it;
+    const int r = i / (kSplitH / 4), c = 4 * (i % (kSplitH / 4));
+    if (c < kn && e0 + r < E)
+      cp_async16(&ws[r][c], Wr + static_cast<size_t>(e0 + r) * H + k0 + c, pol);
+    else
+      *reinterpret_cast<float4*>(&ws[r][c]) = make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  uint32_t phase = 0;
-  float4 wv[kRowRegs];
-  {
-    // unconditional loads from clamped addresses (all in flight together),
-    // then zero the slots past the row's end
-    const float* row = Wr + static_cast<size_t>(have ? e : 0) * H;
+  const uint64_t pol_x = policy_evict_last();
 #pragma unroll
-    for (int j = 0; j < kRowRegs; ++j)
-      wv[j] = *reinterpret_cast<const float4*>(row + min(4 * lane + 128 * j, H - 4));
-#pragma unroll
-    for (int j = 0; j < kRowRegs; ++j)
-      if (4 * lane + 128 * j >= H) wv[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int it = 0; it < kSmallT * kSplitH / 8 / 256; ++it) {
+    const int i = tid + 256 * it;
+    const int r = i / (kSplitH / 8), c = 8 * (i % (kSplitH / 8));
+    if (r < T && c < kn)
+      cp_async16(&xs[r][c], x + static_cast<size_t>(r) * H + k0 + c, pol_x);
+    else
+      *reinterpret_cast<uint4*>(&xs[r][c]) = make_uint4(0u, 0u, 0u, 0u);
   }
-  const uint32_t row_bytes = static_cast<uint32_t>(H) * 2;
-  for (int c0 = 0; c0 < n; c0 += kSmallT) {
-    const int nc = min(kSmallT, n - c0);
-    __syncthreads();  // everyone is done with the previous chunk
-    if (tid == 0) {
-      // one bulk copy per token row, all in flight at once
-      fence_proxy_async_smem();
-      mbar_arrive_expect_tx(&bar, row_bytes * nc);
-      for (int r = 0; r < nc; ++r) {
-        const int t = list ? list[c0 + r] : c0 + r;
-        bulk_load(xs + r * H, x + static_cast<size_t>(t) * H, row_bytes, &bar);
-      }
-    }
-    mbar_wait(&bar, phase, &abort_flag, err, MOE_DEVERR_TIMEOUT);
-    phase ^= 1;
-    if (!have) continue;
-    for (int r0 = split * ILP; r0 < nc; r0 += ILP * kTokSplit) {
-      Acc acc[ILP];
-#pragma unroll
-      for (int q = 0; q < ILP; ++q) acc[q] = Acc(0);
-#pragma unroll
-      for (int j = 0; j < kRowRegs; ++j) {
-        const int k = 4 * lane + 128 * j;
-        if (k < H) {
-          Acc w0, w1, w2, w3;
-          if (EXACT) {
-            w0 = static_cast<Acc>(wv[j].x); w1 = static_cast<Acc>(wv[j].y);
-            w2 = static_cast<Acc>(wv[j].z); w3 = static_cast<Acc>(wv[j].w);
-          } else {
-            w0 = wv[j].x; w1 = wv[j].y; w2 = wv[j].z; w3 = wv[j].w;
-          }
-#pragma unroll
-          for (int q = 0; q < ILP; ++q) {
-            const int r = min(r0 + q, nc - 1);
-            const uint2 p = *reinterpret_cast<const uint2*>(xs + r * H + k);
-            if (EXACT) {
-              acc[q] = fma(w0, static_cast<Acc>(bf16_bits_to_double(p.x & 0xFFFFu)), acc[q]);
-              acc[q] = fma(w1, static_cast<Acc>(bf16_bits_to_double(p.x >> 16)), acc[q]);
-              acc[q] = fma(w2, static_cast<Acc>(bf16_bits_to_double(p.y & 0xFFFFu)), acc[q]);
-              acc[q] = fma(w3, static_cast<Acc>(bf16_bits_to_double(p.y >> 16)), acc[q]);
-            } else {
-              acc[q] = fmaf(w0, __uint_as_float(p.x << 16), acc[q]);
-              acc[q] = fmaf(w1, __uint_as_float(p.x & 0xFFFF0000u), acc[q]);
-              acc[q] = fmaf(w2, __uint_as_float(p.y << 16), acc[q]);
-              acc[q] = fmaf(w3, __uint_as_float(p.y & 0xFFFF0000u), acc[q]);
-            }
-          }
-        }
-      }
-#pragma unroll
-      for (int q = 0; q < ILP; ++q) {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc[q] += __shfl_xor_sync(0xffffffffu, acc[q], o);
-      }
-      if (lane < ILP) {
-        Acc v = acc[0];
-#pragma unroll
-        for (int q = 1; q < ILP; ++q)
-          if (lane == q) v = acc[q];
-        if (r0 + lane < nc) {
-          const int t = list ? list[c0 + r0 + lane] : c0 + r0 + lane;
-          z[static_cast<size_t>(t) * E + e] = static_cast<float>(v);
-        }
-      }
-    }
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Logits for larger batches: a 128 (tokens) x 128 (experts) fp32 SIMT tile
-// per CTA, 8x8 outputs per thread, K streamed in chunks of 16 through
-// double-buffered shared memory.
-// ---------------------------------------------------------------------------
-constexpr int kRT = 128, kRE = 128, kRK = 16;
-
-__global__ void __launch_bounds__(256) router_logits_tiled(int T, int H, int E,
-                                                          const uint16_t* __restrict__ x,
-                                                          const float* __restrict__ Wr,
-                                                          float* __restrict__ z) {
-  __shared__ __align__(16) float xs[2][kRK][kRT + 4];
-  __shared__ __align__(16) float ws[2][kRK][kRE + 4];
-  const int tid = threadIdx.x;
-  const int t0 = blockIdx.x * kRT, e0 = blockIdx.y * kRE;
-  // loader mapping: row = tid / 2 (token or expert), 8 consecutive k per thread
-  const int lrow = tid >> 1, lk = (tid & 1) * 8;
-  const bool xok = (t0 + lrow) < T, wok = (e0 + lrow) < E;
-  const uint16_t* xsrc = x + static_cast<size_t>(t0 + lrow) * H + lk;
-  const float* wsrc = Wr + static_cast<size_t>(e0 + lrow) * H + lk;
-
-  uint4 xr;
-  float4 wr0, wr1;
-  auto gload = [&](int kc) {
-    xr = xok ? *reinterpret_cast<const uint4*>(xsrc + kc) : make_uint4(0, 0, 0, 0);
-    wr0 = wok ? *reinterpret_cast<const float4*>(wsrc + kc) : make_float4(0.f, 0.f, 0.f, 0.f);
-    wr1 = wok ? *reinterpret_cast<const float4*>(wsrc + kc + 4) : make_float4(0.f, 0.f, 0.f, 0.f);
-  };
-  auto sstore = [&](int buf) {
-    const uint32_t xv[4] = {xr.x, xr.y, xr.z, xr.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      xs[buf][lk + 2 * i][lrow] = __uint_as_float(xv[i] << 16);
-      xs[buf][lk + 2 * i + 1][lrow] = __uint_as_float(xv[i] & 0xFFFF0000u);
-    }
-    ws[buf][lk + 0][lrow] = wr0.x;
-    ws[buf][lk + 1][lrow] = wr0.y;
-    ws[buf][lk + 2][lrow] = wr0.z;
-    ws[buf][lk + 3][lrow] = wr0.w;
-    ws[buf][lk + 4][lrow] = wr1.x;
-    ws[buf][lk + 5][lrow] = wr1.y;
-    ws[buf][lk + 6][lrow] = wr1.z;
-    ws[buf][lk + 7][lrow] = wr1.w;
-  };
-
-  const int ty = tid >> 4, tx = tid & 15;
-  float acc[8][8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
-
-  const int nk = H / kRK;
-  gload(0);
-  sstore(0);
+  cp_async_commit();
+  cp_async_wait<0>();
   __syncthreads();
-  for (int kc = 0; kc < nk; ++kc) {
-    const int buf = kc & 1;
-    if (kc + 1 < nk) gload((kc + 1) * kRK);
+  constexpr int EW = kSplitE / 8;  // experts per warp
+  float acc[EW];
 #pragma unroll
-    for (int k = 0; k < kRK; ++k) {
-      const float4 a0 = *reinterpret_cast<const float4*>(&xs[buf][k][ty * 4]);
-      const float4 a1 = *reinterpret_cast<const float4*>(&xs[buf][k][64 + ty * 4]);
-      const float4 b0 = *reinterpret_cast<const float4*>(&ws[buf][k][tx * 4]);
-      const float4 b1 = *reinterpret_cast<const float4*>(&ws[buf][k][64 + tx * 4]);
-      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-      const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+  for (int q = 0; q < EW; ++q) acc[q] = 0.f;
+#pragma unroll 4
+  for (int i = 0; i < kSplitH / 8; ++i) {
+    const uint4 xv8 = *reinterpret_cast<const uint4*>(&xs[lane][8 * i]);
+    const uint32_t pk[4] = {xv8.x, xv8.y, xv8.z, xv8.w};
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
+    for (int h = 0; h < 2; ++h) {
+      const float xv0 = __uint_as_float(pk[2 * h] << 16);
+      const float xv1 = __uint_as_float(pk[2 * h] & 0xFFFF0000u);
+      const float xv2 = __uint_as_float(pk[2 * h + 1] << 16);
+      const float xv3 = __uint_as_float(pk[2 * h + 1] & 0xFFFF0000u);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+      for (int q = 0; q < EW; ++q) {
+        const float4 wv = *reinterpret_cast<const float4*>(&ws[warp * EW + q][8 * i + 4 * h]);
+        acc[q] = fmaf(xv0, wv.x, acc[q]);
+        acc[q] = fmaf(xv1, wv.y, acc[q]);
+        acc[q] = fmaf(xv2, wv.z, acc[q]);
+        acc[q] = fmaf(xv3, wv.w, acc[q]);
+      }
     }
-    if (kc + 1 < nk) sstore(buf ^ 1);
-    __syncthreads();
   }
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int t = t0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + i - 4);
-    if (t >= T) continue;
+  for (int q = 0; q < EW; ++q) out[lane][warp * EW + q] = acc[q];
+  __syncthreads();
+  for (int i = tid; i < T * kSplitE; i += blockDim.x) {
+    const int t = i / kSplitE, c = i % kSplitE;
+    if (e0 + c < E) zpart[(static_cast<size_t>(s) * T + t) * E + e0 + c] = out[t][c];
+  }
+  // The last CTA of this expert block to finish adds the block's partials in
+  // split order (so z does not depend on which CTA came last).
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) is_last = atomicAdd(&block_cnt[blockIdx.y], 1) == static_cast<int>(gridDim.x) - 1;
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  const int nsplit = gridDim.x;
+  const size_t stride = static_cast<size_t>(T) * E;
+  constexpr int kPer = kSmallT * kSplitE / 256;  // outputs per thread, taken two at a time
+#pragma unroll 1
+  for (int r0 = 0; r0 < kPer; r0 += 2) {
+    float v[2][kMaxSplit];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int e = e0 + (j < 4 ? tx * 4 + j : 64 + tx * 4 + j - 4);
-      if (e < E) z[static_cast<size_t>(t) * E + e] = acc[i][j];
+    for (int r = 0; r < 2; ++r) {
+      const int i = tid + 256 * (r0 + r), t = i / kSplitE, c = i % kSplitE;
+      const bool ok = t < T && e0 + c < E;
+      const float* pp = zpart + static_cast<size_t>(ok ? t : 0) * E + (ok ? e0 + c : 0);
+#pragma unroll
+      for (int sp = 0; sp < kMaxSplit; ++sp) v[r][sp] = sp < nsplit ? __ldcg(pp + sp * stride) : 0.f;
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int i = tid + 256 * (r0 + r), t = i / kSplitE, c = i % kSplitE;
+      float sum = 0.f;
+#pragma unroll
+      for (int sp = 0; sp < kMaxSplit; ++sp)
+        if (sp < nsplit) sum += v[r][sp];
+      if (t < T && e0 + c < E) z[static_cast<size_t>(t) * E + e0 + c] = sum;
     }
   }
 }
 
-// ---------------------------------------------------------------------------
-// Scores and group-limited top-k: one warp per token. Lane l holds experts
-// e = l + 32*j. The combine weights are computed in float64 from the fp32
-// scores and rounded once.
-//
-// Two modes:
-//  certified (tau > 0): scores from an fp32 sigmoid of the fp32 logits; the
-//    kernel also measures its own decision margins (the topk_group-th minus
-//    the next group score, and every gap between neighbours in the ranking
-//    of the K+1 best candidates, since slot order is rank order) and appends
-//    the token to `unc` when one is below tau (scaled by the token's logit
-//    RMS); those tokens get exact logits and a second, exact pass.
-//  exact (tau == 0): scores from a float64 sigmoid rounded to fp32 (the
-//    reference definition), over the tokens in `list`.
-// GJ > 0: every group spans GJ whole register slots (E/n_group a multiple of
-// 32), so group maxima are reduced in registers, all groups at once.
-// ---------------------------------------------------------------------------
+// Order-preserving map of a (non-NaN) float onto nonzero uint32 keys, and back.
+__device__ __forceinline__ uint32_t order_key(float v) {
+  const uint32_t u = __float_as_uint(v + 0.0f);  // -0 -> +0: equal values, equal keys
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
 template <int NV, int GJ>
 __global__ void __launch_bounds__(256) router_topk(int T, int E, int n_group, int topk_group,
                                                    int K, float scale, int renorm,
@@ -281,9 +191,9 @@ __global__ void __launch_bounds__(256) router_topk(int T, int E, int n_group, in
     // all loads first, from clamped (always valid) addresses, so they are in
     // flight together; lanes past E are masked afterwards
 #pragma unroll
-    for (int j = 0; j < NV; ++j) zv[j] = zr[min(lane + 32 * j, E - 1)];
-#pragma unroll
     for (int j = 0; j < NV; ++j) bv0[j] = bias ? bias[min(lane + 32 * j, E - 1)] : 0.f;
+#pragma unroll
+    for (int j = 0; j < NV; ++j) zv[j] = zr[min(lane + 32 * j, E - 1)];
     float zz = 0.f;
 #pragma unroll
     for (int j = 0; j < NV; ++j) {
@@ -308,9 +218,8 @@ __global__ void __launch_bounds__(256) router_topk(int T, int E, int n_group, in
         gs[g] = m;
       }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-        for (int g = 0; g < G; ++g) gs[g] = fmaxf(gs[g], __shfl_xor_sync(0xffffffffu, gs[g], o));
+      for (int g = 0; g < G; ++g)
+        gs[g] = key_value(__reduce_max_sync(0xffffffffu, order_key(gs[g])));
       float last = 0.f;
       for (int r = 0; r <= topk_group && r < G; ++r) {
         float bv = -INFINITY;
@@ -372,39 +281,45 @@ __global__ void __launch_bounds__(256) router_topk(int T, int E, int n_group, in
       if (e < E && ((kept_groups >> g) & 1u)) cand |= 1u << j;
     }
     // ---- K rounds of warp argmax over candidates (ties -> lower expert id),
-    // plus one more for the last gap of the ranking
+    // plus one more for the last gap of the ranking. Each lane keeps its own
+    // best candidate (lowest j among equals, i.e. lowest expert id); a round
+    // is a warp max of the order-preserving keys, then the lowest expert id
+    // among the lanes that hold that key, and only the winning lane rescans.
     int my_e = -1;
     float my_s = 0.f, last_b = 0.f, emargin = INFINITY;
-    for (int k = 0; k <= K; ++k) {
+    uint32_t lkey = 0u;  // 0: no candidate left in this lane
+    int lj = 0;
+    auto rescan = [&]() {
+      lkey = 0u;
       float bv = -INFINITY;
-      int be = 0x7fffffff;
 #pragma unroll
-      for (int j = 0; j < NV; ++j) {
-        if (((cand >> j) & 1u) && (be == 0x7fffffff || b[j] > bv)) {
+      for (int j = 0; j < NV; ++j)
+        if (((cand >> j) & 1u) && (lkey == 0u || b[j] > bv)) {
           bv = b[j];
-          be = lane + 32 * j;
+          lj = j;
+          lkey = order_key(bv);
         }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-        if (ov > bv || (ov == bv && oe < be)) {
-          bv = ov;
-          be = oe;
-        }
-      }
-      if (k > 0 && be != 0x7fffffff) emargin = fminf(emargin, last_b - bv);
+    };
+    rescan();
+    for (int k = 0; k <= K; ++k) {
+      const uint32_t mkey = __reduce_max_sync(0xffffffffu, lkey);
+      const uint32_t be_u = __reduce_min_sync(
+          0xffffffffu, (lkey == mkey && lkey != 0u) ? static_cast<uint32_t>(lj * 32 + lane) : 0xffffffffu);
+      if (be_u == 0xffffffffu) break;  // no candidate left
+      const int be = static_cast<int>(be_u);
+      const float bv = key_value(mkey);
+      if (k > 0) emargin = fminf(emargin, last_b - bv);
       if (k == K) break;
       // owner lane removes the winner and publishes its unbiased score
       const int owner = be & 31, jw = be >> 5;
       float sw = 0.f;
+      if (lane == owner) {
 #pragma unroll
-      for (int j = 0; j < NV; ++j)
-        if (j == jw && lane == owner) {
-          sw = s[j];
-          cand &= ~(1u << j);
-        }
+        for (int j = 0; j < NV; ++j)
+          if (j == jw) sw = s[j];
+        cand &= ~(1u << jw);
+        rescan();
+      }
       sw = __shfl_sync(0xffffffffu, sw, owner);
       if (lane == k) {
         my_e = be;
@@ -433,6 +348,174 @@ __global__ void __launch_bounds__(256) router_topk(int T, int E, int n_group, in
       const float tau_t = tau * fmaxf(1.f, sqrtf(zz / E));
       if (lane == 0 && (gmargin < tau_t || emargin < tau_t)) unc[atomicAdd(unc_n, 1)] = t;
     }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// The same certified selection with one CTA per token and one warp per
+// expert group, for groups of 32 or 64 experts (NG = 1 or 2 per lane), at
+// most 16 groups and topk_group * (K+1) <= 64. Warp g scores its group
+// (fp32 sigmoid + bias), finds the group maximum and its own top K+1 by
+// rounds of warp max over order-preserving keys (ties -> lower expert id);
+// warp 0 keeps topk_group groups (ties -> lower group) and ranks the kept
+// groups' candidates (the overall top K+1 among the kept groups is among
+// them). Margins, weights and the flagged-token list are as in router_topk.
+// ---------------------------------------------------------------------------
+constexpr int kSelMaxGroups = 16;
+constexpr int kSelMaxCand = 33;  // K + 1 <= 33
+
+template <int NG>
+__global__ void __launch_bounds__(kSelMaxGroups * 32) router_select(
+    int T, int E, int n_group, int topk_group, int K, float scale, int renorm,
+    const float* __restrict__ z, const float* __restrict__ bias, int32_t* __restrict__ idx,
+    float* __restrict__ wout, float tau, int32_t* __restrict__ unc, int32_t* __restrict__ unc_n) {
+  __shared__ uint32_t gkey[kSelMaxGroups];
+  __shared__ float gzz[kSelMaxGroups];
+  __shared__ uint32_t ckey[kSelMaxGroups][kSelMaxCand];
+  __shared__ int cid[kSelMaxGroups][kSelMaxCand];
+  __shared__ float cs[kSelMaxGroups][kSelMaxCand];
+  const int lane = threadIdx.x & 31, g = threadIdx.x >> 5;
+  const int per = 32 * NG, KP1 = K + 1;
+  for (int t = blockIdx.x; t < T; t += gridDim.x) {
+    const float* zr = z + static_cast<size_t>(t) * E;
+    if (g < n_group) {
+      float sv[NG];
+      uint32_t key[NG];
+      float zz = 0.f;
+#pragma unroll
+      for (int v = 0; v < NG; ++v) {
+        const int e = g * per + lane + 32 * v;
+        const float zv = zr[e];
+        zz = fmaf(zv, zv, zz);
+        sv[v] = 1.0f / (1.0f + expf(-zv));
+        key[v] = order_key(sv[v] + (bias ? bias[e] : 0.f));
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) zz += __shfl_xor_sync(0xffffffffu, zz, o);
+      uint32_t mine = key[0];
+      int mj = 0;
+#pragma unroll
+      for (int v = 1; v < NG; ++v)
+        if (key[v] > mine) {
+          mine = key[v];
+          mj = v;
+        }
+      const uint32_t gmax = __reduce_max_sync(0xffffffffu, mine);
+      if (lane == 0) {
+        gkey[g] = gmax;
+        gzz[g] = zz;
+      }
+      // this group's top K+1, best first
+      uint32_t live = (1u << NG) - 1u;
+      for (int r = 0; r < KP1; ++r) {
+        const uint32_t mk = __reduce_max_sync(0xffffffffu, live ? mine : 0u);
+        const uint32_t wid = __reduce_min_sync(
+            0xffffffffu, (live && mine == mk) ? static_cast<uint32_t>(32 * mj + lane) : 0xffffffffu);
+        if (wid == 0xffffffffu) {  // fewer candidates than K+1: mark the rest empty
+          for (int rr = r + lane; rr < KP1; rr += 32) ckey[g][rr] = 0u;
+          break;
+        }
+        if (lane == static_cast<int>(wid & 31)) {
+          ckey[g][r] = mk;
+          cid[g][r] = g * per + static_cast<int>(wid);
+          cs[g][r] = sv[mj];
+          live &= ~(1u << mj);
+          mine = 0u;
+#pragma unroll
+          for (int v = 0; v < NG; ++v)
+            if (((live >> v) & 1u) && key[v] > mine) {
+              mine = key[v];
+              mj = v;
+            }
+        }
+      }
+    }
+    __syncthreads();
+    if (g == 0) {
+      // groups: lane gg holds group gg's maximum
+      uint32_t gk = lane < n_group ? gkey[lane] : 0u;
+      bool avail = lane < n_group;
+      uint32_t kept = 0;
+      float last = 0.f, gmargin = INFINITY;
+      const int rounds = topk_group < n_group ? topk_group + 1 : topk_group;
+      for (int r = 0; r < rounds; ++r) {
+        const uint32_t mk = __reduce_max_sync(0xffffffffu, avail ? gk : 0u);
+        const int gi = static_cast<int>(__reduce_min_sync(
+            0xffffffffu, (avail && gk == mk) ? static_cast<uint32_t>(lane) : 0xffffffffu));
+        if (r < topk_group) {
+          kept |= 1u << gi;
+          if (lane == gi) avail = false;
+          last = key_value(mk);
+        } else {
+          gmargin = last - key_value(mk);
+        }
+      }
+      // candidates of the kept groups, two slots per lane
+      uint32_t k2[2];
+      int i2[2];
+      float s2[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int slot = lane + 32 * h;  // candidate number in kept-group order
+        k2[h] = 0u;
+        i2[h] = 0;
+        s2[h] = 0.f;
+        const int gsel = slot / KP1, r = slot - gsel * KP1;
+        if (gsel < topk_group) {
+          // the gsel-th kept group, in increasing group order
+          uint32_t m = kept;
+          for (int q = 0; q < gsel; ++q) m &= m - 1u;
+          const int gg = __ffs(m) - 1;
+          k2[h] = ckey[gg][r];
+          i2[h] = cid[gg][r];
+          s2[h] = cs[gg][r];
+        }
+      }
+      int my_e = -1;
+      float my_s = 0.f, last_b = 0.f, emargin = INFINITY;
+      for (int k = 0; k <= K; ++k) {
+        const uint32_t mine = k2[0] > k2[1] || (k2[0] == k2[1] && i2[0] < i2[1]) ? k2[0] : k2[1];
+        const int mh = (k2[0] > k2[1] || (k2[0] == k2[1] && i2[0] < i2[1])) ? 0 : 1;
+        const uint32_t mk = __reduce_max_sync(0xffffffffu, mine);
+        if (mk == 0u) break;
+        const uint32_t we = __reduce_min_sync(
+            0xffffffffu, mine == mk ? static_cast<uint32_t>(mh ? i2[1] : i2[0]) : 0xffffffffu);
+        const float bv = key_value(mk);
+        if (k > 0) emargin = fminf(emargin, last_b - bv);
+        if (k == K) break;
+        float sw = 0.f;
+        const bool own = mine == mk && static_cast<uint32_t>(mh ? i2[1] : i2[0]) == we;
+        if (own) {
+          sw = mh ? s2[1] : s2[0];
+          if (mh) k2[1] = 0u;
+          else k2[0] = 0u;
+        }
+        const unsigned ob = __ballot_sync(0xffffffffu, own);
+        sw = __shfl_sync(0xffffffffu, sw, __ffs(ob) - 1);
+        if (lane == k) {
+          my_e = static_cast<int>(we);
+          my_s = sw;
+        }
+        last_b = bv;
+      }
+      double den = (lane < K) ? static_cast<double>(my_s) : 0.0;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+      if (lane < K) {
+        const double sk = static_cast<double>(my_s);
+        const double wv = renorm ? static_cast<double>(scale) * (sk / den)
+                                 : static_cast<double>(scale) * sk;
+        idx[static_cast<size_t>(t) * K + lane] = my_e;
+        wout[static_cast<size_t>(t) * K + lane] = static_cast<float>(wv);
+      }
+      if (lane == 0) {
+        float zz = 0.f;
+        for (int q = 0; q < n_group; ++q) zz += gzz[q];
+        const float tau_t = tau * fmaxf(1.f, sqrtf(zz / E));
+        if (gmargin < tau_t || emargin < tau_t) unc[atomicAdd(unc_n, 1)] = t;
+      }
+    }
+    __syncthreads();  // shared candidates are reused by the next token
   }
 }
 
@@ -772,31 +855,41 @@ __global__ void __launch_bounds__(kRefineThreads) router_refine(
 
 template <int NV, int GJ>
 cudaError_t launch_topk(const moe_cfg& c, int T, const float* z, const float* bias, int32_t* idx,
-                        float* w, float tau, int32_t* unc, int32_t* unc_n, const int32_t* list,
-                        cudaStream_t s) {
+                        float* w, float tau, int32_t* unc, int32_t* unc_n, cudaStream_t s) {
   // small batches: one token per CTA, so every token's warp has an SM to itself
   const int warps = T <= 4 * num_sms() ? 1 : 8;
-  int grid = cdiv(T, warps);
-  if (list) grid = std::min(grid, num_sms() * 4);
+  const int grid = cdiv(T, warps);
   router_topk<NV, GJ><<<grid, warps * 32, 0, s>>>(T, c.E, c.n_group, c.topk_group, c.K, c.scale,
                                                   c.renorm, z, bias, idx, w, tau, unc, unc_n,
-                                                  list, list ? unc_n : nullptr);
+                                                  nullptr, nullptr);
   return cudaGetLastError();
 }
 
 cudaError_t topk_dispatch(const moe_cfg& c, int T, const float* z, const float* bias,
                           int32_t* idx, float* w, float tau, int32_t* unc, int32_t* unc_n,
-                          const int32_t* list, cudaStream_t s) {
+                          cudaStream_t s) {
   const int nv = cdiv(c.E, 32);
   const int per = c.E / c.n_group;
-#define SGL_TOPK(NV_)                                                                    \
-  if (nv <= NV_) {                                                                       \
-    if (c.E == NV_ * 32 && per % 32 == 0 && per / 32 == 2 && NV_ >= 2)                   \
-      return launch_topk<NV_, (NV_ >= 2 ? 2 : 1)>(c, T, z, bias, idx, w, tau, unc, unc_n, \
-                                                  list, s);                              \
-    if (c.E == NV_ * 32 && per % 32 == 0 && per / 32 == 1)                               \
-      return launch_topk<NV_, 1>(c, T, z, bias, idx, w, tau, unc, unc_n, list, s);       \
-    return launch_topk<NV_, 0>(c, T, z, bias, idx, w, tau, unc, unc_n, list, s);         \
+  if ((per == 32 || per == 64) && c.n_group <= kSelMaxGroups && c.K + 1 <= kSelMaxCand &&
+      c.topk_group * (c.K + 1) <= 64) {
+    const int grid = std::min(T, num_sms() * 8);
+    if (per == 32)
+      router_select<1><<<grid, c.n_group * 32, 0, s>>>(T, c.E, c.n_group, c.topk_group, c.K,
+                                                       c.scale, c.renorm, z, bias, idx, w, tau,
+                                                       unc, unc_n);
+    else
+      router_select<2><<<grid, c.n_group * 32, 0, s>>>(T, c.E, c.n_group, c.topk_group, c.K,
+                                                       c.scale, c.renorm, z, bias, idx, w, tau,
+                                                       unc, unc_n);
+    return cudaGetLastError();
+  }
+#define SGL_TOPK(NV_)                                                                   \
+  if (nv <= NV_) {                                                                      \
+    if (c.E == NV_ * 32 && per % 32 == 0 && per / 32 == 2 && NV_ >= 2)                  \
+      return launch_topk<NV_, (NV_ >= 2 ? 2 : 1)>(c, T, z, bias, idx, w, tau, unc, unc_n, s); \
+    if (c.E == NV_ * 32 && per % 32 == 0 && per / 32 == 1)                              \
+      return launch_topk<NV_, 1>(c, T, z, bias, idx, w, tau, unc, unc_n, s);            \
+    return launch_topk<NV_, 0>(c, T, z, bias, idx, w, tau, unc, unc_n, s);              \
   }
   SGL_TOPK(1)
   SGL_TOPK(2)
@@ -853,20 +946,6 @@ cudaError_t launch_refine(const moe_cfg& c, int T, const uint16_t* x, const floa
   return launch_refine_nv<32>(c, T, x, Wr, z, bias, idx, w, tau, list, list_n, s);
 }
 
-template <bool EXACT, int ILP>
-cudaError_t launch_rows(const moe_cfg& c, int T, const uint16_t* x, const float* Wr, float* z,
-                        const int32_t* list, const int32_t* list_n, int32_t* err, cudaStream_t s) {
-  const size_t smem = static_cast<size_t>(kSmallT) * c.H * sizeof(uint16_t);
-  auto kern = router_logits_rows<EXACT, ILP>;
-  cudaError_t e = ensure_dyn_smem(reinterpret_cast<const void*>(kern),
-                                  kSmallT * kRowRegs * 128 * static_cast<int>(sizeof(uint16_t)));
-  if (e != cudaSuccess) return e;
-  kern<<<cdiv(c.E, kRowWarps), kRowWarps * kTokSplit * 32, smem, s>>>(T, c.H, c.E, x, Wr, z, list,
-                                                                      list_n,
-                                                          err);
-  return cudaGetLastError();
-}
-
 }  // namespace
 
 // Margin (on biased scores, per unit of logit RMS) below which an fp32
@@ -878,13 +957,19 @@ constexpr float kCertifyMargin = 1.0f / 32768.0f;
 
 cudaError_t launch_router(const moe_cfg& c, int T, const uint16_t* x, const float* Wr,
                           const float* bias, float* z, int32_t* idx, float* w, int32_t* unc,
-                          int32_t* unc_n, int32_t* err, uint16_t* wr_split, cudaStream_t s) {
+                          int32_t* unc_n, int32_t* err, uint16_t* wr_split, float* zpart,
+                          int32_t* split_cnt, cudaStream_t s) {
   cudaError_t e;
   if (c.H > kRowRegs * 128) return cudaErrorInvalidValue;
   if (T <= kSmallT) {
-    e = launch_rows<false, 4>(c, T, x, Wr, z, nullptr, nullptr, err, s);
-  } else if (wr_split != nullptr) {
+    // fp32 split-K partials, added in order by the last CTA of each expert block
+    if (zpart == nullptr || split_cnt == nullptr) return cudaErrorInvalidValue;
+    const int nsplit = cdiv(c.H, kSplitH);
+    router_logits_splitk<<<dim3(nsplit, cdiv(c.E, kSplitE)), 256, 0, s>>>(T, c.H, c.E, x, Wr,
+                                                                           zpart, split_cnt, z);
+  } else {
     // tensor cores: split the router matrix, then one bf16 x 3 GEMM into z
+    if (wr_split == nullptr) return cudaErrorInvalidValue;
     const long long n = static_cast<long long>(c.E) * c.H;
     uint16_t* hi = wr_split;
     uint16_t* mid = hi + n;
@@ -892,16 +977,10 @@ cudaError_t launch_router(const moe_cfg& c, int T, const uint16_t* x, const floa
     split_router<<<num_sms() * 4, 256, 0, s>>>(n, Wr, hi, mid, lo);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     e = launch_router_gemm(c, T, x, hi, mid, lo, z, err, s);
-  } else {
-    dim3 grid(cdiv(T, kRT), cdiv(c.E, kRE));
-    router_logits_tiled<<<grid, 256, 0, s>>>(T, c.H, c.E, x, Wr, z);
-    e = cudaGetLastError();
   }
-  if (e != cudaSuccess) return e;
-  if ((e = topk_dispatch(c, T, z, bias, idx, w, kCertifyMargin, unc, unc_n, nullptr, s)) !=
-      cudaSuccess)
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = topk_dispatch(c, T, z, bias, idx, w, kCertifyMargin, unc, unc_n, s)) != cudaSuccess)
     return e;
-  (void)err;
   return launch_refine(c, T, x, Wr, z, bias, idx, w, kCertifyMargin, unc, unc_n, s);
 }
 
