@@ -446,6 +446,22 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
     int pend[2] = {-1, -1};  // stages issued and not yet retired, oldest first (kLag used)
     bool live = true;
     for (int n = 0; live; ++n) {
+      // The scheduler may hold the next item back until gate/up tiles that
+      // this CTA is still finishing are published, and the MMA cannot finish
+      // them before their stages retire: if the next item is not queued yet,
+      // retire the pending stages before waiting for it.
+      const bool queued =
+          __shfl_sync(0xffffffffu, lane == 0 ? (mbar_try_wait(&qfull[n % kQueue], (n / kQueue) & 1) ? 1 : 0) : 0, 0) != 0;
+      if (!queued && (pend[0] >= 0 || pend[1] >= 0)) {
+        cp_async_wait<0>();
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if (pend[0] >= 0) mbar_arrive(&full[pend[0]]);
+          if (pend[1] >= 0) mbar_arrive(&full[pend[1]]);
+        }
+        pend[0] = pend[1] = -1;
+      }
       int item;
       if (!next_item(n, item, true)) break;
       bool gu;
@@ -500,7 +516,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
     __syncwarp();
     if (live && lane == 0) {
       if (pend[0] >= 0) mbar_arrive(&full[pend[0]]);
-      if (kLag == 2 && pend[1] >= 0) mbar_arrive(&full[pend[1]]);
+      if (pend[1] >= 0) mbar_arrive(&full[pend[1]]);
     }
   } else {
     // ------------------------------------------------------------ epilogue

@@ -189,6 +189,16 @@ def test_decode_full_size():
 
 
 @pytest.mark.slow
+@pytest.mark.parametrize("E", [64, 128])
+def test_decode_fewer_experts(E):
+    # several row tiles per expert at decode size: down items that wait on the
+    # gate/up tiles their own CTA is still finishing
+    cfg = workloads.CONFIGS["decode"].with_(E=E)
+    d = workloads.generate(cfg, DEV)
+    _full_check(cfg, d)
+
+
+@pytest.mark.slow
 @pytest.mark.parametrize("name", ["prefill", "prefill_bias0", "zipf", "mxfp4"])
 def test_full_size_sampled(name):
     cfg = workloads.CONFIGS[name]
