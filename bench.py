@@ -21,7 +21,6 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -97,60 +96,95 @@ def load_peaks():
 
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,utilization.gpu,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event reasons of this process's GPU, polled through NVML
+    every 2 ms while a timed loop runs (timed() windows), so that even a few
+    milliseconds of timed steps get samples."""
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.path = os.path.join("/tmp", f"sgl_clocks_{os.getpid()}.csv")
+    def __init__(self, device: str):
+        self.device = device
+        self.samples = []
+        self.active = False
+        self.stop = False
+        self.thread = None
+        self.nvml = None
+
+    def _handle(self):
+        import torch
+        nv = self.nvml
+        idx = torch.device(self.device).index or 0
+        try:
+            uuid = str(torch.cuda.get_device_properties(idx).uuid)
+            return nv.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(idx)
 
     def __enter__(self):
+        import threading
         try:
-            self.fh = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.fh,
-                stderr=subprocess.DEVNULL)
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = self._handle()
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.reason_fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+            self.masks = [(n, getattr(pynvml, a)) for n, a in self.REASONS]
         except Exception:
-            self.proc = None
+            self.nvml = None
+            return self
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
         return self
 
+    def _run(self):
+        nv = self.nvml
+        while not self.stop:
+            if self.active:
+                try:
+                    mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                    bits = self.reason_fn(self.h)
+                    self.samples.append((mhz, [n for n, m in self.masks if bits & m]))
+                except Exception:
+                    pass
+            time.sleep(0.002)
+
+    class _Window:
+        def __init__(self, owner):
+            self.owner = owner
+
+        def __enter__(self):
+            self.owner.active = True
+
+        def __exit__(self, *a):
+            self.owner.active = False
+
+    def timed(self):
+        return ClockSampler._Window(self)
+
     def __exit__(self, *a):
-        if self.proc is not None:
-            self.proc.terminate()
+        self.stop = True
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+        if self.nvml is not None:
             try:
-                self.proc.wait(timeout=5)
+                self.nvml.nvmlShutdown()
             except Exception:
-                self.proc.kill()
-            self.fh.close()
+                pass
 
     def summary(self):
-        if self.proc is None or not os.path.exists(self.path):
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
-        rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 9 and parts[1].isdigit():
-                    rows.append(parts)
-        try:
-            os.unlink(self.path)
-        except OSError:
-            pass
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        load = [r for r in rows if r[3].isdigit() and int(r[3]) > 0] or rows
-        reasons = set()
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        for r in load:
-            for n, v in zip(names, r[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(int(r[1]) for r in load),
-                "sm_max_mhz": max(int(r[2]) for r in rows if r[2].isdigit()),
-                "reasons": sorted(reasons), "samples": len(load)}
+        if self.nvml is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["no samples"],
+                    "samples": 0}
+        reasons = sorted({r for _, rs in self.samples for r in rs})
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples),
+                "source": "NVML, every 2 ms during the timed loops"}
 
 
 # ------------------------------------------------------------------ roofline arithmetic
@@ -185,6 +219,38 @@ def roofline_entry(bytes_, flops, seconds, peaks, sustained=False):
             "frac": round(ach / pk, 4)}
 
 
+# DRAM traffic of moe_ffn per algorithmic byte (dram__bytes_read.sum +
+# dram__bytes_write.sum over the bytes of algorithmic_work), from full ncu
+# captures of the same kernel on the small cases named in profiles/
+# (moe_ffn_decode_e128_t32.md: BN=16; moe_ffn_prefill_e128_t1024.md: BN=128).
+# Weight bytes dominate and scale with the experts touched, so the ratio
+# scales the counters to a full launch. Valid only for the ffn.cu they were
+# taken on: any other source reports traffic null.
+FFN_TRAFFIC_SOURCE_SHA256 = "fed4426034d42ce7cb4ae1a0d472869ff856ba64cb88c83bd8a24edb6c3e857f"
+FFN_TRAFFIC_RATIO = {16: (424.9 + 4.4) / 424.9, 128: (795.8 + 48.5) / 760.2}
+
+
+def ffn_tile_n(cfg) -> int:
+    """Token-tile width the library picks for a batch (same rule as choose_bn)."""
+    avg = cfg.T * cfg.K / cfg.E
+    return 16 if avg <= 12 else 32 if avg <= 24 else 64 if avg <= 48 else 128
+
+
+def ffn_traffic(cfg, algorithmic_bytes: float):
+    import hashlib
+    src = os.path.join(os.path.dirname(os.path.abspath(__file__)), "sigmoid_group_limited_b200",
+                       "csrc", "ffn.cu")
+    try:
+        with open(src, "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()
+    except OSError:
+        return None
+    ratio = FFN_TRAFFIC_RATIO.get(ffn_tile_n(cfg))
+    if digest != FFN_TRAFFIC_SOURCE_SHA256 or ratio is None or cfg.wfmt != workloads.MOE_W_BF16:
+        return None
+    return round(ratio * algorithmic_bytes)
+
+
 # ------------------------------------------------------------------ GPU arm
 
 STAGES = ("route", "permute", "gateup", "down", "combine")
@@ -200,7 +266,7 @@ def kernels_per_step(cfg) -> int:
     return n + (2 if cfg.wfmt == workloads.MOE_W_MXFP4 else 0)
 
 
-def measure_gpu(cfg, steps, warmup, device, rank, with_e2e=True):
+def measure_gpu(cfg, steps, warmup, device, rank, clk, with_e2e=True):
     import torch
 
     import sigmoid_group_limited_b200 as sgl
@@ -235,10 +301,11 @@ def measure_gpu(cfg, steps, warmup, device, rank, with_e2e=True):
     barrier(device)
     torch.cuda.synchronize(device)
     t0 = time.perf_counter()
-    for i in range(steps):
-        flush.zero_()
-        fwd(evs[i])
-    torch.cuda.synchronize(device)
+    with clk.timed():
+        for i in range(steps):
+            flush.zero_()
+            fwd(evs[i])
+        torch.cuda.synchronize(device)
     barrier(device)
     wall = time.perf_counter() - t0
     per_step_plain = [evs[i][0].elapsed_time(evs[i][5]) for i in range(steps)]
@@ -263,12 +330,13 @@ def measure_gpu(cfg, steps, warmup, device, rank, with_e2e=True):
     g1 = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     barrier(device)
     torch.cuda.synchronize(device)
-    for i in range(steps):
-        flush.zero_()
-        g0[i].record(stream)
-        graph.replay()
-        g1[i].record(stream)
-    torch.cuda.synchronize(device)
+    with clk.timed():
+        for i in range(steps):
+            flush.zero_()
+            g0[i].record(stream)
+            graph.replay()
+            g1[i].record(stream)
+        torch.cuda.synchronize(device)
     barrier(device)
     per_step = [g0[i].elapsed_time(g1[i]) for i in range(steps)]
     dev_ms = sum(per_step)
@@ -293,14 +361,15 @@ def measure_gpu(cfg, steps, warmup, device, rank, with_e2e=True):
             sgl.moe_layer_forward(cfg, xd, d["Wr"], d["bias"], W, y, ws, stream=stream)
             yh.copy_(y, non_blocking=True)
         torch.cuda.synchronize(device)
-        for i in range(steps):
-            flush.zero_()
-            e0[i].record(stream)
-            xd.copy_(xh, non_blocking=True)
-            sgl.moe_layer_forward(cfg, xd, d["Wr"], d["bias"], W, y, ws, stream=stream)
-            yh.copy_(y, non_blocking=True)
-            e1[i].record(stream)
-        torch.cuda.synchronize(device)
+        with clk.timed():
+            for i in range(steps):
+                flush.zero_()
+                e0[i].record(stream)
+                xd.copy_(xh, non_blocking=True)
+                sgl.moe_layer_forward(cfg, xd, d["Wr"], d["bias"], W, y, ws, stream=stream)
+                yh.copy_(y, non_blocking=True)
+                e1[i].record(stream)
+            torch.cuda.synchronize(device)
         out["e2e_ms_total"] = sum(e0[i].elapsed_time(e1[i]) for i in range(steps))
         out["launches"] += kernels_per_step(cfg) * steps
         out["e2e_h2d"] = T * cfg.H * 2
@@ -443,12 +512,13 @@ def run_native(args, rank, world, local):
     torch.cuda.set_device(device)
     peaks = load_peaks()
     cfg = workload_cfg(args)
-    with ClockSampler(local) as clk:
-        m = measure_gpu(cfg, args.steps, args.warmup, device, rank)
+    with ClockSampler(device) as clk:
+        m = measure_gpu(cfg, args.steps, args.warmup, device, rank, clk)
         also = None
         if args.also and args.also != args.workload:
             acfg = workloads.CONFIGS[args.also]
-            also = (acfg, measure_gpu(acfg, args.steps, args.warmup, device, rank, with_e2e=False))
+            also = (acfg, measure_gpu(acfg, args.steps, args.warmup, device, rank, clk,
+                                      with_e2e=False))
     clocks = clk.summary()
     dev_s = reduce_max(m["device_ms_total"], device) / 1e3
     plain_s = reduce_max(m["plain_ms_total"], device) / 1e3
@@ -462,7 +532,9 @@ def run_native(args, rank, world, local):
         f = work["gateup"][1] + work["down"][1]
         t_ffn = (mm["stage_ms"]["ffn"]) / 1e3
         ent = roofline_entry(b, f, t_ffn, peaks)
-        ent.update(kernel="moe_ffn (gate/up + down)", traffic=None,
+        ent.update(kernel="moe_ffn (gate/up + down)", traffic=ffn_traffic(cfg_, b),
+                   traffic_unit="bytes per launch (ncu DRAM read+write, scaled from the "
+                                "small-case capture of the same kernel)",
                    peak_source=f"{peaks['source']} ({'HBM copy' if ent['bound'] == 'hbm' else 'cuBLAS bf16 burst'})",
                    units_per_launch=f"{cfg_.T} tokens, {mm['touched']} routed experts + shared")
         lb, lf = work["layer"]

@@ -870,9 +870,11 @@ cudaError_t topk_dispatch(const moe_cfg& c, int T, const float* z, const float* 
                           cudaStream_t s) {
   const int nv = cdiv(c.E, 32);
   const int per = c.E / c.n_group;
-  if ((per == 32 || per == 64) && c.n_group <= kSelMaxGroups && c.K + 1 <= kSelMaxCand &&
-      c.topk_group * (c.K + 1) <= 64) {
-    const int grid = std::min(T, num_sms() * 8);
+  // small batches: a CTA per token (its groups in parallel); larger ones keep
+  // the warp per token, which has more tokens in flight per SM
+  if (T <= 4 * num_sms() && (per == 32 || per == 64) && c.n_group <= kSelMaxGroups &&
+      c.K + 1 <= kSelMaxCand && c.topk_group * (c.K + 1) <= 64) {
+    const int grid = T;
     if (per == 32)
       router_select<1><<<grid, c.n_group * 32, 0, s>>>(T, c.E, c.n_group, c.topk_group, c.K,
                                                        c.scale, c.renorm, z, bias, idx, w, tau,

@@ -234,11 +234,13 @@ def test_all_scores_tied(T):
     assert torch.all(w == 0.3125)
 
 
-@pytest.mark.parametrize("T", [32, 4096])
-def test_route_full_size_every_token(T):
-    """Routing of every token at full size, bit-exact outside listed near ties."""
-    cfg = workloads.CONFIGS["prefill"]
-    g = torch.Generator(device=DEV).manual_seed(77 + T)
+@pytest.mark.parametrize("T,E", [(32, 512), (4096, 512), (32, 256), (700, 256), (32, 128)])
+def test_route_full_size_every_token(T, E):
+    """Routing of every token at full size, bit-exact outside listed near ties.
+    Groups of 64 (E=512) and 32 (E=256) experts take the CTA-per-token
+    selection at small T; groups of 16 (E=128) the warp-per-token one."""
+    cfg = workloads.CONFIGS["prefill"].with_(E=E)
+    g = torch.Generator(device=DEV).manual_seed(77 + T + E)
     x = torch.randn(T, cfg.H, device=DEV, generator=g).to(torch.bfloat16)
     Wr = torch.randn(cfg.E, cfg.H, device=DEV, generator=g) / cfg.H ** 0.5
     bias = torch.randn(cfg.E, device=DEV, generator=g) * 0.1 ** 0.5
