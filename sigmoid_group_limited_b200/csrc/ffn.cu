@@ -28,13 +28,14 @@
 // gate/up item runs on its CTA's pipeline whatever that CTA's scheduler is
 // waiting for, so every wait ends.
 //
-// Warp roles per CTA (352 threads):
+// Warp roles per CTA (480 threads):
 //   0      TMA producer (lane 0): weight tiles, and h tiles of down items
 //   1      MMA issuer (lane 0), owner of the TMEM accumulators
-//   2..5   epilogue (TMEM lane quarter warp % 4)
-//   6..9   token gatherers: cp.async of the routed x rows into the swizzled
+//   2..9   epilogue: two warps per TMEM lane quarter (warp % 4), alternate
+//          column chunks
+//   10..13 token gatherers: cp.async of the routed x rows into the swizzled
 //          B tile of gate/up stages
-//   10     scheduler (lane 0): claims the next item while the current one is
+//   14     scheduler (lane 0): claims the next item while the current one is
 //          still streaming, waits for its inputs, and queues it for the others
 // Pipelines: STAGES shared-memory stages (full / empty mbarriers), two TMEM
 // accumulator buffers (tfull / tempty) so the epilogue of one item overlaps
@@ -48,14 +49,17 @@
 #include <stdint.h>
 #include <string.h>
 
+#include "ffn_common.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 
 namespace sgl {
 namespace {
 
-constexpr int kGatherWarps = 4;
-constexpr int kSchedWarp = 10;
+constexpr int kEpiWarps = 8;      // warps 2..9: two per TMEM lane quarter
+constexpr int kGatherWarp0 = 2 + kEpiWarps;
+constexpr int kGatherWarps = 4;   // warps 10..13
+constexpr int kSchedWarp = kGatherWarp0 + kGatherWarps;  // warp 14
 constexpr int kFfnThreads = 32 * (kSchedWarp + 1);
 constexpr int kQueue = 4;                 // item queue entries
 constexpr int kLead = 4;                  // claim the next item this many k-blocks early
@@ -82,111 +86,6 @@ struct Cfg {
   static_assert(8 * (2 * 8 + 2 * 2 + 2 * kQueue) + 8 + 4 * (2 + kQueue) <= CTRL_BYTES,
                 "control block");
 };
-
-struct FfnParams {
-  int T, K, E, H, I, Is;
-  int has_shared;
-  float lim_r, lim_s;        // <= 0: no limit
-  const uint16_t* x;         // [T, H]
-  const int32_t* perm;       // [T*K] sorted position -> flat slot j
-  const float* w;            // [T*K] routing weights
-  uint16_t* h_r;             // [T*K, I] permuted rows
-  uint16_t* h_s;             // [T, Is]
-  float* y_slot;             // [(T*K + T), H] fp32
-  const int32_t* offsets;    // [E+1]
-  const int32_t* wslot;      // nullable: weight row block of expert e
-  const int32_t* gu_start;   // [E+2]
-  const int32_t* dn_start;   // [E+2]
-  const int32_t* nitems;     // [2] item totals; [2] is the claim counter
-  int32_t* counter;
-  int32_t* ready;            // [max_gu] finished gate/up tiles per (slot, row tile)
-  int max_gu, max_dn;
-  int32_t* err;
-};
-
-__device__ __forceinline__ void epilogue_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-
-__device__ __forceinline__ float clampL(float v, float L) {
-  return L > 0.f ? fminf(fmaxf(v, -L), L) : v;
-}
-
-__device__ __forceinline__ uint16_t f2bf(float v) {
-  return __bfloat16_as_ushort(__float2bfloat16_rn(v));
-}
-
-__device__ __forceinline__ void fence_proxy_async_global() {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
-__device__ __forceinline__ int ld_acquire(const int32_t* a) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
-  return v;
-}
-
-// Bounded wait until *addr >= need (acquire), with mbar_wait's abort protocol.
-__device__ __forceinline__ bool wait_count(const int32_t* addr, int need, volatile int* abort_flag,
-                                           int* err) {
-  const long long t0 = clock64();
-  while (ld_acquire(addr) < need) {
-    if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitLimitCycles) {
-      *abort_flag = 1;
-      atomicExch(err, MOE_DEVERR_TIMEOUT);
-      return false;
-    }
-    __nanosleep(100);
-  }
-  return true;
-}
-
-// Bounded wait until the producer's progress word reaches `need`.
-__device__ __forceinline__ bool wait_progress(const volatile long long* prog, long long need,
-                                              volatile int* abort_flag, int* err) {
-  const long long t0 = clock64();
-  while (*prog < need) {
-    if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitLimitCycles) {
-      *abort_flag = 1;
-      atomicExch(err, MOE_DEVERR_TIMEOUT);
-      return false;
-    }
-    __nanosleep(32);
-  }
-  return true;
-}
-
-// Same validity rule in every role, so all roles skip the same items.
-__device__ __forceinline__ bool item_ok(const FfnParams& p, const WorkItem& it, bool gu, int bn) {
-  const bool sh = it.e == p.E;
-  if (it.e < 0 || it.e > p.E || (sh && !p.has_shared)) return false;
-  if (it.nrows <= 0 || it.nrows > bn || it.row0 < 0) return false;
-  if (it.row0 + it.nrows > (sh ? p.T : p.T * p.K)) return false;
-  if (it.ntile < 0) return false;
-  return gu ? it.ntile * kTileN < (sh ? p.Is : p.I) : it.ntile * kDownTile < p.H;
-}
-
-// Work item `i` of one kind from its per-slot item prefix sums (in shared
-// memory): the slot is the last one whose first item is <= i; within a slot
-// the row tile varies fastest, so CTAs that run at the same time share a
-// weight tile in L2.
-__device__ __forceinline__ WorkItem decode_item(int i, const int* s_start, const int* s_off,
-                                                int nslots, int E, int T, int bn) {
-  int lo = 0, hi = nslots;
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (s_start[mid] <= i) lo = mid;
-    else hi = mid;
-  }
-  const int e = lo;
-  const bool sh = e == E;
-  const int rows = sh ? T : s_off[e + 1] - s_off[e];
-  const int r0 = sh ? 0 : s_off[e];
-  const int nm = max(1, (rows + bn - 1) / bn);
-  const int local = i - s_start[e];
-  const int n = local / nm, m = local - n * nm;
-  return WorkItem{e, r0 + m * bn, min(bn, rows - m * bn), n};
-}
 
 template <int BN>
 __global__ void __launch_bounds__(kFfnThreads, 1)
@@ -224,11 +123,11 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4);
+      mbar_init(&tempty[a], kEpiWarps);
     }
     for (int q = 0; q < kQueue; ++q) {
       mbar_init(&qfull[q], 1);
-      mbar_init(&qempty[q], 1 + 1 + 4 + kGatherWarps);  // producer, MMA, epilogue, gatherers
+      mbar_init(&qempty[q], 1 + 1 + kEpiWarps + kGatherWarps);  // producer, MMA, epilogue, gatherers
     }
     *prog = 0;
     *abort_flag = 0;
@@ -424,7 +323,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp >= 6) {
+  } else if (warp >= kGatherWarp0) {
     // ------------------------------------------------------------ token gatherers
     // Gate/up items: thread g copies 16-byte chunk (g % 8) of rows g/8,
     // g/8 + 16, ... of the stage's BN x 64 token tile straight into the
@@ -438,7 +337,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
     // one when the ring has only three stages (else the MMA would never run
     // ahead of the gatherers)
     constexpr int kLag = C::STAGES >= 4 ? 2 : 1;
-    const int g = tid - 6 * 32;
+    const int g = tid - kGatherWarp0 * 32;
     const int chunk = g & 7, rbase = g >> 3;
     const uint64_t pol_x = policy_evict_last();
     int stage = 0;
@@ -522,6 +421,9 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;            // TMEM lane quarter of this warp
     const int orow = q * 32 + lane;    // output feature within a 128-row half
+    const int et = tid - 2 * 32;       // epilogue thread 0..255
+    const int cpart = et >> 7;         // which of the two warps of the quarter: column chunks
+    constexpr int kEpiThreads = 32 * kEpiWarps;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int n = 0;; ++n) {
@@ -534,8 +436,8 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
       if (!gu) {
         // destination slot and routing weight of every row, staged while the
         // item's MMAs run (the store loop then touches no metadata in global)
-        epilogue_bar();  // all four warps are done with the previous item's rows
-        for (int rr = orow; rr < BN; rr += 4 * 32) {
+        epi_bar<kEpiThreads>();  // every epilogue warp is done with the previous item's rows
+        for (int rr = et; rr < BN; rr += kEpiThreads) {
           int j = -1;
           float wt = 0.f;
           if (rr < it.nrows) {
@@ -556,7 +458,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
           meta_j[rr] = j;
           meta_w[rr] = wt;
         }
-        epilogue_bar();
+        epi_bar<kEpiThreads>();
       }
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) break;
       tc_fence_after();
@@ -568,8 +470,9 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
         const float L = sh ? p.lim_s : p.lim_r;
         uint16_t* hout = sh ? p.h_s : p.h_r;
         const int ncol = mma_n(it);
+        // the two warps of a lane quarter take alternate 16-column chunks
 #pragma unroll 1
-        for (int c0 = 0; c0 < ncol; c0 += 16) {
+        for (int c0 = 16 * cpart; c0 < ncol; c0 += 32) {
           float gv[16], uv[16];
           tmem_ld16(taddr + c0, gv);
           tmem_ld16(taddr + BN + c0, uv);
@@ -578,11 +481,8 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
               const int r = c0 + c;
-              if (r < it.nrows) {
-                const float gg = clampL(gv[c], L), uu = clampL(uv[c], L);
-                hout[static_cast<size_t>(it.row0 + r) * ncols + nfeat] =
-                    f2bf((gg / (1.0f + expf(-gg))) * uu);
-              }
+              if (r < it.nrows)
+                hout[static_cast<size_t>(it.row0 + r) * ncols + nfeat] = f2bf(swiglu(gv[c], uv[c], L));
             }
           }
         }
@@ -592,14 +492,18 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
         for (int half = 0; half < 2; ++half) {
           const int nfeat = it.ntile * kDownTile + half * kTileN + orow;
           const bool ok = nfeat < p.H;
+          // kCols columns per TMEM wait (the loads of one group are in flight
+          // together); the two warps of a lane quarter take alternate groups
+          constexpr int kCols = BN >= 32 ? 32 : 16;
 #pragma unroll 1
-          for (int c0 = 0; c0 < ncol; c0 += 16) {
-            float ov[16];
-            tmem_ld16(taddr + half * BN + c0, ov);
+          for (int c0 = kCols * cpart; c0 < ncol; c0 += 2 * kCols) {
+            float ov[kCols];
+#pragma unroll
+            for (int u = 0; u < kCols; u += 16) tmem_ld16(taddr + half * BN + c0 + u, ov + u);
             tmem_ld_wait();
             if (ok) {
 #pragma unroll
-              for (int c = 0; c < 16; ++c) {
+              for (int c = 0; c < kCols; ++c) {
                 const int j = meta_j[c0 + c];
                 if (j >= 0) p.y_slot[static_cast<size_t>(j) * p.H + nfeat] = meta_w[c0 + c] * ov[c];
               }
@@ -617,7 +521,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
       if (gu) {
         // publish this output tile of h: stores -> async proxy -> CTA -> GPU
         fence_proxy_async_global();
-        epilogue_bar();
+        epi_bar<kEpiThreads>();
         if (warp == 2 && lane == 0) {
           __threadfence();
           const int r0 = sh ? 0 : s_off[it.e];
@@ -711,6 +615,7 @@ cudaError_t launch_ffn(const GemmArgs& a, cudaStream_t s) {
     case 32: return launch_bn<32>(a, s);
     case 64: return launch_bn<64>(a, s);
     case 128: return launch_bn<128>(a, s);
+    case kPairTileN: return launch_ffn_pair(a, s);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -1,0 +1,132 @@
+// ffn_common.cuh - parameters and device helpers shared by the two expert-FFN
+// kernels (ffn.cu: one CTA per item; ffn_pair.cu: a CTA pair per item).
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace sgl {
+namespace {
+
+struct FfnParams {
+  int T, K, E, H, I, Is;
+  int has_shared;
+  float lim_r, lim_s;        // <= 0: no limit
+  const uint16_t* x;         // [T, H]
+  const int32_t* perm;       // [T*K] sorted position -> flat slot j
+  const float* w;            // [T*K] routing weights
+  uint16_t* h_r;             // [T*K, I] permuted rows
+  uint16_t* h_s;             // [T, Is]
+  float* y_slot;             // [(T*K + T), H] fp32
+  const int32_t* offsets;    // [E+1]
+  const int32_t* wslot;      // nullable: weight row block of expert e
+  const int32_t* gu_start;   // [E+2]
+  const int32_t* dn_start;   // [E+2]
+  const int32_t* nitems;     // [2] item totals; [2] is the claim counter
+  int32_t* counter;
+  int32_t* ready;            // [max_gu] finished gate/up tiles per (slot, row tile)
+  int max_gu, max_dn;
+  int32_t* err;
+};
+
+__device__ __forceinline__ float clampL(float v, float L) {
+  return L > 0.f ? fminf(fmaxf(v, -L), L) : v;
+}
+
+// Named barrier 1 over the epilogue warps (NT threads).
+template <int NT>
+__device__ __forceinline__ void epi_bar() {
+  asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory");
+}
+
+// silu(g) * u after the clamp, with the hardware exponential and a rounded
+// reciprocal (h is rounded to bf16 right after).
+__device__ __forceinline__ float swiglu(float g, float u, float L) {
+  const float gg = clampL(g, L), uu = clampL(u, L);
+  return gg * __frcp_rn(1.0f + __expf(-gg)) * uu;
+}
+
+
+__device__ __forceinline__ uint16_t f2bf(float v) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
+
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__device__ __forceinline__ int ld_acquire(const int32_t* a) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
+  return v;
+}
+
+// Bounded wait until *addr >= need (acquire), with mbar_wait's abort protocol.
+__device__ __forceinline__ bool wait_count(const int32_t* addr, int need, volatile int* abort_flag,
+                                           int* err) {
+  const long long t0 = clock64();
+  while (ld_acquire(addr) < need) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitLimitCycles) {
+      *abort_flag = 1;
+      atomicExch(err, MOE_DEVERR_TIMEOUT);
+      return false;
+    }
+    __nanosleep(100);
+  }
+  return true;
+}
+
+// Bounded wait until the producer's progress word reaches `need`.
+__device__ __forceinline__ bool wait_progress(const volatile long long* prog, long long need,
+                                              volatile int* abort_flag, int* err) {
+  const long long t0 = clock64();
+  while (*prog < need) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitLimitCycles) {
+      *abort_flag = 1;
+      atomicExch(err, MOE_DEVERR_TIMEOUT);
+      return false;
+    }
+    __nanosleep(32);
+  }
+  return true;
+}
+
+// Same validity rule in every role, so all roles skip the same items.
+__device__ __forceinline__ bool item_ok(const FfnParams& p, const WorkItem& it, bool gu, int bn) {
+  const bool sh = it.e == p.E;
+  if (it.e < 0 || it.e > p.E || (sh && !p.has_shared)) return false;
+  if (it.nrows <= 0 || it.nrows > bn || it.row0 < 0) return false;
+  if (it.row0 + it.nrows > (sh ? p.T : p.T * p.K)) return false;
+  if (it.ntile < 0) return false;
+  return gu ? it.ntile * kTileN < (sh ? p.Is : p.I) : it.ntile * kDownTile < p.H;
+}
+
+// Work item `i` of one kind from its per-slot item prefix sums (in shared
+// memory): the slot is the last one whose first item is <= i; within a slot
+// the row tile varies fastest, so CTAs that run at the same time share a
+// weight tile in L2.
+__device__ __forceinline__ WorkItem decode_item(int i, const int* s_start, const int* s_off,
+                                                int nslots, int E, int T, int bn) {
+  int lo = 0, hi = nslots;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (s_start[mid] <= i) lo = mid;
+    else hi = mid;
+  }
+  const int e = lo;
+  const bool sh = e == E;
+  const int rows = sh ? T : s_off[e + 1] - s_off[e];
+  const int r0 = sh ? 0 : s_off[e];
+  const int nm = max(1, (rows + bn - 1) / bn);
+  const int local = i - s_start[e];
+  const int n = local / nm, m = local - n * nm;
+  return WorkItem{e, r0 + m * bn, min(bn, rows - m * bn), n};
+}
+
+}  // namespace
+}  // namespace sgl

@@ -1,0 +1,553 @@
+// ffn_pair.cu - stages 7 and 8 for large batches: the grouped SwiGLU experts
+// and the shared expert on CTA pairs (tcgen05 cta_group::2).
+//
+// Page "Ling-3.0-flash-VL MoE sparse routing" (lqnn.cn/news/282163): sec. 2
+// (an expert is a gate / up / down SwiGLU FFN, hidden 2560, intermediate 768;
+// one shared expert sees every token) and sec. 4 (SwiGLU limits).
+//
+// Same items and scheduling as ffn.cu, but each item runs on a pair of CTAs
+// (a cluster of two) that issue one M = 256 MMA: each CTA holds 128 rows of A
+// and half of the item's N token rows of B, and gets its 128 rows of D in its
+// own TMEM. Per CTA and 64-wide k-block that is 16 KB of A and up to 16 KB of
+// B for up to 256 x 256 x 64 MACs of the pair: twice the flops per byte of
+// shared-memory fill of a single CTA with 128-token tiles, with the
+// accumulators still double-buffered (two 256-column buffers).
+//   gate/up item (slot, 256-token tile, 128 features f0..f0+127): CTA r holds
+//       gate rows f0 + 64r .. +63 over up rows f0 + 64r .. +63 (lanes 0-63 /
+//       64-127 of its D); the epilogue pairs lane l with lane l + 64 through
+//       shared memory. B = the item's rows of the token matrix gathered into
+//       routed-row order beforehand (x_perm), or x itself for the shared expert.
+//   down item (slot, 256-token tile, 256 hidden features): CTA r holds Wd rows
+//       256 n + 128 r .. +127; B = h rows.
+// Both operands arrive by TMA (no multicast): each CTA loads its own halves
+// and the byte counts complete on the leader CTA's full barrier; the leader's
+// MMA thread releases a stage in both CTAs with one multicast commit.
+//
+// Warp roles per CTA (352 threads):
+//   0     TMA producer (lane 0), both CTAs
+//   1     TMEM allocation in both CTAs; MMA issuer (lane 0) in the leader
+//   2..9  epilogue, both CTAs: two warps per TMEM lane quarter (warp % 4),
+//         alternate column chunks
+//   10    scheduler (lane 0), leader: claims items, waits for their inputs
+//         and writes them into the item queues of both CTAs
+// Barriers filled by TMA bytes or by tcgen05.commit are waited on at CTA
+// scope; the ones other threads of the pair arrive on (item queues, the
+// leader's accumulator-empty barriers) at cluster scope.
+// Every wait is bounded; the two CTAs meet at a cluster barrier after setup
+// and before exit, so no CTA touches the other's shared memory after it left.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "ffn_common.cuh"
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace sgl {
+namespace {
+
+constexpr int kPEpiWarps = 8;              // warps 2..9, two per TMEM lane quarter
+constexpr int kPEpiThreads = 32 * kPEpiWarps;
+constexpr int kPSchedWarp = 2 + kPEpiWarps;
+constexpr int kPThreads = 32 * (kPSchedWarp + 1);
+constexpr int kPQueue = 4;
+constexpr int kPLead = 4;                  // claim the next item this many k-blocks early
+constexpr long long kPProgStride = 1024;
+constexpr int kPStages = 6;
+constexpr int kPA = 128 * 128;             // A half: 128 rows x 64 bf16
+constexpr int kPB = kPairTileN / 2 * 128;  // B half: up to 128 rows x 64 bf16
+constexpr int kPStage = kPA + kPB;
+constexpr int kPBox = 32;                  // token rows per B box
+constexpr int kPAccCols = kPairTileN;      // fp32 columns of one accumulator
+constexpr int kPTmemCols = 2 * kPAccCols;  // two buffers
+constexpr int kPCtrl = 512;
+constexpr int kPXchRow = 9;                // 8 floats + 1 (bank spread)
+constexpr int kPXchFloats = 2 * 2 * 64 * kPXchRow;  // [column part][gate/up][feature][8]
+constexpr int kPSmem = kPStages * kPStage + 1024 + kPCtrl + kPXchFloats * 4 + kPairTileN * 8;
+static_assert(kPTmemCols <= 512, "TMEM");
+// consumers of a queue entry, counted on the leader's qempty: leader producer,
+// MMA and epilogue warps; peer producer and epilogue warps
+constexpr int kPQueueConsumers = 1 + 1 + kPEpiWarps + 1 + kPEpiWarps;
+
+// MMA N of an item: its rows rounded up to 64 (each CTA then holds a whole
+// number of 32-row boxes of B)
+__device__ __forceinline__ int pair_n(const WorkItem& it) {
+  return (min(it.nrows, kPairTileN) + 63) & ~63;
+}
+
+struct PairMaps {
+  CUtensorMap wg, wu, wgs, wus;  // gate / up rows, 64-row boxes
+  CUtensorMap wd, wds;           // down rows, 128-row boxes
+  CUtensorMap xp, x;             // token rows (routed order / token order), 32-row boxes
+  CUtensorMap h, hs;             // h rows, 32-row boxes
+};
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
+    moe_ffn_pair(const __grid_constant__ FfnParams p, const __grid_constant__ PairMaps m) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* ctrl = smem + kPStages * kPStage;
+  uint64_t* full = reinterpret_cast<uint64_t*>(ctrl);  // [kPStages] (the leader's count)
+  uint64_t* empty = full + kPStages;                    // [kPStages]
+  uint64_t* tfull = empty + kPStages;                   // [2]
+  uint64_t* tempty = tfull + 2;                         // [2] (the leader's count)
+  uint64_t* qfull = tempty + 2;                         // [kPQueue]
+  uint64_t* qempty = qfull + kPQueue;                   // [kPQueue] (the leader's count)
+  volatile long long* prog = reinterpret_cast<volatile long long*>(qempty + kPQueue);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(const_cast<long long*>(prog) + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* qitem = abort_flag + 1;  // [kPQueue]
+  float* xch = reinterpret_cast<float*>(ctrl + kPCtrl);             // [kPXchFloats]
+  int* meta_j = reinterpret_cast<int*>(xch + kPXchFloats);          // [kPairTileN]
+  float* meta_w = reinterpret_cast<float*>(meta_j + kPairTileN);    // [kPairTileN]
+  int* s_gu = reinterpret_cast<int*>(meta_w + kPairTileN);          // [E+2]
+  int* s_dn = s_gu + (p.E + 2);                                      // [E+2]
+  int* s_off = s_dn + (p.E + 2);                                     // [E+1]
+  static_assert(8 * (2 * kPStages + 4 + 2 * kPQueue) + 8 + 4 * (2 + kPQueue) <= kPCtrl, "ctrl");
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_ctarank() & 1u;
+  const bool leader = rank == 0;
+  if (tid == 0) {
+    for (int s = 0; s < kPStages; ++s) {
+      mbar_init(&full[s], 1);   // the leader's expect_tx arrival (+ both CTAs' bytes)
+      mbar_init(&empty[s], 1);  // the leader's multicast commit
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);   // multicast commit
+      mbar_init(&tempty[a], 2 * kPEpiWarps);  // the epilogue warps of both CTAs
+    }
+    for (int q = 0; q < kPQueue; ++q) {
+      mbar_init(&qfull[q], 1);
+      mbar_init(&qempty[q], kPQueueConsumers);
+    }
+    *prog = 0;
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&m.wg);
+    prefetch_tmap(&m.wd);
+    prefetch_tmap(&m.xp);
+    prefetch_tmap(&m.h);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, kPTmemCols);
+    tmem_relinquish_pair();
+  }
+  for (int i = tid; i < p.E + 2; i += blockDim.x) {
+    s_gu[i] = p.gu_start[i];
+    s_dn[i] = p.dn_start[i];
+  }
+  for (int i = tid; i < p.E + 1; i += blockDim.x) s_off[i] = p.offsets[i];
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before any remote arrival
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int nslots = p.E + (p.has_shared ? 1 : 0);
+  const int n_gu = min(p.nitems[0], p.max_gu);
+  const int n_dn = min(p.nitems[1], p.max_dn);
+  const int n_all = n_gu + n_dn;
+  auto item_at = [&](int i, bool& gu) {
+    gu = i < n_gu;
+    return gu ? decode_item(i, s_gu, s_off, nslots, p.E, p.T, kPairTileN)
+              : decode_item(i - n_gu, s_dn, s_off, nslots, p.E, p.T, kPairTileN);
+  };
+  const int KB_gu = p.H / 64, KB_dn_r = p.I / 64, KB_dn_s = p.Is / 64;
+  auto nkb_of = [&](bool gu, bool sh) { return gu ? KB_gu : (sh ? KB_dn_s : KB_dn_r); };
+  // the leader's copy of a barrier, as a cluster address
+  auto at_leader = [&](uint64_t* bar) { return mapa_shared(smem_u32(bar), 0); };
+  // queue entry n: wait, read, release (one arrival per warp, on the leader's qempty)
+  auto next_item = [&](int n, int& item, bool whole_warp) -> bool {
+    const int q = n % kPQueue;
+    if (!mbar_wait_cluster(&qfull[q], (n / kPQueue) & 1, abort_flag, p.err, MOE_DEVERR_TIMEOUT))
+      return false;
+    item = qitem[q];
+    if (whole_warp) __syncwarp();
+    if (lane == 0) {
+      if (leader) mbar_arrive(&qempty[q]);
+      else mbar_arrive_cluster(at_leader(&qempty[q]));
+    }
+    return item >= 0;
+  };
+
+  if (warp == kPSchedWarp) {
+    // ------------------------------------------------------------ scheduler (leader)
+    if (leader && lane == 0) {
+      int prev_nkb = 0;
+      for (int n = 0;; ++n) {
+        const int q = n % kPQueue;
+        if (!mbar_wait_cluster(&qempty[q], ((n / kPQueue) & 1) ^ 1, abort_flag, p.err,
+                               MOE_DEVERR_TIMEOUT))
+          break;
+        // claim item n when the producer is kPLead k-blocks from the end of item n-1
+        if (n > 0 && !wait_progress(prog, (n - 1) * kPProgStride + max(0, prev_nkb - kPLead),
+                                    abort_flag, p.err))
+          break;
+        int item = atomicAdd(p.counter, 1);
+        if (item >= n_all) item = -1;
+        prev_nkb = 0;
+        if (item >= 0) {
+          bool gu;
+          const WorkItem it = item_at(item, gu);
+          if (item_ok(p, it, gu, kPairTileN)) {
+            const bool sh = it.e == p.E;
+            prev_nkb = nkb_of(gu, sh);
+            if (!gu) {
+              // both halves of every gate/up output tile of this (slot, row tile) are in h
+              const int r0 = sh ? 0 : s_off[it.e];
+              const int ridx = s_gu[it.e] + (it.row0 - r0) / kPairTileN;
+              if (!wait_count(p.ready + ridx, 2 * cdiv_dev(sh ? p.Is : p.I, kTileN), abort_flag,
+                              p.err))
+                item = -1;
+            }
+          } else {
+            atomicExch(p.err, MOE_DEVERR_SCHEDULE);
+          }
+        }
+        // the peer's copy first, then both arrivals (release at cluster scope)
+        st_shared_cluster(mapa_shared(smem_u32(const_cast<int*>(&qitem[q])), 1), item);
+        qitem[q] = item;
+        mbar_arrive_cluster(mapa_shared(smem_u32(&qfull[q]), 1));
+        mbar_arrive(&qfull[q]);
+        if (item < 0) break;
+      }
+    }
+    __syncwarp();
+  } else if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_b = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      bool live = true;
+      for (int n = 0; live; ++n) {
+        int item;
+        if (!next_item(n, item, false)) break;
+        if (leader) *prog = n * kPProgStride;
+        bool gu;
+        const WorkItem it = item_at(item, gu);
+        if (!item_ok(p, it, gu, kPairTileN)) continue;
+        const bool sh = it.e == p.E;
+        // h rows of a down item were published by other CTAs (acquired by the
+        // leader's scheduler, released to this CTA through the queue)
+        if (!gu) fence_proxy_async_global();
+        const int wblk = sh ? 0 : (p.wslot ? p.wslot[it.e] : it.e);
+        const int nkb = nkb_of(gu, sh);
+        const int nhalf = pair_n(it) / 2;       // this CTA's B rows
+        const int nbox = nhalf / kPBox;
+        const int brow = it.row0 + static_cast<int>(rank) * nhalf;
+        const uint32_t pair_bytes = 2u * (kPA + nbox * kPBox * 128);
+        const CUtensorMap* mb = gu ? (sh ? &m.x : &m.xp) : (sh ? &m.hs : &m.h);
+        int arow0, arow1 = 0;
+        const CUtensorMap *ma0, *ma1 = nullptr;
+        if (gu) {
+          const int f = it.ntile * kTileN + static_cast<int>(rank) * 64;
+          arow0 = (sh ? 0 : wblk * p.I) + f;
+          arow1 = arow0;
+          ma0 = sh ? &m.wgs : &m.wg;
+          ma1 = sh ? &m.wus : &m.wu;
+        } else {
+          arow0 = (sh ? 0 : wblk * p.H) + it.ntile * kDownTile + static_cast<int>(rank) * kTileN;
+          ma0 = sh ? &m.wds : &m.wd;
+        }
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) {
+            live = false;
+            break;
+          }
+          uint8_t* sA = smem + stage * kPStage;
+          uint8_t* sB = sA + kPA;
+          const uint32_t lbar = at_leader(&full[stage]);
+          if (leader) mbar_arrive_expect_tx(&full[stage], pair_bytes);
+          if (gu) {
+            tma_load_2d_pair(sA, ma0, lbar, kb * 64, arow0, pol_w);               // gate rows
+            tma_load_2d_pair(sA + kPA / 2, ma1, lbar, kb * 64, arow1, pol_w);     // up rows
+          } else {
+            tma_load_2d_pair(sA, ma0, lbar, kb * 64, arow0, pol_w);
+          }
+          for (int b = 0; b < nbox; ++b)
+            tma_load_2d_pair(sB + b * kPBox * 128, mb, lbar, kb * 64, brow + b * kPBox, pol_b);
+          if (leader) *prog = n * kPProgStride + kb + 1;
+          if (++stage == kPStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      // every stage must be released by the MMA before teardown
+      for (int i = 0; i < kPStages && live; ++i) {
+        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, MOE_DEVERR_TIMEOUT))
+          break;
+        if (++stage == kPStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader)
+    if (leader && lane == 0) {
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool live = true;
+      for (int n = 0; live; ++n) {
+        int item;
+        if (!next_item(n, item, false)) break;
+        bool gu;
+        const WorkItem it = item_at(item, gu);
+        if (!item_ok(p, it, gu, kPairTileN)) continue;
+        const int nkb = nkb_of(gu, it.e == p.E);
+        const uint32_t idesc = idesc_bf16(2 * kTileN, pair_n(it));
+        if (!mbar_wait_cluster(&tempty[acc], acc_phase ^ 1, abort_flag, p.err, MOE_DEVERR_TIMEOUT))
+          break;
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + acc * kPAccCols;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) {
+            live = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + stage * kPStage);
+          const uint32_t b0 = a0 + kPA;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16_pair(d0, sdesc_k128(a0 + kk * 32), sdesc_k128(b0 + kk * 32), idesc,
+                           (kb | kk) != 0 ? 1u : 0u);
+          umma_commit_pair_mc(&empty[stage], 0x3);  // frees the stage in both CTAs
+          if (++stage == kPStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!live) break;
+        umma_commit_pair_mc(&tfull[acc], 0x3);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1;
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 2 && warp < 2 + kPEpiWarps) {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp & 3;            // TMEM lane quarter
+    const int orow = q * 32 + lane;    // row of this CTA's D
+    const int et = tid - 64;           // epilogue thread 0..255
+    const int cpart = et >> 7;         // column chunks of this warp: alternate ones
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int n = 0;; ++n) {
+      int item;
+      if (!next_item(n, item, true)) break;
+      bool gu;
+      const WorkItem it = item_at(item, gu);
+      if (!item_ok(p, it, gu, kPairTileN)) continue;
+      const bool sh = it.e == p.E;
+      const int ncol = pair_n(it);
+      if (!gu) {
+        // destination slot and routing weight of every row, staged while the MMAs run
+        epi_bar<kPEpiThreads>();
+        for (int rr = et; rr < kPairTileN; rr += kPEpiThreads) {
+          int j = -1;
+          float wt = 0.f;
+          if (rr < it.nrows) {
+            const int row = it.row0 + rr;
+            if (sh) {
+              j = p.T * p.K + row;
+              wt = 1.0f;
+            } else {
+              j = p.perm[row];
+              if (j < 0 || j >= p.T * p.K) {
+                atomicExch(p.err, MOE_DEVERR_SCHEDULE);
+                j = -1;
+              } else {
+                wt = p.w[j];
+              }
+            }
+          }
+          meta_j[rr] = j;
+          meta_w[rr] = wt;
+        }
+        epi_bar<kPEpiThreads>();
+      }
+      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kPAccCols;
+      if (gu) {
+        // lanes 0-63 hold gate rows, lanes 64-127 the up rows of the same features.
+        // Per 16-column chunk the gate warps finish columns 0-7 and the up warps
+        // columns 8-15, each taking the other operand through shared memory.
+        const bool is_gate = q < 2;
+        const int fq = q & 1;  // which 32 of the CTA's 64 features
+        const int nfeat = it.ntile * kTileN + static_cast<int>(rank) * 64 + fq * 32 + lane;
+        const int ncols = sh ? p.Is : p.I;
+        const bool ok = nfeat < ncols;
+        const float L = sh ? p.lim_s : p.lim_r;
+        uint16_t* hout = sh ? p.h_s : p.h_r;
+        float* give = xch + ((cpart * 2 + (is_gate ? 0 : 1)) * 64 + fq * 32 + lane) * kPXchRow;
+        const float* take = xch + ((cpart * 2 + (is_gate ? 1 : 0)) * 64 + fq * 32 + lane) * kPXchRow;
+#pragma unroll 1
+        for (int c0 = 16 * cpart; c0 < ncol; c0 += 32) {
+          float v[16];
+          tmem_ld16(taddr + c0, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < 8; ++c) give[c] = is_gate ? v[8 + c] : v[c];
+          epi_bar<kPEpiThreads>();
+          if (ok) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const int r = c0 + (is_gate ? c : 8 + c);
+              const float g = is_gate ? v[c] : take[c];
+              const float u = is_gate ? take[c] : v[8 + c];
+              if (r < it.nrows)
+                hout[static_cast<size_t>(it.row0 + r) * ncols + nfeat] = f2bf(swiglu(g, u, L));
+            }
+          }
+          epi_bar<kPEpiThreads>();
+        }
+      } else {
+        const int nfeat = it.ntile * kDownTile + static_cast<int>(rank) * kTileN + orow;
+        const bool ok = nfeat < p.H;
+        // 32 columns per TMEM wait (ncol is a multiple of 64), alternate groups per warp
+#pragma unroll 1
+        for (int c0 = 32 * cpart; c0 < ncol; c0 += 64) {
+          float ov[32];
+          tmem_ld16(taddr + c0, ov);
+          tmem_ld16(taddr + c0 + 16, ov + 16);
+          tmem_ld_wait();
+          if (ok) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              const int j = meta_j[c0 + c];
+              if (j >= 0) p.y_slot[static_cast<size_t>(j) * p.H + nfeat] = meta_w[c0 + c] * ov[c];
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader) mbar_arrive(&tempty[acc]);
+        else mbar_arrive_cluster(at_leader(&tempty[acc]));
+      }
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1;
+      if (gu) {
+        // publish this CTA's half of the output tile of h
+        fence_proxy_async_global();
+        epi_bar<kPEpiThreads>();
+        if (warp == 2 && lane == 0) {
+          __threadfence();
+          const int r0 = sh ? 0 : s_off[it.e];
+          atomicAdd(p.ready + s_gu[it.e] + (it.row0 - r0) / kPairTileN, 1);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // no CTA leaves while the other may still arrive on its barriers
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, kPTmemCols);
+  }
+}
+
+// x_perm[r] = x[perm[r] / K]: the routed token rows in permuted order, so that
+// the pair kernel loads its B tiles of gate/up items with plain TMA boxes.
+// 16-byte copies; one grid-stride loop over (row, 8-column chunk).
+__global__ void __launch_bounds__(256) gather_rows(int TK, int K, int T, int H,
+                                                   const int32_t* __restrict__ perm,
+                                                   const uint16_t* __restrict__ x,
+                                                   uint16_t* __restrict__ x_perm) {
+  const int chunks = H / 8;
+  const long long total = static_cast<long long>(TK) * chunks;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long r = i / chunks;
+    const int c = static_cast<int>(i - r * chunks);
+    int t = perm[r] / K;
+    t = min(max(t, 0), T - 1);
+    reinterpret_cast<uint4*>(x_perm)[r * chunks + c] =
+        reinterpret_cast<const uint4*>(x)[static_cast<long long>(t) * chunks + c];
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_ffn_pair(const GemmArgs& a, cudaStream_t s) {
+  const moe_cfg& c = *a.cfg;
+  if (a.x_perm == nullptr) return cudaErrorInvalidValue;
+  const int T = a.T, TK = a.T * c.K;
+  {
+    const long long total = static_cast<long long>(TK) * (c.H / 8);
+    long long blocks = (total + 255) / 256;
+    const long long cap = static_cast<long long>(num_sms()) * 8;
+    if (blocks > cap) blocks = cap;
+    gather_rows<<<static_cast<int>(blocks), 256, 0, s>>>(TK, c.K, T, c.H, a.perm, a.x, a.x_perm);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  FfnParams p;
+  memset(&p, 0, sizeof(p));
+  p.T = T;
+  p.K = c.K;
+  p.E = c.E;
+  p.H = c.H;
+  p.I = c.I;
+  p.Is = c.I_shared;
+  p.has_shared = (c.I_shared > 0 && a.W->Wg_s != nullptr) ? 1 : 0;
+  p.lim_r = (c.limit_routed > 0.f && isfinite(c.limit_routed)) ? c.limit_routed : 0.f;
+  p.lim_s = (c.limit_shared > 0.f && isfinite(c.limit_shared)) ? c.limit_shared : 0.f;
+  p.x = a.x;
+  p.perm = a.perm;
+  p.w = a.w;
+  p.h_r = a.h_r;
+  p.h_s = a.h_s;
+  p.y_slot = a.y_slot;
+  p.offsets = a.offsets;
+  p.wslot = a.wslot;
+  p.gu_start = a.gu_start;
+  p.dn_start = a.dn_start;
+  p.nitems = a.nitems;
+  p.counter = const_cast<int32_t*>(a.nitems) + 2;
+  p.ready = a.ready;
+  p.max_gu = a.max_items_gu;
+  p.max_dn = a.max_items_dn;
+  p.err = a.err;
+  PairMaps m;
+  const uint64_t wr = static_cast<uint64_t>(a.wrows);
+  bool ok = map_bf16(&m.wg, a.Wg, wr * c.I, c.H, 64) && map_bf16(&m.wu, a.Wu, wr * c.I, c.H, 64) &&
+            map_bf16(&m.wd, a.Wd, wr * c.H, c.I, kTileN) &&
+            map_bf16(&m.xp, a.x_perm, TK, c.H, kPBox) && map_bf16(&m.x, a.x, T, c.H, kPBox) &&
+            map_bf16(&m.h, a.h_r, TK, c.I, kPBox);
+  if (p.has_shared) {
+    ok = ok && map_bf16(&m.wgs, a.W->Wg_s, c.I_shared, c.H, 64) &&
+         map_bf16(&m.wus, a.W->Wu_s, c.I_shared, c.H, 64) &&
+         map_bf16(&m.wds, a.W->Wd_s, c.H, c.I_shared, kTileN) &&
+         map_bf16(&m.hs, a.h_s, T, c.I_shared, kPBox);
+  } else {
+    m.wgs = m.wg;
+    m.wus = m.wu;
+    m.wds = m.wd;
+    m.hs = m.h;
+  }
+  if (!ok) return cudaErrorInvalidValue;
+  const int smem_max = kPSmem + (3 * kMaxExpertsCfg + 5) * static_cast<int>(sizeof(int));
+  const int smem = kPSmem + (3 * c.E + 5) * static_cast<int>(sizeof(int));
+  cudaError_t e = ensure_dyn_smem(reinterpret_cast<const void*>(moe_ffn_pair), smem_max);
+  if (e != cudaSuccess) return e;
+  // clusters of two CTAs, one per SM; items are claimed by running CTAs only,
+  // so every wait is on work a resident CTA has already taken
+  const int grid = num_sms() & ~1;
+  moe_ffn_pair<<<grid, kPThreads, smem, s>>>(p, m);
+  return cudaGetLastError();
+}
+
+}  // namespace sgl

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
 
 #include "../../include/moe.h"
 
@@ -27,7 +29,17 @@ struct WorkItem {
 constexpr int kPermTile = 2048;   // (token, slot) entries per permutation tile
 constexpr int kTileN = 128;       // output features per GEMM tile (MMA M)
 constexpr int kDownTile = 256;    // hidden features per down item (two MMA tiles)
+constexpr int kPairTileN = 256;   // token tile of the CTA-pair FFN (large batches)
 constexpr int kMaxExpertsCfg = 1024;  // largest E a configuration may have
+
+// The expert-FFN kernel for large batches: one CTA per item (default), or a
+// CTA pair per item (tcgen05 cta_group::2, token tile kPairTileN) when the
+// environment variable SGL_MOE_FFN is "pair". Read at every call, so the
+// workspace layout and the launch always agree.
+inline bool ffn_pair_requested() {
+  const char* v = getenv("SGL_MOE_FFN");
+  return v != nullptr && strcmp(v, "pair") == 0;
+}
 
 // Token-tile width (MMA N) for a batch: small for decode, wide for prefill.
 inline int choose_bn(int T, int K, int E) {
@@ -35,7 +47,7 @@ inline int choose_bn(int T, int K, int E) {
   if (avg <= 12.0) return 16;
   if (avg <= 24.0) return 32;
   if (avg <= 48.0) return 64;
-  return 128;
+  return ffn_pair_requested() ? kPairTileN : 128;
 }
 
 inline int cdiv(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
@@ -55,6 +67,7 @@ struct WsLayout {
   size_t slot_of, touched, ntouched, wq_g, wq_u, wq_d;
   size_t wr_split;  // router matrix as three bf16 terms (batches above 32 tokens)
   size_t zpart;     // split-K router partials [H/128][T][E] fp32 (batches up to 32 tokens)
+  size_t x_perm;    // routed token rows in permuted order [T*K][H] bf16 (pair FFN only)
   int max_touched;
   int n_ptiles, bn, max_items_gu, max_items_dn;
 };
@@ -105,6 +118,7 @@ struct GemmArgs {
   int wrows;                 // row blocks in Wg/Wu/Wd (E, or the slot capacity)
   uint16_t* h_r;
   uint16_t* h_s;
+  uint16_t* x_perm;         // [T*K, H] scratch: routed token rows in permuted order (pair FFN)
   float* y_slot;
   const int32_t* offsets;   // [E+1] routed row offsets
   const int32_t* gu_start;  // [E+2] item prefix sums, gate/up
@@ -120,6 +134,8 @@ struct GemmArgs {
 // The expert FFN: gate/up and down in one cooperative persistent launch
 // (counters in a.ready and a.nitems[2], zeroed by the schedule builder).
 cudaError_t launch_ffn(const GemmArgs& a, cudaStream_t s);
+// The expert FFN on CTA pairs (token tile kPairTileN); gathers a.x_perm first.
+cudaError_t launch_ffn_pair(const GemmArgs& a, cudaStream_t s);
 cudaError_t launch_router_gemm(const moe_cfg& c, int T, const uint16_t* x, const uint16_t* w_hi,
                                const uint16_t* w_mid, const uint16_t* w_lo, float* z,
                                int32_t* err, cudaStream_t s);

@@ -56,6 +56,26 @@ def test_tiny_layer(T):
     _full_check(cfg, d)
 
 
+@pytest.mark.parametrize("T,variant", [(300, {}), (600, {}), (600, dict(limit_routed=0.5, limit_shared=0.7)),
+                                       (600, dict(I_shared=0)), (600, dict(I=192, I_shared=320))])
+def test_tiny_layer_pair_ffn(T, variant, monkeypatch):
+    """The CTA-pair expert FFN (tcgen05 cta_group::2), selected explicitly."""
+    monkeypatch.setenv("SGL_MOE_FFN", "pair")
+    cfg = TINY.with_(**variant)
+    d = workloads.generate(cfg, DEV, T=T)
+    _full_check(cfg, d)
+
+
+@pytest.mark.slow
+def test_prefill_sampled_pair_ffn(monkeypatch):
+    monkeypatch.setenv("SGL_MOE_FFN", "pair")
+    cfg = workloads.CONFIGS["prefill"]
+    d = workloads.generate(cfg, DEV)
+    _full_check(cfg, d, tokens=_sample(cfg.T, 12, cfg.seed))
+    del d
+    torch.cuda.empty_cache()
+
+
 @pytest.mark.parametrize("variant", [
     dict(limit_routed=0.5, limit_shared=0.7),           # clamps that bite
     dict(n_group=1, topk_group=1),                      # plain top-k
