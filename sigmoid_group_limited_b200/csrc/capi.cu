@@ -167,6 +167,7 @@ size_t moe_workspace_size(const moe_cfg* cfg, int32_t T) {
 moe_status moe_route(const moe_cfg* cfg, int32_t T, const void* x, const float* Wr,
                      const float* bias, int32_t* idx, float* w, void* ws, size_t ws_bytes,
                      void* stream) {
+  PdlScope pdl_scope(T);  // programmatic dependent launch for small batches
   if (!cfg_ok(cfg) || !T_ok(T)) return MOE_ERR_CFG;
   if (!x || !Wr || !idx || !w) return MOE_ERR_NULL;
   if (!al16(x) || !al16(Wr) || !al16(idx) || !al16(w) || (bias && !al16(bias))) return MOE_ERR_ALIGN;
@@ -186,6 +187,7 @@ moe_status moe_route(const moe_cfg* cfg, int32_t T, const void* x, const float* 
 moe_status moe_permute(const moe_cfg* cfg, int32_t T, const int32_t* idx, int32_t* counts,
                        int32_t* offsets, int32_t* perm, int32_t* inv_perm, void* ws,
                        size_t ws_bytes, void* stream) {
+  PdlScope pdl_scope(T);  // programmatic dependent launch for small batches
   if (!cfg_ok(cfg) || !T_ok(T)) return MOE_ERR_CFG;
   if (!idx || !counts || !offsets || !perm) return MOE_ERR_NULL;
   if (!al16(idx) || !al16(counts) || !al16(offsets) || !al16(perm) || (inv_perm && !al16(inv_perm)))
@@ -218,6 +220,7 @@ moe_status moe_permute_static(const moe_cfg* cfg, int32_t T, const int32_t* idx,
 moe_status moe_grouped_swiglu(const moe_cfg* cfg, int32_t T, const void* x, const int32_t* perm,
                               const int32_t* offsets, const float* w, const moe_weights* W,
                               void* y_slot, void* ws, size_t ws_bytes, void* stream) {
+  PdlScope pdl_scope(T);  // programmatic dependent launch for small batches
   if (!cfg_ok(cfg) || !T_ok(T)) return MOE_ERR_CFG;
   if (!x || !perm || !offsets || !w || !y_slot) return MOE_ERR_NULL;
   if (!al16(x) || !al16(perm) || !al16(offsets) || !al16(w) || !al16(y_slot)) return MOE_ERR_ALIGN;
@@ -276,6 +279,7 @@ moe_status moe_grouped_swiglu(const moe_cfg* cfg, int32_t T, const void* x, cons
 
 moe_status moe_combine(const moe_cfg* cfg, int32_t T, const void* y_slot, int32_t with_shared,
                        void* y, void* stream) {
+  PdlScope pdl_scope(T);  // programmatic dependent launch for small batches
   if (!cfg_ok(cfg) || !T_ok(T)) return MOE_ERR_CFG;
   if (!y_slot || !y) return MOE_ERR_NULL;
   if (!al16(y_slot) || !al16(y)) return MOE_ERR_ALIGN;
@@ -289,6 +293,7 @@ moe_status moe_layer_forward(const moe_cfg* cfg, int32_t T, const void* x, const
                              const float* bias, const moe_weights* W, void* y, int32_t* idx_out,
                              float* w_out, int32_t* counts_out, void* ws, size_t ws_bytes,
                              void* stream, void* const* stage_events) {
+  PdlScope pdl_scope(T);  // programmatic dependent launch for small batches
   if (!cfg_ok(cfg) || !T_ok(T)) return MOE_ERR_CFG;
   if (!x || !Wr || !y) return MOE_ERR_NULL;
   if (!al16(x) || !al16(Wr) || !al16(y) || (bias && !al16(bias)) || (idx_out && !al16(idx_out)) ||

@@ -11,6 +11,7 @@
 #include <stdint.h>
 
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace sgl {
 namespace {
@@ -29,6 +30,8 @@ __device__ __forceinline__ void add8(float* acc, const float4 a, const float4 b)
 __global__ void __launch_bounds__(256) combine_kernel(int T, int H, int K, int with_shared,
                                                       const float* __restrict__ y_slot,
                                                       uint16_t* __restrict__ y) {
+  pdl_trigger();
+  pdl_wait();  // inputs come from earlier kernels on the stream
   const int chunks = H / 8;
   const long long total = static_cast<long long>(T) * chunks;
   const float4* src = reinterpret_cast<const float4*>(y_slot);
@@ -69,8 +72,8 @@ cudaError_t launch_combine(const moe_cfg& c, int T, const float* y_slot, int wit
   long long blocks = (total + threads - 1) / threads;
   const long long cap = static_cast<long long>(num_sms()) * 8;
   if (blocks > cap) blocks = cap;
-  combine_kernel<<<static_cast<int>(blocks), threads, 0, s>>>(T, c.H, c.K, with_shared, y_slot, y);
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel, dim3(static_cast<int>(blocks)), dim3(threads), 0, s, T, c.H, c.K,
+                    with_shared, y_slot, y);
 }
 
 }  // namespace sgl

@@ -116,6 +116,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
   int* s_off = s_dn + (p.E + 2);                     // [E+1]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  pdl_trigger();
   if (tid == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1 + kGatherWarps);  // weight TMA + one arrival per gatherer warp
@@ -141,6 +142,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
+  pdl_wait();  // the schedule, the routing and x come from earlier kernels
   for (int i = tid; i < p.E + 2; i += blockDim.x) {
     s_gu[i] = p.gu_start[i];
     s_dn[i] = p.dn_start[i];
@@ -592,19 +594,11 @@ cudaError_t launch_bn(const GemmArgs& a, cudaStream_t s) {
   const int smem = C::SMEM + (3 * c.E + 5) * static_cast<int>(sizeof(int));
   cudaError_t e = ensure_dyn_smem(reinterpret_cast<const void*>(kern), smem_max);
   if (e != cudaSuccess) return e;
-  // one CTA per SM, all resident at once (down items wait on other CTAs)
-  cudaLaunchConfig_t lc;
-  memset(&lc, 0, sizeof(lc));
-  lc.gridDim = dim3(num_sms());
-  lc.blockDim = dim3(kFfnThreads);
-  lc.dynamicSmemBytes = smem;
-  lc.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
-  lc.attrs = attr;
-  lc.numAttrs = 1;
-  return cudaLaunchKernelEx(&lc, kern, p, tWg, tWu, tWgS, tWuS, tWd, tWdS, tH, tHs);
+  // One CTA per SM. Items are claimed only by running CTAs, so a down item
+  // only ever waits on gate/up tiles a resident CTA has taken: no
+  // co-residency guarantee is needed.
+  return launch_pdl(kern, dim3(num_sms()), dim3(kFfnThreads), smem, s, p, tWg, tWu, tWgS, tWuS, tWd,
+                    tWdS, tH, tHs);
 }
 
 }  // namespace

@@ -112,6 +112,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_ctarank() & 1u;
   const bool leader = rank == 0;
+  pdl_trigger();
   if (tid == 0) {
     for (int s = 0; s < kPStages; ++s) {
       mbar_init(&full[s], 1);   // the leader's expect_tx arrival (+ both CTAs' bytes)
@@ -137,6 +138,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
     tmem_alloc_pair(tmem_slot, kPTmemCols);
     tmem_relinquish_pair();
   }
+  pdl_wait();  // the schedule, the routing and x_perm come from earlier kernels
   for (int i = tid; i < p.E + 2; i += blockDim.x) {
     s_gu[i] = p.gu_start[i];
     s_dn[i] = p.dn_start[i];
@@ -466,6 +468,8 @@ __global__ void __launch_bounds__(256) gather_rows(int TK, int K, int T, int H,
                                                    const int32_t* __restrict__ perm,
                                                    const uint16_t* __restrict__ x,
                                                    uint16_t* __restrict__ x_perm) {
+  pdl_trigger();
+  pdl_wait();  // inputs come from earlier kernels on the stream
   const int chunks = H / 8;
   const long long total = static_cast<long long>(TK) * chunks;
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
@@ -490,8 +494,8 @@ cudaError_t launch_ffn_pair(const GemmArgs& a, cudaStream_t s) {
     long long blocks = (total + 255) / 256;
     const long long cap = static_cast<long long>(num_sms()) * 8;
     if (blocks > cap) blocks = cap;
-    gather_rows<<<static_cast<int>(blocks), 256, 0, s>>>(TK, c.K, T, c.H, a.perm, a.x, a.x_perm);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(gather_rows, dim3(static_cast<int>(blocks)), dim3(256), 0, s, TK, c.K,
+                               T, c.H, a.perm, a.x, a.x_perm);
     if (e != cudaSuccess) return e;
   }
   FfnParams p;
@@ -546,8 +550,7 @@ cudaError_t launch_ffn_pair(const GemmArgs& a, cudaStream_t s) {
   // clusters of two CTAs, one per SM; items are claimed by running CTAs only,
   // so every wait is on work a resident CTA has already taken
   const int grid = num_sms() & ~1;
-  moe_ffn_pair<<<grid, kPThreads, smem, s>>>(p, m);
-  return cudaGetLastError();
+  return launch_pdl(moe_ffn_pair, dim3(grid), dim3(kPThreads), smem, s, p, m);
 }
 
 }  // namespace sgl

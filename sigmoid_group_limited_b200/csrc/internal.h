@@ -148,6 +148,40 @@ cudaError_t launch_mxfp4_expand(const moe_cfg& c, const int32_t* offsets, const 
 cudaError_t launch_combine(const moe_cfg& c, int T, const float* y_slot, int with_shared,
                            uint16_t* y, cudaStream_t s);
 
+// Whether launches on this host thread use programmatic dependent launch.
+// It pays for small batches, whose kernels are short and latency-bound; on
+// large ones the early-resident grids cost more than the launch gaps they
+// hide. Set per call by the entry points (PdlScope).
+constexpr int kPdlMaxTokens = 256;
+inline bool& pdl_enabled() {
+  static thread_local bool on = false;
+  return on;
+}
+struct PdlScope {
+  bool prev;
+  explicit PdlScope(int T) : prev(pdl_enabled()) { pdl_enabled() = T <= kPdlMaxTokens; }
+  ~PdlScope() { pdl_enabled() = prev; }
+};
+
+// Launches `kern`, with programmatic stream serialization when enabled (see
+// pdl_wait in ptx.cuh); returns cudaLaunchKernelEx's status.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args&&... args) {
+  cudaLaunchConfig_t lc;
+  memset(&lc, 0, sizeof(lc));
+  lc.gridDim = grid;
+  lc.blockDim = block;
+  lc.dynamicSmemBytes = smem;
+  lc.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&lc, kern, static_cast<Args&&>(args)...);
+}
+
 int num_sms();
 
 // Tensor map of a bf16 row-major [rows, cols] matrix for TMA: box of

@@ -14,6 +14,7 @@
 #include <stdint.h>
 
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace sgl {
 namespace {
@@ -24,6 +25,8 @@ __global__ void __launch_bounds__(1024) mxfp4_slots(int E, const int32_t* __rest
                                                     int32_t* __restrict__ slot_of,
                                                     int32_t* __restrict__ touched,
                                                     int32_t* __restrict__ ntouched) {
+  pdl_trigger();
+  pdl_wait();  // inputs come from earlier kernels on the stream
   __shared__ int wsum[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int base = 0;
@@ -80,6 +83,8 @@ __global__ void __launch_bounds__(256) mxfp4_dequant(
     const uint8_t* __restrict__ uq, const uint8_t* __restrict__ us,
     const uint8_t* __restrict__ dq, const uint8_t* __restrict__ ds, uint16_t* __restrict__ gout,
     uint16_t* __restrict__ uout, uint16_t* __restrict__ dout) {
+  pdl_trigger();
+  pdl_wait();  // inputs come from earlier kernels on the stream
   const long long per_mat = static_cast<long long>(I) * H / 8;  // units per matrix
   const long long total = static_cast<long long>(*ntouched) * 3 * per_mat;
   for (long long u = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; u < total;
@@ -104,14 +109,14 @@ __global__ void __launch_bounds__(256) mxfp4_dequant(
 cudaError_t launch_mxfp4_expand(const moe_cfg& c, const int32_t* offsets, const moe_weights* W,
                                 int32_t* slot_of, int32_t* touched, int32_t* ntouched,
                                 uint16_t* gout, uint16_t* uout, uint16_t* dout, cudaStream_t s) {
-  mxfp4_slots<<<1, 1024, 0, s>>>(c.E, offsets, slot_of, touched, ntouched);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(mxfp4_slots, dim3(1), dim3(1024), 0, s, c.E, offsets, slot_of, touched,
+                             ntouched);
   if (e != cudaSuccess) return e;
-  mxfp4_dequant<<<num_sms() * 8, 256, 0, s>>>(
-      c.I, c.H, touched, ntouched, static_cast<const uint8_t*>(W->Wg), W->Wg_scale,
-      static_cast<const uint8_t*>(W->Wu), W->Wu_scale, static_cast<const uint8_t*>(W->Wd),
-      W->Wd_scale, gout, uout, dout);
-  return cudaGetLastError();
+  return launch_pdl(mxfp4_dequant, dim3(num_sms() * 8), dim3(256), 0, s, c.I, c.H,
+                    static_cast<const int32_t*>(touched), static_cast<const int32_t*>(ntouched),
+                    static_cast<const uint8_t*>(W->Wg), W->Wg_scale,
+                    static_cast<const uint8_t*>(W->Wu), W->Wu_scale,
+                    static_cast<const uint8_t*>(W->Wd), W->Wd_scale, gout, uout, dout);
 }
 
 }  // namespace sgl

@@ -18,17 +18,21 @@
 #include <mutex>
 
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace sgl {
 namespace {
 
 constexpr int kMaxE = 1024;
+constexpr int kScanSmemInts = 48 * 1024;  // tile counts perm_scan stages in shared memory (192 KB)
 constexpr int kScatterWarps = 8;
 
 __global__ void __launch_bounds__(256) perm_hist(int TK, int E, int n_ptiles,
                                                  const int32_t* __restrict__ idx,
                                                  int32_t* __restrict__ tile_cnt,  // [E][n_ptiles]
                                                  int32_t* __restrict__ err) {
+  pdl_trigger();
+  pdl_wait();  // inputs come from earlier kernels on the stream
   __shared__ int hist[kMaxE];
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
@@ -145,15 +149,26 @@ __global__ void __launch_bounds__(1024) perm_scan(int E, int n_ptiles,
                                                   int32_t* __restrict__ tile_base,
                                                   int32_t* __restrict__ counts,
                                                   int32_t* __restrict__ offsets, SchedArgs sa,
-                                                  int build) {
+                                                  int build, int stage_smem) {
+  pdl_trigger();
+  pdl_wait();  // inputs come from earlier kernels on the stream
   __shared__ int cnt[kMaxE + 1];
   __shared__ int off[kMaxE + 1];
   __shared__ int scratch[33];
+  extern __shared__ int tc_s[];  // the tile counts, when they fit (else read from global)
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int ncnt = E * n_ptiles;
+  const int32_t* tc = tile_cnt;
+  if (stage_smem && ncnt <= kScanSmemInts) {  // the launch provided E * n_ptiles ints
+    // one coalesced sweep, all loads in flight, instead of a dependent load per expert
+    for (int i = threadIdx.x; i < ncnt; i += blockDim.x) tc_s[i] = tile_cnt[i];
+    __syncthreads();
+    tc = tc_s;
+  }
   // per-expert totals: one warp per expert, lanes over tiles
   for (int e = warp; e < E; e += nw) {
     int s = 0;
-    for (int t = lane; t < n_ptiles; t += 32) s += tile_cnt[static_cast<size_t>(e) * n_ptiles + t];
+    for (int t = lane; t < n_ptiles; t += 32) s += tc[static_cast<size_t>(e) * n_ptiles + t];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
     if (lane == 0) cnt[e] = s;
@@ -176,7 +191,7 @@ __global__ void __launch_bounds__(1024) perm_scan(int E, int n_ptiles,
     int carry = off[e];
     for (int t0 = 0; t0 < n_ptiles; t0 += 32) {
       const int t = t0 + lane;
-      const int v = t < n_ptiles ? tile_cnt[static_cast<size_t>(e) * n_ptiles + t] : 0;
+      const int v = t < n_ptiles ? tc[static_cast<size_t>(e) * n_ptiles + t] : 0;
       int incl = v;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -192,6 +207,8 @@ __global__ void __launch_bounds__(1024) perm_scan(int E, int n_ptiles,
 
 __global__ void __launch_bounds__(1024) schedule_only(const int32_t* __restrict__ offsets,
                                                       SchedArgs sa) {
+  pdl_trigger();
+  pdl_wait();  // inputs come from earlier kernels on the stream
   __shared__ int cnt[kMaxE + 1];
   __shared__ int scratch[33];
   for (int e = threadIdx.x; e < sa.E; e += blockDim.x) cnt[e] = offsets[e + 1] - offsets[e];
@@ -203,6 +220,8 @@ __global__ void __launch_bounds__(kScatterWarps * 32) perm_scatter(
     int TK, int E, int n_ptiles, const int32_t* __restrict__ idx,
     const int32_t* __restrict__ tile_base, int32_t* __restrict__ perm,
     int32_t* __restrict__ inv_perm, int32_t* __restrict__ err) {
+  pdl_trigger();
+  pdl_wait();  // inputs come from earlier kernels on the stream
   __shared__ int whist[kScatterWarps][kMaxE];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < kScatterWarps * E; i += blockDim.x) whist[i / E][i % E] = 0;
@@ -273,6 +292,8 @@ __global__ void __launch_bounds__(1024) perm_single(int TK, int E, const int32_t
                                                     int32_t* __restrict__ inv_perm,
                                                     int32_t* __restrict__ err, SchedArgs sa,
                                                     int build) {
+  pdl_trigger();
+  pdl_wait();  // inputs come from earlier kernels on the stream
   extern __shared__ int whist[];  // [32 warps][E]
   __shared__ int cnt[kMaxE + 1];
   __shared__ int off[kMaxE + 1];
@@ -383,17 +404,24 @@ cudaError_t launch_permute(const moe_cfg& c, int T, const int32_t* idx, int32_t*
     cudaError_t e = ensure_dyn_smem(reinterpret_cast<const void*>(perm_single),
                                     32 * kMaxE * static_cast<int>(sizeof(int)));
     if (e != cudaSuccess) return e;
-    perm_single<<<1, 1024, smem, s>>>(TK, c.E, idx, counts, offsets, perm, inv_perm, err, sa,
-                                      gu_start != nullptr ? 1 : 0);
-    return cudaGetLastError();
+    return launch_pdl(perm_single, dim3(1), dim3(1024), smem, s, TK, c.E, idx, counts, offsets, perm,
+                      inv_perm, err, sa, gu_start != nullptr ? 1 : 0);
   }
   int32_t* tile_base = tile_cnt + static_cast<size_t>(c.E) * np;
-  perm_hist<<<np, 256, 0, s>>>(TK, c.E, np, idx, tile_cnt, err);
-  perm_scan<<<1, 1024, 0, s>>>(c.E, np, tile_cnt, tile_base, counts, offsets, sa,
-                               gu_start != nullptr ? 1 : 0);
-  perm_scatter<<<np, kScatterWarps * 32, 0, s>>>(TK, c.E, np, idx, tile_base, perm, inv_perm,
-                                                 err);
-  return cudaGetLastError();
+  cudaError_t e = launch_pdl(perm_hist, dim3(np), dim3(256), 0, s, TK, c.E, np, idx, tile_cnt, err);
+  if (e != cudaSuccess) return e;
+  const int scan_smem = c.E * np <= kScanSmemInts ? c.E * np * static_cast<int>(sizeof(int)) : 0;
+  if (scan_smem > 0) {
+    e = ensure_dyn_smem(reinterpret_cast<const void*>(perm_scan),
+                        kScanSmemInts * static_cast<int>(sizeof(int)));
+    if (e != cudaSuccess) return e;
+  }
+  e = launch_pdl(perm_scan, dim3(1), dim3(1024), scan_smem, s, c.E, np,
+                 static_cast<const int32_t*>(tile_cnt), tile_base, counts, offsets, sa,
+                 gu_start != nullptr ? 1 : 0, scan_smem > 0 ? 1 : 0);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(perm_scatter, dim3(np), dim3(kScatterWarps * 32), 0, s, TK, c.E, np, idx,
+                    static_cast<const int32_t*>(tile_base), perm, inv_perm, err);
 }
 
 // ---------------------------------------------------------------------------
@@ -442,7 +470,7 @@ cudaError_t launch_permute_static(const moe_cfg& c, int T, const int32_t* idx, i
   SchedArgs sa{};
   sa.nitems = base + 1;
   sa.ready = nullptr;
-  perm_scan<<<1, 1024, 0, s>>>(c.E, np, tile_cnt, tile_base, counts, offsets, sa, 0);
+  perm_scan<<<1, 1024, 0, s>>>(c.E, np, tile_cnt, tile_base, counts, offsets, sa, 0, 0);
   perm_scatter<<<np, kScatterWarps * 32, 0, s>>>(TK, c.E, np, idx, tile_base, perm, inv_perm,
                                                  err);
   return cudaGetLastError();
@@ -452,8 +480,7 @@ cudaError_t launch_schedule(const moe_cfg& c, int T, const int32_t* offsets, con
                             int32_t* gu_start, int32_t* dn_start, int32_t* ready,
                             int32_t* nitems, cudaStream_t s) {
   SchedArgs sa = make_sched(c, T, L, gu_start, dn_start, ready, nitems);
-  schedule_only<<<1, 1024, 0, s>>>(offsets, sa);
-  return cudaGetLastError();
+  return launch_pdl(schedule_only, dim3(1), dim3(1024), 0, s, offsets, sa);
 }
 
 }  // namespace sgl

@@ -60,6 +60,8 @@ __global__ void __launch_bounds__(256) router_logits_splitk(int T, int H, int E,
                                                            float* __restrict__ zpart,
                                                            int32_t* __restrict__ block_cnt,
                                                            float* __restrict__ z) {
+  pdl_trigger();
+  pdl_wait();  // inputs come from earlier kernels on the stream
   __shared__ __align__(16) float ws[kSplitE][kSplitH];
   // token rows of the chunk, padded by 16 bytes so that 8 lanes reading the
   // same column of 8 rows hit 8 different bank groups
@@ -180,6 +182,8 @@ __global__ void __launch_bounds__(256) router_topk(int T, int E, int n_group, in
                                                    int32_t* __restrict__ unc_n,
                                                    const int32_t* __restrict__ list,
                                                    const int32_t* __restrict__ list_n) {
+  pdl_trigger();
+  pdl_wait();  // inputs come from earlier kernels on the stream
   const int lane = threadIdx.x & 31;
   const int wpb = blockDim.x >> 5;
   const int n = list ? min(*list_n, T) : T;
@@ -369,6 +373,8 @@ __global__ void __launch_bounds__(kSelMaxGroups * 32) router_select(
     int T, int E, int n_group, int topk_group, int K, float scale, int renorm,
     const float* __restrict__ z, const float* __restrict__ bias, int32_t* __restrict__ idx,
     float* __restrict__ wout, float tau, int32_t* __restrict__ unc, int32_t* __restrict__ unc_n) {
+  pdl_trigger();
+  pdl_wait();  // inputs come from earlier kernels on the stream
   __shared__ uint32_t gkey[kSelMaxGroups];
   __shared__ float gzz[kSelMaxGroups];
   __shared__ uint32_t ckey[kSelMaxGroups][kSelMaxCand];
@@ -534,7 +540,7 @@ __global__ void __launch_bounds__(kSelMaxGroups * 32) router_select(
 // then the float64 sigmoid rounded to fp32, plus the bias in fp32: the same
 // arithmetic as the reference definition.
 // ---------------------------------------------------------------------------
-constexpr int kRefineThreads = 128;
+constexpr int kRefineThreads = 256;  // 8 warps: exact scores of 8 experts at a time
 
 template <int NV>
 __device__ __forceinline__ void load_scores(const float* zr, const float* bias, int E, int lane,
@@ -563,6 +569,8 @@ __global__ void __launch_bounds__(kRefineThreads) router_refine(
     const float* __restrict__ z, const float* __restrict__ bias, int32_t* __restrict__ idx,
     float* __restrict__ wout, const int32_t* __restrict__ list,
     const int32_t* __restrict__ list_n) {
+  pdl_trigger();
+  pdl_wait();  // inputs come from earlier kernels on the stream
   __shared__ __align__(16) uint16_t xs[kRowRegs * 128];
   __shared__ int need[kMaxExperts];
   __shared__ float bex[kMaxExperts], sex[kMaxExperts];
@@ -638,18 +646,21 @@ __global__ void __launch_bounds__(kRefineThreads) router_refine(
 #pragma unroll
         for (int j = 0; j < kRowRegs; ++j)
           wv[j] = *reinterpret_cast<const float4*>(row + min(4 * lane + 128 * j, H - 4));
-        double acc = 0.0;
+        // every product is exact in float64; four independent float64 sums keep
+        // the FMA units busy, then a fixed tree adds them
+        double a4[4] = {0.0, 0.0, 0.0, 0.0};
 #pragma unroll
         for (int j = 0; j < kRowRegs; ++j) {
           const int k = 4 * lane + 128 * j;
           if (k < H) {
             const uint2 p = *reinterpret_cast<const uint2*>(xs + k);
-            acc = fma(static_cast<double>(wv[j].x), bf16_bits_to_double(p.x & 0xFFFFu), acc);
-            acc = fma(static_cast<double>(wv[j].y), bf16_bits_to_double(p.x >> 16), acc);
-            acc = fma(static_cast<double>(wv[j].z), bf16_bits_to_double(p.y & 0xFFFFu), acc);
-            acc = fma(static_cast<double>(wv[j].w), bf16_bits_to_double(p.y >> 16), acc);
+            a4[0] = fma(static_cast<double>(wv[j].x), bf16_bits_to_double(p.x & 0xFFFFu), a4[0]);
+            a4[1] = fma(static_cast<double>(wv[j].y), bf16_bits_to_double(p.x >> 16), a4[1]);
+            a4[2] = fma(static_cast<double>(wv[j].z), bf16_bits_to_double(p.y & 0xFFFFu), a4[2]);
+            a4[3] = fma(static_cast<double>(wv[j].w), bf16_bits_to_double(p.y >> 16), a4[3]);
           }
         }
+        double acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
         if (lane == 0) {
@@ -859,10 +870,9 @@ cudaError_t launch_topk(const moe_cfg& c, int T, const float* z, const float* bi
   // small batches: one token per CTA, so every token's warp has an SM to itself
   const int warps = T <= 4 * num_sms() ? 1 : 8;
   const int grid = cdiv(T, warps);
-  router_topk<NV, GJ><<<grid, warps * 32, 0, s>>>(T, c.E, c.n_group, c.topk_group, c.K, c.scale,
-                                                  c.renorm, z, bias, idx, w, tau, unc, unc_n,
-                                                  nullptr, nullptr);
-  return cudaGetLastError();
+  return launch_pdl(router_topk<NV, GJ>, dim3(grid), dim3(warps * 32), 0, s, T, c.E, c.n_group,
+                    c.topk_group, c.K, c.scale, c.renorm, z, bias, idx, w, tau, unc, unc_n,
+                    static_cast<const int32_t*>(nullptr), static_cast<const int32_t*>(nullptr));
 }
 
 cudaError_t topk_dispatch(const moe_cfg& c, int T, const float* z, const float* bias,
@@ -875,15 +885,9 @@ cudaError_t topk_dispatch(const moe_cfg& c, int T, const float* z, const float* 
   if (T <= 4 * num_sms() && (per == 32 || per == 64) && c.n_group <= kSelMaxGroups &&
       c.K + 1 <= kSelMaxCand && c.topk_group * (c.K + 1) <= 64) {
     const int grid = T;
-    if (per == 32)
-      router_select<1><<<grid, c.n_group * 32, 0, s>>>(T, c.E, c.n_group, c.topk_group, c.K,
-                                                       c.scale, c.renorm, z, bias, idx, w, tau,
-                                                       unc, unc_n);
-    else
-      router_select<2><<<grid, c.n_group * 32, 0, s>>>(T, c.E, c.n_group, c.topk_group, c.K,
-                                                       c.scale, c.renorm, z, bias, idx, w, tau,
-                                                       unc, unc_n);
-    return cudaGetLastError();
+    auto kern = per == 32 ? router_select<1> : router_select<2>;
+    return launch_pdl(kern, dim3(grid), dim3(c.n_group * 32), 0, s, T, c.E, c.n_group,
+                      c.topk_group, c.K, c.scale, c.renorm, z, bias, idx, w, tau, unc, unc_n);
   }
 #define SGL_TOPK(NV_)                                                                   \
   if (nv <= NV_) {                                                                      \
@@ -912,6 +916,8 @@ __global__ void __launch_bounds__(256) split_router(long long n, const float* __
                                                     uint16_t* __restrict__ hi,
                                                     uint16_t* __restrict__ mid,
                                                     uint16_t* __restrict__ lo) {
+  pdl_trigger();
+  pdl_wait();  // inputs come from earlier kernels on the stream
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
     const float v = w[i];
@@ -930,10 +936,9 @@ cudaError_t launch_refine_nv(const moe_cfg& c, int T, const uint16_t* x, const f
                              const float* z, const float* bias, int32_t* idx, float* w, float tau,
                              const int32_t* list, const int32_t* list_n, cudaStream_t s) {
   const int grid = std::max(1, std::min(T, num_sms() * 4));
-  router_refine<NV><<<grid, kRefineThreads, 0, s>>>(T, c.H, c.E, c.n_group, c.topk_group, c.K,
-                                                    c.scale, c.renorm, tau, x, Wr, z, bias, idx,
-                                                    w, list, list_n);
-  return cudaGetLastError();
+  return launch_pdl(router_refine<NV>, dim3(grid), dim3(kRefineThreads), 0, s, T, c.H, c.E,
+                    c.n_group, c.topk_group, c.K, c.scale, c.renorm, tau, x, Wr, z, bias, idx, w,
+                    list, list_n);
 }
 
 cudaError_t launch_refine(const moe_cfg& c, int T, const uint16_t* x, const float* Wr,
@@ -967,8 +972,8 @@ cudaError_t launch_router(const moe_cfg& c, int T, const uint16_t* x, const floa
     // fp32 split-K partials, added in order by the last CTA of each expert block
     if (zpart == nullptr || split_cnt == nullptr) return cudaErrorInvalidValue;
     const int nsplit = cdiv(c.H, kSplitH);
-    router_logits_splitk<<<dim3(nsplit, cdiv(c.E, kSplitE)), 256, 0, s>>>(T, c.H, c.E, x, Wr,
-                                                                           zpart, split_cnt, z);
+    e = launch_pdl(router_logits_splitk, dim3(nsplit, cdiv(c.E, kSplitE)), dim3(256), 0, s, T, c.H,
+                   c.E, x, Wr, zpart, split_cnt, z);
   } else {
     // tensor cores: split the router matrix, then one bf16 x 3 GEMM into z
     if (wr_split == nullptr) return cudaErrorInvalidValue;
@@ -976,8 +981,9 @@ cudaError_t launch_router(const moe_cfg& c, int T, const uint16_t* x, const floa
     uint16_t* hi = wr_split;
     uint16_t* mid = hi + n;
     uint16_t* lo = mid + n;
-    split_router<<<num_sms() * 4, 256, 0, s>>>(n, Wr, hi, mid, lo);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_pdl(split_router, dim3(num_sms() * 4), dim3(256), 0, s, n, Wr, hi, mid, lo)) !=
+        cudaSuccess)
+      return e;
     e = launch_router_gemm(c, T, x, hi, mid, lo, z, err, s);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -63,6 +63,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  pdl_trigger();
   if (tid == 0) {
     for (int s = 0; s < kRStages; ++s) {
       mbar_init(&full[s], 1);
@@ -83,6 +84,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
     tmem_alloc(tmem_slot, kRTmemCols);
     tmem_relinquish();
   }
+  pdl_wait();  // the split router matrix comes from the kernel before
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -257,8 +259,7 @@ cudaError_t launch_router_gemm(const moe_cfg& c, int T, const uint16_t* x, const
   if (e != cudaSuccess) return e;
   const int n_items = cdiv(c.E, kTileN) * cdiv(T, kRBN);
   const int grid = std::max(1, std::min(num_sms(), n_items));
-  router_logits_tc<<<grid, kRThreads, kRSmem, s>>>(p, tHi, tMid, tLo, tX);
-  return cudaGetLastError();
+  return launch_pdl(router_logits_tc, dim3(grid), dim3(kRThreads), kRSmem, s, p, tHi, tMid, tLo, tX);
 }
 
 }  // namespace sgl
