@@ -226,8 +226,8 @@ def roofline_entry(bytes_, flops, seconds, peaks, sustained=False):
 # Weight bytes dominate and scale with the experts touched, so the ratio
 # scales the counters to a full launch. Valid only for the ffn.cu they were
 # taken on: any other source reports traffic null.
-FFN_TRAFFIC_SOURCE_SHA256 = "fed4426034d42ce7cb4ae1a0d472869ff856ba64cb88c83bd8a24edb6c3e857f"
-FFN_TRAFFIC_RATIO = {16: (424.9 + 4.4) / 424.9, 128: (795.8 + 48.5) / 760.2}
+FFN_TRAFFIC_SOURCE_SHA256 = "48e27a9659764bd394e28d2e553ed03ee0bf6861e6ea5ae2eaf0e108fcd84afb"
+FFN_TRAFFIC_RATIO = {16: (424.91 + 4.26) / 424.82, 128: (778.64 + 48.90) / 760.2}
 
 
 def ffn_tile_n(cfg) -> int:
