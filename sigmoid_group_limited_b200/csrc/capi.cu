@@ -78,7 +78,6 @@ WsLayout ws_layout(const moe_cfg& c, int T) {
   L.h_s = take(static_cast<size_t>(T) * (c.I_shared > 0 ? c.I_shared : 0) * 2);
   L.y_slot = take((TK + T) * c.H * 4);
   L.wr_split = T > 32 ? take(static_cast<size_t>(3) * c.E * c.H * 2) : 0;
-  L.zpart = T <= 32 ? take(static_cast<size_t>(cdiv(c.H, 128)) * T * c.E * 4) : 0;
   L.x_perm = L.bn == kPairTileN ? take(TK * c.H * 2) : 0;
   if (c.wfmt == MOE_W_MXFP4) {
     L.max_touched = static_cast<int>(TK < static_cast<size_t>(c.E) ? TK : c.E);
@@ -180,8 +179,7 @@ moe_status moe_route(const moe_cfg* cfg, int32_t T, const void* x, const float* 
   return cu(launch_router(*cfg, T, static_cast<const uint16_t*>(x), Wr, bias, at<float>(ws, L.z),
                           idx, w, at<int32_t>(ws, L.unc), at<int32_t>(ws, L.err) + 1,
                           at<int32_t>(ws, L.err), T > 32 ? at<uint16_t>(ws, L.wr_split) : nullptr,
-                          T <= 32 ? at<float>(ws, L.zpart) : nullptr,
-                          at<int32_t>(ws, L.err) + kCtrlSplitCnt, s));
+                          s));
 }
 
 moe_status moe_permute(const moe_cfg* cfg, int32_t T, const int32_t* idx, int32_t* counts,
@@ -325,9 +323,7 @@ moe_status moe_layer_forward(const moe_cfg* cfg, int32_t T, const void* x, const
   if (cudaMemsetAsync(err, 0, kCtrlBytes, s) != cudaSuccess) return MOE_ERR_CUDA;
   if ((e = launch_router(*cfg, T, static_cast<const uint16_t*>(x), Wr, bias, at<float>(ws, L.z),
                          idx, w, at<int32_t>(ws, L.unc), err + 1, err,
-                         T > 32 ? at<uint16_t>(ws, L.wr_split) : nullptr,
-                         T <= 32 ? at<float>(ws, L.zpart) : nullptr, err + kCtrlSplitCnt, s)) !=
-      cudaSuccess)
+                         T > 32 ? at<uint16_t>(ws, L.wr_split) : nullptr, s)) != cudaSuccess)
     return MOE_ERR_CUDA;
   rec(1);
   if ((e = launch_permute(*cfg, T, idx, at<int32_t>(ws, L.tile_hist), counts, offsets, perm,

@@ -55,10 +55,8 @@ __host__ __device__ inline int cdiv_dev(int a, int b) { return (a + b - 1) / b; 
 
 // Per-call control block at the start of the workspace, zeroed by every
 // entry point that routes: [0] device error word, [1] count of tokens whose
-// routing is re-derived exactly, [32 .. 64) split-K router block counters.
+// routing is re-derived exactly.
 constexpr int kCtrlBytes = 256;
-constexpr int kCtrlSplitCnt = 32;
-static_assert(kCtrlSplitCnt + kMaxExpertsCfg / 32 <= kCtrlBytes / 4, "control block");
 
 struct WsLayout {
   size_t z, unc, tile_hist, idx, w, counts, offsets, perm, inv_perm, gu_start, dn_start, ready, nitems, h_r,
@@ -66,7 +64,6 @@ struct WsLayout {
   // MXFP4 routed weights only: touched-expert slots and their bf16 copies
   size_t slot_of, touched, ntouched, wq_g, wq_u, wq_d;
   size_t wr_split;  // router matrix as three bf16 terms (batches above 32 tokens)
-  size_t zpart;     // split-K router partials [H/128][T][E] fp32 (batches up to 32 tokens)
   size_t x_perm;    // routed token rows in permuted order [T*K][H] bf16 (pair FFN only)
   int max_touched;
   int n_ptiles, bn, max_items_gu, max_items_dn;
@@ -77,14 +74,11 @@ WsLayout ws_layout(const moe_cfg& c, int T);
 // Launchers (return cudaGetLastError()).
 // Routing. unc [T] / unc_n: scratch list (and its count, zeroed by the
 // caller) of tokens whose fp32 decision is re-derived from exact logits.
-// Scratch, by batch size: wr_split [3][E][H] bf16 for the router matrix as
-// three bf16 terms (tensor-core logits, T > 32); zpart [H/128][T][E] fp32 for
-// the split-K fp32 logits (T <= 32), with split_cnt [E/32] counters zeroed
-// by the caller. The ones the batch size does not use may be nullptr.
+// wr_split: scratch [3][E][H] bf16 for the router matrix as three bf16 terms
+// (tensor-core logits, T > 32); nullptr for smaller batches.
 cudaError_t launch_router(const moe_cfg& c, int T, const uint16_t* x, const float* Wr,
                           const float* bias, float* z, int32_t* idx, float* w, int32_t* unc,
-                          int32_t* unc_n, int32_t* err, uint16_t* wr_split, float* zpart,
-                          int32_t* split_cnt, cudaStream_t s);
+                          int32_t* unc_n, int32_t* err, uint16_t* wr_split, cudaStream_t s);
 
 cudaError_t launch_permute(const moe_cfg& c, int T, const int32_t* idx, int32_t* tile_hist,
                            int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv_perm,

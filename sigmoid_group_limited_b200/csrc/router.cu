@@ -26,22 +26,24 @@ namespace sgl {
 namespace {
 
 // ---------------------------------------------------------------------------
-// Logits for small batches (T <= 32), split over K: CTA (s, eb) forms the
-// partial dot products of all tokens with experts [32 eb, 32 eb + 32) over
-// hidden columns [128 s, 128 s + 128), in fp32, and writes them to
-// zpart[s][t][e]. Lane t
-// of every warp holds token t's 128 columns in registers, the 32 router rows
-// of the block sit in shared memory and are read as broadcasts, and warp w
-// accumulates experts 4w .. 4w+3 of the block: no cross-lane reduction.
-// block_cnt[eb] counts the finished CTAs of expert block eb (zeroed by the
-// caller); the last one writes z[t][e] = sum over s of zpart[s][t][e].
+// Logits for small batches (T <= 32), split over K inside thread-block
+// clusters: cluster b (8 CTAs) owns experts [32 b, 32 b + 32); CTA r of it
+// forms the fp32 partial dot products of all tokens with those experts over
+// hidden columns [r C, r C + C), C = H / 8 rounded up to 64. Lane t of every
+// warp is token t, the block's router rows sit in shared memory and are read
+// as broadcasts, and warp w accumulates experts 4w .. 4w+3: no cross-lane
+// reduction. The eight partials are then added in rank order through
+// distributed shared memory, each CTA finishing 4 of the 32 tokens, so z is
+// the same whichever CTA finishes first.
 // ---------------------------------------------------------------------------
 constexpr int kSmallT = 32;
 constexpr int kRowRegs = 24;  // float4 per lane in router_refine: H <= 24 * 128 = 3072
 constexpr int kMaxExperts = 1024;
-constexpr int kSplitH = 128;  // hidden columns per partial
-constexpr int kSplitE = 32;   // experts per CTA
-constexpr int kMaxSplit = kRowRegs * 128 / kSplitH;  // H <= 3072
+constexpr int kClusterK = 8;                               // CTAs splitting H
+constexpr int kSplitE = 32;                                // experts per cluster
+constexpr int kMaxChunk = kRowRegs * 128 / kClusterK;      // H <= 3072: 384 columns per CTA
+constexpr int kXRow = kMaxChunk + 8;                       // bf16, padded: 8 lanes hit 8 bank groups
+constexpr int kLogitsSmem = kSplitE * kMaxChunk * 4 + kSmallT * kXRow * 2 + kSmallT * (kSplitE + 1) * 4;
 
 // bf16 bits -> float64 by field arithmetic (no conversion instruction):
 // sign, exponent rebiased from 127 to 1023, 7 mantissa bits on top.
@@ -54,45 +56,39 @@ __device__ __forceinline__ double bf16_bits_to_double(uint32_t b) {
   return __longlong_as_double(static_cast<long long>(bits));
 }
 
-__global__ void __launch_bounds__(256) router_logits_splitk(int T, int H, int E,
-                                                           const uint16_t* __restrict__ x,
-                                                           const float* __restrict__ Wr,
-                                                           float* __restrict__ zpart,
-                                                           int32_t* __restrict__ block_cnt,
-                                                           float* __restrict__ z) {
+__global__ void __cluster_dims__(kClusterK, 1, 1) __launch_bounds__(256)
+    router_logits_cluster(int T, int H, int E, const uint16_t* __restrict__ x,
+                          const float* __restrict__ Wr, float* __restrict__ z) {
   pdl_trigger();
-  pdl_wait();  // inputs come from earlier kernels on the stream
-  __shared__ __align__(16) float ws[kSplitE][kSplitH];
-  // token rows of the chunk, padded by 16 bytes so that 8 lanes reading the
-  // same column of 8 rows hit 8 different bank groups
-  constexpr int kXRow = kSplitH + 8;  // bf16 elements
-  __shared__ __align__(16) uint16_t xs[kSmallT][kXRow];
-  __shared__ float out[kSmallT][kSplitE + 1];
-  __shared__ int is_last;
+  extern __shared__ __align__(16) uint8_t lsm[];
+  float* ws = reinterpret_cast<float*>(lsm);                                  // [32][kMaxChunk]
+  uint16_t* xs = reinterpret_cast<uint16_t*>(ws + kSplitE * kMaxChunk);       // [32][kXRow]
+  float* out = reinterpret_cast<float*>(xs + kSmallT * kXRow);                // [32][33]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int s = blockIdx.x, e0 = blockIdx.y * kSplitE;
-  const int k0 = s * kSplitH, kn = min(kSplitH, H - k0);  // kn is a multiple of 64
-  // the block's router rows and the batch's token columns, all copies in
-  // flight at once (16-byte cp.async); zeros past the ends
+  const uint32_t r = cluster_ctarank();
+  const int e0 = blockIdx.y * kSplitE;
+  const int chunk = ((H / 64 + kClusterK - 1) / kClusterK) * 64;
+  const int k0 = static_cast<int>(r) * chunk;
+  const int kn = max(0, min(chunk, H - k0));  // a multiple of 64, possibly 0
+  pdl_wait();  // x may come from an earlier kernel on the stream
+  // the block's router rows and the batch's token columns, all copies in flight
   const uint64_t pol = policy_evict_first();
-#pragma unroll
-  for (int it = 0; it < kSplitE * kSplitH / 4 / 256; ++it) {
-    const int i = tid + 256 * it;
-    const int r = i / (kSplitH / 4), c = 4 * (i % (kSplitH / 4));
-    if (c < kn && e0 + r < E)
-      cp_async16(&ws[r][c], Wr + static_cast<size_t>(e0 + r) * H + k0 + c, pol);
+  for (int i = tid; i < kSplitE * (kMaxChunk / 4); i += blockDim.x) {
+    const int row = i / (kMaxChunk / 4), c = 4 * (i % (kMaxChunk / 4));
+    float* dst = ws + row * kMaxChunk + c;
+    if (c < kn && e0 + row < E)
+      cp_async16(dst, Wr + static_cast<size_t>(e0 + row) * H + k0 + c, pol);
     else
-      *reinterpret_cast<float4*>(&ws[r][c]) = make_float4(0.f, 0.f, 0.f, 0.f);
+      *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
   }
   const uint64_t pol_x = policy_evict_last();
-#pragma unroll
-  for (int it = 0; it < kSmallT * kSplitH / 8 / 256; ++it) {
-    const int i = tid + 256 * it;
-    const int r = i / (kSplitH / 8), c = 8 * (i % (kSplitH / 8));
-    if (r < T && c < kn)
-      cp_async16(&xs[r][c], x + static_cast<size_t>(r) * H + k0 + c, pol_x);
+  for (int i = tid; i < kSmallT * (kMaxChunk / 8); i += blockDim.x) {
+    const int row = i / (kMaxChunk / 8), c = 8 * (i % (kMaxChunk / 8));
+    uint16_t* dst = xs + row * kXRow + c;
+    if (row < T && c < kn)
+      cp_async16(dst, x + static_cast<size_t>(row) * H + k0 + c, pol_x);
     else
-      *reinterpret_cast<uint4*>(&xs[r][c]) = make_uint4(0u, 0u, 0u, 0u);
+      *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
   }
   cp_async_commit();
   cp_async_wait<0>();
@@ -102,8 +98,8 @@ __global__ void __launch_bounds__(256) router_logits_splitk(int T, int H, int E,
 #pragma unroll
   for (int q = 0; q < EW; ++q) acc[q] = 0.f;
 #pragma unroll 4
-  for (int i = 0; i < kSplitH / 8; ++i) {
-    const uint4 xv8 = *reinterpret_cast<const uint4*>(&xs[lane][8 * i]);
+  for (int i = 0; i < kn / 8; ++i) {
+    const uint4 xv8 = *reinterpret_cast<const uint4*>(xs + lane * kXRow + 8 * i);
     const uint32_t pk[4] = {xv8.x, xv8.y, xv8.z, xv8.w};
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -113,7 +109,7 @@ __global__ void __launch_bounds__(256) router_logits_splitk(int T, int H, int E,
       const float xv3 = __uint_as_float(pk[2 * h + 1] & 0xFFFF0000u);
 #pragma unroll
       for (int q = 0; q < EW; ++q) {
-        const float4 wv = *reinterpret_cast<const float4*>(&ws[warp * EW + q][8 * i + 4 * h]);
+        const float4 wv = *reinterpret_cast<const float4*>(ws + (warp * EW + q) * kMaxChunk + 8 * i + 4 * h);
         acc[q] = fmaf(xv0, wv.x, acc[q]);
         acc[q] = fmaf(xv1, wv.y, acc[q]);
         acc[q] = fmaf(xv2, wv.z, acc[q]);
@@ -122,44 +118,18 @@ __global__ void __launch_bounds__(256) router_logits_splitk(int T, int H, int E,
     }
   }
 #pragma unroll
-  for (int q = 0; q < EW; ++q) out[lane][warp * EW + q] = acc[q];
-  __syncthreads();
-  for (int i = tid; i < T * kSplitE; i += blockDim.x) {
-    const int t = i / kSplitE, c = i % kSplitE;
-    if (e0 + c < E) zpart[(static_cast<size_t>(s) * T + t) * E + e0 + c] = out[t][c];
+  for (int q = 0; q < EW; ++q) out[lane * (kSplitE + 1) + warp * EW + q] = acc[q];
+  cluster_sync();  // every CTA's partials are in its shared memory
+  // CTA r adds tokens 4r .. 4r+3 over the eight partials, in rank order
+  if (tid < (kSmallT / kClusterK) * kSplitE) {
+    const int t = static_cast<int>(r) * (kSmallT / kClusterK) + tid / kSplitE, c = tid % kSplitE;
+    const uint32_t loc = smem_u32(out + t * (kSplitE + 1) + c);
+    float sum = 0.f;
+#pragma unroll
+    for (int q = 0; q < kClusterK; ++q) sum += ld_shared_cluster_f32(mapa_shared(loc, q));
+    if (t < T && e0 + c < E) z[static_cast<size_t>(t) * E + e0 + c] = sum;
   }
-  // The last CTA of this expert block to finish adds the block's partials in
-  // split order (so z does not depend on which CTA came last).
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) is_last = atomicAdd(&block_cnt[blockIdx.y], 1) == static_cast<int>(gridDim.x) - 1;
-  __syncthreads();
-  if (!is_last) return;
-  __threadfence();
-  const int nsplit = gridDim.x;
-  const size_t stride = static_cast<size_t>(T) * E;
-  constexpr int kPer = kSmallT * kSplitE / 256;  // outputs per thread, taken two at a time
-#pragma unroll 1
-  for (int r0 = 0; r0 < kPer; r0 += 2) {
-    float v[2][kMaxSplit];
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int i = tid + 256 * (r0 + r), t = i / kSplitE, c = i % kSplitE;
-      const bool ok = t < T && e0 + c < E;
-      const float* pp = zpart + static_cast<size_t>(ok ? t : 0) * E + (ok ? e0 + c : 0);
-#pragma unroll
-      for (int sp = 0; sp < kMaxSplit; ++sp) v[r][sp] = sp < nsplit ? __ldcg(pp + sp * stride) : 0.f;
-    }
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int i = tid + 256 * (r0 + r), t = i / kSplitE, c = i % kSplitE;
-      float sum = 0.f;
-#pragma unroll
-      for (int sp = 0; sp < kMaxSplit; ++sp)
-        if (sp < nsplit) sum += v[r][sp];
-      if (t < T && e0 + c < E) z[static_cast<size_t>(t) * E + e0 + c] = sum;
-    }
-  }
+  cluster_sync();  // no CTA exits while another may still read its partials
 }
 
 // Order-preserving map of a (non-NaN) float onto nonzero uint32 keys, and back.
@@ -964,16 +934,15 @@ constexpr float kCertifyMargin = 1.0f / 32768.0f;
 
 cudaError_t launch_router(const moe_cfg& c, int T, const uint16_t* x, const float* Wr,
                           const float* bias, float* z, int32_t* idx, float* w, int32_t* unc,
-                          int32_t* unc_n, int32_t* err, uint16_t* wr_split, float* zpart,
-                          int32_t* split_cnt, cudaStream_t s) {
+                          int32_t* unc_n, int32_t* err, uint16_t* wr_split, cudaStream_t s) {
   cudaError_t e;
   if (c.H > kRowRegs * 128) return cudaErrorInvalidValue;
   if (T <= kSmallT) {
-    // fp32 split-K partials, added in order by the last CTA of each expert block
-    if (zpart == nullptr || split_cnt == nullptr) return cudaErrorInvalidValue;
-    const int nsplit = cdiv(c.H, kSplitH);
-    e = launch_pdl(router_logits_splitk, dim3(nsplit, cdiv(c.E, kSplitE)), dim3(256), 0, s, T, c.H,
-                   c.E, x, Wr, zpart, split_cnt, z);
+    // fp32 split-K logits in clusters of kClusterK CTAs
+    e = ensure_dyn_smem(reinterpret_cast<const void*>(router_logits_cluster), kLogitsSmem);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(router_logits_cluster, dim3(kClusterK, cdiv(c.E, kSplitE)), dim3(256),
+                   static_cast<size_t>(kLogitsSmem), s, T, c.H, c.E, x, Wr, z);
   } else {
     // tensor cores: split the router matrix, then one bf16 x 3 GEMM into z
     if (wr_split == nullptr) return cudaErrorInvalidValue;
