@@ -532,6 +532,42 @@ __device__ __forceinline__ void load_scores(const float* zr, const float* bias, 
   *zz_out = zz;
 }
 
+// Value of the kth candidate (1-based) in the ranking by biased score, ties
+// to the lower expert id; the last one found if there are fewer. Each lane
+// keeps its own best; a round is a warp max of the keys, then the lowest id
+// among the lanes holding it, and only the winning lane rescans.
+template <int NV>
+__device__ __forceinline__ float kth_candidate_value(uint32_t cand, const float* b, int kth,
+                                                     int lane) {
+  uint32_t lkey = 0u;
+  int lj = 0;
+  auto rescan = [&]() {
+    lkey = 0u;
+    float bv = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < NV; ++j)
+      if (((cand >> j) & 1u) && (lkey == 0u || b[j] > bv)) {
+        bv = b[j];
+        lj = j;
+        lkey = order_key(bv);
+      }
+  };
+  rescan();
+  float v = -INFINITY;
+  for (int k = 0; k < kth; ++k) {
+    const uint32_t mk = __reduce_max_sync(0xffffffffu, lkey);
+    if (mk == 0u) break;
+    const uint32_t be = __reduce_min_sync(
+        0xffffffffu, (lkey == mk) ? static_cast<uint32_t>(lj * 32 + lane) : 0xffffffffu);
+    v = key_value(mk);
+    if (lane == static_cast<int>(be & 31)) {
+      cand &= ~(1u << (be >> 5));
+      rescan();
+    }
+  }
+  return v;
+}
+
 template <int NV>
 __global__ void __launch_bounds__(kRefineThreads) router_refine(
     int T, int H, int E, int n_group, int topk_group, int K, float scale, int renorm,
@@ -561,18 +597,20 @@ __global__ void __launch_bounds__(kRefineThreads) router_refine(
 
     // ---- warp 0: fp32 scores, group scores, the experts that decide group maxima
     float b[NV];
+    int gj[NV];  // group of register slot j (-1 past E)
     float tau_t = 0.f, gth = -INFINITY;
     if (warp == 0) {
       float zz;
       load_scores<NV>(z + static_cast<size_t>(t) * E, bias, E, lane, b, &zz);
       tau_t = tau * fmaxf(1.f, sqrtf(zz / E));
+#pragma unroll
+      for (int j = 0; j < NV; ++j) gj[j] = lane + 32 * j < E ? (lane + 32 * j) / per : -1;
       for (int g = 0; g < n_group; ++g) {
         float m = -INFINITY;
 #pragma unroll
         for (int j = 0; j < NV; ++j)
-          if ((lane + 32 * j) / per == g && b[j] > m) m = b[j];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+          if (gj[j] == g && b[j] > m) m = b[j];
+        m = key_value(__reduce_max_sync(0xffffffffu, order_key(m)));
         if (lane == 0) gsc[g] = m;
       }
       __syncwarp();
@@ -592,7 +630,7 @@ __global__ void __launch_bounds__(kRefineThreads) router_refine(
         const int e = lane + 32 * j;
         bool nd = false;
         if (e < E) {
-          const float gs = gsc[e / per];
+          const float gs = gsc[gj[j]];
           nd = gs >= gth - tau_t && b[j] >= gs - tau_t;
         }
         const unsigned bal = __ballot_sync(0xffffffffu, nd);
@@ -654,59 +692,25 @@ __global__ void __launch_bounds__(kRefineThreads) router_refine(
               const int e = need[i];
               if (e / per == g) m = fmaxf(m, bex[e]);
             }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            m = key_value(__reduce_max_sync(0xffffffffu, order_key(m)));
           }
           if (lane == g) gex = m;
         }
         uint32_t kept = 0;
         for (int r = 0; r < topk_group; ++r) {
-          float bv = lane < n_group && !((kept >> lane) & 1u) ? gex : -INFINITY;
-          int bi = lane < n_group && !((kept >> lane) & 1u) ? lane : 0x7fffffff;
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            if (ov > bv || (ov == bv && oi < bi)) {
-              bv = ov;
-              bi = oi;
-            }
-          }
+          // best remaining group, ties to the lower group
+          const bool avail = lane < n_group && !((kept >> lane) & 1u);
+          const uint32_t mk = __reduce_max_sync(0xffffffffu, avail ? order_key(gex) : 0u);
+          const uint32_t bi = __reduce_min_sync(
+              0xffffffffu, (avail && order_key(gex) == mk) ? static_cast<uint32_t>(lane) : 0xffffffffu);
           kept |= 1u << bi;
         }
         // (K+1)-th largest fp32 score among the kept groups' experts
         uint32_t cand = 0;
 #pragma unroll
-        for (int j = 0; j < NV; ++j) {
-          const int e = lane + 32 * j;
-          if (e < E && ((kept >> (e / per)) & 1u)) cand |= 1u << j;
-        }
-        float bth = -INFINITY;
-        {
-          uint32_t c2 = cand;
-          for (int k = 0; k <= K; ++k) {
-            float bv = -INFINITY;
-            int be = 0x7fffffff;
-#pragma unroll
-            for (int j = 0; j < NV; ++j)
-              if (((c2 >> j) & 1u) && (be == 0x7fffffff || b[j] > bv)) {
-                bv = b[j];
-                be = lane + 32 * j;
-              }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-              const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-              const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-              if (ov > bv || (ov == bv && oe < be)) {
-                bv = ov;
-                be = oe;
-              }
-            }
-            if (be == 0x7fffffff) break;
-            bth = bv;
-            if ((be & 31) == lane) c2 &= ~(1u << (be >> 5));
-          }
-        }
+        for (int j = 0; j < NV; ++j)
+          if (gj[j] >= 0 && ((kept >> gj[j]) & 1u)) cand |= 1u << j;
+        const float bth = kth_candidate_value<NV>(cand, b, K + 1, lane);
         if (lane == 0) {
           kept_mask_s = static_cast<int>(kept);
           n_need = 0;
@@ -756,36 +760,9 @@ __global__ void __launch_bounds__(kRefineThreads) router_refine(
       // recompute the pool membership (same rule as above) from registers
       uint32_t cand = 0;
 #pragma unroll
-      for (int j = 0; j < NV; ++j) {
-        const int e = lane + 32 * j;
-        if (e < E && ((kept >> (e / per)) & 1u)) cand |= 1u << j;
-      }
-      float bth = -INFINITY;
-      {
-        uint32_t c2 = cand;
-        for (int k = 0; k <= K; ++k) {
-          float bv = -INFINITY;
-          int be = 0x7fffffff;
-#pragma unroll
-          for (int j = 0; j < NV; ++j)
-            if (((c2 >> j) & 1u) && (be == 0x7fffffff || b[j] > bv)) {
-              bv = b[j];
-              be = lane + 32 * j;
-            }
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-            if (ov > bv || (ov == bv && oe < be)) {
-              bv = ov;
-              be = oe;
-            }
-          }
-          if (be == 0x7fffffff) break;
-          bth = bv;
-          if ((be & 31) == lane) c2 &= ~(1u << (be >> 5));
-        }
-      }
+      for (int j = 0; j < NV; ++j)
+        if (gj[j] >= 0 && ((kept >> gj[j]) & 1u)) cand |= 1u << j;
+      const float bth = kth_candidate_value<NV>(cand, b, K + 1, lane);
       uint32_t pool = 0;
 #pragma unroll
       for (int j = 0; j < NV; ++j)
@@ -805,15 +782,11 @@ __global__ void __launch_bounds__(kRefineThreads) router_refine(
             }
           }
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-          const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-          if (ov > bv || (ov == bv && oe < be)) {
-            bv = ov;
-            be = oe;
-          }
-        }
+        // best remaining pool member by exact score, ties to the lower expert id
+        const uint32_t lk = be != 0x7fffffff ? order_key(bv) : 0u;
+        const uint32_t mk = __reduce_max_sync(0xffffffffu, lk);
+        be = static_cast<int>(__reduce_min_sync(
+            0xffffffffu, (lk != 0u && lk == mk) ? static_cast<uint32_t>(be) : 0xffffffffu));
         if ((be & 31) == lane) pool &= ~(1u << (be >> 5));
         if (lane == k) {
           my_e = be;
