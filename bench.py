@@ -342,11 +342,18 @@ def measure_gpu(cfg, steps, warmup, device, rank, clk, with_e2e=True):
     dev_ms = sum(per_step)
     assert sgl.moe_read_error(cfg, T, ws) == 0
     del graph
-    touched = int((counts > 0).sum().item())
-    cnt = counts.cpu().numpy()
+    # load statistics of the last step's routing, from the library (outside the timed region)
+    rstats = torch.empty(sgl.MOE_N_ROUTE_STATS, dtype=torch.float64, device=device)
+    sgl.moe_route_stats(cfg, counts, rstats, stream=stream)
+    st = dict(zip(sgl.ROUTE_STATS_NAMES, rstats.cpu().tolist()))
     out = dict(device_ms_total=dev_ms, plain_ms_total=sum(per_step_plain), wall_s=wall,
                per_step_ms=per_step, stage_ms=stage_ms,
-               touched=touched, load_max=int(cnt.max()), load_mean=float(cnt.mean()),
+               routing={"experts_touched": cfg.E - int(st["idle_experts"]),
+                        "idle_experts": int(st["idle_experts"]), "load_max": int(st["load_max"]),
+                        "load_mean": round(st["load_mean"], 2),
+                        "max_over_mean": round(st["max_over_mean"], 3),
+                        "entropy_bits": round(st["entropy_bits"], 4),
+                        "entropy_normalized": round(st["entropy_normalized"], 4)},
                d=d, launches=kernels_per_step(cfg) * 2 * steps)
 
     if with_e2e:
@@ -526,7 +533,7 @@ def run_native(args, rank, world, local):
     tokens = cfg.T * args.steps * world
 
     def roof(cfg_, mm):
-        work = algorithmic_work(cfg_, cfg_.T, mm["touched"])
+        work = algorithmic_work(cfg_, cfg_.T, mm["routing"]["experts_touched"])
         # the dominant kernel is the fused expert FFN (gate/up and down in one launch)
         b = work["gateup"][0] + work["down"][0]
         f = work["gateup"][1] + work["down"][1]
@@ -536,7 +543,7 @@ def run_native(args, rank, world, local):
                    traffic_unit="bytes per launch (ncu DRAM read+write, scaled from the "
                                 "small-case capture of the same kernel)",
                    peak_source=f"{peaks['source']} ({'HBM copy' if ent['bound'] == 'hbm' else 'cuBLAS bf16 burst'})",
-                   units_per_launch=f"{cfg_.T} tokens, {mm['touched']} routed experts + shared")
+                   units_per_launch=f"{cfg_.T} tokens, {mm['routing']['experts_touched']} routed experts + shared")
         lb, lf = work["layer"]
         t_roof = max(lb / (peaks["hbm_gbs"] * 1e9), lf / (peaks["bf16_tflops"] * 1e12))
         step_s = statistics.mean(mm["per_step_ms"]) / 1e3
@@ -553,8 +560,7 @@ def run_native(args, rank, world, local):
             "config": config_block(cfg, world), "roofline": ent,
             "layer_roofline_frac": layer_frac,
             "stage_ms": {k: round(v, 4) for k, v in m["stage_ms"].items()},
-            "routing": {"experts_touched": m["touched"], "load_max": m["load_max"],
-                        "load_mean": round(m["load_mean"], 2)},
+            "routing": m["routing"],
             "e2e": {"value": round(tokens / e2e_s, 1), "unit": "tokens/s",
                     "h2d_bytes_per_step": m["e2e_h2d"], "d2h_bytes_per_step": m["e2e_d2h"]},
             "gpu_launches": m["launches"], "clocks": clocks}
@@ -568,8 +574,7 @@ def run_native(args, rank, world, local):
                            "ms_per_step": round(1e3 * a_s / args.steps, 4), "roofline": aent,
                            "layer_roofline_frac": afrac,
                            "stage_ms": {k: round(v, 4) for k, v in am["stage_ms"].items()},
-                           "routing": {"experts_touched": am["touched"], "load_max": am["load_max"],
-                                       "load_mean": round(am["load_mean"], 2)},
+                           "routing": am["routing"],
                            "config": config_block(acfg, world)}
         line["gpu_launches"] += am["launches"]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

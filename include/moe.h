@@ -176,6 +176,22 @@ MOE_API moe_status moe_layer_forward(const moe_cfg* cfg, int32_t T, const void* 
                              float* w_out, int32_t* counts_out, void* ws, size_t ws_bytes,
                              void* stream, void* const* stage_events);
 
+/* Routing statistics from the expert counts that moe_permute and
+ * moe_layer_forward produce: the load monitoring of page 1 ("Ling-3.0-flash-VL：
+ * 层级化稀疏路由大模型硬核解析", sec. 4.1: routing entropy and experts that are
+ * never selected), for the balancing that page 3 sec. 3 step 3 describes.
+ * in: counts [E] int32 (device; negative entries count as 0);
+ * out: stats [MOE_N_ROUTE_STATS] float64 (device):
+ *   [0] entropy H = -sum_e p_e log2 p_e, p_e = counts_e / sum(counts), bits
+ *       (0 when the sum is 0)
+ *   [1] H / log2(E)  (1 = every expert equally loaded)
+ *   [2] max load      [3] mean load = sum / E      [4] max / mean
+ *   [5] idle experts (count 0)                      [6] sum of the counts
+ * Deterministic (fixed summation order). Asynchronous on `stream`. */
+#define MOE_N_ROUTE_STATS 7
+MOE_API moe_status moe_route_stats(const moe_cfg* cfg, const int32_t* counts, double* stats,
+                                   void* stream);
+
 /* Reads (synchronously, on `stream`) and clears the workspace error word.
  * *code = 0 when no kernel reported a problem; otherwise one of the
  * MOE_DEVERR_* values below. Returns MOE_OK or MOE_ERR_CUDA. */

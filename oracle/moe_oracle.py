@@ -23,6 +23,9 @@ Sources (page title, section):
                       gate/up/down, hidden 2560, intermediate 768
   [P4] "Ling-3.0-flash-VL 42-layer hybrid backbone" (lpnh.cn/news/2815793),
        spec table: routed-expert weights in MXFP4 (4 bit).
+  [P1] "Ling-3.0-flash-VL：层级化稀疏路由大模型硬核解析" (sheratonhq.com/news/113555),
+       sec. 4.1: monitor the routing entropy of the expert selection
+       frequencies and the experts that are never selected.
 
 Readings where the pages are silent (each also listed in the design notes):
   R1 group score = max over the group of the BIASED score b = s + bias.
@@ -212,6 +215,26 @@ def permute(idx: np.ndarray, E: int):
     inv_perm = np.empty_like(perm)
     inv_perm[perm] = np.arange(perm.size, dtype=np.int32)
     return counts, offsets, perm, inv_perm
+
+
+def route_stats(counts: np.ndarray, E: int) -> np.ndarray:
+    """Load statistics of one routing pass from its expert counts ([P1] sec. 4.1).
+
+    p_e = counts[e] / sum(counts); returns float64 [7]:
+      0 H = -sum_{p_e > 0} p_e log2 p_e (bits), 1 H / log2 E, 2 max count,
+      3 mean count (sum / E), 4 max / mean, 5 experts with count 0, 6 sum.
+    With no slots at all every entry but the idle count (= E) is 0.
+    """
+    c = np.asarray(counts, dtype=np.int64)[:E]
+    tot = float(c.sum())
+    H = 0.0
+    if tot > 0:
+        p = c[c > 0] / tot
+        H = float(-(p * np.log2(p)).sum())
+    mx = float(c.max()) if E > 0 else 0.0
+    mean = tot / E
+    return np.array([H, H / math.log2(E) if E > 1 else 0.0, mx, mean,
+                     mx / mean if mean > 0 else 0.0, float((c == 0).sum()), tot])
 
 
 # --------------------------------------------------------------------------

@@ -29,7 +29,7 @@ STATUS = {0: "MOE_OK", -1: "MOE_ERR_CFG", -2: "MOE_ERR_NULL", -3: "MOE_ERR_ALIGN
 DEVERR = {0: "none", 1: "expert id out of range", 2: "pipeline wait timed out",
           3: "work item out of range"}
 
-C_FUNCTIONS = ("moe_workspace_size", "moe_route", "moe_permute", "moe_permute_static",
+C_FUNCTIONS = ("moe_workspace_size", "moe_route", "moe_permute", "moe_permute_static", "moe_route_stats",
                "moe_grouped_swiglu",
                "moe_combine", "moe_layer_forward", "moe_read_error", "moe_status_string",
                "moe_version")
@@ -77,11 +77,13 @@ def lib() -> ctypes.CDLL:
     L.moe_grouped_swiglu.argtypes = [cp, i32, vp, vp, vp, vp, wp, vp, vp, sz, vp]
     L.moe_combine.argtypes = [cp, i32, vp, i32, vp, vp]
     L.moe_layer_forward.argtypes = [cp, i32, vp, vp, vp, wp, vp, vp, vp, vp, vp, sz, vp, vp]
+    L.moe_route_stats.argtypes = [cp, vp, vp, vp]
     L.moe_read_error.argtypes = [cp, i32, vp, sz, vp, ctypes.POINTER(i32)]
     L.moe_status_string.argtypes = [i32]
     L.moe_status_string.restype = ctypes.c_char_p
     L.moe_version.restype = ctypes.c_char_p
-    for f in ("moe_route", "moe_permute", "moe_permute_static", "moe_grouped_swiglu", "moe_combine",
+    for f in ("moe_route", "moe_permute", "moe_permute_static", "moe_route_stats", "moe_grouped_swiglu",
+              "moe_combine",
               "moe_layer_forward", "moe_read_error"):
         getattr(L, f).restype = i32
     _lib = L
@@ -152,6 +154,19 @@ def moe_permute_static(cfg, T, idx, counts, offsets, perm, inv_perm, stream=None
     c = make_cfg(cfg)
     _check(lib().moe_permute_static(ctypes.byref(c), int(T), _p(idx), _p(counts), _p(offsets),
                                     _p(perm), _p(inv_perm), _stream(stream)), "moe_permute_static")
+
+
+MOE_N_ROUTE_STATS = 7
+ROUTE_STATS_NAMES = ("entropy_bits", "entropy_normalized", "load_max", "load_mean", "max_over_mean",
+                     "idle_experts", "slots")
+
+
+def moe_route_stats(cfg, counts, stats, stream=None):
+    """Routing statistics from expert counts into `stats` (float64 [7], device);
+    see ROUTE_STATS_NAMES for the entries."""
+    c = make_cfg(cfg)
+    _check(lib().moe_route_stats(ctypes.byref(c), _p(counts), _p(stats), _stream(stream)),
+           "moe_route_stats")
 
 
 def moe_grouped_swiglu(cfg, T, x, perm, offsets, w, weights: moe_weights, y_slot, ws, stream=None):

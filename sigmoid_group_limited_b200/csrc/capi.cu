@@ -379,6 +379,16 @@ moe_status moe_layer_forward(const moe_cfg* cfg, int32_t T, const void* x, const
   return MOE_OK;
 }
 
+moe_status moe_route_stats(const moe_cfg* cfg, const int32_t* counts, double* stats,
+                           void* stream) {
+  if (!cfg_ok(cfg)) return MOE_ERR_CFG;
+  if (!counts || !stats) return MOE_ERR_NULL;
+  if (!al16(counts) || !al16(stats)) return MOE_ERR_ALIGN;
+  moe_status st = device_ok();
+  if (st != MOE_OK) return st;
+  return cu(launch_route_stats(*cfg, counts, stats, static_cast<cudaStream_t>(stream)));
+}
+
 moe_status moe_read_error(const moe_cfg* cfg, int32_t T, void* ws, size_t ws_bytes, void* stream,
                           int32_t* code) {
   if (!cfg_ok(cfg) || !T_ok(T)) return MOE_ERR_CFG;

@@ -176,6 +176,10 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   return cudaLaunchKernelEx(&lc, kern, static_cast<Args&&>(args)...);
 }
 
+// Routing statistics from expert counts (see moe_route_stats in moe.h).
+cudaError_t launch_route_stats(const moe_cfg& c, const int32_t* counts, double* stats,
+                               cudaStream_t s);
+
 int num_sms();
 
 // Tensor map of a bf16 row-major [rows, cols] matrix for TMA: box of

@@ -274,6 +274,56 @@ def test_route_full_size_every_token(T, E):
     assert len(near) <= max(2, T // 500)
 
 
+# ------------------------------------------------------------------ load statistics
+
+def _stat_counts(kind, E, seed):
+    rng = np.random.default_rng(seed)
+    if kind == "uniform":
+        return np.full(E, 64, np.int32)
+    if kind == "zipf":
+        c = rng.zipf(1.3, size=E).clip(max=1 << 20)
+        return (c * (rng.random(E) < 0.6)).astype(np.int32)
+    if kind == "one":
+        c = np.zeros(E, np.int32)
+        c[E // 3] = 4096 * 8
+        return c
+    return np.zeros(E, np.int32)
+
+
+@pytest.mark.parametrize("E", [32, 128, 512, 1024])
+@pytest.mark.parametrize("kind", ["uniform", "zipf", "one", "empty"])
+def test_route_stats(E, kind):
+    """Entropy, load and idle experts against the oracle on the same counts.
+    Integer entries exact; entropy terms are summed in another order, so
+    H and H / log2 E agree to 1e-12 relative."""
+    cfg = workloads.CONFIGS["prefill"].with_(E=E, n_group=1, topk_group=1, K=1)
+    counts = _stat_counts(kind, E, seed=E)
+    st = torch.full((sgl.MOE_N_ROUTE_STATS,), float("nan"), dtype=torch.float64, device=DEV)
+    sgl.moe_route_stats(cfg, torch.from_numpy(counts).to(DEV), st)
+    torch.cuda.synchronize()
+    got, ref = st.cpu().numpy(), oracle.route_stats(counts, E)
+    assert np.array_equal(got[[2, 5, 6]], ref[[2, 5, 6]])
+    assert np.allclose(got, ref, rtol=1e-12, atol=1e-13)
+
+
+def test_route_stats_after_routing():
+    """The statistics read the counts that routing and the permutation left in
+    device memory, on the same stream, with no copy in between."""
+    cfg = workloads.CONFIGS["prefill"]
+    T = 4096
+    idx = torch.randint(0, cfg.E, (T, cfg.K), dtype=torch.int32,
+                        generator=torch.Generator().manual_seed(5))
+    ws = sgl.alloc_workspace(cfg, T)
+    out = [torch.empty(n, dtype=torch.int32, device=DEV)
+           for n in (cfg.E, cfg.E + 1, T * cfg.K, T * cfg.K)]
+    st = torch.empty(sgl.MOE_N_ROUTE_STATS, dtype=torch.float64, device=DEV)
+    sgl.moe_permute(cfg, T, idx.to(DEV), *out, ws)
+    sgl.moe_route_stats(cfg, out[0], st)
+    torch.cuda.synchronize()
+    ref = oracle.route_stats(oracle.permute(idx.numpy(), cfg.E)[0], cfg.E)
+    assert np.allclose(st.cpu().numpy(), ref, rtol=1e-12, atol=1e-13)
+
+
 @pytest.mark.parametrize("T,variant", [(64, {}), (300, dict(limit_routed=0.5, limit_shared=0.7)),
                                        (7, dict(I=128, I_shared=192))])
 def test_tiny_mxfp4(T, variant):

@@ -270,3 +270,51 @@ def test_permutation_one_expert_takes_all():
     counts, offsets, perm, _ = oracle.permute(idx, 8)
     assert counts[5] == 10 and offsets[5] == 0 and offsets[6] == 10
     assert np.array_equal(perm, np.arange(10))
+
+
+# ---------------------------------------------------------------- load statistics
+
+@pytest.mark.parametrize("E", [2, 8, 128, 512])
+def test_route_stats_uniform_load_has_full_entropy(E):
+    st = oracle.route_stats(np.full(E, 3, np.int32), E)
+    assert st[0] == pytest.approx(math.log2(E), rel=1e-14)   # H of a uniform law
+    assert st[1] == pytest.approx(1.0, rel=1e-14)
+    assert st[2] == 3 and st[3] == 3 and st[4] == 1 and st[5] == 0 and st[6] == 3 * E
+
+
+def test_route_stats_one_expert_takes_all():
+    c = np.zeros(64, np.int32)
+    c[17] = 40
+    st = oracle.route_stats(c, 64)
+    assert st[0] == 0 and st[1] == 0
+    assert st[2] == 40 and st[3] == 40 / 64 and st[4] == 64      # max/mean = E
+    assert st[5] == 63 and st[6] == 40
+
+
+def test_route_stats_worked_dyadic_law():
+    # p = (1/4, 1/4, 1/2, 0): H = 2*(1/4)*2 + (1/2)*1 = 1.5 bits exactly
+    st = oracle.route_stats(np.array([1, 1, 2, 0], np.int32), 4)
+    assert st[0] == 1.5 and st[1] == 0.75
+    assert st[2] == 2 and st[3] == 1 and st[4] == 2 and st[5] == 1 and st[6] == 4
+
+
+def test_route_stats_no_slots():
+    st = oracle.route_stats(np.zeros(32, np.int32), 32)
+    assert list(st) == [0, 0, 0, 0, 0, 32, 0]
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_route_stats_against_counting_loop(seed):
+    rng = np.random.default_rng(seed)
+    E = int(rng.integers(2, 300))
+    counts = rng.zipf(1.5, size=E).clip(max=1000) * (rng.random(E) < 0.7)
+    tot = int(counts.sum())
+    H = sum(-(n / tot) * math.log(n / tot) / math.log(2) for n in counts if n > 0)
+    st = oracle.route_stats(counts.astype(np.int32), E)
+    assert st[0] == pytest.approx(H, rel=1e-12)
+    assert 0 <= st[0] <= math.log2(E - st[5]) + 1e-12          # H <= log2(#experts used)
+    assert st[5] == sum(1 for n in counts if n == 0)
+    assert st[2] == max(counts) and st[6] == tot
+    # relabelling the experts changes nothing
+    assert np.allclose(oracle.route_stats(rng.permutation(counts).astype(np.int32), E), st,
+                       rtol=1e-14, atol=0)
