@@ -78,7 +78,6 @@ WsLayout ws_layout(const moe_cfg& c, int T) {
   L.h_s = take(static_cast<size_t>(T) * (c.I_shared > 0 ? c.I_shared : 0) * 2);
   L.y_slot = take((TK + T) * c.H * 4);
   L.wr_split = T > 32 ? take(static_cast<size_t>(3) * c.E * c.H * 2) : 0;
-  L.x_perm = L.bn == kPairTileN ? take(TK * c.H * 2) : 0;
   if (c.wfmt == MOE_W_MXFP4) {
     L.max_touched = static_cast<int>(TK < static_cast<size_t>(c.E) ? TK : c.E);
     const size_t mat = static_cast<size_t>(L.max_touched) * c.I * c.H * 2;
@@ -261,7 +260,6 @@ moe_status moe_grouped_swiglu(const moe_cfg* cfg, int32_t T, const void* x, cons
   }
   a.h_r = at<uint16_t>(ws, L.h_r);
   a.h_s = at<uint16_t>(ws, L.h_s);
-  a.x_perm = L.bn == kPairTileN ? at<uint16_t>(ws, L.x_perm) : nullptr;
   a.y_slot = static_cast<float*>(y_slot);
   a.offsets = offsets;
   a.gu_start = gu;
@@ -358,7 +356,6 @@ moe_status moe_layer_forward(const moe_cfg* cfg, int32_t T, const void* x, const
   }
   a.h_r = at<uint16_t>(ws, L.h_r);
   a.h_s = at<uint16_t>(ws, L.h_s);
-  a.x_perm = L.bn == kPairTileN ? at<uint16_t>(ws, L.x_perm) : nullptr;
   a.y_slot = y_slot;
   a.offsets = offsets;
   a.gu_start = gu;

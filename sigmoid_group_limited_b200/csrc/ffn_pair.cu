@@ -15,24 +15,26 @@
 //   gate/up item (slot, 256-token tile, 128 features f0..f0+127): CTA r holds
 //       gate rows f0 + 64r .. +63 over up rows f0 + 64r .. +63 (lanes 0-63 /
 //       64-127 of its D); the epilogue pairs lane l with lane l + 64 through
-//       shared memory. B = the item's rows of the token matrix gathered into
-//       routed-row order beforehand (x_perm), or x itself for the shared expert.
+//       shared memory. B = the item's token rows, copied from x by the
+//       gatherer warps of each CTA (16-byte cp.async into the swizzled tile).
 //   down item (slot, 256-token tile, 256 hidden features): CTA r holds Wd rows
 //       256 n + 128 r .. +127; B = h rows.
-// Both operands arrive by TMA (no multicast): each CTA loads its own halves
-// and the byte counts complete on the leader CTA's full barrier; the leader's
+// A and the h rows of down items arrive by TMA (no multicast): each CTA loads
+// its own halves and the byte counts complete on the leader CTA's full
+// barrier, where the gatherer warps of both CTAs also arrive; the leader's
 // MMA thread releases a stage in both CTAs with one multicast commit.
 //
-// Warp roles per CTA (352 threads):
-//   0     TMA producer (lane 0), both CTAs
-//   1     TMEM allocation in both CTAs; MMA issuer (lane 0) in the leader
-//   2..9  epilogue, both CTAs: two warps per TMEM lane quarter (warp % 4),
-//         alternate column chunks
-//   10    scheduler (lane 0), leader: claims items, waits for their inputs
-//         and writes them into the item queues of both CTAs
-// Barriers filled by TMA bytes or by tcgen05.commit are waited on at CTA
-// scope; the ones other threads of the pair arrive on (item queues, the
-// leader's accumulator-empty barriers) at cluster scope.
+// Warp roles per CTA (480 threads):
+//   0      TMA producer (lane 0), both CTAs
+//   1      TMEM allocation in both CTAs; MMA issuer (lane 0) in the leader
+//   2..9   epilogue, both CTAs: two warps per TMEM lane quarter (warp % 4),
+//          alternate column chunks
+//   10..13 token gatherers, both CTAs
+//   14     scheduler (lane 0), leader: claims items, waits for their inputs
+//          and writes them into the item queues of both CTAs
+// Barriers filled by TMA bytes or by tcgen05.commit only are waited on at
+// CTA scope; the ones other threads of the pair arrive on (full stages, item
+// queues, the leader's accumulator-empty barriers) at cluster scope.
 // Every wait is bounded; the two CTAs meet at a cluster barrier after setup
 // and before exit, so no CTA touches the other's shared memory after it left.
 #include <cuda.h>
@@ -51,7 +53,9 @@ namespace {
 
 constexpr int kPEpiWarps = 8;              // warps 2..9, two per TMEM lane quarter
 constexpr int kPEpiThreads = 32 * kPEpiWarps;
-constexpr int kPSchedWarp = 2 + kPEpiWarps;
+constexpr int kPGatherWarp0 = 2 + kPEpiWarps;   // warps 10..13
+constexpr int kPGatherWarps = 4;
+constexpr int kPSchedWarp = kPGatherWarp0 + kPGatherWarps;  // warp 14
 constexpr int kPThreads = 32 * (kPSchedWarp + 1);
 constexpr int kPQueue = 4;
 constexpr int kPLead = 4;                  // claim the next item this many k-blocks early
@@ -69,8 +73,8 @@ constexpr int kPXchFloats = 2 * 2 * 64 * kPXchRow;  // [column part][gate/up][fe
 constexpr int kPSmem = kPStages * kPStage + 1024 + kPCtrl + kPXchFloats * 4 + kPairTileN * 8;
 static_assert(kPTmemCols <= 512, "TMEM");
 // consumers of a queue entry, counted on the leader's qempty: leader producer,
-// MMA and epilogue warps; peer producer and epilogue warps
-constexpr int kPQueueConsumers = 1 + 1 + kPEpiWarps + 1 + kPEpiWarps;
+// MMA, epilogue and gatherer warps; peer producer, epilogue and gatherer warps
+constexpr int kPQueueConsumers = 1 + 1 + kPEpiWarps + kPGatherWarps + 1 + kPEpiWarps + kPGatherWarps;
 
 // MMA N of an item: its rows rounded up to 64 (each CTA then holds a whole
 // number of 32-row boxes of B)
@@ -81,7 +85,6 @@ __device__ __forceinline__ int pair_n(const WorkItem& it) {
 struct PairMaps {
   CUtensorMap wg, wu, wgs, wus;  // gate / up rows, 64-row boxes
   CUtensorMap wd, wds;           // down rows, 128-row boxes
-  CUtensorMap xp, x;             // token rows (routed order / token order), 32-row boxes
   CUtensorMap h, hs;             // h rows, 32-row boxes
 };
 
@@ -115,7 +118,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
   pdl_trigger();
   if (tid == 0) {
     for (int s = 0; s < kPStages; ++s) {
-      mbar_init(&full[s], 1);   // the leader's expect_tx arrival (+ both CTAs' bytes)
+      // the leader's expect_tx arrival (+ both CTAs' TMA bytes) and one
+      // arrival per gatherer warp of both CTAs (the peer's are remote)
+      mbar_init(&full[s], 1 + 2 * kPGatherWarps);
       mbar_init(&empty[s], 1);  // the leader's multicast commit
     }
     for (int a = 0; a < 2; ++a) {
@@ -131,14 +136,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
     fence_mbar_init();
     prefetch_tmap(&m.wg);
     prefetch_tmap(&m.wd);
-    prefetch_tmap(&m.xp);
     prefetch_tmap(&m.h);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, kPTmemCols);
     tmem_relinquish_pair();
   }
-  pdl_wait();  // the schedule, the routing and x_perm come from earlier kernels
+  pdl_wait();  // the schedule, the routing and x come from earlier kernels
   for (int i = tid; i < p.E + 2; i += blockDim.x) {
     s_gu[i] = p.gu_start[i];
     s_dn[i] = p.dn_start[i];
@@ -221,9 +225,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
     __syncwarp();
   } else if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
+    // This CTA's 128 rows of A, and for down items its half of the h rows;
+    // the token rows of gate/up items come from the gatherer warps.
     if (lane == 0) {
       const uint64_t pol_w = policy_evict_first();
-      const uint64_t pol_b = policy_evict_last();
+      const uint64_t pol_h = policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
       bool live = true;
@@ -240,11 +246,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
         if (!gu) fence_proxy_async_global();
         const int wblk = sh ? 0 : (p.wslot ? p.wslot[it.e] : it.e);
         const int nkb = nkb_of(gu, sh);
-        const int nhalf = pair_n(it) / 2;       // this CTA's B rows
-        const int nbox = nhalf / kPBox;
+        const int nhalf = pair_n(it) / 2;  // this CTA's B rows (a multiple of 32)
         const int brow = it.row0 + static_cast<int>(rank) * nhalf;
+        const int nbox = gu ? 0 : nhalf / kPBox;
         const uint32_t pair_bytes = 2u * (kPA + nbox * kPBox * 128);
-        const CUtensorMap* mb = gu ? (sh ? &m.x : &m.xp) : (sh ? &m.hs : &m.h);
         int arow0, arow1 = 0;
         const CUtensorMap *ma0, *ma1 = nullptr;
         if (gu) {
@@ -267,13 +272,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
           const uint32_t lbar = at_leader(&full[stage]);
           if (leader) mbar_arrive_expect_tx(&full[stage], pair_bytes);
           if (gu) {
-            tma_load_2d_pair(sA, ma0, lbar, kb * 64, arow0, pol_w);               // gate rows
-            tma_load_2d_pair(sA + kPA / 2, ma1, lbar, kb * 64, arow1, pol_w);     // up rows
+            tma_load_2d_pair(sA, ma0, lbar, kb * 64, arow0, pol_w);            // gate rows
+            tma_load_2d_pair(sA + kPA / 2, ma1, lbar, kb * 64, arow1, pol_w);  // up rows
           } else {
             tma_load_2d_pair(sA, ma0, lbar, kb * 64, arow0, pol_w);
           }
           for (int b = 0; b < nbox; ++b)
-            tma_load_2d_pair(sB + b * kPBox * 128, mb, lbar, kb * 64, brow + b * kPBox, pol_b);
+            tma_load_2d_pair(sB + b * kPBox * 128, sh ? &m.hs : &m.h, lbar, kb * 64,
+                             brow + b * kPBox, pol_h);
           if (leader) *prog = n * kPProgStride + kb + 1;
           if (++stage == kPStages) {
             stage = 0;
@@ -311,7 +317,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
         tc_fence_after();
         const uint32_t d0 = tmem_base + acc * kPAccCols;
         for (int kb = 0; kb < nkb; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) {
+          // acquire at cluster scope: the peer's gatherers arrive from the other CTA
+          if (!mbar_wait_cluster(&full[stage], phase, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) {
             live = false;
             break;
           }
@@ -335,6 +342,107 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
       }
     }
     __syncwarp();
+  } else if (warp >= kPGatherWarp0 && warp < kPSchedWarp) {
+    // ------------------------------------------------------------ token gatherers (both CTAs)
+    // Gate/up items: thread g copies 16-byte chunk (g % 8) of rows g/8,
+    // g/8 + 16, ... of this CTA's half of the token tile into the
+    // 128-byte-swizzled layout (chunk c of row r lands at c ^ (r % 8)). A
+    // stage's copies retire two stages later: wait for the group, make it
+    // visible to the tensor cores (proxy fence), then one arrival per warp on
+    // the leader's full barrier. Down items copy nothing but keep the stage
+    // sequence and the arrivals.
+    constexpr int kRowsPerThread = kPairTileN / 2 / 16;
+    constexpr int kLag = 2;
+    const int g = tid - kPGatherWarp0 * 32;
+    const int chunk = g & 7, rbase = g >> 3;
+    const uint64_t pol_x = policy_evict_last();
+    int stage = 0;
+    uint32_t phase = 0;
+    int pend[2] = {-1, -1};  // stages issued and not yet retired, oldest first
+    bool live = true;
+    // The peer's copies are in its own shared memory: a release restricted to
+    // shared memory, then a relaxed arrive on the leader's barrier (a full
+    // cluster-scope release would also wait for the copies still in flight).
+    auto retire = [&](int st) {
+      if (leader) {
+        mbar_arrive(&full[st]);
+      } else {
+        fence_release_shared_cluster();
+        mbar_arrive_cluster_relaxed(at_leader(&full[st]));
+      }
+    };
+    for (int n = 0; live; ++n) {
+      // The scheduler may hold the next item back until gate/up tiles this
+      // pair is still finishing are published, and the MMA cannot finish them
+      // before their stages retire: if the next item is not queued yet,
+      // retire the pending stages before waiting for it.
+      const int q = n % kPQueue;
+      const bool queued = __shfl_sync(
+          0xffffffffu, lane == 0 ? (mbar_try_wait_cluster(&qfull[q], (n / kPQueue) & 1) ? 1 : 0) : 0, 0) != 0;
+      if (!queued && (pend[0] >= 0 || pend[1] >= 0)) {
+        cp_async_wait<0>();
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if (pend[0] >= 0) retire(pend[0]);
+          if (pend[1] >= 0) retire(pend[1]);
+        }
+        pend[0] = pend[1] = -1;
+      }
+      int item;
+      if (!next_item(n, item, true)) break;
+      bool gu;
+      const WorkItem it = item_at(item, gu);
+      if (!item_ok(p, it, gu, kPairTileN)) continue;
+      const bool sh = it.e == p.E;
+      const int nkb = nkb_of(gu, sh);
+      const int nhalf = pair_n(it) / 2;  // this CTA's B rows
+      const int brow = it.row0 + static_cast<int>(rank) * nhalf;
+      const uint16_t* src[kRowsPerThread];
+#pragma unroll
+      for (int i = 0; i < kRowsPerThread; ++i) {
+        // rows past the item repeat its last row (their columns are never stored)
+        const int row = min(brow + rbase + 16 * i, it.row0 + it.nrows - 1);
+        int t = 0;
+        if (gu) t = sh ? row : p.perm[row] / p.K;
+        t = min(max(t, 0), p.T - 1);
+        src[i] = p.x + static_cast<size_t>(t) * p.H + chunk * 8;
+      }
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) {
+          live = false;
+          break;
+        }
+        if (gu) {
+          uint8_t* sB = smem + stage * kPStage + kPA;
+#pragma unroll
+          for (int i = 0; i < kRowsPerThread; ++i) {
+            const int r = rbase + 16 * i;
+            if (r < nhalf) cp_async16(sB + r * 128 + ((chunk ^ (r & 7)) << 4), src[i] + kb * 64, pol_x);
+          }
+        }
+        cp_async_commit();
+        if (pend[0] >= 0) {
+          cp_async_wait<kLag>();     // this lane's copies for the oldest pending stage landed
+          fence_proxy_async_smem();  // ... and are visible to the tensor cores
+          __syncwarp();
+          if (lane == 0) retire(pend[0]);
+        }
+        pend[0] = pend[1];
+        pend[1] = stage;
+        if (++stage == kPStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+    cp_async_wait<0>();  // nothing may still be landing in shared memory at exit
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (live && lane == 0) {
+      if (pend[0] >= 0) retire(pend[0]);
+      if (pend[1] >= 0) retire(pend[1]);
+    }
   } else if (warp >= 2 && warp < 2 + kPEpiWarps) {
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int q = warp & 3;            // TMEM lane quarter
@@ -461,43 +569,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
   }
 }
 
-// x_perm[r] = x[perm[r] / K]: the routed token rows in permuted order, so that
-// the pair kernel loads its B tiles of gate/up items with plain TMA boxes.
-// 16-byte copies; one grid-stride loop over (row, 8-column chunk).
-__global__ void __launch_bounds__(256) gather_rows(int TK, int K, int T, int H,
-                                                   const int32_t* __restrict__ perm,
-                                                   const uint16_t* __restrict__ x,
-                                                   uint16_t* __restrict__ x_perm) {
-  pdl_trigger();
-  pdl_wait();  // inputs come from earlier kernels on the stream
-  const int chunks = H / 8;
-  const long long total = static_cast<long long>(TK) * chunks;
-  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
-       i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const long long r = i / chunks;
-    const int c = static_cast<int>(i - r * chunks);
-    int t = perm[r] / K;
-    t = min(max(t, 0), T - 1);
-    reinterpret_cast<uint4*>(x_perm)[r * chunks + c] =
-        reinterpret_cast<const uint4*>(x)[static_cast<long long>(t) * chunks + c];
-  }
-}
-
 }  // namespace
 
 cudaError_t launch_ffn_pair(const GemmArgs& a, cudaStream_t s) {
   const moe_cfg& c = *a.cfg;
-  if (a.x_perm == nullptr) return cudaErrorInvalidValue;
   const int T = a.T, TK = a.T * c.K;
-  {
-    const long long total = static_cast<long long>(TK) * (c.H / 8);
-    long long blocks = (total + 255) / 256;
-    const long long cap = static_cast<long long>(num_sms()) * 8;
-    if (blocks > cap) blocks = cap;
-    cudaError_t e = launch_pdl(gather_rows, dim3(static_cast<int>(blocks)), dim3(256), 0, s, TK, c.K,
-                               T, c.H, a.perm, a.x, a.x_perm);
-    if (e != cudaSuccess) return e;
-  }
   FfnParams p;
   memset(&p, 0, sizeof(p));
   p.T = T;
@@ -529,7 +605,6 @@ cudaError_t launch_ffn_pair(const GemmArgs& a, cudaStream_t s) {
   const uint64_t wr = static_cast<uint64_t>(a.wrows);
   bool ok = map_bf16(&m.wg, a.Wg, wr * c.I, c.H, 64) && map_bf16(&m.wu, a.Wu, wr * c.I, c.H, 64) &&
             map_bf16(&m.wd, a.Wd, wr * c.H, c.I, kTileN) &&
-            map_bf16(&m.xp, a.x_perm, TK, c.H, kPBox) && map_bf16(&m.x, a.x, T, c.H, kPBox) &&
             map_bf16(&m.h, a.h_r, TK, c.I, kPBox);
   if (p.has_shared) {
     ok = ok && map_bf16(&m.wgs, a.W->Wg_s, c.I_shared, c.H, 64) &&

@@ -64,7 +64,6 @@ struct WsLayout {
   // MXFP4 routed weights only: touched-expert slots and their bf16 copies
   size_t slot_of, touched, ntouched, wq_g, wq_u, wq_d;
   size_t wr_split;  // router matrix as three bf16 terms (batches above 32 tokens)
-  size_t x_perm;    // routed token rows in permuted order [T*K][H] bf16 (pair FFN only)
   int max_touched;
   int n_ptiles, bn, max_items_gu, max_items_dn;
 };
@@ -112,7 +111,6 @@ struct GemmArgs {
   int wrows;                 // row blocks in Wg/Wu/Wd (E, or the slot capacity)
   uint16_t* h_r;
   uint16_t* h_s;
-  uint16_t* x_perm;         // [T*K, H] scratch: routed token rows in permuted order (pair FFN)
   float* y_slot;
   const int32_t* offsets;   // [E+1] routed row offsets
   const int32_t* gu_start;  // [E+2] item prefix sums, gate/up
@@ -128,7 +126,7 @@ struct GemmArgs {
 // The expert FFN: gate/up and down in one cooperative persistent launch
 // (counters in a.ready and a.nitems[2], zeroed by the schedule builder).
 cudaError_t launch_ffn(const GemmArgs& a, cudaStream_t s);
-// The expert FFN on CTA pairs (token tile kPairTileN); gathers a.x_perm first.
+// The expert FFN on CTA pairs (token tile kPairTileN).
 cudaError_t launch_ffn_pair(const GemmArgs& a, cudaStream_t s);
 cudaError_t launch_router_gemm(const moe_cfg& c, int T, const uint16_t* x, const uint16_t* w_hi,
                                const uint16_t* w_mid, const uint16_t* w_lo, float* z,

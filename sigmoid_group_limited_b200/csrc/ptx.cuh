@@ -1,5 +1,6 @@
 // ptx.cuh - thin inline-PTX wrappers for sm_100a: mbarriers, TMA (tiled and
-// gather4), tcgen05 MMA / TMEM, and the shared-memory matrix descriptor.
+// bulk), cp.async, clusters, tcgen05 MMA / TMEM, and the shared-memory matrix
+// descriptor.
 // Written for this library; every wait is bounded (see mbar_wait).
 #pragma once
 #include <cuda.h>
@@ -101,18 +102,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m, uin
       : "memory");
 }
 
-// Gather four rows (r0..r3) of a 2D tensor, columns [c0, c0 + box width),
-// into four consecutive box rows in smem. The tensor map's box is 1 row high.
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* m, uint64_t* bar, int c0,
-                                            int r0, int r1, int r2, int r3, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      ".L2::cache_hint [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(c0), "r"(r0), "r"(r1), "r"(r2),
-      "r"(r3), "l"(policy)
-      : "memory");
-}
-
 // 1D bulk copy global -> shared (16-byte aligned addresses, size a multiple of
 // 16), completion counted on `bar` in bytes.
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -168,6 +157,17 @@ __device__ __forceinline__ void st_shared_cluster(uint32_t addr, int v) {
 // Arrive on an mbarrier of another CTA of the cluster (release at cluster scope).
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t remote_bar) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar)
+               : "memory");
+}
+// Release at cluster scope restricted to this CTA's shared-memory operations,
+// to be followed by a relaxed remote arrive (mbar_arrive_cluster_relaxed).
+// Unlike a full cluster-scope release it does not wait for this thread's
+// global-memory traffic still in flight (e.g. cp.async of later stages).
+__device__ __forceinline__ void fence_release_shared_cluster() {
+  asm volatile("fence.release.sync_restrict::shared::cta.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t remote_bar) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar)
                : "memory");
 }
 // Wait-test that acquires at cluster scope (for barriers that other CTAs arrive on).
