@@ -57,6 +57,15 @@ extern "C" {
 
 #define MOE_W_BF16 0   /* routed weights are bf16 */
 #define MOE_W_MXFP4 1  /* routed weights are MXFP4 codes + e8m0 scales */
+/* Routed weights MXFP4 as above, and the routed experts' activations MXFP8:
+ * page "Ling-3.0-flash-VL 42-layer hybrid backbone" (lpnh.cn/news/2815793),
+ * spec table, gives the quantisation scheme as FP8 + MXFP4. x is quantised
+ * before gate/up and h before down (OCP Microscaling v1.0: e4m3 elements, one
+ * e8m0 scale per 32 consecutive elements along the contraction; scale
+ * 2^(floor(log2(amax)) - 8), elements rounded to nearest even, saturating at
+ * 448), and the routed GEMMs run on block-scaled tensor cores. The shared
+ * expert stays bf16. Needs H % 128 == 0 and I % 128 == 0. */
+#define MOE_W_MXFP4_A8 2
 
 /* Layer configuration; field names follow the model's config keys. */
 typedef struct moe_cfg {
@@ -71,7 +80,7 @@ typedef struct moe_cfg {
   int32_t renorm;       /* norm_topk_prob (1) */
   float limit_routed;   /* SwiGLU limit of routed experts; <= 0 or inf: off */
   float limit_shared;   /* SwiGLU limit of the shared expert; <= 0 or inf: off */
-  int32_t wfmt;         /* MOE_W_BF16 or MOE_W_MXFP4 */
+  int32_t wfmt;         /* MOE_W_BF16, MOE_W_MXFP4 or MOE_W_MXFP4_A8 */
 } moe_cfg;
 
 typedef enum moe_status {
@@ -86,8 +95,10 @@ typedef enum moe_status {
 } moe_status;
 
 /* Expert weights. Routed bf16: Wg,Wu [E,I,H], Wd [E,H,I] bf16, scales NULL.
- * Routed MXFP4: Wg,Wu [E,I,H/2], Wd [E,H,I/2] uint8 codes (element 2j in the
- * low nibble) and Wg_scale,Wu_scale [E,I,H/32], Wd_scale [E,H,I/32] e8m0.
+ * Routed MXFP4 (MOE_W_MXFP4 and MOE_W_MXFP4_A8): Wg,Wu [E,I,H/2], Wd [E,H,I/2]
+ * uint8 codes (element 2j in the low nibble) and Wg_scale,Wu_scale [E,I,H/32],
+ * Wd_scale [E,H,I/32] e8m0; with MOE_W_MXFP4_A8 the codes must be 32-byte
+ * aligned.
  * Shared expert (bf16): Wg_s,Wu_s [I_s,H], Wd_s [H,I_s]; all three NULL when
  * cfg->I_shared == 0. All device pointers. */
 typedef struct moe_weights {

@@ -45,6 +45,15 @@ Readings where the pages are silent (each also listed in the design notes):
      expert = ascending flat index j = t*K + k (stable counting sort).
   R9 MXFP4 weights are used through their exact dequantised values
      (e2m1 magnitude * sign * 2^(scale - 127)).
+  R10 block-scaled variant (weight format MXFP4_A8): the spec table of [P4]
+     lists the quantisation scheme as FP8 + MXFP4. It is read as MXFP8
+     activations (OCP Microscaling v1.0: e4m3 elements, one e8m0 scale per
+     32 consecutive elements along the contraction) for the routed experts:
+     x is quantised before gate/up, h (fp32) before down, instead of R7's
+     bf16 h. Scale = 2^(floor(log2(amax)) - 8) (8 = e4m3's largest exponent),
+     its byte clamped to [0, 254] (amax = 0 gives byte 0); elements are
+     v / scale rounded to nearest e4m3, ties to even, saturating at +-448.
+     The shared expert keeps the bf16 path of R7.
 
 Parity pins: see tests/test_oracle_*.py (brute-force group enumeration, rank
 counting, reductions to plain top-k and argmax, the all-ties case, closed
@@ -99,6 +108,65 @@ def mxfp4_dequantize(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
     scale = np.where(scales == 0xFF, np.nan, np.exp2(s - 127.0))
     scale = np.repeat(scale, 32, axis=-1)
     return val * scale
+
+
+E4M3_MAX = 448.0
+MOE_W_MXFP4_A8 = 2   # weight-format code of the block-scaled variant (R10)
+
+
+def e4m3_decode(codes: np.ndarray) -> np.ndarray:
+    """OCP e4m3 (the "fn" variant: no infinities) -> float64.
+
+    Bit 7 sign, bits 6..3 exponent (bias 7), bits 2..0 mantissa; exponent 0
+    is subnormal (m/8 * 2^-6); exponent 15 with mantissa 7 is NaN."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    mag = np.where((e == 15) & (m == 7), np.nan, mag)
+    return sign * mag
+
+
+# the 127 finite non-negative e4m3 values, in code order (increasing)
+_E4M3_POS = e4m3_decode(np.arange(0x7F, dtype=np.uint8))
+
+
+def e4m3_encode(v: np.ndarray) -> np.ndarray:
+    """Nearest e4m3 code to each finite float64 value, ties to the even code
+    (mantissa bit 0 clear), magnitudes above 448 saturate to 448 (R10); the
+    sign bit is the input's, also when the magnitude rounds to zero."""
+    v = np.asarray(v, dtype=np.float64)
+    a = np.minimum(np.abs(v), E4M3_MAX)
+    hi = np.clip(np.searchsorted(_E4M3_POS, a, side="left"), 0, 0x7E)  # first value >= a
+    lo = np.maximum(hi - 1, 0)
+    dlo = a - _E4M3_POS[lo]
+    dhi = _E4M3_POS[hi] - a
+    take_hi = (dhi < dlo) | ((dhi == dlo) & (hi % 2 == 0))
+    code = np.where(take_hi, hi, lo).astype(np.uint8)
+    return np.where(np.signbit(v), code | 0x80, code).astype(np.uint8)   # the sign is kept
+
+
+def mxfp8_quantize(v: np.ndarray):
+    """MXFP8 (e4m3 elements, e8m0 scale per 32 along the last axis), R10.
+
+    v [..., K] float (K a multiple of 32) -> (codes uint8 [..., K],
+    scales uint8 [..., K/32])."""
+    v = np.asarray(v, dtype=np.float64)
+    blk = v.reshape(*v.shape[:-1], v.shape[-1] // 32, 32)
+    amax = np.abs(blk).max(axis=-1)
+    _, ex = np.frexp(amax)                      # amax = f * 2^ex, f in [0.5, 1)
+    floor_log2 = ex.astype(np.int64) - 1
+    byte = np.where(amax > 0, np.clip(floor_log2 - 8 + 127, 0, 254), 0).astype(np.uint8)
+    scale = np.exp2(byte.astype(np.float64) - 127.0)
+    codes = e4m3_encode(blk / scale[..., None]).reshape(v.shape)
+    return codes, byte
+
+
+def mxfp8_dequantize(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """Exact float64 values of MXFP8 codes and their e8m0 scales."""
+    s = np.exp2(np.asarray(scales, dtype=np.float64) - 127.0)
+    return e4m3_decode(codes) * np.repeat(s, 32, axis=-1)
 
 
 # --------------------------------------------------------------------------
@@ -243,12 +311,14 @@ def route_stats(counts: np.ndarray, E: int) -> np.ndarray:
 
 
 def swiglu_expert(x64: np.ndarray, Wg64: np.ndarray, Wu64: np.ndarray, Wd64: np.ndarray,
-                  limit: float = 0.0) -> Tuple[np.ndarray, np.ndarray]:
-    """One SwiGLU expert on rows x64 [n,H] (float64 copies of bf16 values).
+                  limit: float = 0.0, h_mxfp8: bool = False) -> Tuple[np.ndarray, np.ndarray]:
+    """One SwiGLU expert on rows x64 [n,H] (float64 values of its inputs).
 
     g = x Wg^T, u = x Wu^T (fp32 results); with a limit L > 0 both are clamped
-    to [-L, L] (R6); h = bf16(fp32(silu(g) * u)), silu(g) = g / (1 + e^-g);
-    o = h Wd^T (fp32).  Returns (o fp32 [n,H_out], h bf16 bits [n,I])."""
+    to [-L, L] (R6); h = fp32(silu(g) * u), silu(g) = g / (1 + e^-g), rounded
+    to bf16 (R7) or, with h_mxfp8, quantised to MXFP8 along I (R10);
+    o = h Wd^T (fp32).  Returns (o fp32 [n,H_out], h): h as bf16 bits [n,I],
+    or with h_mxfp8 the pair (codes [n,I], scales [n,I/32])."""
     g = (x64 @ Wg64.T).astype(np.float32)
     u = (x64 @ Wu64.T).astype(np.float32)
     if limit is not None and limit > 0.0 and math.isfinite(limit):
@@ -256,8 +326,12 @@ def swiglu_expert(x64: np.ndarray, Wg64: np.ndarray, Wu64: np.ndarray, Wd64: np.
         g = np.clip(g, -L, L)
         u = np.clip(u, -L, L)
     g64 = g.astype(np.float64)
-    a = (g64 / (1.0 + np.exp(-g64))) * u.astype(np.float64)
-    h_bits = f32_to_bf16_bits(a.astype(np.float32))
+    a = ((g64 / (1.0 + np.exp(-g64))) * u.astype(np.float64)).astype(np.float32)
+    if h_mxfp8:
+        hq, hs = mxfp8_quantize(a)
+        o = (mxfp8_dequantize(hq, hs) @ Wd64.T).astype(np.float32)
+        return o, (hq, hs)
+    h_bits = f32_to_bf16_bits(a)
     o = (bf16_bits_to_f64(h_bits) @ Wd64.T).astype(np.float32)
     return o, h_bits
 
@@ -298,13 +372,16 @@ def layer_forward(cfg, x_bits: np.ndarray, Wr: np.ndarray, bias: np.ndarray,
     tok = np.arange(T) if tokens is None else np.asarray(tokens, dtype=np.int64)
     x64 = bf16_bits_to_f64(x_bits[tok])
     n, K, H = tok.size, cfg.K, cfg.H
+    act_mx = getattr(cfg, "wfmt", 0) == MOE_W_MXFP4_A8
+    # R10: the routed experts see x through its MXFP8 values
+    xr64 = mxfp8_dequantize(*mxfp8_quantize(x64)) if act_mx else x64
     y_slot = np.zeros((n, K, H), dtype=np.float32)
     idx = r["idx"][tok]
     w = r["w"][tok]
     for e in np.unique(idx):
         rows, ks = np.nonzero(idx == e)
         Wg, Wu, Wd = expert(int(e))
-        o, _ = swiglu_expert(x64[rows], Wg, Wu, Wd, cfg.limit_routed)
+        o, _ = swiglu_expert(xr64[rows], Wg, Wu, Wd, cfg.limit_routed, h_mxfp8=act_mx)
         y_slot[rows, ks, :] = (w[rows, ks][:, None].astype(np.float32) * o).astype(np.float32)
     o_sh, h_sh = swiglu_expert(x64, bf16_bits_to_f64(Wg_s), bf16_bits_to_f64(Wu_s),
                                bf16_bits_to_f64(Wd_s), cfg.limit_shared)

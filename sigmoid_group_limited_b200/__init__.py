@@ -22,6 +22,7 @@ LIB_PATH = os.path.join(_PKG, "libsgl_moe.so")
 
 MOE_W_BF16 = 0
 MOE_W_MXFP4 = 1
+MOE_W_MXFP4_A8 = 2
 MOE_N_STAGE_EVENTS = 6
 STATUS = {0: "MOE_OK", -1: "MOE_ERR_CFG", -2: "MOE_ERR_NULL", -3: "MOE_ERR_ALIGN",
           -4: "MOE_ERR_WORKSPACE", -5: "MOE_ERR_CUDA", -6: "MOE_ERR_DEVICE",
