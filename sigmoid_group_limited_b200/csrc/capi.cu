@@ -47,12 +47,15 @@ WsLayout ws_layout(const moe_cfg& c, int T) {
   memset(&L, 0, sizeof(L));
   const size_t TK = static_cast<size_t>(T) * c.K;
   L.n_ptiles = cdiv(static_cast<long long>(TK), kPermTile);
-  L.bn = choose_bn(T, c.K, c.E);
-  const int rt_gu = cdiv(c.I, kTileN), st_gu = cdiv(c.I_shared, kTileN), nt_dn = cdiv(c.H, kDownTile);
+  const bool mx = c.wfmt == MOE_W_MXFP4_A8;
+  L.bn = mx ? kMxTileN : choose_bn(T, c.K, c.E);
+  const int gu_ft = mx ? kMxGuTile : kTileN, dn_ft = mx ? kMxDnTile : kDownTile;
+  const int rt_gu = cdiv(c.I, gu_ft), st_gu = cdiv(c.I_shared, gu_ft), nt_dn = cdiv(c.H, dn_ft);
   const long long mt_r = cdiv(static_cast<long long>(TK), L.bn) +
                          (static_cast<long long>(TK) < c.E ? static_cast<long long>(TK) : c.E);
   const long long mt_s = c.I_shared > 0 ? cdiv(T, L.bn) : 0;
   L.max_items_gu = static_cast<int>(mt_r * rt_gu + mt_s * st_gu);
+  L.max_row_tiles = static_cast<int>(mt_r);
   L.max_items_dn = static_cast<int>((mt_r + mt_s) * nt_dn);
   size_t o = 0;
   auto take = [&](size_t bytes) {
@@ -78,6 +81,19 @@ WsLayout ws_layout(const moe_cfg& c, int T) {
   L.h_s = take(static_cast<size_t>(T) * (c.I_shared > 0 ? c.I_shared : 0) * 2);
   L.y_slot = take((TK + T) * c.H * 4);
   L.wr_split = T > 32 ? take(static_cast<size_t>(3) * c.E * c.H * 2) : 0;
+  if (mx) {
+    // h_r holds the e4m3 h codes; the rest is scales
+    L.max_touched = static_cast<int>(TK < static_cast<size_t>(c.E) ? TK : c.E);
+    const size_t kb_h = static_cast<size_t>(c.H / 128), kb_i = static_cast<size_t>(c.I / 128);
+    L.slot_of = take(static_cast<size_t>(c.E) * 4);
+    L.touched = take(static_cast<size_t>(c.E) * 4);
+    L.ntouched = take(16);
+    L.x_q = take(static_cast<size_t>(T) * c.H);
+    L.x_sf = take(static_cast<size_t>(T) * (c.H / 32));
+    L.h_sf = take(static_cast<size_t>(L.max_row_tiles) * kb_i * 512);
+    L.sf_gu = take(static_cast<size_t>(L.max_touched) * (c.I / kMxGuTile) * kb_h * 512);
+    L.sf_dn = take(static_cast<size_t>(L.max_touched) * kb_h * kb_i * 512);
+  }
   if (c.wfmt == MOE_W_MXFP4) {
     L.max_touched = static_cast<int>(TK < static_cast<size_t>(c.E) ? TK : c.E);
     const size_t mat = static_cast<size_t>(L.max_touched) * c.I * c.H * 2;
@@ -109,7 +125,8 @@ bool cfg_ok(const moe_cfg* c) {
   if (c->I_shared < 0 || c->I_shared % 64 != 0 || c->I_shared > 16384) return false;
   if (isnan(c->scale) || isinf(c->scale)) return false;
   if (isnan(c->limit_routed) || isnan(c->limit_shared)) return false;
-  if (c->wfmt != MOE_W_BF16 && c->wfmt != MOE_W_MXFP4) return false;
+  if (c->wfmt != MOE_W_BF16 && c->wfmt != MOE_W_MXFP4 && c->wfmt != MOE_W_MXFP4_A8) return false;
+  if (c->wfmt == MOE_W_MXFP4_A8 && (c->H % 128 != 0 || c->I % 128 != 0)) return false;
   return true;
 }
 
@@ -142,15 +159,80 @@ moe_status cu(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; 
 moe_status check_weights(const moe_cfg* c, const moe_weights* W) {
   if (W == nullptr || W->Wg == nullptr || W->Wu == nullptr || W->Wd == nullptr) return MOE_ERR_NULL;
   if (!al16(W->Wg) || !al16(W->Wu) || !al16(W->Wd)) return MOE_ERR_ALIGN;
-  if (c->wfmt == MOE_W_MXFP4) {
+  if (c->wfmt == MOE_W_MXFP4 || c->wfmt == MOE_W_MXFP4_A8) {
     if (!W->Wg_scale || !W->Wu_scale || !W->Wd_scale) return MOE_ERR_NULL;
     if (!al16(W->Wg_scale) || !al16(W->Wu_scale) || !al16(W->Wd_scale)) return MOE_ERR_ALIGN;
+  }
+  if (c->wfmt == MOE_W_MXFP4_A8) {  // TMA of unpacked 4-bit codes wants 32-byte bases
+    auto al32 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; };
+    if (!al32(W->Wg) || !al32(W->Wu) || !al32(W->Wd)) return MOE_ERR_ALIGN;
   }
   if (c->I_shared > 0) {
     if (W->Wg_s == nullptr || W->Wu_s == nullptr || W->Wd_s == nullptr) return MOE_ERR_NULL;
     if (!al16(W->Wg_s) || !al16(W->Wu_s) || !al16(W->Wd_s)) return MOE_ERR_ALIGN;
   }
   return MOE_OK;
+}
+
+// Stages 7-8 after the schedule: the weight-format preparation (MXFP4: the
+// touched experts' bf16 copies; MXFP4_A8: scale atoms and MXFP8 x), then the
+// expert FFN kernel of the format.
+cudaError_t run_ffn(const moe_cfg* cfg, int T, const uint16_t* x, const int32_t* perm,
+                    const int32_t* offsets, const float* w, const moe_weights* W, float* y_slot,
+                    void* ws, const WsLayout& L, cudaStream_t s) {
+  GemmArgs a;
+  memset(&a, 0, sizeof(a));
+  a.cfg = cfg;
+  a.T = T;
+  a.x = x;
+  a.perm = perm;
+  a.w = w;
+  a.W = W;
+  a.Wg = W->Wg;
+  a.Wu = W->Wu;
+  a.Wd = W->Wd;
+  a.wslot = nullptr;
+  a.wrows = cfg->E;
+  if (cfg->wfmt == MOE_W_MXFP4) {
+    cudaError_t e = launch_mxfp4_expand(*cfg, offsets, W, at<int32_t>(ws, L.slot_of),
+                                        at<int32_t>(ws, L.touched), at<int32_t>(ws, L.ntouched),
+                                        at<uint16_t>(ws, L.wq_g), at<uint16_t>(ws, L.wq_u),
+                                        at<uint16_t>(ws, L.wq_d), s);
+    if (e != cudaSuccess) return e;
+    a.Wg = at<uint16_t>(ws, L.wq_g);
+    a.Wu = at<uint16_t>(ws, L.wq_u);
+    a.Wd = at<uint16_t>(ws, L.wq_d);
+    a.wslot = at<int32_t>(ws, L.slot_of);
+    a.wrows = L.max_touched;
+  }
+  a.h_r = at<uint16_t>(ws, L.h_r);
+  a.h_s = at<uint16_t>(ws, L.h_s);
+  a.y_slot = y_slot;
+  a.offsets = offsets;
+  a.gu_start = at<int32_t>(ws, L.gu_start);
+  a.dn_start = at<int32_t>(ws, L.dn_start);
+  a.ready = at<int32_t>(ws, L.ready);
+  a.nitems = at<int32_t>(ws, L.nitems);
+  a.err = at<int32_t>(ws, L.err);
+  a.bn = L.bn;
+  a.max_items_gu = L.max_items_gu;
+  a.max_items_dn = L.max_items_dn;
+  if (cfg->wfmt == MOE_W_MXFP4_A8) {
+    cudaError_t e = launch_mx_prep(*cfg, T, offsets, W, x, at<int32_t>(ws, L.slot_of),
+                                   at<int32_t>(ws, L.touched), at<int32_t>(ws, L.ntouched),
+                                   at<uint8_t>(ws, L.sf_gu), at<uint8_t>(ws, L.sf_dn),
+                                   at<uint8_t>(ws, L.x_q), at<uint8_t>(ws, L.x_sf), s);
+    if (e != cudaSuccess) return e;
+    a.x_q = at<uint8_t>(ws, L.x_q);
+    a.x_sf = at<uint8_t>(ws, L.x_sf);
+    a.h_q = at<uint8_t>(ws, L.h_r);
+    a.h_sf = at<uint8_t>(ws, L.h_sf);
+    a.sf_gu = at<uint8_t>(ws, L.sf_gu);
+    a.sf_dn = at<uint8_t>(ws, L.sf_dn);
+    a.slot_of = at<int32_t>(ws, L.slot_of);
+    return launch_ffn_mx(a, s);
+  }
+  return launch_ffn(a, s);
 }
 
 }  // namespace
@@ -233,44 +315,8 @@ moe_status moe_grouped_swiglu(const moe_cfg* cfg, int32_t T, const void* x, cons
   int32_t* nitems = at<int32_t>(ws, L.nitems);
   cudaError_t e = launch_schedule(*cfg, T, offsets, L, gu, dn, at<int32_t>(ws, L.ready), nitems, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
-  const int32_t* a_offsets = offsets;
-  GemmArgs a;
-  a.cfg = cfg;
-  a.T = T;
-  a.x = static_cast<const uint16_t*>(x);
-  a.perm = perm;
-  a.w = w;
-  a.W = W;
-  a.Wg = W->Wg;
-  a.Wu = W->Wu;
-  a.Wd = W->Wd;
-  a.wslot = nullptr;
-  a.wrows = cfg->E;
-  if (cfg->wfmt == MOE_W_MXFP4) {
-    if (launch_mxfp4_expand(*cfg, a_offsets, W, at<int32_t>(ws, L.slot_of),
-                            at<int32_t>(ws, L.touched), at<int32_t>(ws, L.ntouched),
-                            at<uint16_t>(ws, L.wq_g), at<uint16_t>(ws, L.wq_u),
-                            at<uint16_t>(ws, L.wq_d), s) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    a.Wg = at<uint16_t>(ws, L.wq_g);
-    a.Wu = at<uint16_t>(ws, L.wq_u);
-    a.Wd = at<uint16_t>(ws, L.wq_d);
-    a.wslot = at<int32_t>(ws, L.slot_of);
-    a.wrows = L.max_touched;
-  }
-  a.h_r = at<uint16_t>(ws, L.h_r);
-  a.h_s = at<uint16_t>(ws, L.h_s);
-  a.y_slot = static_cast<float*>(y_slot);
-  a.offsets = offsets;
-  a.gu_start = gu;
-  a.dn_start = dn;
-  a.ready = at<int32_t>(ws, L.ready);
-  a.nitems = nitems;
-  a.err = at<int32_t>(ws, L.err);
-  a.bn = L.bn;
-  a.max_items_gu = L.max_items_gu;
-  a.max_items_dn = L.max_items_dn;
-  return cu(launch_ffn(a, s));
+  return cu(run_ffn(cfg, T, static_cast<const uint16_t*>(x), perm, offsets, w, W,
+                    static_cast<float*>(y_slot), ws, L, s));
 }
 
 moe_status moe_combine(const moe_cfg* cfg, int32_t T, const void* y_slot, int32_t with_shared,
@@ -329,44 +375,9 @@ moe_status moe_layer_forward(const moe_cfg* cfg, int32_t T, const void* x, const
                           nitems, s)) != cudaSuccess)
     return MOE_ERR_CUDA;
   rec(2);
-  const int32_t* a_offsets = offsets;
-  GemmArgs a;
-  a.cfg = cfg;
-  a.T = T;
-  a.x = static_cast<const uint16_t*>(x);
-  a.perm = perm;
-  a.w = w;
-  a.W = W;
-  a.Wg = W->Wg;
-  a.Wu = W->Wu;
-  a.Wd = W->Wd;
-  a.wslot = nullptr;
-  a.wrows = cfg->E;
-  if (cfg->wfmt == MOE_W_MXFP4) {
-    if (launch_mxfp4_expand(*cfg, a_offsets, W, at<int32_t>(ws, L.slot_of),
-                            at<int32_t>(ws, L.touched), at<int32_t>(ws, L.ntouched),
-                            at<uint16_t>(ws, L.wq_g), at<uint16_t>(ws, L.wq_u),
-                            at<uint16_t>(ws, L.wq_d), s) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    a.Wg = at<uint16_t>(ws, L.wq_g);
-    a.Wu = at<uint16_t>(ws, L.wq_u);
-    a.Wd = at<uint16_t>(ws, L.wq_d);
-    a.wslot = at<int32_t>(ws, L.slot_of);
-    a.wrows = L.max_touched;
-  }
-  a.h_r = at<uint16_t>(ws, L.h_r);
-  a.h_s = at<uint16_t>(ws, L.h_s);
-  a.y_slot = y_slot;
-  a.offsets = offsets;
-  a.gu_start = gu;
-  a.dn_start = dn;
-  a.ready = at<int32_t>(ws, L.ready);
-  a.nitems = nitems;
-  a.err = err;
-  a.bn = L.bn;
-  a.max_items_gu = L.max_items_gu;
-  a.max_items_dn = L.max_items_dn;
-  if ((e = launch_ffn(a, s)) != cudaSuccess) return MOE_ERR_CUDA;
+  if ((e = run_ffn(cfg, T, static_cast<const uint16_t*>(x), perm, offsets, w, W, y_slot, ws, L,
+                   s)) != cudaSuccess)
+    return MOE_ERR_CUDA;
   rec(3);
   rec(4);
   if ((e = launch_combine(*cfg, T, y_slot, cfg->I_shared > 0 ? 1 : 0, static_cast<uint16_t*>(y),

@@ -1,5 +1,6 @@
-// ffn_common.cuh - parameters and device helpers shared by the two expert-FFN
-// kernels (ffn.cu: one CTA per item; ffn_pair.cu: a CTA pair per item).
+// ffn_common.cuh - parameters and device helpers shared by the expert-FFN
+// kernels (ffn.cu: one CTA per item; ffn_pair.cu: a CTA pair per item;
+// ffn_mx.cu: block-scaled MXFP8 x MXFP4).
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -97,13 +98,15 @@ __device__ __forceinline__ bool wait_progress(const volatile long long* prog, lo
 }
 
 // Same validity rule in every role, so all roles skip the same items.
-__device__ __forceinline__ bool item_ok(const FfnParams& p, const WorkItem& it, bool gu, int bn) {
+// gu_tile / dn_tile: output features per gate/up and per down item.
+__device__ __forceinline__ bool item_ok(const FfnParams& p, const WorkItem& it, bool gu, int bn,
+                                        int gu_tile = kTileN, int dn_tile = kDownTile) {
   const bool sh = it.e == p.E;
   if (it.e < 0 || it.e > p.E || (sh && !p.has_shared)) return false;
   if (it.nrows <= 0 || it.nrows > bn || it.row0 < 0) return false;
   if (it.row0 + it.nrows > (sh ? p.T : p.T * p.K)) return false;
   if (it.ntile < 0) return false;
-  return gu ? it.ntile * kTileN < (sh ? p.Is : p.I) : it.ntile * kDownTile < p.H;
+  return gu ? it.ntile * gu_tile < (sh ? p.Is : p.I) : it.ntile * dn_tile < p.H;
 }
 
 // Work item `i` of one kind from its per-slot item prefix sums (in shared

@@ -30,6 +30,12 @@ constexpr int kPermTile = 2048;   // (token, slot) entries per permutation tile
 constexpr int kTileN = 128;       // output features per GEMM tile (MMA M)
 constexpr int kDownTile = 256;    // hidden features per down item (two MMA tiles)
 constexpr int kPairTileN = 256;   // token tile of the CTA-pair FFN (large batches)
+// Block-scaled FFN (MOE_W_MXFP4_A8): token tile, intermediate features per
+// gate/up item (their gate and up rows share one 128-row MMA tile) and hidden
+// features per down item.
+constexpr int kMxTileN = 128;
+constexpr int kMxGuTile = 64;
+constexpr int kMxDnTile = 128;
 constexpr int kMaxExpertsCfg = 1024;  // largest E a configuration may have
 
 // The expert-FFN kernel for large batches: one CTA per item (default), or a
@@ -63,6 +69,12 @@ struct WsLayout {
       h_s, y_slot, err, total;
   // MXFP4 routed weights only: touched-expert slots and their bf16 copies
   size_t slot_of, touched, ntouched, wq_g, wq_u, wq_d;
+  // MOE_W_MXFP4_A8 only: MXFP8 x (codes [T,H], scales [T,H/32]); the scales
+  // of h (codes reuse h_r) as 512-byte atoms per (row tile, 128-wide k-block);
+  // the touched experts' weight scales as atoms (gate/up: per 64-feature
+  // tile and k-block; down: per 128-row tile and k-block)
+  size_t x_q, x_sf, h_sf, sf_gu, sf_dn;
+  int max_row_tiles;
   size_t wr_split;  // router matrix as three bf16 terms (batches above 32 tokens)
   int max_touched;
   int n_ptiles, bn, max_items_gu, max_items_dn;
@@ -121,6 +133,14 @@ struct GemmArgs {
   int bn;
   int max_items_gu;
   int max_items_dn;
+  // MOE_W_MXFP4_A8: the MXFP4 codes are a.Wg/Wu/Wd (expert-major), read in place
+  const uint8_t* x_q;        // [T, H] e4m3
+  const uint8_t* x_sf;       // [T, H/32] e8m0
+  uint8_t* h_q;              // [T*K, I] e4m3 (permuted rows)
+  uint8_t* h_sf;             // [row tiles][I/128][512] e8m0 atoms
+  const uint8_t* sf_gu;      // [slot][I/64][H/128][512]
+  const uint8_t* sf_dn;      // [slot][H/128][I/128][512]
+  const int32_t* slot_of;    // [E] touched slot of expert e
 };
 
 // The expert FFN: gate/up and down in one cooperative persistent launch
@@ -131,6 +151,20 @@ cudaError_t launch_ffn_pair(const GemmArgs& a, cudaStream_t s);
 cudaError_t launch_router_gemm(const moe_cfg& c, int T, const uint16_t* x, const uint16_t* w_hi,
                                const uint16_t* w_mid, const uint16_t* w_lo, float* z,
                                int32_t* err, cudaStream_t s);
+
+// The block-scaled expert FFN (MOE_W_MXFP4_A8): routed items on
+// tcgen05.mma kind::mxf8f6f4 (e2m1 weights x e4m3 activations, e8m0 scales),
+// shared-expert items on kind::f16, in one persistent launch.
+cudaError_t launch_ffn_mx(const GemmArgs& a, cudaStream_t s);
+// MOE_W_MXFP4_A8 inputs of that FFN: touched-expert slots, their weight
+// scales repacked as atoms (sf_gu / sf_dn) and x quantised to MXFP8.
+cudaError_t launch_mx_prep(const moe_cfg& c, int T, const int32_t* offsets, const moe_weights* W,
+                           const uint16_t* x, int32_t* slot_of, int32_t* touched,
+                           int32_t* ntouched, uint8_t* sf_gu, uint8_t* sf_dn, uint8_t* x_q,
+                           uint8_t* x_sf, cudaStream_t s);
+// Touched experts of a batch in increasing id order (slot_of[e], -1 if none).
+cudaError_t launch_mxfp4_slots(const moe_cfg& c, const int32_t* offsets, int32_t* slot_of,
+                               int32_t* touched, int32_t* ntouched, cudaStream_t s);
 
 // MXFP4: list the touched experts and dequantise each once into bf16 slots.
 cudaError_t launch_mxfp4_expand(const moe_cfg& c, const int32_t* offsets, const moe_weights* W,
@@ -183,6 +217,15 @@ int num_sms();
 // Tensor map of a bf16 row-major [rows, cols] matrix for TMA: box of
 // box_rows x 64 columns, 128-byte swizzle. False if it cannot be encoded.
 bool map_bf16(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows);
+// Row-major [rows, cols] bytes (e4m3 codes): box of box_rows x 128 bytes,
+// 128-byte swizzle.
+bool map_u8(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows);
+// MXFP4 codes [rows, cols/2] (cols 4-bit elements per row, two per byte):
+// box of box_rows x 128 elements, unpacked to one byte per element in shared
+// memory (16 elements per 16 bytes: 8 code bytes + 8 bytes of gap) with the
+// 128-byte swizzle, the operand layout of tcgen05.mma kind::mxf8f6f4.
+// Needs a 32-byte aligned base and cols % 128 == 0.
+bool map_fp4(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows);
 
 // Raises `func`'s dynamic shared-memory limit to at least `bytes`, once per
 // device (later calls with a size already granted cost a table lookup).

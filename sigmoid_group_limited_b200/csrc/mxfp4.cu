@@ -106,11 +106,16 @@ __global__ void __launch_bounds__(256) mxfp4_dequant(
 
 }  // namespace
 
+cudaError_t launch_mxfp4_slots(const moe_cfg& c, const int32_t* offsets, int32_t* slot_of,
+                               int32_t* touched, int32_t* ntouched, cudaStream_t s) {
+  return launch_pdl(mxfp4_slots, dim3(1), dim3(1024), 0, s, c.E, offsets, slot_of, touched,
+                    ntouched);
+}
+
 cudaError_t launch_mxfp4_expand(const moe_cfg& c, const int32_t* offsets, const moe_weights* W,
                                 int32_t* slot_of, int32_t* touched, int32_t* ntouched,
                                 uint16_t* gout, uint16_t* uout, uint16_t* dout, cudaStream_t s) {
-  cudaError_t e = launch_pdl(mxfp4_slots, dim3(1), dim3(1024), 0, s, c.E, offsets, slot_of, touched,
-                             ntouched);
+  cudaError_t e = launch_mxfp4_slots(c, offsets, slot_of, touched, ntouched, s);
   if (e != cudaSuccess) return e;
   return launch_pdl(mxfp4_dequant, dim3(num_sms() * 8), dim3(256), 0, s, c.I, c.H,
                     static_cast<const int32_t*>(touched), static_cast<const int32_t*>(ntouched),

@@ -85,6 +85,7 @@ __device__ int block_exscan2(int v0, int v1, int* scratch /*32*/, int* total) {
 
 struct SchedArgs {
   int T, K, E, H, I, Is, has_shared, bn;
+  int gu_ft, dn_ft;   // output features per gate/up item and per down item
   int32_t* gu_start;  // [E+2] first gate/up work item of slot e (e == E: shared expert)
   int32_t* dn_start;  // [E+2] first down work item of slot e
   int32_t* ready;     // nullable: [gate/up items] zeroed for the fused FFN's row-tile counters
@@ -98,8 +99,8 @@ struct SchedArgs {
 // these starts. Needs blockDim.x == 1024 and counts in shared memory.
 __device__ void build_schedule(const SchedArgs& a, const int* cnt, int* scratch) {
   const int nslots = a.E + (a.has_shared ? 1 : 0);
-  const int nt_gu_r = cdiv_dev(a.I, kTileN), nt_gu_s = cdiv_dev(a.Is, kTileN);
-  const int nt_dn = cdiv_dev(a.H, kDownTile);
+  const int nt_gu_r = cdiv_dev(a.I, a.gu_ft), nt_gu_s = cdiv_dev(a.Is, a.gu_ft);
+  const int nt_dn = cdiv_dev(a.H, a.dn_ft);
   int ngu[2] = {0, 0}, ndn[2] = {0, 0};
 #pragma unroll
   for (int q = 0; q < 2; ++q) {
@@ -383,6 +384,9 @@ SchedArgs make_sched(const moe_cfg& c, int T, const WsLayout& L, int32_t* gu_sta
   a.Is = c.I_shared;
   a.has_shared = c.I_shared > 0;
   a.bn = L.bn;
+  const bool mx = c.wfmt == MOE_W_MXFP4_A8;
+  a.gu_ft = mx ? kMxGuTile : kTileN;
+  a.dn_ft = mx ? kMxDnTile : kDownTile;
   a.gu_start = gu_start;
   a.dn_start = dn_start;
   a.ready = ready;

@@ -119,6 +119,12 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src, uint64_t 
                "l"(reinterpret_cast<uint64_t>(src)), "l"(policy)
                : "memory");
 }
+// 4-byte asynchronous copy global -> shared (both 4-byte aligned).
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)),
+               "l"(reinterpret_cast<uint64_t>(src))
+               : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;" ::: "memory");
 }
@@ -326,11 +332,56 @@ __device__ __forceinline__ uint64_t sdesc_k128(uint32_t saddr) {
   return d;
 }
 
+// Block-scaled MMA, kind::mxf8f6f4: D (fp32, TMEM) (+)= (A * scaleA) x
+// (B * scaleB)^T over K = 32, A and B K-major 8-bit-per-element tiles in
+// shared memory (4-bit codes sit unpacked, 16 per 16 bytes), one e8m0 scale
+// per row and 32-element chunk read from tensor memory at sfa / sfb; bits
+// 30-31 of those addresses pick the byte (chunk) of each 32-bit column and
+// must equal the descriptor's scale ids.
+__device__ __forceinline__ void umma_mx(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                        uint32_t idesc, uint32_t accumulate, uint32_t sfa,
+                                        uint32_t sfb) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+// Shared-memory descriptor of a 32-row x 16-byte block with no swizzle (rows
+// 16 bytes apart, 8-row groups 128 bytes apart): the source of tcgen05.cp.
+__device__ __forceinline__ uint64_t sdesc_rows16(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(128u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  return d;
+}
+// Copies a 512-byte scale atom (32 rows x 16 bytes) from shared memory into
+// 4 tensor-memory columns at `taddr`, repeated into all four 32-lane
+// quarters; ordered before later tcgen05.mma of the same thread.
+__device__ __forceinline__ void tmem_cp_atom(uint32_t taddr, uint32_t saddr) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr),
+               "l"(sdesc_rows16(saddr))
+               : "memory");
+}
+
 // Instruction descriptor, kind::f16: D fp32, A and B bf16, both K-major,
 // N >> 3 at [17,23), M >> 4 at [24,29).
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Instruction descriptor, kind::mxf8f6f4 with e8m0 scales: A e2m1 (format 5)
+// and B e4m3 (format 0), both K-major; B's scale id at [4,6), formats at
+// [7,10) and [10,13), N >> 3 at [17,23), scale type e8m0 at bit 23, M >> 4
+// at [24,29), A's scale id at [29,31), K = 32.
+__host__ __device__ constexpr uint32_t idesc_mx_e2m1_e4m3(int M, int N, int sf_id) {
+  return (static_cast<uint32_t>(sf_id) << 4) | (5u << 7) | (0u << 10) |
+         (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) | (static_cast<uint32_t>(M >> 4) << 24) |
+         (static_cast<uint32_t>(sf_id) << 29);
 }
 
 }  // namespace sgl

@@ -79,3 +79,23 @@ def test_null_misaligned_and_small_workspace_rejected_before_launch():
                                None, A, need, None, None) == -3
     assert L.moe_combine(ctypes.byref(c), 32, None, 1, A, None) == -2
     assert L.moe_grouped_swiglu(ctypes.byref(c), 32, A, A, A, A, None, A, A, need, None) == -2
+
+
+def test_block_scaled_format_validation():
+    """MOE_W_MXFP4_A8 needs H and I multiples of 128 and 32-byte aligned codes."""
+    L = sgl.lib()
+    full = workloads.CONFIGS["mxfp4_a8"]
+    assert sgl.workspace_size(full, 32) > 0
+    assert sgl.workspace_size(workloads.CONFIGS["tiny_a8"], 64) > 0
+    assert L.moe_workspace_size(ctypes.byref(sgl.make_cfg(full.with_(I=704))), 32) == 0
+    assert L.moe_workspace_size(ctypes.byref(sgl.make_cfg(full.with_(H=2496))), 32) == 0
+    assert L.moe_workspace_size(ctypes.byref(sgl.make_cfg(full.with_(wfmt=3))), 32) == 0
+    c = sgl.make_cfg(full)
+    need = sgl.workspace_size(full, 32)
+    A = 1 << 20
+    w = sgl.moe_weights(A, A + 16, A, A, A, A, A, A, A)         # 16- but not 32-byte aligned codes
+    assert L.moe_layer_forward(ctypes.byref(c), 32, A, A, None, ctypes.byref(w), A, None, None,
+                               None, A, need, None, None) == -3
+    w = sgl.moe_weights(A, A, A, None, A, A, A, A, A)           # a scale array missing
+    assert L.moe_layer_forward(ctypes.byref(c), 32, A, A, None, ctypes.byref(w), A, None, None,
+                               None, A, need, None, None) == -2
