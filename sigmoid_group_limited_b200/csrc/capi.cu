@@ -91,8 +91,10 @@ WsLayout ws_layout(const moe_cfg& c, int T) {
     L.x_q = take(static_cast<size_t>(T) * c.H);
     L.x_sf = take(static_cast<size_t>(T) * (c.H / 32));
     L.h_sf = take(static_cast<size_t>(L.max_row_tiles) * kb_i * 512);
-    L.sf_gu = take(static_cast<size_t>(L.max_touched) * (c.I / kMxGuTile) * kb_h * 512);
-    L.sf_dn = take(static_cast<size_t>(L.max_touched) * kb_h * kb_i * 512);
+    const size_t atoms = static_cast<size_t>(L.max_touched) * kb_h * kb_i * 512;
+    L.sf_g = take(atoms);
+    L.sf_u = take(atoms);
+    L.sf_d = take(atoms);
   }
   if (c.wfmt == MOE_W_MXFP4) {
     L.max_touched = static_cast<int>(TK < static_cast<size_t>(c.E) ? TK : c.E);
@@ -220,15 +222,17 @@ cudaError_t run_ffn(const moe_cfg* cfg, int T, const uint16_t* x, const int32_t*
   if (cfg->wfmt == MOE_W_MXFP4_A8) {
     cudaError_t e = launch_mx_prep(*cfg, T, offsets, W, x, at<int32_t>(ws, L.slot_of),
                                    at<int32_t>(ws, L.touched), at<int32_t>(ws, L.ntouched),
-                                   at<uint8_t>(ws, L.sf_gu), at<uint8_t>(ws, L.sf_dn),
-                                   at<uint8_t>(ws, L.x_q), at<uint8_t>(ws, L.x_sf), s);
+                                   at<uint8_t>(ws, L.sf_g), at<uint8_t>(ws, L.sf_u),
+                                   at<uint8_t>(ws, L.sf_d), at<uint8_t>(ws, L.x_q),
+                                   at<uint8_t>(ws, L.x_sf), s);
     if (e != cudaSuccess) return e;
     a.x_q = at<uint8_t>(ws, L.x_q);
     a.x_sf = at<uint8_t>(ws, L.x_sf);
     a.h_q = at<uint8_t>(ws, L.h_r);
     a.h_sf = at<uint8_t>(ws, L.h_sf);
-    a.sf_gu = at<uint8_t>(ws, L.sf_gu);
-    a.sf_dn = at<uint8_t>(ws, L.sf_dn);
+    a.sf_g = at<uint8_t>(ws, L.sf_g);
+    a.sf_u = at<uint8_t>(ws, L.sf_u);
+    a.sf_d = at<uint8_t>(ws, L.sf_d);
     a.slot_of = at<int32_t>(ws, L.slot_of);
     return launch_ffn_mx(a, s);
   }

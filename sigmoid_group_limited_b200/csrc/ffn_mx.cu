@@ -8,25 +8,26 @@
 // (lpnh.cn/news/2815793) spec table (quantisation FP8 + MXFP4, routed experts
 // in 4 bits). Formats per the OCP Microscaling spec v1.0 (see mxfp8.cu).
 //
-// Every product is D = W_tile * X_tile^T with a 128-row weight tile as the
-// MMA's A operand and a tile of up to 128 token rows as its N, K = 128 per
-// pipeline stage for the 8-bit kinds (64 for bf16):
-//   gate/up (slot e, row tile m, feature tile n of 64): A rows 0..63 = Wg rows
-//       64n.., rows 64..127 = Wu rows of the same features, B = routed rows
-//       of x (MXFP8 codes and scales, gathered); one accumulator holds gate
-//       over up, and the epilogue pairs TMEM lane l with lane l + 64 through
-//       shared memory. Routed h = silu(g) * u is quantised to MXFP8 (one
-//       warp = 32 consecutive features = one scale block); shared h -> bf16.
-//   down (slot e, row tile m, output tile n of 128): A = Wd rows 128n..,
-//       B = h rows; y_slot[j] = w_j * D (fp32).
+// Same items as the bf16 kernel (ffn.cu), with a token tile of 112 rows:
+//   gate/up (slot e, row tile m, feature tile n of 128): A0 = Wg rows, A1 = Wu
+//       rows, B = the routed rows of x (MXFP8 codes and scales, gathered);
+//       two accumulators, so the gate and up MMAs of a k step are independent
+//       (a chain of MMAs into one accumulator runs at its latency, ~1.4x
+//       slower). Routed h = silu(g) * u is quantised to MXFP8 in the epilogue
+//       (one warp = 32 consecutive features = one scale block); shared h ->
+//       bf16.
+//   down (slot e, row tile m, output tile n of 256): A0 / A1 = Wd rows
+//       [256n, 256n+128) / [256n+128, 256n+256), B = h rows; y_slot[j] = w_j * D.
 // Routed items run tcgen05.mma kind::mxf8f6f4.block_scale (e2m1 weights read
-// in place by TMA, unpacked to one byte per element; e4m3 activations); their
-// scales go shared memory -> tensor memory with tcgen05.cp once per stage.
-// Shared-expert items run kind::f16 on the same pipeline.
+// in place by TMA, unpacked to one byte per element; e4m3 activations; K = 128
+// per stage); their scale atoms go shared memory -> tensor memory with
+// tcgen05.cp once per stage. Shared-expert items run kind::f16 (K = 64 per
+// stage) on the same pipeline. TMEM: two buffers of gate | up accumulators
+// (2 x 2 x 112 columns), then the three scale atoms.
 //
-// Items, claiming, readiness counters, warp roles and bounded waits are those
-// of ffn.cu (480 threads: TMA producer, MMA issuer, 8 epilogue warps, 4
-// gatherer warps, scheduler).
+// Claiming, readiness counters, warp roles and bounded waits are those of
+// ffn.cu (480 threads: TMA producer, MMA issuer, 8 epilogue warps, 4 gatherer
+// warps, scheduler).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
@@ -51,21 +52,19 @@ constexpr int kXThreads = 32 * (kXSchedWarp + 1);
 constexpr int kXQueue = 4;
 constexpr int kXLead = 4;
 constexpr long long kXProgStride = 1024;
-constexpr int kXA = 128 * 128;             // A tile: 128 rows x 128 bytes
-constexpr int kXB = kMxTileN * 128;        // B tile: up to 128 rows x 128 bytes
-constexpr int kXStage = kXA + kXB + 1024;  // + the A and B scale atoms
-constexpr int kXStages = 6;
-constexpr int kXAccCols = kMxTileN;        // one fp32 accumulator: N columns
-constexpr int kXSfaCol = 2 * kXAccCols;    // two accumulators, then the scale atoms
-constexpr int kXSfbCol = kXSfaCol + 4;
+constexpr int kXA = 128 * 128;              // one A tile: 128 rows x 128 bytes
+constexpr int kXB = kMxTileN * 128;         // B tile: up to 112 rows x 128 bytes
+constexpr int kXSfOff = 2 * kXA + kXB;      // scale atoms: A0, A1, B (512 bytes each)
+constexpr int kXStage = (kXSfOff + 3 * 512 + 1023) / 1024 * 1024;
+constexpr int kXStages = 4;
+constexpr int kXAccCols = 2 * kMxTileN;     // gate | up of one buffer
+constexpr int kXSfCol = 2 * kXAccCols;      // scale atoms after the two buffers
 constexpr int kXTmemCols = 512;
 constexpr int kXCtrl = 512;
-constexpr int kXXchRow = 9;
-constexpr int kXXchFloats = 2 * 2 * 64 * kXXchRow;  // [column part][gate/up][feature][8]
-constexpr int kXHBox = 32;                 // h rows per TMA box
-constexpr int kXSmem = kXStages * kXStage + 1024 + kXCtrl + kXXchFloats * 4 + kMxTileN * 8;
-static_assert(kXSfbCol + 4 <= kXTmemCols, "TMEM");
-static_assert(kXStage % 1024 == 0, "stage alignment");
+constexpr int kXHBox = 16;                  // h rows per TMA box
+constexpr int kXSmem = kXStages * kXStage + 1024 + kXCtrl + kMxTileN * 8;
+static_assert(kXSfCol + 12 <= kXTmemCols, "TMEM");
+static_assert(kMxTileN % 16 == 0 && kMxTileN <= 128, "token tile");
 
 struct MxParams {
   FfnParams f;
@@ -73,21 +72,22 @@ struct MxParams {
   const uint8_t* x_sf;   // [T, H/32] e8m0
   uint8_t* h_q;          // [T*K, I] e4m3, permuted rows
   uint8_t* h_sf;         // [routed row tiles][I/128][512] atoms
-  const uint8_t* sf_gu;  // [slot][I/64][H/128][512]
-  const uint8_t* sf_dn;  // [slot][H/128][I/128][512]
+  const uint8_t* sf_g;   // [slot][I/128][H/128][512]
+  const uint8_t* sf_u;   // [slot][I/128][H/128][512]
+  const uint8_t* sf_d;   // [slot][H/128][I/128][512]
   const int32_t* slot_of;
 };
 
 struct MxMaps {
-  CUtensorMap wg, wu, wd;     // MXFP4 codes: 64-row (gate/up) and 128-row (down) boxes
-  CUtensorMap hq;             // h codes [T*K, I] bytes, 32-row boxes
-  CUtensorMap wgs, wus, wds;  // shared expert bf16: 64-row / 128-row boxes
-  CUtensorMap hs;             // shared h [T, Is] bf16, 32-row boxes
+  CUtensorMap wg, wu, wd;     // MXFP4 codes, 128-row boxes
+  CUtensorMap hq;             // h codes [T*K, I] bytes, 16-row boxes
+  CUtensorMap wgs, wus, wds;  // shared expert bf16, 128-row boxes
+  CUtensorMap hs;             // shared h [T, Is] bf16, 16-row boxes
 };
 
 __device__ __forceinline__ int atom_off(int r, int k) { return (r & 31) * 16 + (r >> 5) * 4 + k; }
 
-// e4m3 code of v * inv (inv a power of two), nearest even, saturating.
+// e4m3 code of v (already divided by the block scale), nearest even, saturating.
 __device__ __forceinline__ uint8_t to_e4m3(float v) {
   return static_cast<uint8_t>(__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3));
 }
@@ -109,8 +109,7 @@ __global__ void __launch_bounds__(kXThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(const_cast<long long*>(prog) + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* qitem = abort_flag + 1;  // [kXQueue]
-  float* xch = reinterpret_cast<float*>(ctrl + kXCtrl);
-  int* meta_j = reinterpret_cast<int*>(xch + kXXchFloats);
+  int* meta_j = reinterpret_cast<int*>(ctrl + kXCtrl);
   float* meta_w = reinterpret_cast<float*>(meta_j + kMxTileN);
   int* s_gu = reinterpret_cast<int*>(meta_w + kMxTileN);  // [E+2]
   int* s_dn = s_gu + (p.E + 2);                           // [E+2]
@@ -158,7 +157,7 @@ __global__ void __launch_bounds__(kXThreads, 1)
   const int n_gu = min(p.nitems[0], p.max_gu);
   const int n_dn = min(p.nitems[1], p.max_dn);
   const int n_all = n_gu + n_dn;
-  const int kbh = p.H / 128, kbi = p.I / 128, ftg = p.I / kMxGuTile, rtd = p.H / kMxDnTile;
+  const int kbh = p.H / 128, kbi = p.I / 128, ftg = cdiv_dev(p.I, kMxGuTile);
   auto item_at = [&](int i, bool& gu) {
     gu = i < n_gu;
     return gu ? decode_item(i, s_gu, s_off, nslots, p.E, p.T, kMxTileN)
@@ -170,6 +169,10 @@ __global__ void __launch_bounds__(kXThreads, 1)
   // k-blocks: 128 wide for the 8-bit routed operands, 64 for bf16
   auto nkb_of = [&](bool gu, bool sh) {
     return gu ? (sh ? p.H / 64 : kbh) : (sh ? p.Is / 64 : kbi);
+  };
+  // a down item's second 128-row half exists unless it starts past H
+  auto two_halves = [&](const WorkItem& it, bool gu) {
+    return gu || it.ntile * kMxDnTile + 128 < p.H;
   };
   auto mma_n = [&](const WorkItem& it) { return (min(it.nrows, kMxTileN) + 15) & ~15; };
   // dense index of a routed (slot, row tile): every routed slot has ftg gate/up tiles per row tile
@@ -223,8 +226,8 @@ __global__ void __launch_bounds__(kXThreads, 1)
     __syncwarp();
   } else if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    // Weight tiles (and their scale atoms), and for down items the h rows
-    // (and their scale atom). Routed MXFP4 boxes count their packed bytes.
+    // Weight tiles and their scale atoms; for down items also the h rows and
+    // their scale atom. MXFP4 boxes count their packed bytes.
     if (lane == 0) {
       const uint64_t pol_w = policy_evict_first();
       const uint64_t pol_h = policy_evict_last();
@@ -241,52 +244,59 @@ __global__ void __launch_bounds__(kXThreads, 1)
         const bool sh = it.e == p.E;
         if (!gu) fence_proxy_async_global();  // h was published by other CTAs
         const int nkb = nkb_of(gu, sh);
-        const int nhbox = gu ? 0 : (mma_n(it) + kXHBox - 1) / kXHBox;
+        const bool two = two_halves(it, gu);
+        const int na = two ? 2 : 1;
+        const int nhbox = gu ? 0 : mma_n(it) / kXHBox;
         const int slot = sh ? 0 : q.slot_of[it.e];
-        const int rt = sh ? 0 : row_tile(it);
         uint32_t bytes;
-        if (gu) bytes = sh ? 2 * 64 * 128 : 2 * 64 * 64 + 512;
-        else bytes = (sh ? 128 * 128 : 128 * 64 + 512 + 512) + nhbox * kXHBox * 128;
-        const uint8_t* sfa_src = nullptr;
-        if (!sh)
-          sfa_src = gu ? q.sf_gu + (static_cast<size_t>(slot) * ftg + it.ntile) * kbh * 512
-                       : q.sf_dn + (static_cast<size_t>(slot) * rtd + it.ntile) * kbi * 512;
-        const uint8_t* sfb_src = (!sh && !gu) ? q.h_sf + static_cast<size_t>(rt) * kbi * 512 : nullptr;
+        if (sh) bytes = na * kXA + nhbox * kXHBox * 128;
+        else bytes = na * (128 * 64 + 512) + (gu ? 0 : nhbox * kXHBox * 128 + 512);
+        // first weight row of A0 (A1 follows 128 rows later for down items)
+        const int arow = gu ? it.ntile * kMxGuTile : it.ntile * kMxDnTile;
+        const uint8_t* sfa0 = nullptr;
+        const uint8_t* sfa1 = nullptr;
+        const uint8_t* sfb = nullptr;
+        if (!sh) {
+          if (gu) {
+            sfa0 = q.sf_g + (static_cast<size_t>(slot) * (p.I / 128) + arow / 128) * kbh * 512;
+            sfa1 = q.sf_u + (static_cast<size_t>(slot) * (p.I / 128) + arow / 128) * kbh * 512;
+          } else {
+            sfa0 = q.sf_d + (static_cast<size_t>(slot) * (p.H / 128) + arow / 128) * kbi * 512;
+            sfa1 = sfa0 + static_cast<size_t>(kbi) * 512;  // the next 128-row tile
+            sfb = q.h_sf + static_cast<size_t>(row_tile(it)) * kbi * 512;
+          }
+        }
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) {
             live = false;
             break;
           }
           uint8_t* sA = smem + stage * kXStage;
-          uint8_t* sB = sA + kXA;
-          uint8_t* sSFA = sB + kXB;
-          uint8_t* sSFB = sSFA + 512;
+          uint8_t* sB = sA + 2 * kXA;
+          uint8_t* sSF = sA + kXSfOff;
           mbar_arrive_expect_tx(&full[stage], bytes);
-          if (gu) {
-            const int frow = it.ntile * kMxGuTile;
-            if (sh) {
-              tma_load_2d(sA, &m.wgs, &full[stage], kb * 64, frow, pol_w);
-              tma_load_2d(sA + kXA / 2, &m.wus, &full[stage], kb * 64, frow, pol_w);
-            } else {
-              tma_load_2d(sA, &m.wg, &full[stage], kb * 128, it.e * p.I + frow, pol_w);
-              tma_load_2d(sA + kXA / 2, &m.wu, &full[stage], kb * 128, it.e * p.I + frow, pol_w);
-              bulk_load(sSFA, sfa_src + kb * 512, 512, &full[stage]);
-            }
+          if (sh) {
+            const CUtensorMap* a0 = gu ? &m.wgs : &m.wds;
+            const CUtensorMap* a1 = gu ? &m.wus : &m.wds;
+            tma_load_2d(sA, a0, &full[stage], kb * 64, arow, pol_w);
+            if (two) tma_load_2d(sA + kXA, a1, &full[stage], kb * 64, gu ? arow : arow + 128, pol_w);
+            for (int hb = 0; hb < nhbox; ++hb)
+              tma_load_2d(sB + hb * kXHBox * 128, &m.hs, &full[stage], kb * 64, it.row0 + hb * kXHBox,
+                          pol_h);
           } else {
-            const int orow = it.ntile * kMxDnTile;
-            if (sh) {
-              tma_load_2d(sA, &m.wds, &full[stage], kb * 64, orow, pol_w);
-              for (int hb = 0; hb < nhbox; ++hb)
-                tma_load_2d(sB + hb * kXHBox * 128, &m.hs, &full[stage], kb * 64,
-                            it.row0 + hb * kXHBox, pol_h);
+            if (gu) {
+              tma_load_2d(sA, &m.wg, &full[stage], kb * 128, it.e * p.I + arow, pol_w);
+              tma_load_2d(sA + kXA, &m.wu, &full[stage], kb * 128, it.e * p.I + arow, pol_w);
             } else {
-              tma_load_2d(sA, &m.wd, &full[stage], kb * 128, it.e * p.H + orow, pol_w);
-              bulk_load(sSFA, sfa_src + kb * 512, 512, &full[stage]);
+              tma_load_2d(sA, &m.wd, &full[stage], kb * 128, it.e * p.H + arow, pol_w);
+              if (two) tma_load_2d(sA + kXA, &m.wd, &full[stage], kb * 128, it.e * p.H + arow + 128, pol_w);
               for (int hb = 0; hb < nhbox; ++hb)
                 tma_load_2d(sB + hb * kXHBox * 128, &m.hq, &full[stage], kb * 128,
                             it.row0 + hb * kXHBox, pol_h);
-              bulk_load(sSFB, sfb_src + kb * 512, 512, &full[stage]);
+              bulk_load(sSF + 1024, sfb + kb * 512, 512, &full[stage]);
             }
+            bulk_load(sSF, sfa0 + kb * 512, 512, &full[stage]);
+            if (two) bulk_load(sSF + 512, sfa1 + kb * 512, 512, &full[stage]);
           }
           *prog = n * kXProgStride + kb + 1;
           if (++stage == kXStages) {
@@ -311,7 +321,7 @@ __global__ void __launch_bounds__(kXThreads, 1)
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool live = true;
-      const uint32_t sfa_t = tmem_base + kXSfaCol, sfb_t = tmem_base + kXSfbCol;
+      const uint32_t sf_t = tmem_base + kXSfCol;  // A0, A1, B scale atoms: 4 columns each
       for (int n = 0; live; ++n) {
         int item;
         if (!next_item(n, item, false)) break;
@@ -320,35 +330,44 @@ __global__ void __launch_bounds__(kXThreads, 1)
         if (!ok_item(it, gu)) continue;
         const bool sh = it.e == p.E;
         const int nkb = nkb_of(gu, sh);
+        const bool two = two_halves(it, gu);
         const int N = mma_n(it);
         const uint32_t idesc_f16 = idesc_bf16(128, N);
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) break;
         tc_fence_after();
-        const uint32_t d0 = tmem_base + acc * kXAccCols;
+        const uint32_t d0 = tmem_base + acc * kXAccCols, d1 = d0 + kMxTileN;
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) {
             live = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(smem + stage * kXStage);
-          const uint32_t b0 = a0 + kXA;
+          const uint32_t a0 = smem_u32(smem + stage * kXStage), a1 = a0 + kXA, b0 = a0 + 2 * kXA;
           if (sh) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              umma_bf16(d0, sdesc_k128(a0 + kk * 32), sdesc_k128(b0 + kk * 32), idesc_f16,
-                        (kb | kk) != 0 ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t bd = sdesc_k128(b0 + kk * 32);
+              const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
+              umma_bf16(d0, sdesc_k128(a0 + kk * 32), bd, idesc_f16, accum);
+              if (two) umma_bf16(d1, sdesc_k128(a1 + kk * 32), bd, idesc_f16, accum);
+            }
           } else {
-            // this stage's scales into tensor memory (ordered before the MMAs below,
-            // and after the MMAs of the previous stage that read the same columns)
-            tmem_cp_atom(sfa_t, b0 + kXB);
-            tmem_cp_atom(sfb_t, b0 + kXB + 512);
+            // this stage's scales into tensor memory: ordered before the MMAs
+            // below and after those of the previous stage that read the columns
+            const uint32_t sf_s = a0 + kXSfOff;
+            tmem_cp_atom(sf_t, sf_s);
+            if (two) tmem_cp_atom(sf_t + 4, sf_s + 512);
+            tmem_cp_atom(sf_t + 8, sf_s + 1024);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const uint32_t sel = static_cast<uint32_t>(kk) << 30;
-              umma_mx(d0, sdesc_k128(a0 + kk * 32), sdesc_k128(b0 + kk * 32),
-                      idesc_mx_e2m1_e4m3(128, N, kk), (kb | kk) != 0 ? 1u : 0u, sfa_t | sel,
-                      sfb_t | sel);
+              const uint64_t bd = sdesc_k128(b0 + kk * 32);
+              const uint32_t idesc = idesc_mx_e2m1_e4m3(128, N, kk);
+              const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
+              umma_mx(d0, sdesc_k128(a0 + kk * 32), bd, idesc, accum, sf_t | sel, (sf_t + 8) | sel);
+              if (two)
+                umma_mx(d1, sdesc_k128(a1 + kk * 32), bd, idesc, accum, (sf_t + 4) | sel,
+                        (sf_t + 8) | sel);
             }
           }
           umma_commit(&empty[stage]);
@@ -418,20 +437,20 @@ __global__ void __launch_bounds__(kXThreads, 1)
         const int t = min(max(p.perm[row] / p.K, 0), p.T - 1);
         sf_src = q.x_sf + static_cast<size_t>(t) * (p.H / 32);
       }
-      const int kstep = sh ? 128 : 128;  // bytes of one row per k-block (64 bf16 or 128 e4m3)
       for (int kb = 0; kb < nkb; ++kb) {
         if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) {
           live = false;
           break;
         }
         if (gu) {
-          uint8_t* sB = smem + stage * kXStage + kXA;
+          uint8_t* sB = smem + stage * kXStage + 2 * kXA;
+          // 128 bytes of a row per k-block: 64 bf16 or 128 e4m3
 #pragma unroll
           for (int i = 0; i < kRowsPerThread; ++i) {
             const int r = rbase + 16 * i;
-            if (r < nb) cp_async16(sB + r * 128 + ((chunk ^ (r & 7)) << 4), src[i] + kb * kstep, pol_x);
+            if (r < nb) cp_async16(sB + r * 128 + ((chunk ^ (r & 7)) << 4), src[i] + kb * 128, pol_x);
           }
-          if (sf_src) cp_async4(sB + kXB + 512 + atom_off(g, 0), sf_src + kb * 4);
+          if (sf_src) cp_async4(smem + stage * kXStage + kXSfOff + 1024 + atom_off(g, 0), sf_src + kb * 4);
         }
         cp_async_commit();
         if (pend[0] >= 0) {
@@ -457,9 +476,10 @@ __global__ void __launch_bounds__(kXThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int qd = warp & 3;          // TMEM lane quarter
-    const int et = tid - 2 * 32;      // epilogue thread 0..255
-    const int cpart = et >> 7;        // alternate column chunks
+    const int qd = warp & 3;            // TMEM lane quarter
+    const int orow = qd * 32 + lane;    // output feature within a 128-row tile
+    const int et = tid - 2 * 32;        // epilogue thread 0..255
+    const int cpart = et >> 7;          // the two warps of a quarter: alternate column chunks
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int n = 0;; ++n) {
@@ -499,69 +519,56 @@ __global__ void __launch_bounds__(kXThreads, 1)
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(qd * 32) << 16) + acc * kXAccCols;
       const int ncol = mma_n(it);
       if (gu) {
-        // lanes 0-63: gate rows, 64-127: up rows of the same 64 features. Per
-        // 16-column chunk the gate warps finish columns 0-7 and the up warps
-        // columns 8-15, each taking the other operand through shared memory.
-        const bool is_gate = qd < 2;
-        const int fq = qd & 1;
-        const int nfeat = it.ntile * kMxGuTile + fq * 32 + lane;
+        const int nfeat = it.ntile * kMxGuTile + orow;
+        const int ncols = sh ? p.Is : p.I;
+        const bool ok = nfeat < ncols;
         const float L = sh ? p.lim_s : p.lim_r;
-        float* give = xch + ((cpart * 2 + (is_gate ? 0 : 1)) * 64 + fq * 32 + lane) * kXXchRow;
-        const float* take = xch + ((cpart * 2 + (is_gate ? 1 : 0)) * 64 + fq * 32 + lane) * kXXchRow;
-        // routed h scale block of this warp: features 32 * blk .. +31
-        const int blk = (it.ntile * kMxGuTile + fq * 32) / 32;
-        uint8_t* hsf = sh ? nullptr : q.h_sf + (static_cast<size_t>(row_tile(it)) * kbi + blk / 4) * 512;
-        // both column halves run the same iterations (the exchange has CTA
-        // barriers); a chunk past ncol reads unused accumulator columns and
-        // stores nothing (c0 + 16 <= 128 always)
+        // routed: this warp's 32 features are one MXFP8 block, chunk qd of the
+        // h scale atom of (row tile, k-block ntile)
+        uint8_t* hsf = sh ? nullptr : q.h_sf + (static_cast<size_t>(row_tile(it)) * kbi + it.ntile) * 512;
 #pragma unroll 1
-        for (int base = 0; base < ncol; base += 32) {
-          const int c0 = base + 16 * cpart;
-          float v[16];
-          tmem_ld16(taddr + c0, v);
+        for (int c0 = 16 * cpart; c0 < ncol; c0 += 32) {
+          float gv[16], uv[16];
+          tmem_ld16(taddr + c0, gv);
+          tmem_ld16(taddr + kMxTileN + c0, uv);
           tmem_ld_wait();
 #pragma unroll
-          for (int c = 0; c < 8; ++c) give[c] = is_gate ? v[8 + c] : v[c];
-          epi_bar<kXEpiThreads>();
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const int col = c0 + (is_gate ? c : 8 + c);
-            const float gg = is_gate ? v[c] : take[c];
-            const float uu = is_gate ? take[c] : v[8 + c];
-            const float h = swiglu(gg, uu, L);
+          for (int c = 0; c < 16; ++c) {
+            const int col = c0 + c;
+            const float h = ok ? swiglu(gv[c], uv[c], L) : 0.f;
             if (sh) {
-              if (col < it.nrows)
+              if (ok && col < it.nrows)
                 p.h_s[static_cast<size_t>(it.row0 + col) * p.Is + nfeat] = f2bf(h);
             } else {
-              // MXFP8 block = this warp's 32 features of one token
               const uint32_t amax = __reduce_max_sync(0xffffffffu, __float_as_uint(h) & 0x7FFFFFFFu);
               const int byte = min(max(static_cast<int>(amax >> 23) - 8, 0), 254);
-              const int ie = 254 - byte;
+              const int ie = 254 - byte;  // 1 / scale = 2^(127 - byte)
               const float inv = ie > 0 ? __uint_as_float(static_cast<uint32_t>(ie) << 23)
                                        : __uint_as_float(0x00400000u);
               if (col < it.nrows) {
-                q.h_q[static_cast<size_t>(it.row0 + col) * p.I + nfeat] = to_e4m3(h * inv);
-                if (lane == 0) hsf[atom_off(col, blk & 3)] = static_cast<uint8_t>(byte);
+                if (ok) q.h_q[static_cast<size_t>(it.row0 + col) * p.I + nfeat] = to_e4m3(h * inv);
+                if (lane == 0) hsf[atom_off(col, qd)] = static_cast<uint8_t>(byte);
               }
             }
           }
-          epi_bar<kXEpiThreads>();
         }
       } else {
-        const int nfeat = it.ntile * kMxDnTile + qd * 32 + lane;
-        const bool ok = nfeat < p.H;
+        const bool two = two_halves(it, gu);
 #pragma unroll 1
-        for (int c0 = 32 * cpart; c0 < ncol; c0 += 64) {
-          float ov[32];
-          tmem_ld16(taddr + c0, ov);
-          tmem_ld16(taddr + c0 + 16, ov + 16);
-          tmem_ld_wait();
-          if (ok) {
+        for (int half = 0; half < (two ? 2 : 1); ++half) {
+          const int nfeat = it.ntile * kMxDnTile + half * 128 + orow;
+          const bool ok = nfeat < p.H;
+#pragma unroll 1
+          for (int c0 = 16 * cpart; c0 < ncol; c0 += 32) {
+            float ov[16];
+            tmem_ld16(taddr + half * kMxTileN + c0, ov);
+            tmem_ld_wait();
+            if (ok) {
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              if (c0 + c >= ncol) break;
-              const int j = meta_j[c0 + c];
-              if (j >= 0) p.y_slot[static_cast<size_t>(j) * p.H + nfeat] = meta_w[c0 + c] * ov[c];
+              for (int c = 0; c < 16; ++c) {
+                const int j = meta_j[c0 + c];
+                if (j >= 0) p.y_slot[static_cast<size_t>(j) * p.H + nfeat] = meta_w[c0 + c] * ov[c];
+              }
             }
           }
         }
@@ -628,19 +635,19 @@ cudaError_t launch_ffn_mx(const GemmArgs& a, cudaStream_t s) {
   q.x_sf = a.x_sf;
   q.h_q = a.h_q;
   q.h_sf = a.h_sf;
-  q.sf_gu = a.sf_gu;
-  q.sf_dn = a.sf_dn;
+  q.sf_g = a.sf_g;
+  q.sf_u = a.sf_u;
+  q.sf_d = a.sf_d;
   q.slot_of = a.slot_of;
   const int T = a.T, TK = a.T * c.K;
   const uint64_t E = static_cast<uint64_t>(c.E);
   MxMaps m;
-  bool ok = map_fp4(&m.wg, a.Wg, E * c.I, c.H, kMxGuTile) &&
-            map_fp4(&m.wu, a.Wu, E * c.I, c.H, kMxGuTile) &&
-            map_fp4(&m.wd, a.Wd, E * c.H, c.I, kMxDnTile) && map_u8(&m.hq, a.h_q, TK, c.I, kXHBox);
+  bool ok = map_fp4(&m.wg, a.Wg, E * c.I, c.H, 128) && map_fp4(&m.wu, a.Wu, E * c.I, c.H, 128) &&
+            map_fp4(&m.wd, a.Wd, E * c.H, c.I, 128) && map_u8(&m.hq, a.h_q, TK, c.I, kXHBox);
   if (p.has_shared) {
-    ok = ok && map_bf16(&m.wgs, a.W->Wg_s, c.I_shared, c.H, kMxGuTile) &&
-         map_bf16(&m.wus, a.W->Wu_s, c.I_shared, c.H, kMxGuTile) &&
-         map_bf16(&m.wds, a.W->Wd_s, c.H, c.I_shared, kMxDnTile) &&
+    ok = ok && map_bf16(&m.wgs, a.W->Wg_s, c.I_shared, c.H, 128) &&
+         map_bf16(&m.wus, a.W->Wu_s, c.I_shared, c.H, 128) &&
+         map_bf16(&m.wds, a.W->Wd_s, c.H, c.I_shared, 128) &&
          map_bf16(&m.hs, a.h_s, T, c.I_shared, kXHBox);
   } else {
     m.wgs = m.wus = m.wds = m.hs = m.hq;  // never read

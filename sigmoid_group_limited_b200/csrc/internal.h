@@ -30,12 +30,13 @@ constexpr int kPermTile = 2048;   // (token, slot) entries per permutation tile
 constexpr int kTileN = 128;       // output features per GEMM tile (MMA M)
 constexpr int kDownTile = 256;    // hidden features per down item (two MMA tiles)
 constexpr int kPairTileN = 256;   // token tile of the CTA-pair FFN (large batches)
-// Block-scaled FFN (MOE_W_MXFP4_A8): token tile, intermediate features per
-// gate/up item (their gate and up rows share one 128-row MMA tile) and hidden
-// features per down item.
-constexpr int kMxTileN = 128;
-constexpr int kMxGuTile = 64;
-constexpr int kMxDnTile = 128;
+// Block-scaled FFN (MOE_W_MXFP4_A8): token tile (MMA N; two double-buffered
+// gate/up accumulators of this width and the scale columns fill the 512 TMEM
+// columns), intermediate features per gate/up item and hidden features per
+// down item (as the bf16 kernel).
+constexpr int kMxTileN = 112;
+constexpr int kMxGuTile = 128;
+constexpr int kMxDnTile = 256;
 constexpr int kMaxExpertsCfg = 1024;  // largest E a configuration may have
 
 // The expert-FFN kernel for large batches: one CTA per item (default), or a
@@ -71,9 +72,9 @@ struct WsLayout {
   size_t slot_of, touched, ntouched, wq_g, wq_u, wq_d;
   // MOE_W_MXFP4_A8 only: MXFP8 x (codes [T,H], scales [T,H/32]); the scales
   // of h (codes reuse h_r) as 512-byte atoms per (row tile, 128-wide k-block);
-  // the touched experts' weight scales as atoms (gate/up: per 64-feature
-  // tile and k-block; down: per 128-row tile and k-block)
-  size_t x_q, x_sf, h_sf, sf_gu, sf_dn;
+  // the touched experts' weight scales as atoms per (128-row tile, k-block)
+  // of Wg, Wu and Wd
+  size_t x_q, x_sf, h_sf, sf_g, sf_u, sf_d;
   int max_row_tiles;
   size_t wr_split;  // router matrix as three bf16 terms (batches above 32 tokens)
   int max_touched;
@@ -138,8 +139,9 @@ struct GemmArgs {
   const uint8_t* x_sf;       // [T, H/32] e8m0
   uint8_t* h_q;              // [T*K, I] e4m3 (permuted rows)
   uint8_t* h_sf;             // [row tiles][I/128][512] e8m0 atoms
-  const uint8_t* sf_gu;      // [slot][I/64][H/128][512]
-  const uint8_t* sf_dn;      // [slot][H/128][I/128][512]
+  const uint8_t* sf_g;       // [slot][I/128][H/128][512]
+  const uint8_t* sf_u;       // [slot][I/128][H/128][512]
+  const uint8_t* sf_d;       // [slot][H/128][I/128][512]
   const int32_t* slot_of;    // [E] touched slot of expert e
 };
 
@@ -157,11 +159,11 @@ cudaError_t launch_router_gemm(const moe_cfg& c, int T, const uint16_t* x, const
 // shared-expert items on kind::f16, in one persistent launch.
 cudaError_t launch_ffn_mx(const GemmArgs& a, cudaStream_t s);
 // MOE_W_MXFP4_A8 inputs of that FFN: touched-expert slots, their weight
-// scales repacked as atoms (sf_gu / sf_dn) and x quantised to MXFP8.
+// scales repacked as atoms (sf_g / sf_u / sf_d) and x quantised to MXFP8.
 cudaError_t launch_mx_prep(const moe_cfg& c, int T, const int32_t* offsets, const moe_weights* W,
                            const uint16_t* x, int32_t* slot_of, int32_t* touched,
-                           int32_t* ntouched, uint8_t* sf_gu, uint8_t* sf_dn, uint8_t* x_q,
-                           uint8_t* x_sf, cudaStream_t s);
+                           int32_t* ntouched, uint8_t* sf_g, uint8_t* sf_u, uint8_t* sf_d,
+                           uint8_t* x_q, uint8_t* x_sf, cudaStream_t s);
 // Touched experts of a batch in increasing id order (slot_of[e], -1 if none).
 cudaError_t launch_mxfp4_slots(const moe_cfg& c, const int32_t* offsets, int32_t* slot_of,
                                int32_t* touched, int32_t* ntouched, cudaStream_t s);

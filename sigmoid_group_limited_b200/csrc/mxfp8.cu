@@ -28,49 +28,41 @@ namespace {
 
 __device__ __forceinline__ int atom_offset(int r, int k) { return (r & 31) * 16 + (r >> 5) * 4 + k; }
 
-// Weight scales of the touched experts as atoms. Unit = one row of one atom
-// (four scale bytes, read as one 32-bit word):
-//   gate/up: [slot][64-feature tile f][k-block b][atom]; atom rows 0..63 are
-//            gate rows 64f.., rows 64..127 the up rows of the same features;
-//   down:    [slot][128-row tile t][k-block b][atom].
+// Weight scales of the touched experts as atoms, [slot][128-row tile][k-block]
+// for each of Wg, Wu ([I, H]) and Wd ([H, I]). Unit = one row of one atom
+// (four scale bytes, read as one 32-bit word); consecutive threads take
+// consecutive rows of one atom.
 __global__ void __launch_bounds__(256) mx_sf_repack(int H, int I, int max_touched,
                                                      const int32_t* __restrict__ touched,
                                                      const int32_t* __restrict__ ntouched,
                                                      const uint8_t* __restrict__ gs,
                                                      const uint8_t* __restrict__ us,
                                                      const uint8_t* __restrict__ ds,
-                                                     uint8_t* __restrict__ sf_gu,
-                                                     uint8_t* __restrict__ sf_dn) {
+                                                     uint8_t* __restrict__ sf_g,
+                                                     uint8_t* __restrict__ sf_u,
+                                                     uint8_t* __restrict__ sf_d) {
   pdl_trigger();
   pdl_wait();  // the touched list comes from the previous kernel
   const int nt = min(*ntouched, max_touched);
-  const int kbh = H / 128, kbi = I / 128, ftg = I / kMxGuTile, rtd = H / 128;
-  const long long per_gu = static_cast<long long>(ftg) * kbh * 128;
-  const long long per_dn = static_cast<long long>(rtd) * kbi * 128;
-  const long long total = static_cast<long long>(nt) * (per_gu + per_dn);
+  const int kbh = H / 128, kbi = I / 128;
+  const long long per_mat = static_cast<long long>(kbh) * kbi * 128;  // units per matrix (both shapes)
+  const long long total = static_cast<long long>(nt) * 3 * per_mat;
   for (long long u = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; u < total;
        u += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const long long slot = u / (per_gu + per_dn);
-    long long v = u - slot * (per_gu + per_dn);
+    const long long slot = u / (3 * per_mat);
+    long long v = u - slot * 3 * per_mat;
+    const int mat = static_cast<int>(v / per_mat);
+    v -= mat * per_mat;
     const long long e = touched[slot];
     const int r = static_cast<int>(v & 127);
-    v >>= 7;
-    uint32_t word;
-    uint8_t* dst;
-    if (v < per_gu / 128) {
-      const int b = static_cast<int>(v % kbh), f = static_cast<int>(v / kbh);
-      const int row = f * kMxGuTile + (r & 63);
-      const uint8_t* src = (r < 64 ? gs : us) + (e * I + row) * (H / 32) + b * 4;
-      word = *reinterpret_cast<const uint32_t*>(src);
-      dst = sf_gu + ((slot * ftg + f) * kbh + b) * 512;
-    } else {
-      v -= per_gu / 128;
-      const int b = static_cast<int>(v % kbi), t = static_cast<int>(v / kbi);
-      const uint8_t* src = ds + (e * H + t * 128 + r) * (I / 32) + b * 4;
-      word = *reinterpret_cast<const uint32_t*>(src);
-      dst = sf_dn + ((slot * rtd + t) * kbi + b) * 512;
-    }
-    *reinterpret_cast<uint32_t*>(dst + atom_offset(r, 0)) = word;
+    const long long atom = v >> 7;  // (row tile, k-block) of this matrix
+    const int nkb = mat < 2 ? kbh : kbi;  // k-blocks along the contraction
+    const int kc = mat < 2 ? H / 32 : I / 32;  // scale bytes per row
+    const long long rows = mat < 2 ? I : H;
+    const int t = static_cast<int>(atom / nkb), b = static_cast<int>(atom % nkb);
+    const uint8_t* src = (mat == 0 ? gs : mat == 1 ? us : ds) + (e * rows + t * 128 + r) * kc + b * 4;
+    uint8_t* dst = (mat == 0 ? sf_g : mat == 1 ? sf_u : sf_d) + (slot * per_mat / 128 + atom) * 512;
+    *reinterpret_cast<uint32_t*>(dst + atom_offset(r, 0)) = *reinterpret_cast<const uint32_t*>(src);
   }
 }
 
@@ -123,15 +115,15 @@ __global__ void __launch_bounds__(256) mx_quant_x(long long nblocks, int H,
 
 cudaError_t launch_mx_prep(const moe_cfg& c, int T, const int32_t* offsets, const moe_weights* W,
                            const uint16_t* x, int32_t* slot_of, int32_t* touched,
-                           int32_t* ntouched, uint8_t* sf_gu, uint8_t* sf_dn, uint8_t* x_q,
-                           uint8_t* x_sf, cudaStream_t s) {
+                           int32_t* ntouched, uint8_t* sf_g, uint8_t* sf_u, uint8_t* sf_d,
+                           uint8_t* x_q, uint8_t* x_sf, cudaStream_t s) {
   cudaError_t e = launch_mxfp4_slots(c, offsets, slot_of, touched, ntouched, s);
   if (e != cudaSuccess) return e;
   const long long TK = static_cast<long long>(T) * c.K;
   const int max_touched = static_cast<int>(TK < c.E ? TK : c.E);
   e = launch_pdl(mx_sf_repack, dim3(num_sms() * 4), dim3(256), 0, s, c.H, c.I, max_touched,
                  static_cast<const int32_t*>(touched), static_cast<const int32_t*>(ntouched),
-                 W->Wg_scale, W->Wu_scale, W->Wd_scale, sf_gu, sf_dn);
+                 W->Wg_scale, W->Wu_scale, W->Wd_scale, sf_g, sf_u, sf_d);
   if (e != cudaSuccess) return e;
   const long long nblocks = static_cast<long long>(T) * (c.H / 32);
   long long grid = (nblocks + 255) / 256;
