@@ -205,10 +205,20 @@ def algorithmic_work(cfg, T: int, touched: int):
                 layer=(layer_bytes, layer_flops), router_flops=2.0 * T * H * E)
 
 
-def roofline_entry(bytes_, flops, seconds, peaks, sustained=False):
+# the nominal dense fp8 / bf16 tensor ratio (4.5 / 2.25 PFLOP/s): the block-scaled
+# MXFP8 x MXFP4 flops are credited at the measured bf16 peak times this
+FP8_OVER_BF16 = 2.0
+
+
+def roofline_entry(bytes_, flops, seconds, peaks, sustained=False, fp8_flops=0.0):
+    """fp8_flops: the part of `flops` that runs block-scaled 8-bit (its peak
+    is FP8_OVER_BF16 x the bf16 one); the entry's peak is then the effective
+    rate of the mix, flops / (bf16 time + fp8 time)."""
     tp = (peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]) * 1e12
     bw = peaks["hbm_gbs"] * 1e9
-    t_mem, t_tc = bytes_ / bw, flops / tp
+    t_mem = bytes_ / bw
+    t_tc = (flops - fp8_flops) / tp + fp8_flops / (FP8_OVER_BF16 * tp)
+    tp = flops / t_tc if t_tc > 0 else tp
     if t_mem >= t_tc:
         ach = bytes_ / seconds / 1e9
         return {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -256,14 +266,20 @@ def ffn_traffic(cfg, algorithmic_bytes: float):
 STAGES = ("route", "permute", "gateup", "down", "combine")
 
 
+DTYPES = {workloads.MOE_W_BF16: "bf16",
+          workloads.MOE_W_MXFP4: "mxfp4 weights expanded to bf16",
+          workloads.MOE_W_MXFP4_A8: "mxfp8 x mxfp4 (routed, block-scaled), bf16 (shared)"}
+
+
 def kernels_per_step(cfg) -> int:
     """Library kernels launched by one moe_layer_forward: router 3 (logits,
     certified top-k, exact re-derivation; the logits take 2 kernels, split and
     tensor-core GEMM, above 32 tokens), permutation 1 when all T*K slots fit
     one 2048-entry tile else 3, the fused expert FFN 1, combine 1; MXFP4 adds
-    2 (touched-expert list, dequantisation)."""
+    2 (touched-expert list, dequantisation); the block-scaled MXFP4_A8 adds 3
+    (touched-expert list, weight-scale atoms, MXFP8 x)."""
     n = (3 if cfg.T <= 32 else 4) + (1 if cfg.T * cfg.K <= 2048 else 3) + 1 + 1
-    return n + (2 if cfg.wfmt == workloads.MOE_W_MXFP4 else 0)
+    return n + {workloads.MOE_W_MXFP4: 2, workloads.MOE_W_MXFP4_A8: 3}.get(cfg.wfmt, 0)
 
 
 def measure_gpu(cfg, steps, warmup, device, rank, clk, with_e2e=True):
@@ -453,7 +469,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="decode", choices=sorted(workloads.CONFIGS))
-    ap.add_argument("--also", default="prefill", help="second workload for the line ('' = none)")
+    ap.add_argument("--also", default="prefill,mxfp4_a8",
+                    help="further workloads for the line, comma-separated ('' = none)")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--oracle-tokens", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -521,11 +538,11 @@ def run_native(args, rank, world, local):
     cfg = workload_cfg(args)
     with ClockSampler(device) as clk:
         m = measure_gpu(cfg, args.steps, args.warmup, device, rank, clk)
-        also = None
-        if args.also and args.also != args.workload:
-            acfg = workloads.CONFIGS[args.also]
-            also = (acfg, measure_gpu(acfg, args.steps, args.warmup, device, rank, clk,
-                                      with_e2e=False))
+        also = []
+        for name in [a for a in args.also.split(",") if a and a != args.workload]:
+            acfg = workloads.CONFIGS[name]
+            also.append((acfg, measure_gpu(acfg, args.steps, args.warmup, device, rank, clk,
+                                           with_e2e=False)))
     clocks = clk.summary()
     dev_s = reduce_max(m["device_ms_total"], device) / 1e3
     plain_s = reduce_max(m["plain_ms_total"], device) / 1e3
@@ -538,14 +555,24 @@ def run_native(args, rank, world, local):
         b = work["gateup"][0] + work["down"][0]
         f = work["gateup"][1] + work["down"][1]
         t_ffn = (mm["stage_ms"]["ffn"]) / 1e3
-        ent = roofline_entry(b, f, t_ffn, peaks)
-        ent.update(kernel="moe_ffn (gate/up + down)", traffic=ffn_traffic(cfg_, b),
+        mx = cfg_.wfmt == workloads.MOE_W_MXFP4_A8
+        # block-scaled: the routed experts' flops run at the fp8 rate, the shared expert's at bf16
+        f8 = 2.0 * cfg_.T * cfg_.K * 3 * cfg_.H * cfg_.I if mx else 0.0
+        ent = roofline_entry(b, f, t_ffn, peaks, fp8_flops=f8)
+        src = "HBM copy" if ent["bound"] == "hbm" else (
+            f"cuBLAS bf16 burst; routed MXFP8 x MXFP4 flops at {FP8_OVER_BF16:g} x that (nominal fp8/bf16 ratio)"
+            if mx else "cuBLAS bf16 burst")
+        ent.update(kernel="moe_ffn_mx (block-scaled gate/up + down)" if mx else "moe_ffn (gate/up + down)",
+                   traffic=ffn_traffic(cfg_, b),
                    traffic_unit="bytes per launch (ncu DRAM read+write, scaled from the "
                                 "small-case capture of the same kernel)",
-                   peak_source=f"{peaks['source']} ({'HBM copy' if ent['bound'] == 'hbm' else 'cuBLAS bf16 burst'})",
+                   peak_source=f"{peaks['source']} ({src})",
                    units_per_launch=f"{cfg_.T} tokens, {mm['routing']['experts_touched']} routed experts + shared")
+        if mx:
+            ent["time"] = "FFN stage events: scale atoms and MXFP8 x included"
         lb, lf = work["layer"]
-        t_roof = max(lb / (peaks["hbm_gbs"] * 1e9), lf / (peaks["bf16_tflops"] * 1e12))
+        tp = peaks["bf16_tflops"] * 1e12
+        t_roof = max(lb / (peaks["hbm_gbs"] * 1e9), (lf - f8) / tp + f8 / (FP8_OVER_BF16 * tp))
         step_s = statistics.mean(mm["per_step_ms"]) / 1e3
         return ent, round(t_roof / step_s, 4)
 
@@ -564,8 +591,7 @@ def run_native(args, rank, world, local):
             "e2e": {"value": round(tokens / e2e_s, 1), "unit": "tokens/s",
                     "h2d_bytes_per_step": m["e2e_h2d"], "d2h_bytes_per_step": m["e2e_d2h"]},
             "gpu_launches": m["launches"], "clocks": clocks}
-    if also is not None:
-        acfg, am = also
+    for acfg, am in also:
         a_s = reduce_max(am["device_ms_total"], device) / 1e3
         aent, afrac = roof(acfg, am)
         ap_s = reduce_max(am["plain_ms_total"], device) / 1e3
@@ -575,6 +601,7 @@ def run_native(args, rank, world, local):
                            "layer_roofline_frac": afrac,
                            "stage_ms": {k: round(v, 4) for k, v in am["stage_ms"].items()},
                            "routing": am["routing"],
+                           "dtype": DTYPES.get(acfg.wfmt, "bf16"),
                            "config": config_block(acfg, world)}
         line["gpu_launches"] += am["launches"]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
