@@ -272,14 +272,27 @@ DTYPES = {workloads.MOE_W_BF16: "bf16",
 
 
 def kernels_per_step(cfg) -> int:
-    """Library kernels launched by one moe_layer_forward: router 3 (logits,
+    """Library kernels launched by one moe_layer_forward: for decode batches
+    the fused front (routing and permutation) 1; otherwise router 3 (logits,
     certified top-k, exact re-derivation; the logits take 2 kernels, split and
-    tensor-core GEMM, above 32 tokens), permutation 1 when all T*K slots fit
-    one 2048-entry tile else 3, the fused expert FFN 1, combine 1; MXFP4 adds
+    tensor-core GEMM, above 32 tokens) and permutation 1 when all T*K slots
+    fit one 2048-entry tile else 3; then the expert FFN 1 and combine 1; MXFP4 adds
     2 (touched-expert list, dequantisation); the block-scaled MXFP4_A8 adds 3
     (touched-expert list, weight-scale atoms, MXFP8 x)."""
-    n = (3 if cfg.T <= 32 else 4) + (1 if cfg.T * cfg.K <= 2048 else 3) + 1 + 1
+    if fused_front(cfg):
+        n = 1 + 1 + 1  # fused decode front (routing + permutation), FFN, combine
+    else:
+        n = (3 if cfg.T <= 32 else 4) + (1 if cfg.T * cfg.K <= 2048 else 3) + 1 + 1
     return n + {workloads.MOE_W_MXFP4: 2, workloads.MOE_W_MXFP4_A8: 3}.get(cfg.wfmt, 0)
+
+
+def fused_front(cfg) -> bool:
+    """Whether the library routes and permutes a batch in one launch (its
+    decode_front_ok rule; SGL_MOE_FRONT=separate turns it off)."""
+    per = cfg.E // cfg.n_group
+    return (os.environ.get("SGL_MOE_FRONT") != "separate" and cfg.T <= 32 and cfg.E in (128, 256, 512)
+            and per in (32, 64) and cfg.n_group <= 16 and cfg.K + 1 <= 33
+            and cfg.topk_group * (cfg.K + 1) <= 64 and cfg.H <= 3072 and cfg.T * cfg.K <= 2048)
 
 
 def measure_gpu(cfg, steps, warmup, device, rank, clk, with_e2e=True):

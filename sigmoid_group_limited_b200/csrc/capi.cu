@@ -81,6 +81,7 @@ WsLayout ws_layout(const moe_cfg& c, int T) {
   L.h_s = take(static_cast<size_t>(T) * (c.I_shared > 0 ? c.I_shared : 0) * 2);
   L.y_slot = take((TK + T) * c.H * 4);
   L.wr_split = T > 32 ? take(static_cast<size_t>(3) * c.E * c.H * 2) : 0;
+  L.zp = T <= 32 ? take(static_cast<size_t>(8) * 32 * c.E * 4) : 0;
   if (mx) {
     // h_r holds the e4m3 h codes; the rest is scales
     L.max_touched = static_cast<int>(TK < static_cast<size_t>(c.E) ? TK : c.E);
@@ -135,6 +136,13 @@ bool cfg_ok(const moe_cfg* c) {
 bool T_ok(int32_t T) { return T >= 1 && T <= (1 << 20); }
 
 bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// SGL_MOE_FRONT=separate keeps the separate routing and permutation kernels
+// for decode batches (read at every call; for comparisons and tests).
+bool fused_front_disabled() {
+  const char* v = getenv("SGL_MOE_FRONT");
+  return v != nullptr && strcmp(v, "separate") == 0;
+}
 
 // sm_100 check, cached per device.
 moe_status device_ok() {
@@ -369,15 +377,26 @@ moe_status moe_layer_forward(const moe_cfg* cfg, int32_t T, const void* x, const
   cudaError_t e;
   rec(0);
   if (cudaMemsetAsync(err, 0, kCtrlBytes, s) != cudaSuccess) return MOE_ERR_CUDA;
-  if ((e = launch_router(*cfg, T, static_cast<const uint16_t*>(x), Wr, bias, at<float>(ws, L.z),
-                         idx, w, at<int32_t>(ws, L.unc), err + 1, err,
-                         T > 32 ? at<uint16_t>(ws, L.wr_split) : nullptr, s)) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  rec(1);
-  if ((e = launch_permute(*cfg, T, idx, at<int32_t>(ws, L.tile_hist), counts, offsets, perm,
-                          at<int32_t>(ws, L.inv_perm), err, L, gu, dn, at<int32_t>(ws, L.ready),
-                          nitems, s)) != cudaSuccess)
-    return MOE_ERR_CUDA;
+  if (decode_front_ok(*cfg, T) && !fused_front_disabled()) {
+    // routing, permutation and work lists in one launch (decode batches)
+    if ((e = launch_decode_front(*cfg, T, static_cast<const uint16_t*>(x), Wr, bias,
+                                 at<float>(ws, L.zp), at<float>(ws, L.z), idx, w,
+                                 at<int32_t>(ws, L.unc), err + 1, err + 2, err, counts, offsets,
+                                 perm, at<int32_t>(ws, L.inv_perm), L, gu, dn,
+                                 at<int32_t>(ws, L.ready), nitems, s)) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    rec(1);
+  } else {
+    if ((e = launch_router(*cfg, T, static_cast<const uint16_t*>(x), Wr, bias, at<float>(ws, L.z),
+                           idx, w, at<int32_t>(ws, L.unc), err + 1, err,
+                           T > 32 ? at<uint16_t>(ws, L.wr_split) : nullptr, s)) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    rec(1);
+    if ((e = launch_permute(*cfg, T, idx, at<int32_t>(ws, L.tile_hist), counts, offsets, perm,
+                            at<int32_t>(ws, L.inv_perm), err, L, gu, dn, at<int32_t>(ws, L.ready),
+                            nitems, s)) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
   rec(2);
   if ((e = run_ffn(cfg, T, static_cast<const uint16_t*>(x), perm, offsets, w, W, y_slot, ws, L,
                    s)) != cudaSuccess)

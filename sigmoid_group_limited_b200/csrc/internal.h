@@ -62,7 +62,8 @@ __host__ __device__ inline int cdiv_dev(int a, int b) { return (a + b - 1) / b; 
 
 // Per-call control block at the start of the workspace, zeroed by every
 // entry point that routes: [0] device error word, [1] count of tokens whose
-// routing is re-derived exactly.
+// routing is re-derived exactly, [2] grid barrier counter of the fused
+// decode front.
 constexpr int kCtrlBytes = 256;
 
 struct WsLayout {
@@ -77,6 +78,7 @@ struct WsLayout {
   size_t x_q, x_sf, h_sf, sf_g, sf_u, sf_d;
   int max_row_tiles;
   size_t wr_split;  // router matrix as three bf16 terms (batches above 32 tokens)
+  size_t zp;        // partial router logits [8][32][E] of the fused decode front (T <= 32)
   int max_touched;
   int n_ptiles, bn, max_items_gu, max_items_dn;
 };
@@ -91,6 +93,19 @@ WsLayout ws_layout(const moe_cfg& c, int T);
 cudaError_t launch_router(const moe_cfg& c, int T, const uint16_t* x, const float* Wr,
                           const float* bias, float* z, int32_t* idx, float* w, int32_t* unc,
                           int32_t* unc_n, int32_t* err, uint16_t* wr_split, cudaStream_t s);
+
+// The decode front in one cooperative launch (T <= 32, see front.cu):
+// routing (logits via zp, certified selection, exact re-derivation of close
+// calls), then the permutation and the FFN work lists. bar: a zeroed grid
+// barrier counter. decode_front_ok: whether a configuration qualifies.
+bool decode_front_ok(const moe_cfg& c, int T);
+cudaError_t launch_decode_front(const moe_cfg& c, int T, const uint16_t* x, const float* Wr,
+                                const float* bias, float* zp, float* z, int32_t* idx, float* w,
+                                int32_t* unc, int32_t* unc_n, int32_t* bar, int32_t* err,
+                                int32_t* counts, int32_t* offsets, int32_t* perm,
+                                int32_t* inv_perm, const WsLayout& L, int32_t* gu_start,
+                                int32_t* dn_start, int32_t* ready, int32_t* nitems,
+                                cudaStream_t s);
 
 cudaError_t launch_permute(const moe_cfg& c, int T, const int32_t* idx, int32_t* tile_hist,
                            int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv_perm,

@@ -18,12 +18,12 @@
 #include <mutex>
 
 #include "internal.h"
+#include "permute_dev.cuh"
 #include "ptx.cuh"
 
 namespace sgl {
 namespace {
 
-constexpr int kMaxE = 1024;
 constexpr int kScanSmemInts = 48 * 1024;  // tile counts perm_scan stages in shared memory (192 KB)
 constexpr int kScatterWarps = 8;
 
@@ -49,100 +49,6 @@ __global__ void __launch_bounds__(256) perm_hist(int TK, int E, int n_ptiles,
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x)
     tile_cnt[static_cast<size_t>(e) * n_ptiles + blockIdx.x] = hist[e];
-}
-
-// Block-wide exclusive scan of up to 2 values per thread (1024 threads).
-// Returns the exclusive prefix of this thread's first value; *total gets the sum.
-__device__ int block_exscan2(int v0, int v1, int* scratch /*32*/, int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int v = v0 + v1;
-  int incl = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  if (lane == 31) scratch[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    const int nw = blockDim.x >> 5;
-    int s = lane < nw ? scratch[lane] : 0;
-    int si = s;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, si, o);
-      if (lane >= o) si += y;
-    }
-    if (lane < nw) scratch[lane] = si - s;
-    if (lane == 31) scratch[32] = si;
-  }
-  __syncthreads();
-  const int ex = scratch[warp] + incl - v;
-  *total = scratch[32];
-  __syncthreads();
-  return ex;
-}
-
-struct SchedArgs {
-  int T, K, E, H, I, Is, has_shared, bn;
-  int gu_ft, dn_ft;   // output features per gate/up item and per down item
-  int32_t* gu_start;  // [E+2] first gate/up work item of slot e (e == E: shared expert)
-  int32_t* dn_start;  // [E+2] first down work item of slot e
-  int32_t* ready;     // nullable: [gate/up items] zeroed for the fused FFN's row-tile counters
-  int32_t* nitems;    // [2] totals
-};
-
-// Work lists of the two grouped GEMMs, as prefix sums of per-slot item counts.
-// Slot e (e == E: the shared expert, whose rows are the T tokens) has
-// ceil(rows/bn) row tiles times its output tiles; the GEMM kernels decode an
-// item index back to (slot, row tile, output tile) with a binary search over
-// these starts. Needs blockDim.x == 1024 and counts in shared memory.
-__device__ void build_schedule(const SchedArgs& a, const int* cnt, int* scratch) {
-  const int nslots = a.E + (a.has_shared ? 1 : 0);
-  const int nt_gu_r = cdiv_dev(a.I, a.gu_ft), nt_gu_s = cdiv_dev(a.Is, a.gu_ft);
-  const int nt_dn = cdiv_dev(a.H, a.dn_ft);
-  int ngu[2] = {0, 0}, ndn[2] = {0, 0};
-#pragma unroll
-  for (int q = 0; q < 2; ++q) {
-    const int e = 2 * threadIdx.x + q;
-    if (e < nslots) {
-      const bool sh = e == a.E;
-      const int rows = sh ? a.T : cnt[e];
-      const int nm = (rows + a.bn - 1) / a.bn;
-      ngu[q] = nm * (sh ? nt_gu_s : nt_gu_r);
-      ndn[q] = nm * nt_dn;
-    }
-  }
-  int tot_gu, tot_dn;
-  const int base_gu = block_exscan2(ngu[0], ngu[1], scratch, &tot_gu);
-  const int base_dn = block_exscan2(ndn[0], ndn[1], scratch, &tot_dn);
-#pragma unroll
-  for (int q = 0; q < 2; ++q) {
-    const int e = 2 * threadIdx.x + q;
-    if (e <= a.E + 1) {
-      const bool real = e < nslots;
-      a.gu_start[e] = real ? base_gu + (q ? ngu[0] : 0) : tot_gu;
-      a.dn_start[e] = real ? base_dn + (q ? ndn[0] : 0) : tot_dn;
-    }
-  }
-  if (a.ready) {
-    // one counter per (slot, row tile): the slot's first nm gate/up item indices
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      const int e = 2 * threadIdx.x + q;
-      if (e < nslots) {
-        const int ntg = e == a.E ? nt_gu_s : nt_gu_r;
-        const int nm = ntg > 0 ? (q ? ngu[1] : ngu[0]) / ntg : 0;
-        const int b0 = base_gu + (q ? ngu[0] : 0);
-        for (int m = 0; m < nm; ++m) a.ready[b0 + m] = 0;
-      }
-    }
-  }
-  if (threadIdx.x == 0) {
-    a.nitems[0] = tot_gu;
-    a.nitems[1] = tot_dn;
-    a.nitems[2] = 0;  // the fused FFN's item counter
-  }
 }
 
 __global__ void __launch_bounds__(1024) perm_scan(int E, int n_ptiles,
@@ -282,10 +188,7 @@ __global__ void __launch_bounds__(kScatterWarps * 32) perm_scatter(
   }
 }
 
-// The whole permutation in one CTA when all T*K entries fit one tile (decode
-// batches): per-warp histograms of contiguous chunks, per-expert totals and
-// their exclusive scan, per-warp bases, stable positions, and optionally the
-// GEMM work lists, with no round trip through global memory in between.
+// The permutation in one CTA of 1024 threads (decode batches).
 __global__ void __launch_bounds__(1024) perm_single(int TK, int E, const int32_t* __restrict__ idx,
                                                     int32_t* __restrict__ counts,
                                                     int32_t* __restrict__ offsets,
@@ -296,102 +199,7 @@ __global__ void __launch_bounds__(1024) perm_single(int TK, int E, const int32_t
   pdl_trigger();
   pdl_wait();  // inputs come from earlier kernels on the stream
   extern __shared__ int whist[];  // [32 warps][E]
-  __shared__ int cnt[kMaxE + 1];
-  __shared__ int off[kMaxE + 1];
-  __shared__ int scratch[33];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  for (int i = tid; i < 32 * E; i += blockDim.x) whist[i] = 0;
-  __syncthreads();
-  const int chunk = ((cdiv_dev(TK, 32) + 31) / 32) * 32;
-  const int c0 = warp * chunk, c1 = min(c0 + chunk, TK);
-  const unsigned lt = (1u << lane) - 1u;
-  int* wh = whist + warp * E;
-  for (int r = c0; r < c1; r += 32) {
-    const int i = r + lane;
-    int e = -1;
-    if (i < c1) {
-      e = idx[i];
-      if (e < 0 || e >= E) {
-        atomicExch(err, MOE_DEVERR_EXPERT_ID);
-        e = -1;
-      }
-    }
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    if (e >= 0 && (peers & lt) == 0) wh[e] += __popc(peers);
-  }
-  __syncthreads();
-  for (int e = tid; e < E; e += blockDim.x) {
-    int tot = 0;
-    for (int w = 0; w < 32; ++w) tot += whist[w * E + e];
-    cnt[e] = tot;
-  }
-  __syncthreads();
-  int total;
-  const int e0 = 2 * tid;
-  const int v0 = e0 < E ? cnt[e0] : 0, v1 = e0 + 1 < E ? cnt[e0 + 1] : 0;
-  const int ex = block_exscan2(v0, v1, scratch, &total);
-  if (e0 < E) off[e0] = ex;
-  if (e0 + 1 < E) off[e0 + 1] = ex + v0;
-  if (tid == 0) off[E] = total;
-  __syncthreads();
-  for (int e = tid; e <= E; e += blockDim.x) {
-    offsets[e] = off[e];
-    if (e < E) counts[e] = cnt[e];
-  }
-  for (int e = tid; e < E; e += blockDim.x) {
-    int run = off[e];
-    for (int w = 0; w < 32; ++w) {
-      const int v = whist[w * E + e];
-      whist[w * E + e] = run;
-      run += v;
-    }
-  }
-  __syncthreads();
-  for (int r = c0; r < c1; r += 32) {
-    const int i = r + lane;
-    int e = -1;
-    if (i < c1) {
-      e = idx[i];
-      if (e < 0 || e >= E) e = -1;
-    }
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    int pos = -1;
-    if (e >= 0) pos = wh[e] + __popc(peers & lt);
-    __syncwarp();
-    if (e >= 0 && (peers & lt) == 0) wh[e] += __popc(peers);
-    __syncwarp();
-    if (i < c1) {
-      if (e >= 0 && (pos < 0 || pos >= TK)) {
-        atomicExch(err, MOE_DEVERR_SCHEDULE);
-        e = -1;
-        pos = -1;
-      }
-      if (e >= 0) perm[pos] = i;
-      if (inv_perm) inv_perm[i] = pos;
-    }
-  }
-  if (build) build_schedule(sa, cnt, scratch);
-}
-
-SchedArgs make_sched(const moe_cfg& c, int T, const WsLayout& L, int32_t* gu_start,
-                     int32_t* dn_start, int32_t* ready, int32_t* nitems) {
-  SchedArgs a;
-  a.T = T;
-  a.K = c.K;
-  a.E = c.E;
-  a.H = c.H;
-  a.I = c.I;
-  a.Is = c.I_shared;
-  a.has_shared = c.I_shared > 0;
-  a.bn = L.bn;
-  const bool mx = c.wfmt == MOE_W_MXFP4_A8;
-  a.gu_ft = mx ? kMxGuTile : kTileN;
-  a.dn_ft = mx ? kMxDnTile : kDownTile;
-  a.gu_start = gu_start;
-  a.dn_start = dn_start;
-  a.ready = ready;
-  a.nitems = nitems;
-  return a;
+  perm_block(TK, E, idx, counts, offsets, perm, inv_perm, err, sa, build, whist);
 }
 
 }  // namespace

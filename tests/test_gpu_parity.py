@@ -377,3 +377,29 @@ def test_block_scaled_full_size_sampled():
     cfg = workloads.CONFIGS["mxfp4_a8"]
     d = workloads.generate(cfg, DEV)
     _full_check(cfg, d, tokens=_sample(cfg.T, 12, seed=9))
+
+
+# ------------------------------------------------------------------ fused decode front
+
+@pytest.mark.parametrize("T,E", [(1, 512), (7, 512), (32, 512), (32, 256), (16, 128), (32, 128)])
+def test_fused_decode_front_matches_separate_kernels(T, E, monkeypatch):
+    """Decode batches route and permute in one cooperative launch. Its fp32
+    logits add the hidden dimension in another order than the separate
+    kernels, so scores may differ in the last bit; the certified decisions
+    (experts, counts, permutation) are identical, the weights agree to 1e-6,
+    and both outputs meet the bar against the oracle."""
+    cfg = workloads.CONFIGS["decode"].with_(E=E)
+    d = workloads.generate(cfg, DEV, T=T)
+    fused = run_layer(cfg, d)
+    monkeypatch.setenv("SGL_MOE_FRONT", "separate")
+    sep = run_layer(cfg, d)
+    for k in ("idx", "counts"):
+        assert torch.equal(fused[k], sep[k]), k
+    assert torch.allclose(fused["w"], sep["w"], rtol=1e-6, atol=0)
+    tok = list(range(min(T, 6)))
+    ref = _oracle_layer(cfg, d, tokens=tok)
+    near = check_routing(ref, fused["idx"].cpu().numpy(), fused["w"].cpu().numpy())
+    keep = ~np.isin(ref["tokens"], near)
+    for g in (fused, sep):
+        check_y(bits(g["y"])[ref["tokens"][keep]], ref["y_f32"][keep], ref["y"][keep], tol=_tol(cfg))
+
