@@ -236,8 +236,8 @@ def roofline_entry(bytes_, flops, seconds, peaks, sustained=False, fp8_flops=0.0
 # Weight bytes dominate and scale with the experts touched, so the ratio
 # scales the counters to a full launch. Valid only for the ffn.cu they were
 # taken on: any other source reports traffic null.
-FFN_TRAFFIC_SOURCE_SHA256 = "48e27a9659764bd394e28d2e553ed03ee0bf6861e6ea5ae2eaf0e108fcd84afb"
-FFN_TRAFFIC_RATIO = {16: (424.91 + 4.26) / 424.82, 128: (778.64 + 48.90) / 760.2}
+FFN_TRAFFIC_SOURCE_SHA256 = "d33a6269069f76958d4a7790d645868ac93165e48d69db81ea7357839416ce75"
+FFN_TRAFFIC_RATIO = {16: (424.91 + 4.68) / 424.82, 128: (781.17 + 50.85) / 760.2}
 
 
 def ffn_tile_n(cfg) -> int:

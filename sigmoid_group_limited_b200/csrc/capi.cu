@@ -48,8 +48,14 @@ WsLayout ws_layout(const moe_cfg& c, int T) {
   const size_t TK = static_cast<size_t>(T) * c.K;
   L.n_ptiles = cdiv(static_cast<long long>(TK), kPermTile);
   const bool mx = c.wfmt == MOE_W_MXFP4_A8;
-  L.bn = mx ? kMxTileN : choose_bn(T, c.K, c.E);
-  const int gu_ft = mx ? kMxGuTile : kTileN, dn_ft = mx ? kMxDnTile : kDownTile;
+  if (mx) {
+    L.bn = kMxTileN;
+    L.ffn = kFfnMx;
+  } else {
+    L.ffn = choose_ffn(T, c.K, c.E, &L.bn);
+  }
+  ffn_tiles(L.ffn, &L.gu_ft, &L.dn_ft);
+  const int gu_ft = L.gu_ft, dn_ft = L.dn_ft;
   const int rt_gu = cdiv(c.I, gu_ft), st_gu = cdiv(c.I_shared, gu_ft), nt_dn = cdiv(c.H, dn_ft);
   const long long mt_r = cdiv(static_cast<long long>(TK), L.bn) +
                          (static_cast<long long>(TK) < c.E ? static_cast<long long>(TK) : c.E);
@@ -225,6 +231,7 @@ cudaError_t run_ffn(const moe_cfg* cfg, int T, const uint16_t* x, const int32_t*
   a.nitems = at<int32_t>(ws, L.nitems);
   a.err = at<int32_t>(ws, L.err);
   a.bn = L.bn;
+  a.ffn = L.ffn;
   a.max_items_gu = L.max_items_gu;
   a.max_items_dn = L.max_items_dn;
   if (cfg->wfmt == MOE_W_MXFP4_A8) {

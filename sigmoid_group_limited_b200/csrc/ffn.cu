@@ -34,7 +34,7 @@
 //   2..9   epilogue: two warps per TMEM lane quarter (warp % 4), alternate
 //          column chunks
 //   10..13 token gatherers: cp.async of the routed x rows into the swizzled
-//          B tile of gate/up stages
+//          B tile of gate/up stages, completion tracked by the stage's barrier
 //   14     scheduler (lane 0): claims the next item while the current one is
 //          still streaming, waits for its inputs, and queues it for the others
 // Pipelines: STAGES shared-memory stages (full / empty mbarriers), two TMEM
@@ -119,7 +119,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
   pdl_trigger();
   if (tid == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&full[s], 1 + kGatherWarps);  // weight TMA + one arrival per gatherer warp
+      mbar_init(&full[s], 1 + 32 * kGatherWarps);  // weight TMA + one arrival per gatherer thread
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -329,40 +329,19 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
     // ------------------------------------------------------------ token gatherers
     // Gate/up items: thread g copies 16-byte chunk (g % 8) of rows g/8,
     // g/8 + 16, ... of the stage's BN x 64 token tile straight into the
-    // 128-byte-swizzled layout (chunk c of row r lands at c ^ (r % 8)). A
-    // stage's copies retire kLag stages later: wait for the group, make it
-    // visible to the tensor cores (proxy fence), then one arrival per warp on
-    // the stage's full barrier. Down items copy nothing, but keep the stage
-    // sequence and the arrivals (an empty copy group completes at once).
+    // 128-byte-swizzled layout (chunk c of row r lands at c ^ (r % 8)). Each
+    // thread then hands the stage's full barrier an arrival that fires when
+    // its copies have landed (cp.async.mbarrier.arrive.noinc), so gatherers
+    // run as far ahead as the free stages allow. Down items copy nothing but
+    // keep the stage sequence and the arrivals.
     constexpr int kRowsPerThread = BN / 16;
-    // stages a gatherer keeps in flight before retiring the oldest: two, but
-    // one when the ring has only three stages (else the MMA would never run
-    // ahead of the gatherers)
-    constexpr int kLag = C::STAGES >= 4 ? 2 : 1;
     const int g = tid - kGatherWarp0 * 32;
     const int chunk = g & 7, rbase = g >> 3;
     const uint64_t pol_x = policy_evict_last();
     int stage = 0;
     uint32_t phase = 0;
-    int pend[2] = {-1, -1};  // stages issued and not yet retired, oldest first (kLag used)
     bool live = true;
     for (int n = 0; live; ++n) {
-      // The scheduler may hold the next item back until gate/up tiles that
-      // this CTA is still finishing are published, and the MMA cannot finish
-      // them before their stages retire: if the next item is not queued yet,
-      // retire the pending stages before waiting for it.
-      const bool queued =
-          __shfl_sync(0xffffffffu, lane == 0 ? (mbar_try_wait(&qfull[n % kQueue], (n / kQueue) & 1) ? 1 : 0) : 0, 0) != 0;
-      if (!queued && (pend[0] >= 0 || pend[1] >= 0)) {
-        cp_async_wait<0>();
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          if (pend[0] >= 0) mbar_arrive(&full[pend[0]]);
-          if (pend[1] >= 0) mbar_arrive(&full[pend[1]]);
-        }
-        pend[0] = pend[1] = -1;
-      }
       int item;
       if (!next_item(n, item, true)) break;
       bool gu;
@@ -393,32 +372,14 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
             if (r < nb) cp_async16(sB + r * 128 + ((chunk ^ (r & 7)) << 4), src[i] + kb * 64, pol_x);
           }
         }
-        cp_async_commit();
-        if (pend[0] >= 0) {
-          cp_async_wait<kLag>();      // this lane's copies for the oldest pending stage landed
-          fence_proxy_async_smem();   // ... and are visible to the tensor cores
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&full[pend[0]]);
-        }
-        if (kLag == 2) {
-          pend[0] = pend[1];
-          pend[1] = stage;
-        } else {
-          pend[0] = stage;
-        }
+        cp_async_mbar_arrive_noinc(&full[stage]);
         if (++stage == C::STAGES) {
           stage = 0;
           phase ^= 1;
         }
       }
     }
-    cp_async_wait<0>();  // nothing may still be landing in shared memory at exit
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (live && lane == 0) {
-      if (pend[0] >= 0) mbar_arrive(&full[pend[0]]);
-      if (pend[1] >= 0) mbar_arrive(&full[pend[1]]);
-    }
+    cp_async_wait_all();  // nothing may still be landing in shared memory at exit
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;            // TMEM lane quarter of this warp
@@ -604,12 +565,13 @@ cudaError_t launch_bn(const GemmArgs& a, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_ffn(const GemmArgs& a, cudaStream_t s) {
+  if (a.ffn == kFfnPair) return a.bn == kPairTileN ? launch_ffn_pair(a, s) : cudaErrorInvalidValue;
+  if (a.ffn != kFfnNarrow) return cudaErrorInvalidValue;
   switch (a.bn) {
     case 16: return launch_bn<16>(a, s);
     case 32: return launch_bn<32>(a, s);
     case 64: return launch_bn<64>(a, s);
     case 128: return launch_bn<128>(a, s);
-    case kPairTileN: return launch_ffn_pair(a, s);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(kXThreads, 1)
   pdl_trigger();
   if (tid == 0) {
     for (int s = 0; s < kXStages; ++s) {
-      mbar_init(&full[s], 1 + kXGatherWarps);  // producer's expect_tx + one per gatherer warp
+      mbar_init(&full[s], 1 + 32 * kXGatherWarps);  // producer's expect_tx + one per gatherer thread
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -389,30 +389,17 @@ __global__ void __launch_bounds__(kXThreads, 1)
     // g/8 + 16, ... of the stage's token tile (128 bytes per row: 128 e4m3
     // codes, or 64 bf16 for the shared expert) into the 128-byte-swizzled
     // layout, and for routed items the four scale bytes of row g into the B
-    // scale atom. Retirement as in ffn.cu: two stages late, proxy fence, one
-    // arrival per warp; down items keep the stage sequence with empty groups.
+    // scale atom. Each thread then hands the stage's full barrier an arrival
+    // that fires when its copies have landed (as in ffn.cu); down items keep
+    // the stage sequence and the arrivals.
     constexpr int kRowsPerThread = kMxTileN / 16;
-    constexpr int kLag = 2;
     const int g = tid - kXGatherWarp0 * 32;
     const int chunk = g & 7, rbase = g >> 3;
     const uint64_t pol_x = policy_evict_last();
     int stage = 0;
     uint32_t phase = 0;
-    int pend[2] = {-1, -1};
     bool live = true;
     for (int n = 0; live; ++n) {
-      const bool queued =
-          __shfl_sync(0xffffffffu, lane == 0 ? (mbar_try_wait(&qfull[n % kXQueue], (n / kXQueue) & 1) ? 1 : 0) : 0, 0) != 0;
-      if (!queued && (pend[0] >= 0 || pend[1] >= 0)) {
-        cp_async_wait<0>();
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          if (pend[0] >= 0) mbar_arrive(&full[pend[0]]);
-          if (pend[1] >= 0) mbar_arrive(&full[pend[1]]);
-        }
-        pend[0] = pend[1] = -1;
-      }
       int item;
       if (!next_item(n, item, true)) break;
       bool gu;
@@ -452,28 +439,14 @@ __global__ void __launch_bounds__(kXThreads, 1)
           }
           if (sf_src) cp_async4(smem + stage * kXStage + kXSfOff + 1024 + atom_off(g, 0), sf_src + kb * 4);
         }
-        cp_async_commit();
-        if (pend[0] >= 0) {
-          cp_async_wait<kLag>();
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&full[pend[0]]);
-        }
-        pend[0] = pend[1];
-        pend[1] = stage;
+        cp_async_mbar_arrive_noinc(&full[stage]);
         if (++stage == kXStages) {
           stage = 0;
           phase ^= 1;
         }
       }
     }
-    cp_async_wait<0>();
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (live && lane == 0) {
-      if (pend[0] >= 0) mbar_arrive(&full[pend[0]]);
-      if (pend[1] >= 0) mbar_arrive(&full[pend[1]]);
-    }
+    cp_async_wait_all();  // nothing may still be landing in shared memory at exit
   } else {
     // ------------------------------------------------------------ epilogue
     const int qd = warp & 3;            // TMEM lane quarter

@@ -39,22 +39,38 @@ constexpr int kMxGuTile = 128;
 constexpr int kMxDnTile = 256;
 constexpr int kMaxExpertsCfg = 1024;  // largest E a configuration may have
 
+// Which expert-FFN kernel a batch runs on.
+enum FfnKind {
+  kFfnNarrow = 0,  // moe_ffn<BN>: BN <= 128 tokens, 128 gate + 128 up features per item
+  kFfnPair = 1,    // moe_ffn_pair: a CTA pair per item (tcgen05 cta_group::2)
+  kFfnMx = 2,      // moe_ffn_mx: block-scaled MXFP8 x MXFP4
+};
+
 // The expert-FFN kernel for large batches: one CTA per item (default), or a
-// CTA pair per item (tcgen05 cta_group::2, token tile kPairTileN) when the
-// environment variable SGL_MOE_FFN is "pair". Read at every call, so the
-// workspace layout and the launch always agree.
-inline bool ffn_pair_requested() {
+// CTA pair per item when the environment variable SGL_MOE_FFN is "pair".
+// Read at every call, so the workspace layout and the launch always agree.
+inline bool ffn_env_is(const char* name) {
   const char* v = getenv("SGL_MOE_FFN");
-  return v != nullptr && strcmp(v, "pair") == 0;
+  return v != nullptr && strcmp(v, name) == 0;
 }
 
-// Token-tile width (MMA N) for a batch: small for decode, wide for prefill.
-inline int choose_bn(int T, int K, int E) {
+// Kernel and token-tile width (MMA N) for a batch: narrow tiles for decode,
+// wide ones for prefill. T*K/E is the mean load over all experts.
+inline FfnKind choose_ffn(int T, int K, int E, int* bn) {
   const double avg = static_cast<double>(T) * K / E;
-  if (avg <= 12.0) return 16;
-  if (avg <= 24.0) return 32;
-  if (avg <= 48.0) return 64;
-  return ffn_pair_requested() ? kPairTileN : 128;
+  if (avg <= 12.0) return *bn = 16, kFfnNarrow;
+  if (avg <= 24.0) return *bn = 32, kFfnNarrow;
+  if (avg <= 48.0) return *bn = 64, kFfnNarrow;
+  if (ffn_env_is("pair")) return *bn = kPairTileN, kFfnPair;
+  return *bn = 128, kFfnNarrow;
+}
+
+// Output features per gate/up item and per down item of each kernel.
+inline void ffn_tiles(int kind, int* gu_ft, int* dn_ft) {
+  switch (kind) {
+    case kFfnMx: *gu_ft = kMxGuTile, *dn_ft = kMxDnTile; break;
+    default: *gu_ft = kTileN, *dn_ft = kDownTile; break;
+  }
 }
 
 inline int cdiv(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
@@ -81,6 +97,7 @@ struct WsLayout {
   size_t zp;        // partial router logits [8][32][E] of the fused decode front (T <= 32)
   int max_touched;
   int n_ptiles, bn, max_items_gu, max_items_dn;
+  int ffn, gu_ft, dn_ft;  // FfnKind and its output features per gate/up and down item
 };
 
 WsLayout ws_layout(const moe_cfg& c, int T);
@@ -147,6 +164,7 @@ struct GemmArgs {
   const int32_t* nitems;
   int32_t* err;
   int bn;
+  int ffn;  // FfnKind
   int max_items_gu;
   int max_items_dn;
   // MOE_W_MXFP4_A8: the MXFP4 codes are a.Wg/Wu/Wd (expert-major), read in place

@@ -211,9 +211,8 @@ SchedArgs make_sched(const moe_cfg& c, int T, const WsLayout& L, int32_t* gu_sta
   a.Is = c.I_shared;
   a.has_shared = c.I_shared > 0;
   a.bn = L.bn;
-  const bool mx = c.wfmt == MOE_W_MXFP4_A8;
-  a.gu_ft = mx ? kMxGuTile : kTileN;
-  a.dn_ft = mx ? kMxDnTile : kDownTile;
+  a.gu_ft = L.gu_ft;
+  a.dn_ft = L.dn_ft;
   a.gu_start = gu_start;
   a.dn_start = dn_start;
   a.ready = ready;

@@ -132,6 +132,14 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
+// Waits for every cp.async this thread issued, committed to a group or not.
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// One arrival on `bar` once every cp.async this thread issued so far has
+// landed; the arrival counts against the barrier's expected count (.noinc),
+// so the thread never blocks on its own copies.
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
 
 // Orders this thread's earlier generic-proxy shared-memory accesses before
 // later async-proxy (TMA / bulk copy / tensor core) accesses.
