@@ -390,7 +390,7 @@ moe_status moe_layer_forward(const moe_cfg* cfg, int32_t T, const void* x, const
                                  at<float>(ws, L.zp), at<float>(ws, L.z), idx, w,
                                  at<int32_t>(ws, L.unc), err + 1, err + 2, err, counts, offsets,
                                  perm, at<int32_t>(ws, L.inv_perm), L, gu, dn,
-                                 at<int32_t>(ws, L.ready), nitems, s)) != cudaSuccess)
+                                 at<int32_t>(ws, L.ready), nitems, W, s)) != cudaSuccess)
       return MOE_ERR_CUDA;
     rec(1);
   } else {

@@ -22,6 +22,11 @@
 //      K slots at offsets[e] + (the number of earlier flat slots with the
 //      same expert), the stable counting-sort position, and CTA 0 writes the
 //      offsets and the FFN work lists (whose ready counters phase 1 zeroed).
+// L2 prefetch for the expert FFN that follows: HBM is nearly idle while the
+// front runs, so phase 1 asks L2 for the shared expert's weights (known
+// before routing), and after the second barrier the CTAs without a token ask
+// for the gate and up weights of the lowest-numbered touched experts (the
+// FFN's first work items), up to a byte budget.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -61,7 +66,27 @@ struct FrontParams {
   int32_t* inv_perm;
   SchedArgs sa;
   int n_ready;        // ready counters to zero (the FFN's largest gate/up item count)
+  // L2 prefetch (null / 0: none): the shared expert's three matrices, and the
+  // routed gate and up weights (expert e at e * pf_expert_bytes) of at most
+  // pf_experts touched experts
+  const uint8_t* pf_shared[3];
+  uint32_t pf_shared_bytes;
+  const uint8_t* pf_g;
+  const uint8_t* pf_u;
+  uint32_t pf_expert_bytes;
+  int pf_experts;
 };
+
+constexpr uint32_t kPrefetchPiece = 16384;  // bytes per bulk L2 prefetch
+
+// Prefetch pieces [first, n) step `stride` of [base, base + bytes) into L2.
+__device__ __forceinline__ void prefetch_range(const uint8_t* base, uint32_t bytes, int first, int stride) {
+  const int n = static_cast<int>((bytes + kPrefetchPiece - 1) / kPrefetchPiece);
+  for (int c = first; c < n; c += stride) {
+    const uint32_t at = static_cast<uint32_t>(c) * kPrefetchPiece;
+    prefetch_l2_bulk(base + at, min(kPrefetchPiece, bytes - at));
+  }
+}
 
 __device__ __forceinline__ int ld_acquire_gpu(const int32_t* a) {
   int v;
@@ -127,6 +152,9 @@ __global__ void __launch_bounds__(kFrontThreads, 1) decode_front(const __grid_co
         *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
     }
     cp_async_commit();
+    // the shared expert's weights: piece c of each matrix goes to CTA c % grid
+    if (tid < 3 && p.pf_shared[tid])
+      prefetch_range(p.pf_shared[tid], p.pf_shared_bytes, blockIdx.x, gridDim.x);
     cp_async_wait<0>();
     __syncthreads();
     // warp w: experts 4 (w % 8) .. +3 over K half w / 8; lane = token
@@ -254,6 +282,35 @@ __global__ void __launch_bounds__(kFrontThreads, 1) decode_front(const __grid_co
       sa.ready = nullptr;  // zeroed in phase 1
       build_schedule(sa, cnt, scratch);
     }
+  } else if (p.pf_experts > 0) {
+    // gate and up weights of the first touched experts, in the FFN's item
+    // order (increasing expert id); CTA T + i of the idle ones takes piece c
+    // when c % n_idle == i
+    __shared__ int pf_list[kSelMaxCand];
+    __shared__ int pf_n;
+    if (warp == 0) {
+      int n = 0;
+      for (int e0 = 0; e0 < E && n < p.pf_experts; e0 += 32) {
+        const int e = e0 + lane;
+        unsigned m = __ballot_sync(0xffffffffu, e < E && ld_acquire_gpu(p.counts + e) > 0);
+        while (m && n < p.pf_experts) {
+          const int b = __ffs(m) - 1;
+          m &= m - 1;
+          if (lane == 0) pf_list[n] = e0 + b;
+          ++n;
+        }
+      }
+      if (lane == 0) pf_n = n;
+    }
+    __syncthreads();
+    const int n_idle = static_cast<int>(gridDim.x) - T, i = static_cast<int>(blockIdx.x) - T;
+    const int per = static_cast<int>((p.pf_expert_bytes + kPrefetchPiece - 1) / kPrefetchPiece);
+    for (int c = i + n_idle * tid; c < 2 * pf_n * per; c += n_idle * static_cast<int>(blockDim.x)) {
+      const int q = c / per, piece = c - q * per;
+      const uint8_t* base = (q & 1 ? p.pf_u : p.pf_g) + static_cast<size_t>(pf_list[q >> 1]) * p.pf_expert_bytes;
+      const uint32_t at = static_cast<uint32_t>(piece) * kPrefetchPiece;
+      prefetch_l2_bulk(base + at, min(kPrefetchPiece, p.pf_expert_bytes - at));
+    }
   }
 }
 
@@ -272,7 +329,7 @@ cudaError_t launch_decode_front(const moe_cfg& c, int T, const uint16_t* x, cons
                                 int32_t* counts, int32_t* offsets, int32_t* perm,
                                 int32_t* inv_perm, const WsLayout& L, int32_t* gu_start,
                                 int32_t* dn_start, int32_t* ready, int32_t* nitems,
-                                cudaStream_t s) {
+                                const moe_weights* W, cudaStream_t s) {
   if (!decode_front_ok(c, T)) return cudaErrorInvalidValue;
   FrontParams p;
   memset(&p, 0, sizeof(p));
@@ -301,6 +358,26 @@ cudaError_t launch_decode_front(const moe_cfg& c, int T, const uint16_t* x, cons
   p.inv_perm = inv_perm;
   p.sa = make_sched(c, T, L, gu_start, dn_start, ready, nitems);
   p.n_ready = L.max_items_gu;
+  const uint64_t budget = front_prefetch_budget();
+  if (W && budget > 0) {
+    // bf16 matrices whose sizes (multiples of 64 x 64 elements) keep every
+    // piece 16-byte aligned
+    const uint64_t shared_bytes = static_cast<uint64_t>(c.I_shared) * c.H * 2;
+    if (c.I_shared > 0 && W->Wg_s && W->Wu_s && W->Wd_s && shared_bytes < (1ull << 31)) {
+      p.pf_shared[0] = static_cast<const uint8_t*>(W->Wg_s);
+      p.pf_shared[1] = static_cast<const uint8_t*>(W->Wu_s);
+      p.pf_shared[2] = static_cast<const uint8_t*>(W->Wd_s);
+      p.pf_shared_bytes = static_cast<uint32_t>(shared_bytes);
+    }
+    const uint64_t expert_bytes = static_cast<uint64_t>(c.I) * c.H * 2;
+    if (c.wfmt == MOE_W_BF16 && W->Wg && W->Wu && expert_bytes < (1ull << 31)) {
+      p.pf_g = static_cast<const uint8_t*>(W->Wg);
+      p.pf_u = static_cast<const uint8_t*>(W->Wu);
+      p.pf_expert_bytes = static_cast<uint32_t>(expert_bytes);
+      const uint64_t n = budget / (2 * expert_bytes);
+      p.pf_experts = static_cast<int>(n < kSelMaxCand ? n : kSelMaxCand);
+    }
+  }
   const int per = c.E / c.n_group;
   void (*kern)(FrontParams) = nullptr;
   const int nv = c.E / 32;

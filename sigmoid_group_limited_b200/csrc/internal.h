@@ -122,7 +122,17 @@ cudaError_t launch_decode_front(const moe_cfg& c, int T, const uint16_t* x, cons
                                 int32_t* counts, int32_t* offsets, int32_t* perm,
                                 int32_t* inv_perm, const WsLayout& L, int32_t* gu_start,
                                 int32_t* dn_start, int32_t* ready, int32_t* nitems,
-                                cudaStream_t s);
+                                const moe_weights* W, cudaStream_t s);
+// Bytes of routed gate / up weights the decode front asks L2 for (about what
+// HBM delivers between the routing decision and the FFN's first loads): the
+// environment variable SGL_MOE_PREFETCH in MiB, 0 turning every prefetch of
+// the front off; 32 MiB when unset.
+inline uint64_t front_prefetch_budget() {
+  const char* v = getenv("SGL_MOE_PREFETCH");
+  if (v == nullptr || *v == 0) return 32ull << 20;
+  const long mb = strtol(v, nullptr, 10);
+  return mb > 0 ? static_cast<uint64_t>(mb) << 20 : 0;
+}
 
 cudaError_t launch_permute(const moe_cfg& c, int T, const int32_t* idx, int32_t* tile_hist,
                            int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv_perm,

@@ -132,6 +132,13 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
+// Asks L2 to fetch [ptr, ptr + bytes) (16-byte aligned, a multiple of 16
+// bytes); nothing waits for it.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* ptr, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(ptr)),
+               "r"(bytes)
+               : "memory");
+}
 // Waits for every cp.async this thread issued, committed to a group or not.
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 // One arrival on `bar` once every cp.async this thread issued so far has

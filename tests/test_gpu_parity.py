@@ -403,3 +403,16 @@ def test_fused_decode_front_matches_separate_kernels(T, E, monkeypatch):
     for g in (fused, sep):
         check_y(bits(g["y"])[ref["tokens"][keep]], ref["y_f32"][keep], ref["y"][keep], tol=_tol(cfg))
 
+
+
+@pytest.mark.parametrize("T,E", [(32, 512), (8, 128)])
+def test_front_l2_prefetch_changes_nothing(T, E, monkeypatch):
+    """The decode front's L2 prefetch of the shared and first routed experts'
+    weights only warms the cache: outputs are bit-identical with it off."""
+    cfg = workloads.CONFIGS["decode"].with_(E=E)
+    d = workloads.generate(cfg, DEV, T=T)
+    on = run_layer(cfg, d)
+    monkeypatch.setenv("SGL_MOE_PREFETCH", "0")
+    off = run_layer(cfg, d)
+    assert torch.equal(on["idx"], off["idx"])
+    assert np.array_equal(bits(on["y"]), bits(off["y"]))
