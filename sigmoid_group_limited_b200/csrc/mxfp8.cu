@@ -26,13 +26,16 @@
 namespace sgl {
 namespace {
 
-__device__ __forceinline__ int atom_offset(int r, int k) { return (r & 31) * 16 + (r >> 5) * 4 + k; }
-
 // Weight scales of the touched experts as atoms, [slot][128-row tile][k-block]
-// for each of Wg, Wu ([I, H]) and Wd ([H, I]). Unit = one row of one atom
-// (four scale bytes, read as one 32-bit word); consecutive threads take
-// consecutive rows of one atom.
-__global__ void __launch_bounds__(256) mx_sf_repack(int H, int I, int max_touched,
+// for each of Wg, Wu ([I, H]) and Wd ([H, I]). One warp per (slot, matrix,
+// 128-row tile), eight k-blocks at a time: the warp reads the tile's 128 rows
+// x 32 scale bytes with 4-byte loads in which eight lanes cover one row
+// (whole sectors), transposes them through shared memory, and writes each
+// atom as one 512-byte store: lane l's 16 bytes at l * 16 are the four scale
+// bytes of rows l, l+32, l+64 and l+96.
+constexpr int kRepackWarps = 8;
+constexpr int kRepackKb = 8;  // k-blocks per pass
+__global__ void __launch_bounds__(32 * kRepackWarps) mx_sf_repack(int H, int I, int max_touched,
                                                      const int32_t* __restrict__ touched,
                                                      const int32_t* __restrict__ ntouched,
                                                      const uint8_t* __restrict__ gs,
@@ -41,28 +44,42 @@ __global__ void __launch_bounds__(256) mx_sf_repack(int H, int I, int max_touche
                                                      uint8_t* __restrict__ sf_g,
                                                      uint8_t* __restrict__ sf_u,
                                                      uint8_t* __restrict__ sf_d) {
+  __shared__ uint32_t tr[kRepackWarps][128][kRepackKb + 1];  // +1: conflict-free columns
   pdl_trigger();
   pdl_wait();  // the touched list comes from the previous kernel
   const int nt = min(*ntouched, max_touched);
-  const int kbh = H / 128, kbi = I / 128;
-  const long long per_mat = static_cast<long long>(kbh) * kbi * 128;  // units per matrix (both shapes)
-  const long long total = static_cast<long long>(nt) * 3 * per_mat;
-  for (long long u = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; u < total;
-       u += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const long long slot = u / (3 * per_mat);
-    long long v = u - slot * 3 * per_mat;
-    const int mat = static_cast<int>(v / per_mat);
-    v -= mat * per_mat;
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  uint32_t (*sw)[kRepackKb + 1] = tr[wib];
+  const int tiles_gu = I / 128, tiles_d = H / 128;  // 128-row tiles of Wg / Wu, of Wd
+  const int per_slot = 2 * tiles_gu + tiles_d;
+  const long long total = static_cast<long long>(nt) * per_slot;
+  const long long nwarps = static_cast<long long>(gridDim.x) * kRepackWarps;
+  for (long long w = static_cast<long long>(blockIdx.x) * kRepackWarps + wib; w < total; w += nwarps) {
+    const long long slot = w / per_slot;
+    const int v = static_cast<int>(w - slot * per_slot);
+    const int mat = v < tiles_gu ? 0 : (v < 2 * tiles_gu ? 1 : 2);
+    const int t = mat < 2 ? v - mat * tiles_gu : v - 2 * tiles_gu;  // row tile
     const long long e = touched[slot];
-    const int r = static_cast<int>(v & 127);
-    const long long atom = v >> 7;  // (row tile, k-block) of this matrix
-    const int nkb = mat < 2 ? kbh : kbi;  // k-blocks along the contraction
-    const int kc = mat < 2 ? H / 32 : I / 32;  // scale bytes per row
+    const int kw = mat < 2 ? H / 128 : I / 128;  // scale words per row = k-blocks
     const long long rows = mat < 2 ? I : H;
-    const int t = static_cast<int>(atom / nkb), b = static_cast<int>(atom % nkb);
-    const uint8_t* src = (mat == 0 ? gs : mat == 1 ? us : ds) + (e * rows + t * 128 + r) * kc + b * 4;
-    uint8_t* dst = (mat == 0 ? sf_g : mat == 1 ? sf_u : sf_d) + (slot * per_mat / 128 + atom) * 512;
-    *reinterpret_cast<uint32_t*>(dst + atom_offset(r, 0)) = *reinterpret_cast<const uint32_t*>(src);
+    const int tiles = mat < 2 ? tiles_gu : tiles_d;
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(mat == 0 ? gs : mat == 1 ? us : ds) +
+                          (e * rows + t * 128) * kw;
+    uint8_t* dst = (mat == 0 ? sf_g : mat == 1 ? sf_u : sf_d) + ((slot * tiles + t) * kw) * 512 + lane * 16;
+    for (int b0 = 0; b0 < kw; b0 += kRepackKb) {
+      const int nb = min(kRepackKb, kw - b0);
+      __syncwarp();  // the previous pass's reads of sw are done
+      // lane l: word l % 8 of rows l / 8, l / 8 + 4, ...
+      const int c = lane & 7;
+      if (c < nb) {
+#pragma unroll 4
+        for (int r = lane >> 3; r < 128; r += 4) sw[r][c] = src[static_cast<size_t>(r) * kw + b0 + c];
+      }
+      __syncwarp();
+      for (int b = 0; b < nb; ++b)
+        *reinterpret_cast<uint4*>(dst + (b0 + b) * 512) =
+            make_uint4(sw[lane][b], sw[lane + 32][b], sw[lane + 64][b], sw[lane + 96][b]);
+    }
   }
 }
 
@@ -121,7 +138,7 @@ cudaError_t launch_mx_prep(const moe_cfg& c, int T, const int32_t* offsets, cons
   if (e != cudaSuccess) return e;
   const long long TK = static_cast<long long>(T) * c.K;
   const int max_touched = static_cast<int>(TK < c.E ? TK : c.E);
-  e = launch_pdl(mx_sf_repack, dim3(num_sms() * 4), dim3(256), 0, s, c.H, c.I, max_touched,
+  e = launch_pdl(mx_sf_repack, dim3(num_sms() * 4), dim3(32 * kRepackWarps), 0, s, c.H, c.I, max_touched,
                  static_cast<const int32_t*>(touched), static_cast<const int32_t*>(ntouched),
                  W->Wg_scale, W->Wu_scale, W->Wd_scale, sf_g, sf_u, sf_d);
   if (e != cudaSuccess) return e;
