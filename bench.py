@@ -268,7 +268,8 @@ STAGES = ("route", "permute", "gateup", "down", "combine")
 
 DTYPES = {workloads.MOE_W_BF16: "bf16",
           workloads.MOE_W_MXFP4: "mxfp4 weights expanded to bf16",
-          workloads.MOE_W_MXFP4_A8: "mxfp8 x mxfp4 (routed, block-scaled), bf16 (shared)"}
+          workloads.MOE_W_MXFP4_A8: "mxfp8 x mxfp4 (routed, block-scaled), bf16 (shared)",
+          workloads.MOE_W_MXFP4_A8P: "mxfp8 x mxfp4 (routed, block-scaled, prepared scales), bf16 (shared)"}
 
 
 def kernels_per_step(cfg) -> int:
@@ -278,12 +279,13 @@ def kernels_per_step(cfg) -> int:
     tensor-core GEMM, above 32 tokens) and permutation 1 when all T*K slots
     fit one 2048-entry tile else 3; then the expert FFN 1 and combine 1; MXFP4 adds
     2 (touched-expert list, dequantisation); the block-scaled MXFP4_A8 adds 3
-    (touched-expert list, weight-scale atoms, MXFP8 x)."""
+    (touched-expert list, weight-scale atoms, MXFP8 x), and with prepared scale
+    atoms (MXFP4_A8P) 1 (MXFP8 x)."""
     if fused_front(cfg):
         n = 1 + 1 + 1  # fused decode front (routing + permutation), FFN, combine
     else:
         n = (3 if cfg.T <= 32 else 4) + (1 if cfg.T * cfg.K <= 2048 else 3) + 1 + 1
-    return n + {workloads.MOE_W_MXFP4: 2, workloads.MOE_W_MXFP4_A8: 3}.get(cfg.wfmt, 0)
+    return n + {workloads.MOE_W_MXFP4: 2, workloads.MOE_W_MXFP4_A8: 3, workloads.MOE_W_MXFP4_A8P: 1}.get(cfg.wfmt, 0)
 
 
 def fused_front(cfg) -> bool:
@@ -307,6 +309,14 @@ def measure_gpu(cfg, steps, warmup, device, rank, clk, with_e2e=True):
     if "Wg_q" in d:
         W = sgl.make_weights(d["Wg_q"], d["Wu_q"], d["Wd_q"], d["Wg_s"], d["Wu_s"], d["Wd_s"],
                              d["Wg_sc"], d["Wu_sc"], d["Wd_sc"])
+        if cfg.wfmt == workloads.MOE_W_MXFP4_A8P:
+            # one-time weight preparation (load time), outside every timed region
+            atoms = [torch.empty_like(d[k]) for k in ("Wg_sc", "Wu_sc", "Wd_sc")]
+            sgl.moe_prepare_weights(cfg, W, *atoms)
+            torch.cuda.synchronize()
+            d["Wg_sc"], d["Wu_sc"], d["Wd_sc"] = atoms
+            W = sgl.make_weights(d["Wg_q"], d["Wu_q"], d["Wd_q"], d["Wg_s"], d["Wu_s"], d["Wd_s"],
+                                 d["Wg_sc"], d["Wu_sc"], d["Wd_sc"])
     else:
         W = sgl.make_weights(d["Wg"], d["Wu"], d["Wd"], d["Wg_s"], d["Wu_s"], d["Wd_s"])
     ws = sgl.alloc_workspace(cfg, T, device)
@@ -464,8 +474,11 @@ def time_oracle(cfg, h, tokens):
             return g, u, dd
         f = oracle.bf16_bits_to_f64
         return f(g), f(u), f(dd)
+    # prepared scale atoms only re-lay the scale bytes: the oracle's arithmetic
+    # is that of the block-scaled format on the raw scales
+    ocfg = cfg.with_(wfmt=workloads.MOE_W_MXFP4_A8) if cfg.wfmt == workloads.MOE_W_MXFP4_A8P else cfg
     t0 = time.perf_counter()
-    oracle.layer_forward(cfg, h["x"], h["Wr"], h["bias"], ew, h["Wg_s"], h["Wu_s"], h["Wd_s"],
+    oracle.layer_forward(ocfg, h["x"], h["Wr"], h["bias"], ew, h["Wg_s"], h["Wu_s"], h["Wd_s"],
                          tokens=tokens)
     return time.perf_counter() - t0
 
@@ -568,7 +581,7 @@ def run_native(args, rank, world, local):
         b = work["gateup"][0] + work["down"][0]
         f = work["gateup"][1] + work["down"][1]
         t_ffn = (mm["stage_ms"]["ffn"]) / 1e3
-        mx = cfg_.wfmt == workloads.MOE_W_MXFP4_A8
+        mx = cfg_.wfmt in (workloads.MOE_W_MXFP4_A8, workloads.MOE_W_MXFP4_A8P)
         # block-scaled: the routed experts' flops run at the fp8 rate, the shared expert's at bf16
         f8 = 2.0 * cfg_.T * cfg_.K * 3 * cfg_.H * cfg_.I if mx else 0.0
         ent = roofline_entry(b, f, t_ffn, peaks, fp8_flops=f8)

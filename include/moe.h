@@ -66,6 +66,11 @@ extern "C" {
  * 448), and the routed GEMMs run on block-scaled tensor cores. The shared
  * expert stays bf16. Needs H % 128 == 0 and I % 128 == 0. */
 #define MOE_W_MXFP4_A8 2
+/* MOE_W_MXFP4_A8 with the three weight-scale arrays already in the block-
+ * scaled tensor cores' atom layout, written once by moe_prepare_weights: the
+ * forward then skips the per-call repack of the touched experts' scales. The
+ * arithmetic is that of MOE_W_MXFP4_A8, bit for bit. */
+#define MOE_W_MXFP4_A8P 3
 
 /* Layer configuration; field names follow the model's config keys. */
 typedef struct moe_cfg {
@@ -80,7 +85,7 @@ typedef struct moe_cfg {
   int32_t renorm;       /* norm_topk_prob (1) */
   float limit_routed;   /* SwiGLU limit of routed experts; <= 0 or inf: off */
   float limit_shared;   /* SwiGLU limit of the shared expert; <= 0 or inf: off */
-  int32_t wfmt;         /* MOE_W_BF16, MOE_W_MXFP4 or MOE_W_MXFP4_A8 */
+  int32_t wfmt;         /* MOE_W_BF16, MOE_W_MXFP4, MOE_W_MXFP4_A8 or MOE_W_MXFP4_A8P */
 } moe_cfg;
 
 typedef enum moe_status {
@@ -98,7 +103,8 @@ typedef enum moe_status {
  * Routed MXFP4 (MOE_W_MXFP4 and MOE_W_MXFP4_A8): Wg,Wu [E,I,H/2], Wd [E,H,I/2]
  * uint8 codes (element 2j in the low nibble) and Wg_scale,Wu_scale [E,I,H/32],
  * Wd_scale [E,H,I/32] e8m0; with MOE_W_MXFP4_A8 the codes must be 32-byte
- * aligned.
+ * aligned. MOE_W_MXFP4_A8P: the same codes, and the scale arrays in the atom
+ * layout of moe_prepare_weights (same byte counts).
  * Shared expert (bf16): Wg_s,Wu_s [I_s,H], Wd_s [H,I_s]; all three NULL when
  * cfg->I_shared == 0. All device pointers. */
 typedef struct moe_weights {
@@ -186,6 +192,23 @@ MOE_API moe_status moe_layer_forward(const moe_cfg* cfg, int32_t T, const void* 
                              const float* bias, const moe_weights* W, void* y, int32_t* idx_out,
                              float* w_out, int32_t* counts_out, void* ws, size_t ws_bytes,
                              void* stream, void* const* stage_events);
+
+/* One-time preparation of MXFP4 routed weights for MOE_W_MXFP4_A8P (page
+ * "Ling-3.0-flash-VL 42-layer hybrid backbone", spec table: FP8 + MXFP4).
+ * cfg->wfmt: MOE_W_MXFP4_A8 or MOE_W_MXFP4_A8P (only the shapes are read);
+ * in: W->Wg_scale, Wu_scale [E,I,H/32], Wd_scale [E,H,I/32] e8m0 (device);
+ * out (device, caller-owned, the same byte counts as the inputs, 16-byte
+ * aligned): Wg_sf, Wu_sf [E][I/128][H/128][512] and Wd_sf [E][H/128][I/128]
+ * [512]: the 512-byte atom (expert e, 128-row tile t, 128-wide k-block b)
+ * holds the scale of row 128t + r and 32-element chunk 4b + k at byte
+ * (r % 32) * 16 + (r / 32) * 4 + k, the layout tcgen05.cp.32x128b.warpx4
+ * copies into tensor memory for the block-scaled MMA. Pass the three outputs
+ * as the scale pointers of a moe_weights used with MOE_W_MXFP4_A8P.
+ * Errors: MOE_ERR_CFG (not a block-scaled format, or H or I not a multiple
+ * of 128), MOE_ERR_NULL, MOE_ERR_ALIGN, MOE_ERR_CUDA. Asynchronous on
+ * `stream`. */
+MOE_API moe_status moe_prepare_weights(const moe_cfg* cfg, const moe_weights* W, uint8_t* Wg_sf,
+                                       uint8_t* Wu_sf, uint8_t* Wd_sf, void* stream);
 
 /* Routing statistics from the expert counts that moe_permute and
  * moe_layer_forward produce: the load monitoring of page 1 ("Ling-3.0-flash-VL：

@@ -23,6 +23,7 @@ LIB_PATH = os.path.join(_PKG, "libsgl_moe.so")
 MOE_W_BF16 = 0
 MOE_W_MXFP4 = 1
 MOE_W_MXFP4_A8 = 2
+MOE_W_MXFP4_A8P = 3  # MOE_W_MXFP4_A8 with scales prepared by moe_prepare_weights
 MOE_N_STAGE_EVENTS = 6
 STATUS = {0: "MOE_OK", -1: "MOE_ERR_CFG", -2: "MOE_ERR_NULL", -3: "MOE_ERR_ALIGN",
           -4: "MOE_ERR_WORKSPACE", -5: "MOE_ERR_CUDA", -6: "MOE_ERR_DEVICE",
@@ -31,7 +32,7 @@ DEVERR = {0: "none", 1: "expert id out of range", 2: "pipeline wait timed out",
           3: "work item out of range"}
 
 C_FUNCTIONS = ("moe_workspace_size", "moe_route", "moe_permute", "moe_permute_static", "moe_route_stats",
-               "moe_grouped_swiglu",
+               "moe_grouped_swiglu", "moe_prepare_weights",
                "moe_combine", "moe_layer_forward", "moe_read_error", "moe_status_string",
                "moe_version")
 
@@ -79,12 +80,13 @@ def lib() -> ctypes.CDLL:
     L.moe_combine.argtypes = [cp, i32, vp, i32, vp, vp]
     L.moe_layer_forward.argtypes = [cp, i32, vp, vp, vp, wp, vp, vp, vp, vp, vp, sz, vp, vp]
     L.moe_route_stats.argtypes = [cp, vp, vp, vp]
+    L.moe_prepare_weights.argtypes = [cp, wp, vp, vp, vp, vp]
     L.moe_read_error.argtypes = [cp, i32, vp, sz, vp, ctypes.POINTER(i32)]
     L.moe_status_string.argtypes = [i32]
     L.moe_status_string.restype = ctypes.c_char_p
     L.moe_version.restype = ctypes.c_char_p
     for f in ("moe_route", "moe_permute", "moe_permute_static", "moe_route_stats", "moe_grouped_swiglu",
-              "moe_combine",
+              "moe_combine", "moe_prepare_weights",
               "moe_layer_forward", "moe_read_error"):
         getattr(L, f).restype = i32
     _lib = L
@@ -168,6 +170,13 @@ def moe_route_stats(cfg, counts, stats, stream=None):
     c = make_cfg(cfg)
     _check(lib().moe_route_stats(ctypes.byref(c), _p(counts), _p(stats), _stream(stream)),
            "moe_route_stats")
+
+
+def moe_prepare_weights(cfg, weights: moe_weights, Wg_sf, Wu_sf, Wd_sf, stream=None):
+    """Scale atoms of every expert for MOE_W_MXFP4_A8P (uint8 tensors shaped
+    like the scale arrays they replace)."""
+    _check(lib().moe_prepare_weights(ctypes.byref(make_cfg(cfg)), ctypes.byref(weights), _p(Wg_sf),
+                                     _p(Wu_sf), _p(Wd_sf), _stream(stream)), "moe_prepare_weights")
 
 
 def moe_grouped_swiglu(cfg, T, x, perm, offsets, w, weights: moe_weights, y_slot, ws, stream=None):

@@ -47,7 +47,7 @@ WsLayout ws_layout(const moe_cfg& c, int T) {
   memset(&L, 0, sizeof(L));
   const size_t TK = static_cast<size_t>(T) * c.K;
   L.n_ptiles = cdiv(static_cast<long long>(TK), kPermTile);
-  const bool mx = c.wfmt == MOE_W_MXFP4_A8;
+  const bool mx = mx_a8(c.wfmt);
   if (mx) {
     L.bn = kMxTileN;
     L.ffn = kFfnMx;
@@ -92,16 +92,20 @@ WsLayout ws_layout(const moe_cfg& c, int T) {
     // h_r holds the e4m3 h codes; the rest is scales
     L.max_touched = static_cast<int>(TK < static_cast<size_t>(c.E) ? TK : c.E);
     const size_t kb_h = static_cast<size_t>(c.H / 128), kb_i = static_cast<size_t>(c.I / 128);
-    L.slot_of = take(static_cast<size_t>(c.E) * 4);
-    L.touched = take(static_cast<size_t>(c.E) * 4);
-    L.ntouched = take(16);
+    if (c.wfmt == MOE_W_MXFP4_A8) {  // touched-expert slots of the per-call scale repack
+      L.slot_of = take(static_cast<size_t>(c.E) * 4);
+      L.touched = take(static_cast<size_t>(c.E) * 4);
+      L.ntouched = take(16);
+    }
     L.x_q = take(static_cast<size_t>(T) * c.H);
     L.x_sf = take(static_cast<size_t>(T) * (c.H / 32));
     L.h_sf = take(static_cast<size_t>(L.max_row_tiles) * kb_i * 512);
-    const size_t atoms = static_cast<size_t>(L.max_touched) * kb_h * kb_i * 512;
-    L.sf_g = take(atoms);
-    L.sf_u = take(atoms);
-    L.sf_d = take(atoms);
+    if (c.wfmt == MOE_W_MXFP4_A8) {
+      const size_t atoms = static_cast<size_t>(L.max_touched) * kb_h * kb_i * 512;
+      L.sf_g = take(atoms);
+      L.sf_u = take(atoms);
+      L.sf_d = take(atoms);
+    }
   }
   if (c.wfmt == MOE_W_MXFP4) {
     L.max_touched = static_cast<int>(TK < static_cast<size_t>(c.E) ? TK : c.E);
@@ -134,8 +138,8 @@ bool cfg_ok(const moe_cfg* c) {
   if (c->I_shared < 0 || c->I_shared % 64 != 0 || c->I_shared > 16384) return false;
   if (isnan(c->scale) || isinf(c->scale)) return false;
   if (isnan(c->limit_routed) || isnan(c->limit_shared)) return false;
-  if (c->wfmt != MOE_W_BF16 && c->wfmt != MOE_W_MXFP4 && c->wfmt != MOE_W_MXFP4_A8) return false;
-  if (c->wfmt == MOE_W_MXFP4_A8 && (c->H % 128 != 0 || c->I % 128 != 0)) return false;
+  if (c->wfmt != MOE_W_BF16 && c->wfmt != MOE_W_MXFP4 && !mx_a8(c->wfmt)) return false;
+  if (mx_a8(c->wfmt) && (c->H % 128 != 0 || c->I % 128 != 0)) return false;
   return true;
 }
 
@@ -175,11 +179,11 @@ moe_status cu(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; 
 moe_status check_weights(const moe_cfg* c, const moe_weights* W) {
   if (W == nullptr || W->Wg == nullptr || W->Wu == nullptr || W->Wd == nullptr) return MOE_ERR_NULL;
   if (!al16(W->Wg) || !al16(W->Wu) || !al16(W->Wd)) return MOE_ERR_ALIGN;
-  if (c->wfmt == MOE_W_MXFP4 || c->wfmt == MOE_W_MXFP4_A8) {
+  if (c->wfmt == MOE_W_MXFP4 || mx_a8(c->wfmt)) {
     if (!W->Wg_scale || !W->Wu_scale || !W->Wd_scale) return MOE_ERR_NULL;
     if (!al16(W->Wg_scale) || !al16(W->Wu_scale) || !al16(W->Wd_scale)) return MOE_ERR_ALIGN;
   }
-  if (c->wfmt == MOE_W_MXFP4_A8) {  // TMA of unpacked 4-bit codes wants 32-byte bases
+  if (mx_a8(c->wfmt)) {  // TMA of unpacked 4-bit codes wants 32-byte bases
     auto al32 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; };
     if (!al32(W->Wg) || !al32(W->Wu) || !al32(W->Wd)) return MOE_ERR_ALIGN;
   }
@@ -234,21 +238,30 @@ cudaError_t run_ffn(const moe_cfg* cfg, int T, const uint16_t* x, const int32_t*
   a.ffn = L.ffn;
   a.max_items_gu = L.max_items_gu;
   a.max_items_dn = L.max_items_dn;
-  if (cfg->wfmt == MOE_W_MXFP4_A8) {
-    cudaError_t e = launch_mx_prep(*cfg, T, offsets, W, x, at<int32_t>(ws, L.slot_of),
-                                   at<int32_t>(ws, L.touched), at<int32_t>(ws, L.ntouched),
-                                   at<uint8_t>(ws, L.sf_g), at<uint8_t>(ws, L.sf_u),
-                                   at<uint8_t>(ws, L.sf_d), at<uint8_t>(ws, L.x_q),
-                                   at<uint8_t>(ws, L.x_sf), s);
-    if (e != cudaSuccess) return e;
+  if (mx_a8(cfg->wfmt)) {
+    if (cfg->wfmt == MOE_W_MXFP4_A8) {  // touched experts' scales repacked for this call
+      cudaError_t e = launch_mx_prep(*cfg, T, offsets, W, x, at<int32_t>(ws, L.slot_of),
+                                     at<int32_t>(ws, L.touched), at<int32_t>(ws, L.ntouched),
+                                     at<uint8_t>(ws, L.sf_g), at<uint8_t>(ws, L.sf_u),
+                                     at<uint8_t>(ws, L.sf_d), at<uint8_t>(ws, L.x_q),
+                                     at<uint8_t>(ws, L.x_sf), s);
+      if (e != cudaSuccess) return e;
+      a.sf_g = at<uint8_t>(ws, L.sf_g);
+      a.sf_u = at<uint8_t>(ws, L.sf_u);
+      a.sf_d = at<uint8_t>(ws, L.sf_d);
+      a.slot_of = at<int32_t>(ws, L.slot_of);
+    } else {  // prepared atoms of every expert (moe_prepare_weights)
+      cudaError_t e = launch_mx_quant(*cfg, T, x, at<uint8_t>(ws, L.x_q), at<uint8_t>(ws, L.x_sf), s);
+      if (e != cudaSuccess) return e;
+      a.sf_g = W->Wg_scale;
+      a.sf_u = W->Wu_scale;
+      a.sf_d = W->Wd_scale;
+      a.slot_of = nullptr;
+    }
     a.x_q = at<uint8_t>(ws, L.x_q);
     a.x_sf = at<uint8_t>(ws, L.x_sf);
     a.h_q = at<uint8_t>(ws, L.h_r);
     a.h_sf = at<uint8_t>(ws, L.h_sf);
-    a.sf_g = at<uint8_t>(ws, L.sf_g);
-    a.sf_u = at<uint8_t>(ws, L.sf_u);
-    a.sf_d = at<uint8_t>(ws, L.sf_d);
-    a.slot_of = at<int32_t>(ws, L.slot_of);
     return launch_ffn_mx(a, s);
   }
   return launch_ffn(a, s);
@@ -415,6 +428,19 @@ moe_status moe_layer_forward(const moe_cfg* cfg, int32_t T, const void* x, const
     return MOE_ERR_CUDA;
   rec(5);
   return MOE_OK;
+}
+
+moe_status moe_prepare_weights(const moe_cfg* cfg, const moe_weights* W, uint8_t* Wg_sf,
+                               uint8_t* Wu_sf, uint8_t* Wd_sf, void* stream) {
+  if (!cfg_ok(cfg) || !mx_a8(cfg->wfmt)) return MOE_ERR_CFG;
+  if (!W || !W->Wg_scale || !W->Wu_scale || !W->Wd_scale || !Wg_sf || !Wu_sf || !Wd_sf)
+    return MOE_ERR_NULL;
+  if (!al16(W->Wg_scale) || !al16(W->Wu_scale) || !al16(W->Wd_scale) || !al16(Wg_sf) ||
+      !al16(Wu_sf) || !al16(Wd_sf))
+    return MOE_ERR_ALIGN;
+  moe_status st = device_ok();
+  if (st != MOE_OK) return st;
+  return cu(launch_mx_sf_atoms(*cfg, W, Wg_sf, Wu_sf, Wd_sf, static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_route_stats(const moe_cfg* cfg, const int32_t* counts, double* stats,

@@ -75,7 +75,7 @@ struct MxParams {
   const uint8_t* sf_g;   // [slot][I/128][H/128][512]
   const uint8_t* sf_u;   // [slot][I/128][H/128][512]
   const uint8_t* sf_d;   // [slot][H/128][I/128][512]
-  const int32_t* slot_of;
+  const int32_t* slot_of;  // nullptr: prepared atoms, indexed by expert id
 };
 
 struct MxMaps {
@@ -247,7 +247,7 @@ __global__ void __launch_bounds__(kXThreads, 1)
         const bool two = two_halves(it, gu);
         const int na = two ? 2 : 1;
         const int nhbox = gu ? 0 : mma_n(it) / kXHBox;
-        const int slot = sh ? 0 : q.slot_of[it.e];
+        const int slot = sh ? 0 : (q.slot_of ? q.slot_of[it.e] : it.e);  // prepared atoms: by expert
         uint32_t bytes;
         if (sh) bytes = na * kXA + nhbox * kXHBox * 128;
         else bytes = na * (128 * 64 + 512) + (gu ? 0 : nhbox * kXHBox * 128 + 512);
@@ -575,7 +575,7 @@ __global__ void __launch_bounds__(kXThreads, 1)
 
 cudaError_t launch_ffn_mx(const GemmArgs& a, cudaStream_t s) {
   const moe_cfg& c = *a.cfg;
-  if (a.bn != kMxTileN || a.x_q == nullptr || a.slot_of == nullptr) return cudaErrorInvalidValue;
+  if (a.bn != kMxTileN || a.x_q == nullptr) return cudaErrorInvalidValue;
   MxParams q;
   memset(&q, 0, sizeof(q));
   FfnParams& p = q.f;

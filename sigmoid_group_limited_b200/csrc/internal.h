@@ -39,6 +39,9 @@ constexpr int kMxGuTile = 128;
 constexpr int kMxDnTile = 256;
 constexpr int kMaxExpertsCfg = 1024;  // largest E a configuration may have
 
+// The block-scaled weight formats (per-call scale repack, or prepared atoms).
+inline bool mx_a8(int wfmt) { return wfmt == MOE_W_MXFP4_A8 || wfmt == MOE_W_MXFP4_A8P; }
+
 // Which expert-FFN kernel a batch runs on.
 enum FfnKind {
   kFfnNarrow = 0,  // moe_ffn<BN>: BN <= 128 tokens, 128 gate + 128 up features per item
@@ -185,7 +188,7 @@ struct GemmArgs {
   const uint8_t* sf_g;       // [slot][I/128][H/128][512]
   const uint8_t* sf_u;       // [slot][I/128][H/128][512]
   const uint8_t* sf_d;       // [slot][H/128][I/128][512]
-  const int32_t* slot_of;    // [E] touched slot of expert e
+  const int32_t* slot_of;    // [E] touched slot of expert e; nullptr: sf_* indexed by expert
 };
 
 // The expert FFN: gate/up and down in one cooperative persistent launch
@@ -207,6 +210,12 @@ cudaError_t launch_mx_prep(const moe_cfg& c, int T, const int32_t* offsets, cons
                            const uint16_t* x, int32_t* slot_of, int32_t* touched,
                            int32_t* ntouched, uint8_t* sf_g, uint8_t* sf_u, uint8_t* sf_d,
                            uint8_t* x_q, uint8_t* x_sf, cudaStream_t s);
+// MXFP8 x alone (MOE_W_MXFP4_A8P: the weight scales are prepared atoms).
+cudaError_t launch_mx_quant(const moe_cfg& c, int T, const uint16_t* x, uint8_t* x_q, uint8_t* x_sf,
+                            cudaStream_t s);
+// Every expert's weight scales as atoms (moe_prepare_weights).
+cudaError_t launch_mx_sf_atoms(const moe_cfg& c, const moe_weights* W, uint8_t* sf_g, uint8_t* sf_u,
+                               uint8_t* sf_d, cudaStream_t s);
 // Touched experts of a batch in increasing id order (slot_of[e], -1 if none).
 cudaError_t launch_mxfp4_slots(const moe_cfg& c, const int32_t* offsets, int32_t* slot_of,
                                int32_t* touched, int32_t* ntouched, cudaStream_t s);

@@ -47,7 +47,8 @@ __global__ void __launch_bounds__(32 * kRepackWarps) mx_sf_repack(int H, int I, 
   __shared__ uint32_t tr[kRepackWarps][128][kRepackKb + 1];  // +1: conflict-free columns
   pdl_trigger();
   pdl_wait();  // the touched list comes from the previous kernel
-  const int nt = min(*ntouched, max_touched);
+  // touched == nullptr: every expert, slot = expert id (max_touched = E)
+  const int nt = touched ? min(*ntouched, max_touched) : max_touched;
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   uint32_t (*sw)[kRepackKb + 1] = tr[wib];
   const int tiles_gu = I / 128, tiles_d = H / 128;  // 128-row tiles of Wg / Wu, of Wd
@@ -59,7 +60,7 @@ __global__ void __launch_bounds__(32 * kRepackWarps) mx_sf_repack(int H, int I, 
     const int v = static_cast<int>(w - slot * per_slot);
     const int mat = v < tiles_gu ? 0 : (v < 2 * tiles_gu ? 1 : 2);
     const int t = mat < 2 ? v - mat * tiles_gu : v - 2 * tiles_gu;  // row tile
-    const long long e = touched[slot];
+    const long long e = touched ? touched[slot] : slot;
     const int kw = mat < 2 ? H / 128 : I / 128;  // scale words per row = k-blocks
     const long long rows = mat < 2 ? I : H;
     const int tiles = mat < 2 ? tiles_gu : tiles_d;
@@ -142,11 +143,23 @@ cudaError_t launch_mx_prep(const moe_cfg& c, int T, const int32_t* offsets, cons
                  static_cast<const int32_t*>(touched), static_cast<const int32_t*>(ntouched),
                  W->Wg_scale, W->Wu_scale, W->Wd_scale, sf_g, sf_u, sf_d);
   if (e != cudaSuccess) return e;
+  return launch_mx_quant(c, T, x, x_q, x_sf, s);
+}
+
+cudaError_t launch_mx_quant(const moe_cfg& c, int T, const uint16_t* x, uint8_t* x_q, uint8_t* x_sf,
+                            cudaStream_t s) {
   const long long nblocks = static_cast<long long>(T) * (c.H / 32);
   long long grid = (nblocks + 255) / 256;
   if (grid > num_sms() * 8) grid = num_sms() * 8;
   return launch_pdl(mx_quant_x, dim3(static_cast<int>(grid)), dim3(256), 0, s, nblocks, c.H, x,
                     x_q, x_sf);
+}
+
+cudaError_t launch_mx_sf_atoms(const moe_cfg& c, const moe_weights* W, uint8_t* sf_g, uint8_t* sf_u,
+                               uint8_t* sf_d, cudaStream_t s) {
+  return launch_pdl(mx_sf_repack, dim3(num_sms() * 4), dim3(32 * kRepackWarps), 0, s, c.H, c.I, c.E,
+                    static_cast<const int32_t*>(nullptr), static_cast<const int32_t*>(nullptr),
+                    W->Wg_scale, W->Wu_scale, W->Wd_scale, sf_g, sf_u, sf_d);
 }
 
 }  // namespace sgl

@@ -89,7 +89,11 @@ def test_block_scaled_format_validation():
     assert sgl.workspace_size(workloads.CONFIGS["tiny_a8"], 64) > 0
     assert L.moe_workspace_size(ctypes.byref(sgl.make_cfg(full.with_(I=704))), 32) == 0
     assert L.moe_workspace_size(ctypes.byref(sgl.make_cfg(full.with_(H=2496))), 32) == 0
-    assert L.moe_workspace_size(ctypes.byref(sgl.make_cfg(full.with_(wfmt=3))), 32) == 0
+    assert L.moe_workspace_size(ctypes.byref(sgl.make_cfg(full.with_(wfmt=4))), 32) == 0
+    # the prepared variant takes the same shapes and needs no per-call scale atoms
+    prep = full.with_(wfmt=workloads.MOE_W_MXFP4_A8P)
+    assert 0 < sgl.workspace_size(prep, 32) < sgl.workspace_size(full, 32)
+    assert L.moe_workspace_size(ctypes.byref(sgl.make_cfg(prep.with_(I=704))), 32) == 0
     c = sgl.make_cfg(full)
     need = sgl.workspace_size(full, 32)
     A = 1 << 20
@@ -99,3 +103,22 @@ def test_block_scaled_format_validation():
     w = sgl.moe_weights(A, A, A, None, A, A, A, A, A)           # a scale array missing
     assert L.moe_layer_forward(ctypes.byref(c), 32, A, A, None, ctypes.byref(w), A, None, None,
                                None, A, need, None, None) == -2
+
+
+def test_prepare_weights_validation():
+    """moe_prepare_weights: block-scaled formats only, every pointer present
+    and 16-byte aligned; all checked on the host before any device work."""
+    L = sgl.lib()
+    A = 1 << 20
+    full = workloads.CONFIGS["mxfp4_a8"]
+    w = sgl.moe_weights(A, A, A, A, A, A, A, A, A)
+    for bad in (workloads.CONFIGS["prefill"], workloads.CONFIGS["mxfp4"], full.with_(I=704)):
+        assert L.moe_prepare_weights(ctypes.byref(sgl.make_cfg(bad)), ctypes.byref(w), A, A, A, None) == -1
+    c = sgl.make_cfg(full)
+    assert L.moe_prepare_weights(ctypes.byref(c), None, A, A, A, None) == -2
+    assert L.moe_prepare_weights(ctypes.byref(c), ctypes.byref(w), A, None, A, None) == -2
+    no_scale = sgl.moe_weights(A, A, A, A, None, A, A, A, A)
+    assert L.moe_prepare_weights(ctypes.byref(c), ctypes.byref(no_scale), A, A, A, None) == -2
+    assert L.moe_prepare_weights(ctypes.byref(c), ctypes.byref(w), A, A, A + 8, None) == -3
+    odd = sgl.moe_weights(A, A, A, A, A + 4, A, A, A, A)
+    assert L.moe_prepare_weights(ctypes.byref(c), ctypes.byref(odd), A, A, A, None) == -3

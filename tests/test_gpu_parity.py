@@ -416,3 +416,74 @@ def test_front_l2_prefetch_changes_nothing(T, E, monkeypatch):
     off = run_layer(cfg, d)
     assert torch.equal(on["idx"], off["idx"])
     assert np.array_equal(bits(on["y"]), bits(off["y"]))
+
+
+# ------------------------------------------------------------------ prepared block-scaled weights
+
+def _prepared(cfg, d):
+    """moe_prepare_weights on the generated scales; returns the atom arrays."""
+    out = [torch.empty_like(d[k]) for k in ("Wg_sc", "Wu_sc", "Wd_sc")]
+    sgl.moe_prepare_weights(cfg, sgl.make_weights(d["Wg_q"], d["Wu_q"], d["Wd_q"], d.get("Wg_s"),
+                                                  d.get("Wu_s"), d.get("Wd_s"), d["Wg_sc"], d["Wu_sc"],
+                                                  d["Wd_sc"]), *out)
+    torch.cuda.synchronize()
+    return out
+
+
+def _atoms_host(sc: np.ndarray) -> np.ndarray:
+    """The atom layout written out from its definition: [E, rows, kc] scale
+    bytes -> [E, rows/128, kc/4, 512] with row r, chunk k of an atom at byte
+    (r % 32) * 16 + (r / 32) * 4 + k."""
+    E, rows, kc = sc.shape
+    out = np.zeros((E, rows // 128, kc // 4, 512), np.uint8)
+    for r in range(128):
+        for k in range(4):
+            out[:, :, :, (r % 32) * 16 + (r // 32) * 4 + k] = sc[:, r::128, :][:, :rows // 128, k::4]
+    return out
+
+
+@pytest.mark.parametrize("variant", [{}, dict(I=256, H=384)])
+def test_prepare_weights_atom_layout(variant):
+    cfg = TINY_A8.with_(wfmt=workloads.MOE_W_MXFP4_A8, **variant)
+    d = workloads.generate(cfg, DEV, T=8)
+    got = _prepared(cfg, d)
+    for name, g in zip(("Wg_sc", "Wu_sc", "Wd_sc"), got):
+        want = _atoms_host(d[name].cpu().numpy())
+        assert np.array_equal(g.cpu().numpy().reshape(want.shape), want), name
+
+
+@pytest.mark.parametrize("T,variant", [(1, {}), (64, {}), (300, {}), (64, dict(I_shared=0)),
+                                       (200, dict(limit_routed=0.5, limit_shared=0.7))])
+def test_prepared_block_scaled_is_bit_identical(T, variant):
+    """MOE_W_MXFP4_A8P reads the prepared atoms by expert id instead of
+    repacking the touched experts' scales per call; the arithmetic is the
+    same, so y, idx and w are bit-identical to MOE_W_MXFP4_A8 (which is itself
+    checked against the oracle above)."""
+    cfg = TINY_A8.with_(**variant)
+    d = workloads.generate(cfg, DEV, T=T)
+    if cfg.I_shared == 0:
+        d.update(Wg_s=None, Wu_s=None, Wd_s=None)
+    base = run_layer(cfg, d)
+    pcfg = cfg.with_(wfmt=workloads.MOE_W_MXFP4_A8P)
+    g, u, dn = _prepared(pcfg, d)
+    prep = run_layer(pcfg, {**d, "Wg_sc": g, "Wu_sc": u, "Wd_sc": dn})
+    assert torch.equal(base["idx"], prep["idx"]) and torch.equal(base["w"], prep["w"])
+    assert np.array_equal(bits(base["y"]), bits(prep["y"]))
+
+
+@pytest.mark.slow
+def test_prepared_block_scaled_full_size_sampled():
+    """The full T=8192 block-scaled config with prepared scales, against the
+    oracle (which quantises the same way; the format only moves scale bytes)."""
+    cfg = workloads.CONFIGS["mxfp4_a8"]
+    d = workloads.generate(cfg, DEV)
+    pcfg = cfg.with_(wfmt=workloads.MOE_W_MXFP4_A8P)
+    g, u, dn = _prepared(pcfg, d)
+    out = run_layer(pcfg, {**d, "Wg_sc": g, "Wu_sc": u, "Wd_sc": dn})
+    tok = _sample(cfg.T, 8, cfg.seed + 1)
+    ref = _oracle_layer(cfg, d, tokens=tok)
+    near = check_routing(ref, out["idx"].cpu().numpy(), out["w"].cpu().numpy())
+    keep = ~np.isin(ref["tokens"], near)
+    check_y(bits(out["y"])[ref["tokens"][keep]], ref["y_f32"][keep], ref["y"][keep], tol=_tol(cfg))
+    del d
+    torch.cuda.empty_cache()

@@ -29,6 +29,7 @@ import torch
 MOE_W_BF16 = 0
 MOE_W_MXFP4 = 1
 MOE_W_MXFP4_A8 = 2   # MXFP4 routed weights, routed-expert activations in MXFP8
+MOE_W_MXFP4_A8P = 3  # the same, scales prepared once into the tensor cores' atom layout
 
 
 @dataclasses.dataclass(frozen=True)
@@ -81,6 +82,8 @@ CONFIGS: Dict[str, MoEConfig] = {
     "mxfp4": MoEConfig("mxfp4", T=8192, seed=4, wfmt=MOE_W_MXFP4, **_FULL),
     # the same inputs on block-scaled tensor cores: MXFP8 activations x MXFP4 weights
     "mxfp4_a8": MoEConfig("mxfp4_a8", T=8192, seed=4, wfmt=MOE_W_MXFP4_A8, **_FULL),
+    # the same, with the weight scales prepared once into the tensor cores' atom layout
+    "mxfp4_a8p": MoEConfig("mxfp4_a8p", T=8192, seed=4, wfmt=MOE_W_MXFP4_A8P, **_FULL),
     # small case of the block-scaled variant (its tiles need I % 128 == 0)
     "tiny_a8": MoEConfig("tiny_a8", T=64, H=256, E=32, n_group=4, topk_group=2, K=4,
                          I=128, I_shared=64, seed=0, wfmt=MOE_W_MXFP4_A8),
@@ -168,7 +171,7 @@ def generate(cfg: MoEConfig, device="cpu", T: Optional[int] = None) -> Dict[str,
         out["Wg"] = _bf16((E, I, H), 1.0 / H, _gen(device, s + 3), device, chunk)
         out["Wu"] = _bf16((E, I, H), 1.0 / H, _gen(device, s + 4), device, chunk)
         out["Wd"] = _bf16((E, H, I), 1.0 / I, _gen(device, s + 5), device, chunk)
-    elif cfg.wfmt in (MOE_W_MXFP4, MOE_W_MXFP4_A8):
+    elif cfg.wfmt in (MOE_W_MXFP4, MOE_W_MXFP4_A8, MOE_W_MXFP4_A8P):
         for name, shape, var, k in (("Wg", (E, I, H), 1.0 / H, 3), ("Wu", (E, I, H), 1.0 / H, 4),
                                     ("Wd", (E, H, I), 1.0 / I, 5)):
             g = _gen(device, s + k)
