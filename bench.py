@@ -606,7 +606,7 @@ def run_native(args, rank, world, local):
     line = {"metric": METRIC, "value": round(tokens / dev_s, 1), "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(1e3 * dev_s / args.steps, 4), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": DTYPES.get(cfg.wfmt, "bf16"), "data": "synthetic",
             "timing": "CUDA-event time of K graph replays of moe_layer_forward (one capture of "
                       "the C-ABI call); value_no_graph: the same K steps as plain C-ABI calls",
             "value_no_graph": round(tokens / plain_s, 1),
