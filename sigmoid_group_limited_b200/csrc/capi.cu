@@ -199,9 +199,11 @@ moe_status check_weights(const moe_cfg* c, const moe_weights* W) {
 // expert FFN kernel of the format.
 cudaError_t run_ffn(const moe_cfg* cfg, int T, const uint16_t* x, const int32_t* perm,
                     const int32_t* offsets, const float* w, const moe_weights* W, float* y_slot,
-                    void* ws, const WsLayout& L, cudaStream_t s) {
+                    void* ws, const WsLayout& L, cudaStream_t s,
+                    const int32_t* sched_counts = nullptr) {
   GemmArgs a;
   memset(&a, 0, sizeof(a));
+  a.sched_counts = sched_counts;
   a.cfg = cfg;
   a.T = T;
   a.x = x;
@@ -397,13 +399,16 @@ moe_status moe_layer_forward(const moe_cfg* cfg, int32_t T, const void* x, const
   cudaError_t e;
   rec(0);
   if (cudaMemsetAsync(err, 0, kCtrlBytes, s) != cudaSuccess) return MOE_ERR_CUDA;
-  if (decode_front_ok(*cfg, T) && !fused_front_disabled()) {
-    // routing, permutation and work lists in one launch (decode batches)
+  // decode batches: routing and permutation in one launch; the narrow FFN
+  // kernel then derives its work lists from the counts (off the front's tail)
+  const bool front = decode_front_ok(*cfg, T) && !fused_front_disabled();
+  const bool ffn_derives = front && L.ffn == kFfnNarrow;
+  if (front) {
     if ((e = launch_decode_front(*cfg, T, static_cast<const uint16_t*>(x), Wr, bias,
                                  at<float>(ws, L.zp), at<float>(ws, L.z), idx, w,
                                  at<int32_t>(ws, L.unc), err + 1, err + 2, err, counts, offsets,
                                  perm, at<int32_t>(ws, L.inv_perm), L, gu, dn,
-                                 at<int32_t>(ws, L.ready), nitems, W, s)) != cudaSuccess)
+                                 at<int32_t>(ws, L.ready), nitems, W, !ffn_derives, s)) != cudaSuccess)
       return MOE_ERR_CUDA;
     rec(1);
   } else {
@@ -418,8 +423,8 @@ moe_status moe_layer_forward(const moe_cfg* cfg, int32_t T, const void* x, const
       return MOE_ERR_CUDA;
   }
   rec(2);
-  if ((e = run_ffn(cfg, T, static_cast<const uint16_t*>(x), perm, offsets, w, W, y_slot, ws, L,
-                   s)) != cudaSuccess)
+  if ((e = run_ffn(cfg, T, static_cast<const uint16_t*>(x), perm, offsets, w, W, y_slot, ws, L, s,
+                   ffn_derives ? counts : nullptr)) != cudaSuccess)
     return MOE_ERR_CUDA;
   rec(3);
   rec(4);

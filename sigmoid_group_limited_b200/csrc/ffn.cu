@@ -143,18 +143,26 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
     tmem_relinquish();
   }
   pdl_wait();  // the schedule, the routing and x come from earlier kernels
-  for (int i = tid; i < p.E + 2; i += blockDim.x) {
-    s_gu[i] = p.gu_start[i];
-    s_dn[i] = p.dn_start[i];
+  int n_gu_all, n_dn_all;
+  if (p.sched_counts) {
+    __shared__ int wsum[33];
+    derive_schedule(p, s_gu, s_dn, s_off, wsum, &n_gu_all, &n_dn_all);
+  } else {
+    for (int i = tid; i < p.E + 2; i += blockDim.x) {
+      s_gu[i] = p.gu_start[i];
+      s_dn[i] = p.dn_start[i];
+    }
+    for (int i = tid; i < p.E + 1; i += blockDim.x) s_off[i] = p.offsets[i];
+    n_gu_all = p.nitems[0];
+    n_dn_all = p.nitems[1];
   }
-  for (int i = tid; i < p.E + 1; i += blockDim.x) s_off[i] = p.offsets[i];
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int nslots = p.E + (p.has_shared ? 1 : 0);
-  const int n_gu = min(p.nitems[0], p.max_gu);
-  const int n_dn = min(p.nitems[1], p.max_dn);
+  const int n_gu = min(n_gu_all, p.max_gu);
+  const int n_dn = min(n_dn_all, p.max_dn);
   const int n_all = n_gu + n_dn;
   auto item_at = [&](int i, bool& gu) {
     gu = i < n_gu;
@@ -532,6 +540,10 @@ cudaError_t launch_bn(const GemmArgs& a, cudaStream_t s) {
   p.max_gu = a.max_items_gu;
   p.max_dn = a.max_items_dn;
   p.err = a.err;
+  p.sched_counts = a.sched_counts;
+  p.bn = BN;
+  p.gu_ft = kTileN;
+  p.dn_ft = kDownTile;
   const int T = a.T, TK = a.T * c.K;
   CUtensorMap tWg, tWu, tWgS, tWuS, tWd, tWdS, tH, tHs;
   bool ok = map_bf16(&tWg, a.Wg, static_cast<uint64_t>(a.wrows) * c.I, c.H, kTileN) &&

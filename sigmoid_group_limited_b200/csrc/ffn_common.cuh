@@ -31,7 +31,79 @@ struct FfnParams {
   int32_t* ready;            // [max_gu] finished gate/up tiles per (slot, row tile)
   int max_gu, max_dn;
   int32_t* err;
+  const int32_t* sched_counts;  // nullable: derive the work lists from the expert counts
+  int bn, gu_ft, dn_ft;         // token tile and output features per item (for that)
 };
+
+// In-place exclusive scan of a[0..n) in shared memory by the whole CTA
+// (each thread sums a contiguous run, then one block scan of the run sums);
+// wsum: 33 ints of shared memory. Ends with a CTA barrier.
+__device__ __forceinline__ void smem_exscan(int* a, int n, int* wsum) {
+  const int per = (n + static_cast<int>(blockDim.x) - 1) / static_cast<int>(blockDim.x);
+  const int b = static_cast<int>(threadIdx.x) * per, e = min(n, b + per);
+  int s = 0;
+  for (int i = b; i < e; ++i) s += a[i];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = s;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = static_cast<int>(blockDim.x) >> 5;
+    const int v = lane < nw ? wsum[lane] : 0;
+    int vi = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, vi, o);
+      if (lane >= o) vi += y;
+    }
+    if (lane < nw) wsum[lane] = vi - v;
+  }
+  __syncthreads();
+  int run = wsum[warp] + incl - s;
+  for (int i = b; i < e; ++i) {
+    const int v = a[i];
+    a[i] = run;
+    run += v;
+  }
+  __syncthreads();
+}
+
+// The FFN work lists from the expert counts, in shared memory: the row
+// offsets s_off[0..E] (exclusive scan of the counts) and the per-slot item
+// starts s_gu / s_dn [E+2] (slot E the shared expert, entry E+1 the total),
+// exactly as the schedule builder of the permutation writes them. Returns the
+// item totals.
+__device__ __forceinline__ void derive_schedule(const FfnParams& p, int* s_gu, int* s_dn, int* s_off,
+                                                int* wsum, int* n_gu, int* n_dn) {
+  const int nslots = p.E + (p.has_shared ? 1 : 0);
+  const int nt_gu_r = cdiv_dev(p.I, p.gu_ft), nt_gu_s = cdiv_dev(p.Is, p.gu_ft);
+  const int nt_dn = cdiv_dev(p.H, p.dn_ft);
+  for (int e = threadIdx.x; e < p.E + 2; e += blockDim.x) {
+    int gu = 0, dn = 0, c = 0;
+    if (e < p.E) c = max(0, p.sched_counts[e]);
+    if (e < nslots) {
+      const bool sh = e == p.E;
+      const int rows = sh ? p.T : c;
+      const int nm = (rows + p.bn - 1) / p.bn;
+      gu = nm * (sh ? nt_gu_s : nt_gu_r);
+      dn = nm * nt_dn;
+    }
+    s_gu[e] = gu;
+    s_dn[e] = dn;
+    if (e < p.E + 1) s_off[e] = c;
+  }
+  __syncthreads();
+  smem_exscan(s_gu, p.E + 2, wsum);
+  smem_exscan(s_dn, p.E + 2, wsum);
+  smem_exscan(s_off, p.E + 1, wsum);
+  *n_gu = s_gu[p.E + 1];
+  *n_dn = s_dn[p.E + 1];
+}
 
 __device__ __forceinline__ float clampL(float v, float L) {
   return L > 0.f ? fminf(fmaxf(v, -L), L) : v;

@@ -21,7 +21,8 @@
 //      phase 2 (order-free); after the second barrier CTA t places its own
 //      K slots at offsets[e] + (the number of earlier flat slots with the
 //      same expert), the stable counting-sort position, and CTA 0 writes the
-//      offsets and the FFN work lists (whose ready counters phase 1 zeroed).
+//      offsets and, unless the FFN derives them from the counts itself, its
+//      work lists (whose ready counters phase 1 zeroed).
 // L2 prefetch for the expert FFN that follows: HBM is nearly idle while the
 // front runs, so phase 1 asks L2 for the shared expert's weights (known
 // before routing), and after the second barrier the CTAs without a token ask
@@ -66,6 +67,7 @@ struct FrontParams {
   int32_t* inv_perm;
   SchedArgs sa;
   int n_ready;        // ready counters to zero (the FFN's largest gate/up item count)
+  int build_sched;    // 0: the FFN derives its work lists from the counts itself
   // L2 prefetch (null / 0: none): the shared expert's three matrices, and the
   // routed gate and up weights (expert e at e * pf_expert_bytes) of at most
   // pf_experts touched experts
@@ -203,7 +205,9 @@ __global__ void __launch_bounds__(kFrontThreads, 1) decode_front(const __grid_co
   if (blockIdx.x == 0 && p.bias)
     for (int e = tid * 32; e < E; e += blockDim.x * 32)
       asm volatile("prefetch.global.L2 [%0];" ::"l"(p.bias + e));
-  // counts (the selecting CTAs add to them) and the FFN's ready counters start at zero
+  // counts (the selecting CTAs add to them), the FFN's ready counters and its
+  // item claim counter start at zero
+  if (blockIdx.x == 0 && tid == 0) p.sa.nitems[2] = 0;
   for (int i = blockIdx.x * blockDim.x + tid; i < E + p.n_ready; i += gridDim.x * blockDim.x) {
     if (i < E) p.counts[i] = 0;
     else p.sa.ready[i - E] = 0;
@@ -278,9 +282,11 @@ __global__ void __launch_bounds__(kFrontThreads, 1) decode_front(const __grid_co
     }
     if (t == 0) {
       for (int e = tid; e <= E; e += blockDim.x) p.offsets[e] = off[e];
-      SchedArgs sa = p.sa;
-      sa.ready = nullptr;  // zeroed in phase 1
-      build_schedule(sa, cnt, scratch);
+      if (p.build_sched) {
+        SchedArgs sa = p.sa;
+        sa.ready = nullptr;  // zeroed in phase 1
+        build_schedule(sa, cnt, scratch);
+      }
     }
   } else if (p.pf_experts > 0) {
     // gate and up weights of the first touched experts, in the FFN's item
@@ -329,7 +335,7 @@ cudaError_t launch_decode_front(const moe_cfg& c, int T, const uint16_t* x, cons
                                 int32_t* counts, int32_t* offsets, int32_t* perm,
                                 int32_t* inv_perm, const WsLayout& L, int32_t* gu_start,
                                 int32_t* dn_start, int32_t* ready, int32_t* nitems,
-                                const moe_weights* W, cudaStream_t s) {
+                                const moe_weights* W, bool build_sched, cudaStream_t s) {
   if (!decode_front_ok(c, T)) return cudaErrorInvalidValue;
   FrontParams p;
   memset(&p, 0, sizeof(p));
@@ -358,6 +364,7 @@ cudaError_t launch_decode_front(const moe_cfg& c, int T, const uint16_t* x, cons
   p.inv_perm = inv_perm;
   p.sa = make_sched(c, T, L, gu_start, dn_start, ready, nitems);
   p.n_ready = L.max_items_gu;
+  p.build_sched = build_sched ? 1 : 0;
   const uint64_t budget = front_prefetch_budget();
   if (W && budget > 0) {
     // bf16 matrices whose sizes (multiples of 64 x 64 elements) keep every

@@ -125,7 +125,7 @@ cudaError_t launch_decode_front(const moe_cfg& c, int T, const uint16_t* x, cons
                                 int32_t* counts, int32_t* offsets, int32_t* perm,
                                 int32_t* inv_perm, const WsLayout& L, int32_t* gu_start,
                                 int32_t* dn_start, int32_t* ready, int32_t* nitems,
-                                const moe_weights* W, cudaStream_t s);
+                                const moe_weights* W, bool build_sched, cudaStream_t s);
 // Bytes of routed gate / up weights the decode front asks L2 for (about what
 // HBM delivers between the routing decision and the FFN's first loads): the
 // environment variable SGL_MOE_PREFETCH in MiB, 0 turning every prefetch of
@@ -178,6 +178,10 @@ struct GemmArgs {
   int32_t* err;
   int bn;
   int ffn;  // FfnKind
+  // nullable (narrow kernel): the expert counts [E] from which the FFN derives
+  // its work lists and row offsets itself, instead of reading gu_start /
+  // dn_start / offsets / nitems[0..1]
+  const int32_t* sched_counts;
   int max_items_gu;
   int max_items_dn;
   // MOE_W_MXFP4_A8: the MXFP4 codes are a.Wg/Wu/Wd (expert-major), read in place
