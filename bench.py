@@ -236,8 +236,8 @@ def roofline_entry(bytes_, flops, seconds, peaks, sustained=False, fp8_flops=0.0
 # Weight bytes dominate and scale with the experts touched, so the ratio
 # scales the counters to a full launch. Valid only for the ffn.cu they were
 # taken on: any other source reports traffic null.
-FFN_TRAFFIC_SOURCE_SHA256 = "d33a6269069f76958d4a7790d645868ac93165e48d69db81ea7357839416ce75"
-FFN_TRAFFIC_RATIO = {16: (424.91 + 4.68) / 424.82, 128: (781.17 + 50.85) / 760.2}
+FFN_TRAFFIC_SOURCE_SHA256 = "5184b92ea363796e235f0acb8543a7a1bf8b5a2169b71966f45a3ea4770576ce"
+FFN_TRAFFIC_RATIO = {16: (424.94 + 3.77) / 424.82, 128: (780.68 + 48.33) / 760.2}
 
 
 def ffn_tile_n(cfg) -> int:
