@@ -487,3 +487,24 @@ def test_prepared_block_scaled_full_size_sampled():
     check_y(bits(out["y"])[ref["tokens"][keep]], ref["y_f32"][keep], ref["y"][keep], tol=_tol(cfg))
     del d
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("T,E", [(16, 128), (32, 256)])
+def test_fused_front_without_shared_expert(T, E):
+    """Decode batch with no shared expert: the fused front routes and
+    permutes, and the FFN derives its work lists from the counts with no
+    shared slot; checked against the oracle with a zero shared expert."""
+    cfg = workloads.CONFIGS["decode"].with_(E=E, I_shared=0)
+    d = workloads.generate(cfg, DEV, T=T)
+    d.update(Wg_s=None, Wu_s=None, Wd_s=None)
+    g = run_layer(cfg, d)
+    h = host_inputs({**d, "Wg_s": torch.zeros(1, dtype=torch.bfloat16),
+                     "Wu_s": torch.zeros(1, dtype=torch.bfloat16),
+                     "Wd_s": torch.zeros(1, dtype=torch.bfloat16)})
+    z = np.zeros((64, cfg.H), np.uint16)
+    tok = list(range(min(T, 6)))
+    ref = oracle.layer_forward(cfg.with_(I_shared=64), h["x"], h["Wr"], h["bias"], DeviceExperts(d), z, z,
+                               z.T.copy(), tokens=tok)
+    near = check_routing(ref, g["idx"].cpu().numpy(), g["w"].cpu().numpy())
+    keep = ~np.isin(ref["tokens"], near)
+    check_y(bits(g["y"])[ref["tokens"][keep]], ref["y_f32"][keep], ref["y"][keep])
