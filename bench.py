@@ -236,7 +236,7 @@ def roofline_entry(bytes_, flops, seconds, peaks, sustained=False, fp8_flops=0.0
 # Weight bytes dominate and scale with the experts touched, so the ratio
 # scales the counters to a full launch. Valid only for the ffn.cu they were
 # taken on: any other source reports traffic null.
-FFN_TRAFFIC_SOURCE_SHA256 = "5184b92ea363796e235f0acb8543a7a1bf8b5a2169b71966f45a3ea4770576ce"
+FFN_TRAFFIC_SOURCE_SHA256 = "818ebd24c8f7c68dfaf7bd5aef21b8c5f3ce2a25f63a82994be6053fbb104ba0"
 FFN_TRAFFIC_RATIO = {16: (424.94 + 3.77) / 424.82, 128: (780.68 + 48.33) / 760.2}
 
 

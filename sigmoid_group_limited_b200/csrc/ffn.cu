@@ -19,6 +19,10 @@
 //       epilogue y_slot[j] = w_j * D (fp32) at the row's flat slot index j.
 // Slot E is the shared expert: its rows are the T tokens, its weight 1.
 //
+// The work lists (per-slot item starts and row offsets) come from the
+// permutation kernels, or, after the fused decode front, are derived from the
+// expert counts in every CTA's prologue (the same values).
+//
 // Items are claimed dynamically from one global counter: gate/up items
 // [0, Ngu), then down items. A down item reads h rows that other CTAs' gate/up
 // epilogues wrote; those epilogues count finished tiles per (slot, row tile)
