@@ -65,3 +65,20 @@ def test_roofline_arithmetic():
     # the whole layer: 106.2 MFLOP per token in the experts (K routed + 1 shared)
     lb, lf = bench.algorithmic_work(cfg, 1, touched=8)["layer"]
     assert abs(lf - 106.17e6) / 106.17e6 < 1e-3
+
+
+def test_block_scaled_formats_in_bench_accounting():
+    """The prepared block-scaled format counts the same work as the per-call
+    one (only where the scale atoms come from differs), two fewer launches,
+    and every weight format has a dtype label."""
+    import bench
+    a8 = workloads.CONFIGS["mxfp4_a8"]
+    a8p = workloads.CONFIGS["mxfp4_a8p"]
+    assert a8p.wfmt == workloads.MOE_W_MXFP4_A8P and a8p.with_(wfmt=a8.wfmt, name=a8.name) == a8
+    assert bench.algorithmic_work(a8, a8.T, 131) == bench.algorithmic_work(a8p, a8p.T, 131)
+    assert bench.kernels_per_step(a8) - bench.kernels_per_step(a8p) == 2
+    for fmt in (workloads.MOE_W_BF16, workloads.MOE_W_MXFP4, workloads.MOE_W_MXFP4_A8,
+                workloads.MOE_W_MXFP4_A8P):
+        assert fmt in bench.DTYPES
+    # decode batches take the fused front: front, FFN, combine
+    assert bench.kernels_per_step(workloads.CONFIGS["decode"]) == 3
