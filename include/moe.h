@@ -133,8 +133,13 @@ MOE_API moe_status moe_route(const moe_cfg* cfg, int32_t T, const void* x, const
                      const float* bias, int32_t* idx, float* w, void* ws, size_t ws_bytes,
                      void* stream);
 
-/* Stage 6, permutation: stable counting sort of the flat slots j = t*K + k by
- * expert (order inside an expert = ascending j), deterministic.
+/* Stage 6, permutation (page "Ling-3.0-flash-VL MoE sparse routing", sec. 1:
+ * the router picks a few experts for every token, and each expert then works
+ * on the tokens routed to it; page at 2kiu.com/news/4837473 on the sparse
+ * activation of Ling-3.0-flash-VL, sec. 4: the compute fans out from the
+ * router into 8 expert branches per token). The rows routed to each expert
+ * are grouped together: a stable counting sort of the flat slots
+ * j = t*K + k by expert (order inside an expert = ascending j), deterministic.
  * in: idx [T,K] int32; out: counts [E], offsets [E+1] (exclusive prefix sum),
  * perm [T*K] (sorted position -> slot j), inv_perm [T*K] (slot -> position).
  * inv_perm may be NULL. All device. An id outside [0,E) sets the error word. */
@@ -143,21 +148,21 @@ MOE_API moe_status moe_permute(const moe_cfg* cfg, int32_t T, const int32_t* idx
                        size_t ws_bytes, void* stream);
 
 /* moe_permute without a workspace, for callers that cannot allocate device
- * memory: code that runs where cudaMalloc is not allowed or not available
- * (inside a region being captured into a CUDA graph, a plugin whose host
- * framework owns all device memory and hands out no workspace, a real-time
- * loop that must not allocate). The pages describe no such call; it exists
- * only for those callers. Same inputs, outputs and results as moe_permute
- * (all device pointers, owned by the caller).
+ * memory: a plugin whose host framework owns all device memory and hands out
+ * no workspace, or a real-time loop or embedded runtime that must not
+ * allocate once it runs. The pages describe no such call; it exists only for
+ * those callers. Same inputs, outputs and results as moe_permute (all device
+ * pointers, owned by the caller).
  * Scratch: a fixed array inside the library, 256.25 KiB per device, held by
  * every GPU that loads the library until the process exits. Limits:
  * T*K <= 65536 and E <= 1024, else MOE_ERR_WORKSPACE and nothing runs.
- * The first call on a device looks the array's address up (once per
- * device, with that device current): make that first call before any
- * stream capture. All calls share the array, so calls that overlap on the
- * GPU (other streams, other threads) race: serialise them. Expert ids
- * outside [0,E) are dropped as in moe_permute; there is no error word to
- * read back. Allocates nothing (no cudaMalloc, no cudaFree). */
+ * The first call in a CUDA context looks the array's address up (once per
+ * context, with that context current; a device reset or another context on
+ * the device gets a fresh lookup): make that first call before any stream
+ * capture. All calls share the array, so calls that overlap on the GPU (other
+ * streams, other threads) race: serialise them. Expert ids outside [0,E) are
+ * dropped as in moe_permute; there is no error word to read back. Allocates
+ * nothing (no cudaMalloc, no cudaFree). */
 MOE_API moe_status moe_permute_static(const moe_cfg* cfg, int32_t T, const int32_t* idx,
                                       int32_t* counts, int32_t* offsets, int32_t* perm,
                                       int32_t* inv_perm, void* stream);
@@ -173,7 +178,11 @@ MOE_API moe_status moe_grouped_swiglu(const moe_cfg* cfg, int32_t T, const void*
                               const int32_t* offsets, const float* w, const moe_weights* W,
                               void* y_slot, void* ws, size_t ws_bytes, void* stream);
 
-/* Stage 9, weighted combine back to token order:
+/* Stage 9, weighted combine back to token order (page at
+ * 2kiu.com/news/4837473 on the sparse activation of Ling-3.0-flash-VL,
+ * sec. 4: the 8 expert branches' outputs are aggregated before the next
+ * layer; page "Ling-3.0-flash-VL MoE sparse routing", sec. 2: the shared
+ * expert's output is added for every token):
  * y[t] = bf16( (sum over k = 0..K-1 of y_slot[t*K+k]) + y_slot[T*K+t] ),
  * summed in fp32 in slot order; the shared row is added only when
  * with_shared != 0. y_slot (fp32) as produced by moe_grouped_swiglu;

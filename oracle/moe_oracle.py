@@ -45,7 +45,7 @@ Readings where the pages are silent (each also listed in the design notes):
      expert = ascending flat index j = t*K + k (stable counting sort).
   R9 MXFP4 weights are used through their exact dequantised values
      (e2m1 magnitude * sign * 2^(scale - 127)).
-  R10 block-scaled variant (weight format MXFP4_A8): the spec table of [P4]
+  R15 block-scaled variant (weight format MXFP4_A8): the spec table of [P4]
      lists the quantisation scheme as FP8 + MXFP4. It is read as MXFP8
      activations (OCP Microscaling v1.0: e4m3 elements, one e8m0 scale per
      32 consecutive elements along the contraction) for the routed experts:
@@ -111,7 +111,7 @@ def mxfp4_dequantize(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
 
 
 E4M3_MAX = 448.0
-MOE_W_MXFP4_A8 = 2   # weight-format code of the block-scaled variant (R10)
+MOE_W_MXFP4_A8 = 2   # weight-format code of the block-scaled variant (R15)
 
 
 def e4m3_decode(codes: np.ndarray) -> np.ndarray:
@@ -134,7 +134,7 @@ _E4M3_POS = e4m3_decode(np.arange(0x7F, dtype=np.uint8))
 
 def e4m3_encode(v: np.ndarray) -> np.ndarray:
     """Nearest e4m3 code to each finite float64 value, ties to the even code
-    (mantissa bit 0 clear), magnitudes above 448 saturate to 448 (R10); the
+    (mantissa bit 0 clear), magnitudes above 448 saturate to 448 (R15); the
     sign bit is the input's, also when the magnitude rounds to zero."""
     v = np.asarray(v, dtype=np.float64)
     a = np.minimum(np.abs(v), E4M3_MAX)
@@ -148,7 +148,7 @@ def e4m3_encode(v: np.ndarray) -> np.ndarray:
 
 
 def mxfp8_quantize(v: np.ndarray):
-    """MXFP8 (e4m3 elements, e8m0 scale per 32 along the last axis), R10.
+    """MXFP8 (e4m3 elements, e8m0 scale per 32 along the last axis), R15.
 
     v [..., K] float (K a multiple of 32) -> (codes uint8 [..., K],
     scales uint8 [..., K/32])."""
@@ -316,7 +316,7 @@ def swiglu_expert(x64: np.ndarray, Wg64: np.ndarray, Wu64: np.ndarray, Wd64: np.
 
     g = x Wg^T, u = x Wu^T (fp32 results); with a limit L > 0 both are clamped
     to [-L, L] (R6); h = fp32(silu(g) * u), silu(g) = g / (1 + e^-g), rounded
-    to bf16 (R7) or, with h_mxfp8, quantised to MXFP8 along I (R10);
+    to bf16 (R7) or, with h_mxfp8, quantised to MXFP8 along I (R15);
     o = h Wd^T (fp32).  Returns (o fp32 [n,H_out], h): h as bf16 bits [n,I],
     or with h_mxfp8 the pair (codes [n,I], scales [n,I/32])."""
     g = (x64 @ Wg64.T).astype(np.float32)
@@ -373,7 +373,7 @@ def layer_forward(cfg, x_bits: np.ndarray, Wr: np.ndarray, bias: np.ndarray,
     x64 = bf16_bits_to_f64(x_bits[tok])
     n, K, H = tok.size, cfg.K, cfg.H
     act_mx = getattr(cfg, "wfmt", 0) == MOE_W_MXFP4_A8
-    # R10: the routed experts see x through its MXFP8 values
+    # R15: the routed experts see x through its MXFP8 values
     xr64 = mxfp8_dequantize(*mxfp8_quantize(x64)) if act_mx else x64
     y_slot = np.zeros((n, K, H), dtype=np.float32)
     idx = r["idx"][tok]

@@ -12,6 +12,7 @@
 //                tile) bases, and the GEMM work lists,
 //   perm_scatter per tile: stable ranks from warp match/ballot in flat order,
 //                then perm / inv_perm.
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -248,21 +249,51 @@ constexpr int kStaticScratchHead = 64;
 constexpr int kStaticScratchInts =
     kStaticScratchHead + 2 * kStaticMaxExperts * (kStaticMaxSlots / kPermTile);
 static __device__ __align__(256) int32_t g_permute_scratch[kStaticScratchInts];
+// moe_permute_static accepts any E that the configuration check accepts
+static_assert(kStaticMaxExperts >= kMaxExpertsCfg, "static scratch smaller than the largest E");
 
-// Device address of g_permute_scratch on the current device, looked up once
-// per device (with that device current) and cached; nullptr on failure.
+// Device address of g_permute_scratch in the calling thread's current CUDA
+// context, looked up once per context (with that context current) and cached
+// under the context handle, so a device reset or another context on the same
+// device gets its own lookup; nullptr on failure.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+static CUcontext current_context() {
+  static const CtxGetCurrentFn fn = [] {  // the driver's function, found once (thread-safe)
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<CtxGetCurrentFn>(nullptr);
+    return reinterpret_cast<CtxGetCurrentFn>(f);
+  }();
+  CUcontext ctx = nullptr;
+  if (fn == nullptr || fn(&ctx) != CUDA_SUCCESS) return nullptr;
+  return ctx;
+}
+
 static int32_t* static_scratch_address() {
   static std::mutex mu;
+  static CUcontext ctx_of[kMaxDevices] = {};
   static int32_t* addr[kMaxDevices] = {};
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
-    void* p = nullptr;
+  static int used = 0;
+  void* p = nullptr;
+  CUcontext ctx = current_context();
+  if (ctx == nullptr) {
+    // no context bound to this thread yet: the runtime binds the current
+    // device's primary context on this first call
     if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess) return nullptr;
-    addr[dev] = static_cast<int32_t*>(p);
+    ctx = current_context();
+    if (ctx == nullptr) return nullptr;
   }
-  return addr[dev];
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < used; ++i)
+    if (ctx_of[i] == ctx) return addr[i];
+  if (p == nullptr && cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess) return nullptr;
+  const int slot = used < kMaxDevices ? used++ : kMaxDevices - 1;  // keep the newest when full
+  ctx_of[slot] = ctx;
+  addr[slot] = static_cast<int32_t*>(p);
+  return addr[slot];
 }
 
 cudaError_t launch_permute_static(const moe_cfg& c, int T, const int32_t* idx, int32_t* counts,

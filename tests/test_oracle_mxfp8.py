@@ -1,8 +1,9 @@
-"""Pins for the oracle's MXFP8 activation quantisation (reading R10 of the
+"""Pins for the oracle's MXFP8 activation quantisation (reading R15 of the
 block-scaled variant: OCP Microscaling v1.0, e4m3 elements, e8m0 scale per 32
 along the contraction). Each check is against the format's definition, brute
 force over all codes, or a closed form, never a retyped formula."""
 import math
+import struct
 
 import numpy as np
 import pytest
@@ -126,7 +127,7 @@ def test_mxfp8_blocks_follow_the_last_axis():
 
 
 def test_block_scaled_layer_close_to_bf16_layer():
-    """R10 changes only the routed activations' rounding: on the tiny
+    """R15 changes only the routed activations' rounding: on the tiny
     block-scaled config the output stays close to the same layer with bf16
     activations (e4m3 keeps 3 mantissa bits: a relative rounding error of at
     most 2^-4 per element, a few percent of RMS after the dot products) and
@@ -143,3 +144,102 @@ def test_block_scaled_layer_close_to_bf16_layer():
     rms = np.sqrt(np.mean(b16["y_f32"].astype(np.float64) ** 2))
     assert 0 < np.abs(diff).max() < 0.4 * rms
     assert np.sqrt(np.mean(diff.astype(np.float64) ** 2)) < 0.08 * rms
+
+
+# ---------------------------------------------------------------- one token, pure Python
+
+def _py_e4m3_values():
+    """(code, value) of the 127 non-negative finite e4m3 codes from the bit
+    fields: exponent bits 6..3 (bias 7), mantissa bits 2..0, exponent 0
+    subnormal."""
+    out = []
+    for c in range(0x7F):
+        e, m = c >> 3, c & 7
+        out.append((c, (m / 8.0) * 2.0 ** -6 if e == 0 else (1.0 + m / 8.0) * 2.0 ** (e - 7)))
+    return out
+
+
+_PY_E4M3 = _py_e4m3_values()
+
+
+def _py_mx_block(vals):
+    """MXFP8 value of each element of one 32-element block (R15), by linear
+    search over the e4m3 values: scale 2^(floor(log2 amax) - 8) with its byte
+    clamped to [0, 254]; nearest value, ties to the even code, saturation at
+    448; the sign kept."""
+    amax = max(abs(v) for v in vals)
+    if amax == 0.0:
+        byte = 0
+    else:
+        _, ex = math.frexp(amax)                 # amax = f * 2^ex, f in [0.5, 1)
+        byte = min(max(ex - 1 - 8 + 127, 0), 254)
+    X = 2.0 ** (byte - 127)
+    out = []
+    for v in vals:
+        a = min(abs(v) / X, 448.0)
+        best = None
+        for c, q in _PY_E4M3:
+            key = (abs(q - a), c & 1)            # nearer first, then the even code
+            if best is None or key < best[0]:
+                best = (key, q)
+        out.append(math.copysign(best[1] * X, v))
+    return out
+
+
+def _py_mx(row):
+    return [q for b in range(0, len(row), 32) for q in _py_mx_block(row[b:b + 32])]
+
+
+def _f32(v):
+    return struct.unpack("<f", struct.pack("<f", v))[0]
+
+
+def _py_bf16(v):
+    (u,) = struct.unpack("<I", struct.pack("<f", v))
+    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return struct.unpack("<f", struct.pack("<I", u << 16))[0]
+
+
+def _py_swiglu(xrow, Wg, Wu, Wd, L, h_round):
+    I, H = Wg.shape
+    a = []
+    for i in range(I):
+        g = _f32(math.fsum(xrow[k] * Wg[i, k] for k in range(H)))
+        u = _f32(math.fsum(xrow[k] * Wu[i, k] for k in range(H)))
+        if L > 0:
+            g, u = min(max(g, -L), L), min(max(u, -L), L)
+        a.append(_f32(g / (1.0 + math.exp(-g)) * u))
+    h = h_round(a)
+    return [_f32(math.fsum(h[i] * Wd[n, i] for i in range(I))) for n in range(Wd.shape[0])]
+
+
+@pytest.mark.parametrize("t", [5])
+def test_block_scaled_layer_one_token_pure_python(t):
+    """One token of the tiny block-scaled layer from explicit loops: x and the
+    fp32 h of every routed slot quantised to MXFP8 by linear search over the
+    e4m3 values, MXFP4 weights at their exact values, exact dot products
+    (fsum) rounded to fp32, y_slot = w * o, fp32 sum in slot order; the shared
+    expert on bf16 x with a bf16 h. Equal bit for bit to layer_forward."""
+    from helpers import experts_of, host_inputs
+    cfg = workloads.CONFIGS["tiny_a8"]
+    d = workloads.generate(cfg, "cpu", T=8)
+    h = host_inputs(d)
+    ex = experts_of(d)
+    out = oracle.layer_forward(cfg, h["x"], h["Wr"], h["bias"], ex, h["Wg_s"], h["Wu_s"], h["Wd_s"])
+    f = oracle.bf16_bits_to_f64
+    xr = f(h["x"][t]).tolist()
+    xq = _py_mx(xr)
+    assert xq != xr                                   # the quantisation changes x
+    acc = None
+    for k in range(cfg.K):
+        e = int(out["idx"][t, k])
+        Wg, Wu, Wd = ex(e)
+        o = _py_swiglu(xq, Wg, Wu, Wd, cfg.limit_routed, _py_mx)
+        wk = float(out["w"][t, k])
+        contrib = [_f32(wk * v) for v in o]
+        acc = contrib if acc is None else [_f32(a + c) for a, c in zip(acc, contrib)]
+    osh = _py_swiglu(xr, f(h["Wg_s"]), f(h["Wu_s"]), f(h["Wd_s"]), cfg.limit_shared,
+                     lambda a: [_py_bf16(v) for v in a])
+    y32 = [_f32(a + c) for a, c in zip(acc, osh)]
+    assert np.array_equal(out["y_f32"][t], np.array(y32, np.float32))
+    assert np.array_equal(f(out["y"][t]), np.array([_py_bf16(v) for v in y32]))

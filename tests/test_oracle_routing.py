@@ -208,6 +208,53 @@ def test_hand_worked_example():
     assert list(idx[0]) == [int(v) for v in g["idx"].split()]
     w = oracle.combine_weights(s, idx, 2.5, True)
     assert np.allclose(w[0], [float(v) for v in g["w"].split()], rtol=0, atol=1e-7)
+    _, gm, em = oracle.group_limited_topk(b, int(g["n_group"]), int(g["topk_group"]), int(g["K"]))
+    assert gm[0] == float(g["gmargin"]) and em[0] == float(g["emargin"])
+
+
+def test_hand_worked_margins():
+    """Both near-tie margins nonzero and distinct, worked out on paper; a margin
+    taken one rank too early, or over all experts instead of the kept groups'
+    candidates, gives another value (the fixture lists them)."""
+    g = _read_fixture("routing_hand_margins.txt")
+    s = np.array([[float(v) for v in g["s"].split()]], np.float32)
+    bias = np.array([float(v) for v in g["bias"].split()], np.float32)
+    b = oracle.biased_scores(s, bias)
+    idx, gm, em = oracle.group_limited_topk(b, int(g["n_group"]), int(g["topk_group"]), int(g["K"]))
+    assert list(idx[0]) == [int(v) for v in g["idx"].split()]
+    assert gm[0] == float(g["gmargin"]) and em[0] == float(g["emargin"])
+    w = oracle.combine_weights(s, idx, 2.5, True)
+    assert np.allclose(w[0], [float(v) for v in g["w"].split()], rtol=0, atol=1e-7)
+
+
+def _py_margins(row, n_group, topk_group, K):
+    """The two margins from plain sorted Python lists: groups by (max desc,
+    index asc), candidates = experts of the kept groups by (b desc, e asc)."""
+    E = len(row)
+    per = E // n_group
+    gs = [max(float(row[e]) for e in range(g * per, (g + 1) * per)) for g in range(n_group)]
+    order = sorted(range(n_group), key=lambda g: (-gs[g], g))
+    kept = set(order[:topk_group])
+    gm = gs[order[topk_group - 1]] - gs[order[topk_group]] if topk_group < n_group else math.inf
+    cands = sorted((e for e in range(E) if e // per in kept), key=lambda e: (-float(row[e]), e))
+    em = float(row[cands[K - 1]]) - float(row[cands[K]]) if K < len(cands) else math.inf
+    return gm, em
+
+
+@pytest.mark.parametrize("n_group,topk_group,K,E", [(4, 2, 4, 32), (8, 4, 8, 512), (8, 4, 3, 64),
+                                                    (4, 4, 4, 32), (8, 1, 8, 64)])
+def test_margins_brute_force(n_group, topk_group, K, E):
+    rng = np.random.default_rng(E + 7 * K + topk_group)
+    T = 120
+    b = rng.normal(scale=0.3, size=(T, E)).astype(np.float32)
+    per = E // n_group
+    b[::5, :per] = b[::5, per:2 * per]                  # tied groups
+    b[1::7, 3] = b[1::7, 5]                             # tied experts
+    b[2::9] = np.round(b[2::9] * 8) / 8                 # many exact ties at once
+    _, gm, em = oracle.group_limited_topk(b, n_group, topk_group, K)
+    for t in range(T):
+        g_ref, e_ref = _py_margins(b[t], n_group, topk_group, K)
+        assert gm[t] == g_ref and em[t] == e_ref
 
 
 # ---------------------------------------------------------------- weights and invariants

@@ -1,8 +1,9 @@
 """moe_permute_static: the permutation for callers that cannot allocate device
-memory (for example code running while a CUDA graph is being captured, or a
-plugin whose host framework owns all device memory and offers no workspace).
-Its scratch lives in a fixed array inside the library instead of a
-caller-provided workspace. It must give exactly what moe_permute gives.
+memory (for example a plugin whose host framework owns all device memory and
+offers no workspace, or a real-time loop that must not allocate). Its scratch
+lives in a fixed array inside the library instead of a caller-provided
+workspace. It must give exactly what moe_permute gives, and what the oracle's
+stable counting sort gives.
 
 This file is collected last on purpose: if it fails, a run that stops at the
 first failure has already run every other test.
@@ -13,16 +14,17 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import sigmoid_group_limited_b200 as sgl
 import workloads
 
 CFG = workloads.CONFIGS["prefill"]   # 512 experts, 8 groups, K = 8
 
 
-def _outputs(T, fill):
-    n = T * CFG.K
+def _outputs(T, fill, cfg=CFG):
+    n = T * cfg.K
     return [torch.full((m,), fill, dtype=torch.int32, device="cuda")
-            for m in (CFG.E, CFG.E + 1, n, n)]
+            for m in (cfg.E, cfg.E + 1, n, n)]
 
 
 @pytest.mark.gpu
@@ -45,6 +47,30 @@ def test_static_permutation_equals_workspace_permutation_twice():
             assert torch.equal(r, o)
         counts = np.bincount(idx.cpu().numpy().reshape(-1), minlength=CFG.E)
         assert np.array_equal(got[0].cpu().numpy(), counts)
+        for o, r in zip(got, oracle.permute(idx.cpu().numpy(), CFG.E)):
+            assert np.array_equal(o.cpu().numpy(), r)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("E", [512, 1024])
+def test_static_permutation_at_its_size_limit(E):
+    """T*K = 65536 slots (the largest the scratch takes) with 512 and 1024
+    experts: every per-(expert, tile) count and base of the scratch is used."""
+    cfg = CFG.with_(E=E)
+    T = 65536 // cfg.K
+    g = torch.Generator().manual_seed(E)
+    idx = torch.randint(0, E, (T, cfg.K), generator=g, dtype=torch.int32)
+    idx[: T // 2, 0] = E - 1                          # one heavy expert at the top of the range
+    idx = idx.cuda()
+    ws = sgl.alloc_workspace(cfg, T)
+    ref = _outputs(T, -1, cfg)
+    sgl.moe_permute(cfg, T, idx, *ref, ws)
+    got = _outputs(T, -7, cfg)
+    sgl.moe_permute_static(cfg, T, idx, *got)
+    torch.cuda.synchronize()
+    for r, o, p in zip(ref, got, oracle.permute(idx.cpu().numpy(), E)):
+        assert torch.equal(r, o)
+        assert np.array_equal(o.cpu().numpy(), p)
 
 
 def test_static_permutation_rejects_sizes_beyond_its_scratch():

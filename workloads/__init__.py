@@ -22,6 +22,7 @@ from __future__ import annotations
 
 import dataclasses
 import math
+import os
 from typing import Dict, Optional
 
 import torch
@@ -51,8 +52,8 @@ class MoEConfig:
     seed: int = 0
     bias_kind: str = "normal"   # "normal" (N(0, bias_var)), "zero", "zipf"
     bias_var: float = 0.1
-    zipf_s: float = 1.1
-    zipf_beta: float = 0.1
+    zipf_s: float = 1.1         # target popularity law p(r) ~ r^-zipf_s inside each group
+    zipf_beta: float = 0.1      # fixed-formula bias scale (groups without a calibrated table)
 
     def with_(self, **kw) -> "MoEConfig":
         return dataclasses.replace(self, **kw)
@@ -125,14 +126,48 @@ def _bf16(shape, var, g, device, chunk_rows=0) -> torch.Tensor:
     return out
 
 
+ZIPF_TABLE = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "tests",
+                          "golden", "zipf_bias_g64.txt")
+
+
+def zipf_ranks(cfg: MoEConfig):
+    """Within-group popularity rank r = 1..E/G of every expert (int64 [E]):
+    a seeded permutation per group (rank 1 = the most favoured expert)."""
+    import numpy as np
+    per = cfg.experts_per_group
+    gcpu = _gen("cpu", cfg.seed * 16 + 2)
+    ranks = np.empty(cfg.E, dtype=np.int64)
+    for grp in range(cfg.n_group):
+        ranks[grp * per:(grp + 1) * per] = torch.randperm(per, generator=gcpu).numpy() + 1
+    return ranks
+
+
+def zipf_table(per: int):
+    """Calibrated bias per rank (fp32 [per]) from tests/golden/zipf_bias_g64.txt
+    (written by make_zipf_bias.py there), or None when the table is for
+    another group size."""
+    import numpy as np
+    rows = []
+    with open(ZIPF_TABLE) as f:
+        for line in f:
+            line = line.split("#", 1)[0].split()
+            if line:
+                rows.append(int(line[1], 16))
+    if len(rows) != per:
+        return None
+    return np.array(rows, dtype=np.uint32).view(np.float32)
+
+
 def selection_bias(cfg: MoEConfig, device="cpu") -> torch.Tensor:
     """Per-expert additive selection bias [E] fp32.
 
-    normal: N(0, bias_var). zero: all 0. zipf: inside every group a seeded
-    permutation assigns popularity ranks r = 1..E/G and
-    bias_e = -beta * s * ln(r_e), so that rank 1 is the most favoured expert of
-    its group (the pages' balancing bias lowers hot experts and raises cold ones;
-    here it is set to make loads skewed on purpose).
+    normal: N(0, bias_var). zero: all 0. zipf: every expert gets the bias of
+    its within-group popularity rank (zipf_ranks). With 64 experts per group
+    the values per rank are the stored calibration of
+    tests/golden/zipf_bias_g64.txt, which makes expert popularity inside each
+    group follow p(r) ~ r^-1.1; other group sizes (the small test layers) use
+    the fixed formula bias = -zipf_beta * zipf_s * ln(r), which is skewed but
+    not calibrated.
     """
     g = _gen(device, cfg.seed * 16 + 2)
     if cfg.bias_kind == "zero":
@@ -140,14 +175,23 @@ def selection_bias(cfg: MoEConfig, device="cpu") -> torch.Tensor:
     if cfg.bias_kind == "normal":
         return _normal((cfg.E,), cfg.bias_var, g, device)
     if cfg.bias_kind == "zipf":
-        per = cfg.experts_per_group
-        gcpu = _gen("cpu", cfg.seed * 16 + 2)
-        ranks = torch.empty(cfg.E, dtype=torch.float64)
-        for grp in range(cfg.n_group):
-            ranks[grp * per:(grp + 1) * per] = torch.randperm(per, generator=gcpu).double() + 1.0
-        b = -cfg.zipf_beta * cfg.zipf_s * torch.log(ranks)
+        ranks = zipf_ranks(cfg)
+        table = zipf_table(cfg.experts_per_group)
+        if table is not None:
+            return torch.from_numpy(table[ranks - 1].copy()).to(device)
+        b = -cfg.zipf_beta * cfg.zipf_s * torch.log(torch.from_numpy(ranks).double())
         return b.to(torch.float32).to(device)
     raise ValueError(f"unknown bias_kind {cfg.bias_kind}")
+
+
+def router_inputs(cfg: MoEConfig, device="cpu", T: Optional[int] = None) -> Dict[str, torch.Tensor]:
+    """x, Wr and bias of `cfg` alone (the same draws as generate(), without the
+    expert weights)."""
+    T = cfg.T if T is None else T
+    s = cfg.seed * 16
+    return {"x": _bf16((T, cfg.H), 1.0, _gen(device, s + 0), device, chunk_rows=8192),
+            "Wr": _normal((cfg.E, cfg.H), 1.0 / cfg.H, _gen(device, s + 1), device),
+            "bias": selection_bias(cfg, device)}
 
 
 def generate(cfg: MoEConfig, device="cpu", T: Optional[int] = None) -> Dict[str, torch.Tensor]:
