@@ -205,19 +205,31 @@ def algorithmic_work(cfg, T: int, touched: int):
                 layer=(layer_bytes, layer_flops), router_flops=2.0 * T * H * E)
 
 
-# the nominal dense fp8 / bf16 tensor ratio (4.5 / 2.25 PFLOP/s): the block-scaled
-# MXFP8 x MXFP4 flops are credited at the measured bf16 peak times this
-FP8_OVER_BF16 = 2.0
+# the nominal dense fp8 / bf16 and fp4 / bf16 tensor ratios (4.5 and 9 against
+# 2.25 PFLOP/s): used only when the tensor-core probe cannot run
+FP8_OVER_BF16_NOMINAL = 2.0
+FP4_OVER_BF16_NOMINAL = 4.0
 
 
-def roofline_entry(bytes_, flops, seconds, peaks, sustained=False, fp8_flops=0.0):
-    """fp8_flops: the part of `flops` that runs block-scaled 8-bit (its peak
-    is FP8_OVER_BF16 x the bf16 one); the entry's peak is then the effective
-    rate of the mix, flops / (bf16 time + fp8 time)."""
+def tensor_ratios(probe) -> dict:
+    """Block-scaled / bf16 instruction-throughput ratios from the probe
+    (sigmoid_group_limited_b200.peak), else the nominal ones."""
+    if probe:
+        b = probe["bf16"]["tflops"]
+        return {"fp8": probe["e2m1xe4m3"]["tflops"] / b, "fp4": probe["e2m1xe2m1"]["tflops"] / b,
+                "source": "measured (tcgen05 probe on this GPU)"}
+    return {"fp8": FP8_OVER_BF16_NOMINAL, "fp4": FP4_OVER_BF16_NOMINAL, "source": "nominal"}
+
+
+def roofline_entry(bytes_, flops, seconds, peaks, sustained=False, fp8_flops=0.0, fp8_ratio=None):
+    """fp8_flops: the part of `flops` that runs block-scaled 8-bit, whose peak
+    is fp8_ratio x the bf16 one; the entry's peak is then the effective rate of
+    the mix, flops / (bf16 time + fp8 time)."""
+    ratio = FP8_OVER_BF16_NOMINAL if fp8_ratio is None else fp8_ratio
     tp = (peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]) * 1e12
     bw = peaks["hbm_gbs"] * 1e9
     t_mem = bytes_ / bw
-    t_tc = (flops - fp8_flops) / tp + fp8_flops / (FP8_OVER_BF16 * tp)
+    t_tc = (flops - fp8_flops) / tp + fp8_flops / (ratio * tp)
     tp = flops / t_tc if t_tc > 0 else tp
     if t_mem >= t_tc:
         ach = bytes_ / seconds / 1e9
@@ -259,6 +271,35 @@ def ffn_traffic(cfg, algorithmic_bytes: float):
     if digest != FFN_TRAFFIC_SOURCE_SHA256 or ratio is None or cfg.wfmt != workloads.MOE_W_BF16:
         return None
     return round(ratio * algorithmic_bytes)
+
+
+def popularity_slope(cfg, counts) -> float:
+    """Slope of ln(mean expert count per within-group popularity rank) against
+    ln(rank) (a Zipf law p(r) ~ r^-s has slope -s); ranks with no slot are
+    left out of the fit."""
+    ranks = workloads.zipf_ranks(cfg)
+    per = cfg.experts_per_group
+    m = np.array([counts[ranks == r].mean() for r in range(1, per + 1)], dtype=np.float64)
+    ok = m > 0
+    return float(np.polyfit(np.log(np.arange(1, per + 1)[ok]), np.log(m[ok]), 1)[0])
+
+
+def front_prefetch_bytes(cfg, touched: int) -> int:
+    """Bytes of FFN weights the fused decode front asks L2 for before the FFN
+    starts (its rule: the shared expert's three matrices, then the gate and up
+    matrices of the first touched experts, as many whole experts as fit the
+    budget SGL_MOE_PREFETCH MiB, 32 when unset); 0 when the front is not used."""
+    if not fused_front(cfg):
+        return 0
+    v = os.environ.get("SGL_MOE_PREFETCH")
+    budget = (32 << 20) if not v else max(0, int(v)) << 20
+    if budget == 0:
+        return 0
+    shared = 3 * cfg.I_shared * cfg.H * 2
+    if cfg.wfmt != workloads.MOE_W_BF16:
+        return shared
+    gu = 2 * cfg.I * cfg.H * 2
+    return shared + min(touched, budget // gu, 33) * gu
 
 
 # ------------------------------------------------------------------ GPU arm
@@ -385,6 +426,7 @@ def measure_gpu(cfg, steps, warmup, device, rank, clk, with_e2e=True):
     rstats = torch.empty(sgl.MOE_N_ROUTE_STATS, dtype=torch.float64, device=device)
     sgl.moe_route_stats(cfg, counts, rstats, stream=stream)
     st = dict(zip(sgl.ROUTE_STATS_NAMES, rstats.cpu().tolist()))
+    slope = popularity_slope(cfg, counts.cpu().numpy()) if cfg.bias_kind == "zipf" else None
     out = dict(device_ms_total=dev_ms, plain_ms_total=sum(per_step_plain), wall_s=wall,
                per_step_ms=per_step, stage_ms=stage_ms,
                routing={"experts_touched": cfg.E - int(st["idle_experts"]),
@@ -392,7 +434,12 @@ def measure_gpu(cfg, steps, warmup, device, rank, clk, with_e2e=True):
                         "load_mean": round(st["load_mean"], 2),
                         "max_over_mean": round(st["max_over_mean"], 3),
                         "entropy_bits": round(st["entropy_bits"], 4),
-                        "entropy_normalized": round(st["entropy_normalized"], 4)},
+                        "entropy_normalized": round(st["entropy_normalized"], 4),
+                        **({"popularity_slope": round(slope, 3),
+                            "popularity_slope_fit": "least squares of ln(mean count per "
+                                                    "within-group rank) on ln(rank), ranks 1..E/G, "
+                                                    "from the library's expert counts; target -zipf_s"}
+                           if slope is not None else {})},
                d=d, launches=kernels_per_step(cfg) * 2 * steps)
 
     if with_e2e:
@@ -495,7 +542,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="decode", choices=sorted(workloads.CONFIGS))
-    ap.add_argument("--also", default="prefill,mxfp4_a8",
+    ap.add_argument("--also", default="prefill,prefill_bias0,zipf,mxfp4,mxfp4_a8",
                     help="further workloads for the line, comma-separated ('' = none)")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--oracle-tokens", type=int, default=8)
@@ -516,8 +563,24 @@ def workload_cfg(args):
     return cfg
 
 
+WORKLOAD_NOTES = {
+    "decode": "decode batch, bias N(0, 0.1) (memory-bound)",
+    "prefill": "prefill batch, bias N(0, 0.1): skewed loads, about 122 experts touched",
+    "prefill_bias0": "prefill batch with zero bias: near-uniform loads over all 512 experts "
+                     "(memory-bound: 6 GB of weights)",
+    "zipf": "skewed routing: bias calibrated so that expert popularity inside each group "
+            "follows p(r) ~ r^-1.1; SwiGLU limits 4 (routed) / 7 (shared)",
+    "mxfp4": "routed weights MXFP4 (e2m1 codes + e8m0 scale per 32); activations, router and "
+             "shared expert bf16/fp32",
+    "mxfp4_a8": "block-scaled variant: MXFP4 routed weights x MXFP8 routed activations "
+                "(narrower activation arithmetic than the bf16-activation mxfp4 workload)",
+    "mxfp4_a8p": "block-scaled variant with weight scales prepared once (load time)",
+}
+
+
 def config_block(cfg, world):
-    return {"workload": f"{cfg.name}: T={cfg.T} tokens per GPU, H={cfg.H}, E={cfg.E} experts "
+    return {"workload": f"{cfg.name} ({WORKLOAD_NOTES.get(cfg.name, 'custom')}): "
+                        f"T={cfg.T} tokens per GPU, H={cfg.H}, E={cfg.E} experts "
                         f"({cfg.n_group} groups keep {cfg.topk_group}, top-{cfg.K}), I={cfg.I}, "
                         f"shared I={cfg.I_shared}",
             "T": cfg.T, "H": cfg.H, "E": cfg.E, "n_group": cfg.n_group,
@@ -562,13 +625,23 @@ def run_native(args, rank, world, local):
     torch.cuda.set_device(device)
     peaks = load_peaks()
     cfg = workload_cfg(args)
+    # tensor-core instruction throughput per kind on this GPU (about a second)
+    try:
+        from sigmoid_group_limited_b200 import peak as tcprobe
+        probe = tcprobe.peaks(device)
+    except Exception as exc:  # the line then says the ratios are nominal
+        print(f"tensor-core probe unavailable: {exc}", file=sys.stderr)
+        probe = None
+    ratios = tensor_ratios(probe)
     with ClockSampler(device) as clk:
         m = measure_gpu(cfg, args.steps, args.warmup, device, rank, clk)
         also = []
         for name in [a for a in args.also.split(",") if a and a != args.workload]:
             acfg = workloads.CONFIGS[name]
-            also.append((acfg, measure_gpu(acfg, args.steps, args.warmup, device, rank, clk,
-                                           with_e2e=False)))
+            am = measure_gpu(acfg, args.steps, args.warmup, device, rank, clk, with_e2e=False)
+            am.pop("d")                          # free this workload's weights before the next
+            torch.cuda.empty_cache()
+            also.append((acfg, am))
     clocks = clk.summary()
     dev_s = reduce_max(m["device_ms_total"], device) / 1e3
     plain_s = reduce_max(m["plain_ms_total"], device) / 1e3
@@ -583,11 +656,12 @@ def run_native(args, rank, world, local):
         t_ffn = (mm["stage_ms"]["ffn"]) / 1e3
         mx = cfg_.wfmt in (workloads.MOE_W_MXFP4_A8, workloads.MOE_W_MXFP4_A8P)
         # block-scaled: the routed experts' flops run at the fp8 rate, the shared expert's at bf16
-        f8 = 2.0 * cfg_.T * cfg_.K * 3 * cfg_.H * cfg_.I if mx else 0.0
-        ent = roofline_entry(b, f, t_ffn, peaks, fp8_flops=f8)
+        f_routed = 2.0 * cfg_.T * cfg_.K * 3 * cfg_.H * cfg_.I
+        f8 = f_routed if mx else 0.0
+        ent = roofline_entry(b, f, t_ffn, peaks, fp8_flops=f8, fp8_ratio=ratios["fp8"])
         src = "HBM copy" if ent["bound"] == "hbm" else (
-            f"cuBLAS bf16 burst; routed MXFP8 x MXFP4 flops at {FP8_OVER_BF16:g} x that (nominal fp8/bf16 ratio)"
-            if mx else "cuBLAS bf16 burst")
+            f"cuBLAS bf16 burst; routed MXFP8 x MXFP4 flops at {ratios['fp8']:.3f} x that "
+            f"({ratios['source']} kind::mxf8f6f4 / kind::f16 ratio)" if mx else "cuBLAS bf16 burst")
         ent.update(kernel="moe_ffn_mx (block-scaled gate/up + down)" if mx else "moe_ffn (gate/up + down)",
                    traffic=ffn_traffic(cfg_, b),
                    traffic_unit="bytes per launch (ncu DRAM read+write, scaled from the "
@@ -596,9 +670,23 @@ def run_native(args, rank, world, local):
                    units_per_launch=f"{cfg_.T} tokens, {mm['routing']['experts_touched']} routed experts + shared")
         if mx:
             ent["time"] = "FFN stage events: scale atoms and MXFP8 x included"
+        if cfg_.wfmt != workloads.MOE_W_BF16:
+            # the routed flops against the dense FP4 peak (kind::mxf4, e2m1 x e2m1)
+            fp4_peak = peaks["bf16_tflops"] * ratios["fp4"]
+            ent["fp4_peak_tflops"] = round(fp4_peak, 1)
+            ent["frac_of_fp4_peak"] = round(f_routed / t_ffn / 1e12 / fp4_peak, 4)
+            ent["fp4_peak_source"] = f"cuBLAS bf16 burst x {ratios['fp4']:.3f} ({ratios['source']} " \
+                                     f"kind::mxf4 / kind::f16 ratio)"
+        pf = front_prefetch_bytes(cfg_, mm["routing"]["experts_touched"])
+        if ent["bound"] == "hbm" and pf > 0:
+            # the fused front asks L2 for these bytes while routing runs; net of
+            # them, the FFN's own HBM rate is
+            net = (b - pf) / t_ffn / 1e9
+            ent["l2_prefetched_bytes"] = pf
+            ent["frac_net_of_l2_prefetch"] = round(net / peaks["hbm_gbs"], 4)
         lb, lf = work["layer"]
         tp = peaks["bf16_tflops"] * 1e12
-        t_roof = max(lb / (peaks["hbm_gbs"] * 1e9), (lf - f8) / tp + f8 / (FP8_OVER_BF16 * tp))
+        t_roof = max(lb / (peaks["hbm_gbs"] * 1e9), (lf - f8) / tp + f8 / (ratios["fp8"] * tp))
         step_s = statistics.mean(mm["per_step_ms"]) / 1e3
         return ent, round(t_roof / step_s, 4)
 
@@ -616,7 +704,12 @@ def run_native(args, rank, world, local):
             "routing": m["routing"],
             "e2e": {"value": round(tokens / e2e_s, 1), "unit": "tokens/s",
                     "h2d_bytes_per_step": m["e2e_h2d"], "d2h_bytes_per_step": m["e2e_d2h"]},
-            "gpu_launches": m["launches"], "clocks": clocks}
+            "gpu_launches": m["launches"], "clocks": clocks,
+            "tensor_probe": ({k: {"tflops": round(v["tflops"], 1), "ns_per_mma": round(v["ns_per_mma"], 2),
+                                  "shape": f"M=128 N={v['N']} K={v['K']}, {v['chains']} accumulator(s)"}
+                              for k, v in probe.items()} if probe else None),
+            "tensor_ratios": {"fp8_over_bf16": round(ratios["fp8"], 4),
+                              "fp4_over_bf16": round(ratios["fp4"], 4), "source": ratios["source"]}}
     for acfg, am in also:
         a_s = reduce_max(am["device_ms_total"], device) / 1e3
         aent, afrac = roof(acfg, am)

@@ -55,6 +55,26 @@ def build(verbose: bool = False, force: bool = False) -> str:
     return LIB
 
 
+PEAK_SRC = os.path.join(PKG, "peak", "mma_peak.cu")
+PEAK_LIB = os.path.join(PKG, "peak", "libsgl_peak.so")
+
+
+def build_peak(force: bool = False) -> str:
+    """libsgl_peak.so: the tensor-core throughput probe (peak/mma_peak.cu)."""
+    if not force and os.path.exists(PEAK_LIB) and os.path.getmtime(PEAK_LIB) > os.path.getmtime(PEAK_SRC):
+        return PEAK_LIB
+    cmd = [nvcc(), "-O3", "-std=c++17", *ARCH, "-lineinfo", "-Xcompiler", "-fPIC", "-shared",
+           "-Xcompiler", "-fvisibility=hidden", "-o", PEAK_LIB + ".tmp", PEAK_SRC]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    if r.returncode != 0:
+        sys.stderr.write(r.stdout + r.stderr)
+        raise RuntimeError("nvcc failed (peak probe)")
+    os.replace(PEAK_LIB + ".tmp", PEAK_LIB)
+    return PEAK_LIB
+
+
 if __name__ == "__main__":
     build(verbose="--verbose" in sys.argv, force=True)
+    build_peak(force=True)
     print(LIB)
+    print(PEAK_LIB)

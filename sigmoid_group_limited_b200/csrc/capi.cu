@@ -53,6 +53,8 @@ WsLayout ws_layout(const moe_cfg& c, int T) {
     L.ffn = kFfnMx;
   } else {
     L.ffn = choose_ffn(T, c.K, c.E, &L.bn);
+    // MXFP4 weights are expanded by the one-CTA kernel only
+    if (c.wfmt == MOE_W_MXFP4 && L.ffn == kFfnPair) L.ffn = kFfnNarrow, L.bn = kTileN;
   }
   ffn_tiles(L.ffn, &L.gu_ft, &L.dn_ft);
   const int gu_ft = L.gu_ft, dn_ft = L.dn_ft;
@@ -106,16 +108,6 @@ WsLayout ws_layout(const moe_cfg& c, int T) {
       L.sf_u = take(atoms);
       L.sf_d = take(atoms);
     }
-  }
-  if (c.wfmt == MOE_W_MXFP4) {
-    L.max_touched = static_cast<int>(TK < static_cast<size_t>(c.E) ? TK : c.E);
-    const size_t mat = static_cast<size_t>(L.max_touched) * c.I * c.H * 2;
-    L.slot_of = take(static_cast<size_t>(c.E) * 4);
-    L.touched = take(static_cast<size_t>(c.E) * 4);
-    L.ntouched = take(16);
-    L.wq_g = take(mat);
-    L.wq_u = take(mat);
-    L.wq_d = take(mat);
   }
   L.total = o;
   return L;
@@ -194,9 +186,9 @@ moe_status check_weights(const moe_cfg* c, const moe_weights* W) {
   return MOE_OK;
 }
 
-// Stages 7-8 after the schedule: the weight-format preparation (MXFP4: the
-// touched experts' bf16 copies; MXFP4_A8: scale atoms and MXFP8 x), then the
-// expert FFN kernel of the format.
+// Stages 7-8 after the schedule: the weight-format preparation (MXFP4_A8:
+// scale atoms and MXFP8 x), then the expert FFN kernel of the format (MXFP4
+// weights are expanded to bf16 inside the FFN kernel).
 cudaError_t run_ffn(const moe_cfg* cfg, int T, const uint16_t* x, const int32_t* perm,
                     const int32_t* offsets, const float* w, const moe_weights* W, float* y_slot,
                     void* ws, const WsLayout& L, cudaStream_t s,
@@ -215,18 +207,6 @@ cudaError_t run_ffn(const moe_cfg* cfg, int T, const uint16_t* x, const int32_t*
   a.Wd = W->Wd;
   a.wslot = nullptr;
   a.wrows = cfg->E;
-  if (cfg->wfmt == MOE_W_MXFP4) {
-    cudaError_t e = launch_mxfp4_expand(*cfg, offsets, W, at<int32_t>(ws, L.slot_of),
-                                        at<int32_t>(ws, L.touched), at<int32_t>(ws, L.ntouched),
-                                        at<uint16_t>(ws, L.wq_g), at<uint16_t>(ws, L.wq_u),
-                                        at<uint16_t>(ws, L.wq_d), s);
-    if (e != cudaSuccess) return e;
-    a.Wg = at<uint16_t>(ws, L.wq_g);
-    a.Wu = at<uint16_t>(ws, L.wq_u);
-    a.Wd = at<uint16_t>(ws, L.wq_d);
-    a.wslot = at<int32_t>(ws, L.slot_of);
-    a.wrows = L.max_touched;
-  }
   a.h_r = at<uint16_t>(ws, L.h_r);
   a.h_s = at<uint16_t>(ws, L.h_s);
   a.y_slot = y_slot;

@@ -33,6 +33,14 @@ struct FfnParams {
   int32_t* err;
   const int32_t* sched_counts;  // nullable: derive the work lists from the expert counts
   int bn, gu_ft, dn_ft;         // token tile and output features per item (for that)
+  // MXFP4 routed weights (the expanding kernel): codes [E*rows, K/2] and e8m0
+  // scales [E*rows, K/32] of Wg, Wu (K = H) and Wd (K = I), expert-major
+  const uint8_t *q_g, *q_u, *q_d, *s_g, *s_u, *s_d;
+  // test hooks of the scheduler's wait (0 in normal use): its limit in cycles,
+  // and a count added to the tiles it waits for (one that is never reached
+  // makes the wait run out)
+  long long wait_limit;
+  int ready_extra;
 };
 
 // In-place exclusive scan of a[0..n) in shared memory by the whole CTA
@@ -137,14 +145,20 @@ __device__ __forceinline__ int ld_acquire(const int32_t* a) {
   return v;
 }
 
-// Bounded wait until *addr >= need (acquire), with mbar_wait's abort protocol.
+// Bounded wait of a scheduler until *addr >= need (acquire): the count of
+// gate/up tiles that other CTAs have published for a down item's row tile.
+// Gives up after `limit` cycles (kWaitLimitCycles when 0), or at once if the
+// CTA's abort flag is up. A timeout sets the error word but not the abort
+// flag: the scheduler then queues the end of its work, and every role of the
+// CTA finishes the items already queued and leaves, with no copy or MMA left
+// in flight.
 __device__ __forceinline__ bool wait_count(const int32_t* addr, int need, volatile int* abort_flag,
-                                           int* err) {
+                                           int* err, long long limit = 0) {
   const long long t0 = clock64();
+  const long long lim = limit > 0 ? limit : kWaitLimitCycles;
   while (ld_acquire(addr) < need) {
     if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitLimitCycles) {
-      *abort_flag = 1;
+    if (clock64() - t0 > lim) {
       atomicExch(err, MOE_DEVERR_TIMEOUT);
       return false;
     }

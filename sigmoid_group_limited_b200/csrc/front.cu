@@ -90,35 +90,6 @@ __device__ __forceinline__ void prefetch_range(const uint8_t* base, uint32_t byt
   }
 }
 
-__device__ __forceinline__ int ld_acquire_gpu(const int32_t* a) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
-  return v;
-}
-
-// Grid barrier n (1, 2, ...) on a monotonic counter; false if it timed out
-// (the error word is set; every CTA then leaves).
-__device__ bool grid_barrier(int32_t* bar, int n, int32_t* err) {
-  __shared__ int ok_s;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();  // this CTA's writes before its arrival
-    atomicAdd(bar, 1);
-    const int need = n * static_cast<int>(gridDim.x);
-    const long long t0 = clock64();
-    int ok = 1;
-    while (ld_acquire_gpu(bar) < need) {  // waits last a few microseconds: spin
-      if (clock64() - t0 > kWaitLimitCycles) {
-        atomicExch(err, MOE_DEVERR_TIMEOUT);
-        ok = 0;
-        break;
-      }
-    }
-    ok_s = ok;
-  }
-  __syncthreads();
-  return ok_s != 0;
-}
 
 template <int NG, int NV>
 __global__ void __launch_bounds__(kFrontThreads, 1) decode_front(const __grid_constant__ FrontParams p) {

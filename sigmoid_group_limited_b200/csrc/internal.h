@@ -88,8 +88,8 @@ constexpr int kCtrlBytes = 256;
 struct WsLayout {
   size_t z, unc, tile_hist, idx, w, counts, offsets, perm, inv_perm, gu_start, dn_start, ready, nitems, h_r,
       h_s, y_slot, err, total;
-  // MXFP4 routed weights only: touched-expert slots and their bf16 copies
-  size_t slot_of, touched, ntouched, wq_g, wq_u, wq_d;
+  // block-scaled format with per-call scale repack: touched-expert slots
+  size_t slot_of, touched, ntouched;
   // MOE_W_MXFP4_A8 only: MXFP8 x (codes [T,H], scales [T,H/32]); the scales
   // of h (codes reuse h_r) as 512-byte atoms per (row tile, 128-wide k-block);
   // the touched experts' weight scales as atoms per (128-row tile, k-block)
@@ -224,10 +224,6 @@ cudaError_t launch_mx_sf_atoms(const moe_cfg& c, const moe_weights* W, uint8_t* 
 cudaError_t launch_mxfp4_slots(const moe_cfg& c, const int32_t* offsets, int32_t* slot_of,
                                int32_t* touched, int32_t* ntouched, cudaStream_t s);
 
-// MXFP4: list the touched experts and dequantise each once into bf16 slots.
-cudaError_t launch_mxfp4_expand(const moe_cfg& c, const int32_t* offsets, const moe_weights* W,
-                                int32_t* slot_of, int32_t* touched, int32_t* ntouched,
-                                uint16_t* gout, uint16_t* uout, uint16_t* dout, cudaStream_t s);
 
 cudaError_t launch_combine(const moe_cfg& c, int T, const float* y_slot, int with_shared,
                            uint16_t* y, cudaStream_t s);
@@ -278,6 +274,10 @@ bool map_bf16(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uin
 // Row-major [rows, cols] bytes (e4m3 codes): box of box_rows x 128 bytes,
 // 128-byte swizzle.
 bool map_u8(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows);
+// Packed MXFP4 codes as bytes: [rows, row_bytes] uint8, box of 128 rows x 32
+// bytes (64 elements: one k-block), no swizzle (rows 32 bytes apart in
+// shared memory). Needs row_bytes % 32 == 0 and a 16-byte aligned base.
+bool map_codes(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t row_bytes);
 // MXFP4 codes [rows, cols/2] (cols 4-bit elements per row, two per byte):
 // box of box_rows x 128 elements, unpacked to one byte per element in shared
 // memory (16 elements per 16 bytes: 8 code bytes + 8 bytes of gap) with the

@@ -16,6 +16,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <string.h>
+
 #include <mutex>
 
 #include "internal.h"
@@ -203,6 +205,138 @@ __global__ void __launch_bounds__(1024) perm_single(int TK, int E, const int32_t
   perm_block(TK, E, idx, counts, offsets, perm, inv_perm, err, sa, build, whist);
 }
 
+// The permutation of batches that span several tiles, in one cooperative
+// launch of one CTA (1024 threads) per tile of kPermTile flat entries:
+//   phase 1  per-warp expert histograms of the tile's 32 contiguous chunks
+//            (shared memory), the tile's totals to tile_cnt [E][n_tiles];
+//   barrier  (bounded, on a counter that is zero at launch);
+//   phase 2  every CTA reads all tiles' counts, forms the per-expert totals,
+//            their exclusive scan (the offsets) and the counts of the tiles
+//            before its own, turns its warps' histograms into bases and
+//            places its entries in flat order: the same stable counting sort
+//            as the three-kernel form. CTA 0 writes counts, offsets and the
+//            FFN work lists.
+__global__ void __launch_bounds__(1024, 1) perm_fused(int TK, int E, int n_ptiles,
+                                                      const int32_t* __restrict__ idx,
+                                                      int32_t* __restrict__ tile_cnt,
+                                                      int32_t* __restrict__ counts,
+                                                      int32_t* __restrict__ offsets,
+                                                      int32_t* __restrict__ perm,
+                                                      int32_t* __restrict__ inv_perm,
+                                                      int32_t* __restrict__ bar, int32_t* __restrict__ err,
+                                                      SchedArgs sa, int build) {
+  pdl_trigger();
+  pdl_wait();  // inputs come from earlier kernels on the stream
+  extern __shared__ int whist[];  // [32 warps][E]
+  __shared__ int cnt[kMaxE + 1];
+  __shared__ int off[kMaxE + 1];
+  __shared__ int scratch[33];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int kWarps = 32, kChunk = kPermTile / kWarps;
+  const int tbase = blockIdx.x * kPermTile;
+  const int n = min(kPermTile, TK - tbase);
+  const int c0 = warp * kChunk, c1 = min(c0 + kChunk, n);
+  const unsigned lt = (1u << lane) - 1u;
+  int* wh = whist + warp * E;
+  for (int i = tid; i < kWarps * E; i += blockDim.x) whist[i] = 0;
+  __syncthreads();
+  // phase 1: this warp's per-expert counts of its chunk
+  for (int r = c0; r < c1; r += 32) {
+    const int i = r + lane;
+    int e = -1;
+    if (i < c1) {
+      e = idx[tbase + i];
+      if (e < 0 || e >= E) {
+        atomicExch(err, MOE_DEVERR_EXPERT_ID);
+        e = -1;
+      }
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && (peers & lt) == 0) wh[e] += __popc(peers);
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x) {
+    int tot = 0;
+    for (int w = 0; w < kWarps; ++w) tot += whist[w * E + e];
+    tile_cnt[static_cast<size_t>(e) * n_ptiles + blockIdx.x] = tot;
+  }
+  if (!grid_barrier(bar, 1, err)) return;
+  // phase 2: totals, offsets and this tile's base per expert
+  int before[2] = {0, 0};
+  int tot2[2] = {0, 0};
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const int e = 2 * tid + q;
+    if (e < E) {
+      const int32_t* row = tile_cnt + static_cast<size_t>(e) * n_ptiles;
+      int a = 0, b = 0;
+      for (int t = 0; t < n_ptiles; ++t) {
+        const int v = __ldcg(row + t);  // written by other CTAs before the barrier
+        a += v;
+        b += t < static_cast<int>(blockIdx.x) ? v : 0;
+      }
+      tot2[q] = a;
+      before[q] = b;
+      cnt[e] = a;
+    }
+  }
+  int total;
+  const int ex = block_exscan2(tot2[0], tot2[1], scratch, &total);
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const int e = 2 * tid + q;
+    if (e < E) off[e] = ex + (q ? tot2[0] : 0);
+  }
+  if (tid == 0) off[E] = total;
+  __syncthreads();
+  if (blockIdx.x == 0) {
+    for (int e = tid; e <= E; e += blockDim.x) {
+      offsets[e] = off[e];
+      if (e < E) counts[e] = cnt[e];
+    }
+  }
+  // per-warp bases, seeded with the expert's offset plus the earlier tiles' counts
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const int e = 2 * tid + q;
+    if (e < E) {
+      int run = off[e] + before[q];
+      for (int w = 0; w < kWarps; ++w) {
+        const int v = whist[w * E + e];
+        whist[w * E + e] = run;
+        run += v;
+      }
+    }
+  }
+  __syncthreads();
+  // stable positions
+  for (int r = c0; r < c1; r += 32) {
+    const int i = r + lane;
+    int e = -1;
+    if (i < c1) {
+      e = idx[tbase + i];
+      if (e < 0 || e >= E) e = -1;
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    int pos = -1;
+    if (e >= 0) pos = wh[e] + __popc(peers & lt);
+    __syncwarp();
+    if (e >= 0 && (peers & lt) == 0) wh[e] += __popc(peers);
+    __syncwarp();
+    if (i < c1) {
+      const int j = tbase + i;
+      if (e >= 0 && (pos < 0 || pos >= TK)) {  // cannot happen for consistent counts
+        atomicExch(err, MOE_DEVERR_SCHEDULE);
+        pos = -1;
+        e = -1;
+      }
+      if (e >= 0) perm[pos] = j;
+      if (inv_perm) inv_perm[j] = pos;
+    }
+  }
+  if (build && blockIdx.x == 0) build_schedule(sa, cnt, scratch);
+}
+
 }  // namespace
 
 cudaError_t launch_permute(const moe_cfg& c, int T, const int32_t* idx, int32_t* tile_cnt,
@@ -219,6 +353,27 @@ cudaError_t launch_permute(const moe_cfg& c, int T, const int32_t* idx, int32_t*
     if (e != cudaSuccess) return e;
     return launch_pdl(perm_single, dim3(1), dim3(1024), smem, s, TK, c.E, idx, counts, offsets, perm,
                       inv_perm, err, sa, gu_start != nullptr ? 1 : 0);
+  }
+  if (np <= num_sms() && getenv("SGL_MOE_PERM") == nullptr) {
+    // one cooperative launch, one CTA per tile (all resident: the barrier ends);
+    // err[2] of the control block is its barrier counter, zero at this point
+    const int smem = 32 * c.E * static_cast<int>(sizeof(int));
+    cudaError_t e = ensure_dyn_smem(reinterpret_cast<const void*>(perm_fused),
+                                    32 * kMaxE * static_cast<int>(sizeof(int)));
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t lc;
+    memset(&lc, 0, sizeof(lc));
+    lc.gridDim = dim3(np);
+    lc.blockDim = dim3(1024);
+    lc.dynamicSmemBytes = smem;
+    lc.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    return cudaLaunchKernelEx(&lc, perm_fused, TK, c.E, np, idx, tile_cnt, counts, offsets, perm,
+                              inv_perm, err + 2, err, sa, gu_start != nullptr ? 1 : 0);
   }
   int32_t* tile_base = tile_cnt + static_cast<size_t>(c.E) * np;
   cudaError_t e = launch_pdl(perm_hist, dim3(np), dim3(256), 0, s, TK, c.E, np, idx, tile_cnt, err);

@@ -17,6 +17,37 @@ namespace {
 
 constexpr int kMaxE = 1024;
 
+__device__ __forceinline__ int ld_acquire_gpu(const int32_t* a) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
+  return v;
+}
+
+// Grid barrier n (1, 2, ...) of a cooperative launch on a monotonic counter
+// that is zero at launch; false if it timed out (the error word is set;
+// every CTA then leaves).
+__device__ bool grid_barrier(int32_t* bar, int n, int32_t* err) {
+  __shared__ int ok_s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();  // this CTA's writes before its arrival
+    atomicAdd(bar, 1);
+    const int need = n * static_cast<int>(gridDim.x);
+    const long long t0 = clock64();
+    int ok = 1;
+    while (ld_acquire_gpu(bar) < need) {  // waits last a few microseconds: spin
+      if (clock64() - t0 > kWaitLimitCycles) {
+        atomicExch(err, MOE_DEVERR_TIMEOUT);
+        ok = 0;
+        break;
+      }
+    }
+    ok_s = ok;
+  }
+  __syncthreads();
+  return ok_s != 0;
+}
+
 // Block-wide exclusive scan of up to 2 values per thread (1024 threads).
 // Returns the exclusive prefix of this thread's first value; *total gets the sum.
 __device__ int block_exscan2(int v0, int v1, int* scratch /*32*/, int* total) {

@@ -53,6 +53,18 @@ bool map_u8(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint3
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool map_codes(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t row_bytes) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr || ptr == nullptr || rows == 0 || row_bytes % 32 != 0) return false;
+  const cuuint64_t dims[2] = {row_bytes, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {32, 128};
+  const cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool map_fp4(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr || ptr == nullptr || rows == 0 || cols % 128 != 0) return false;

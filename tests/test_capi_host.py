@@ -122,3 +122,18 @@ def test_prepare_weights_validation():
     assert L.moe_prepare_weights(ctypes.byref(c), ctypes.byref(w), A, A, A + 8, None) == -3
     odd = sgl.moe_weights(A, A, A, A, A + 4, A, A, A, A)
     assert L.moe_prepare_weights(ctypes.byref(c), ctypes.byref(odd), A, A, A, None) == -3
+
+
+def test_peak_probe_library_loads_and_checks_arguments():
+    """The tensor-core throughput probe (a separate library) exports its entry
+    point and refuses bad shapes on the host, before any CUDA call."""
+    from sigmoid_group_limited_b200 import peak
+    L = peak.lib()
+    status = ctypes.c_void_p(1 << 20)  # never dereferenced: every call below is refused first
+    for args in ((3, 256, 1, 10, 148, 0), (0, 8, 1, 10, 148, 0), (1, 264, 1, 10, 148, 0),
+                 (2, 136, 3, 10, 148, 0), (0, 128, 1, 0, 148, 0), (0, 128, 1, 10, 0, 0),
+                 (0, 256, 3, 10, 148, 0), (0, 256, 2, 10, 148, 1), (0, 128, 2, 10, 148, 3),
+                 (0, 128, 2, 10, 148, 32)):
+        assert L.sgl_mma_peak(*args, status, None) == 1          # cudaErrorInvalidValue
+    assert L.sgl_mma_peak(0, 128, 1, 10, 148, 0, None, None) == 1   # no status word
+    assert set(peak.KINDS) == {"bf16", "e2m1xe4m3", "e2m1xe2m1"}

@@ -151,6 +151,33 @@ def test_tiny_identical_experts_closed_form():
     check_y(bits(g["y"]), expect, oracle.f32_to_bf16_bits(expect))
 
 
+@pytest.mark.parametrize("T", [33, 600])
+def test_scheduler_wait_runs_out_and_reports(T, monkeypatch):
+    """The FFN's one cross-CTA wait (a down item waits for the gate/up tiles of
+    its row tile) is bounded. With a test limit of about 1 ms and a target no
+    tile count reaches, every CTA's wait runs out: the call returns, the error
+    word reads MOE_DEVERR_TIMEOUT, and the next call on the same context is
+    correct. No fault and no endless wait: the CTAs drain their queued items
+    and leave."""
+    import time
+    cfg = TINY
+    d = workloads.generate(cfg, DEV, T=T)
+    monkeypatch.setenv("SGL_MOE_TEST_WAIT_CYCLES", "2000000")
+    monkeypatch.setenv("SGL_MOE_TEST_READY_EXTRA", "1000000")
+    from helpers import weights
+    ws = sgl.alloc_workspace(cfg, T)
+    y = torch.empty(T, cfg.H, dtype=torch.bfloat16, device=DEV)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    sgl.moe_layer_forward(cfg, d["x"], d["Wr"], d["bias"], weights(d), y, ws)
+    torch.cuda.synchronize()
+    assert time.perf_counter() - t0 < 5.0
+    assert sgl.moe_read_error(cfg, T, ws) == 2                 # MOE_DEVERR_TIMEOUT
+    monkeypatch.delenv("SGL_MOE_TEST_WAIT_CYCLES")
+    monkeypatch.delenv("SGL_MOE_TEST_READY_EXTRA")
+    _full_check(cfg, d)                                        # the context is still usable
+
+
 def test_deterministic_bits():
     cfg = TINY
     d = workloads.generate(cfg, DEV, T=300)
@@ -183,9 +210,32 @@ def test_permute_bit_exact(T, skew):
     assert sgl.moe_read_error(cfg, T, ws) == 0
 
 
-def test_permute_bad_id_sets_error_word():
+@pytest.mark.parametrize("T", [300, 16384])
+def test_permute_forms_agree(T, monkeypatch):
+    """Batches of several 2048-entry tiles take one cooperative launch; the
+    three-kernel form (histograms, scan, scatter), kept for very large batches,
+    gives the same bits."""
     cfg = workloads.CONFIGS["prefill"]
-    T = 40
+    g = torch.Generator().manual_seed(T + 1)
+    idx = torch.randint(0, cfg.E, (T, cfg.K), generator=g, dtype=torch.int32).to(DEV)
+    outs = []
+    for form in ("fused", "split"):
+        if form == "split":
+            monkeypatch.setenv("SGL_MOE_PERM", "split")
+        ws = sgl.alloc_workspace(cfg, T)
+        out = [torch.full((n,), -3, dtype=torch.int32, device=DEV)
+               for n in (cfg.E, cfg.E + 1, T * cfg.K, T * cfg.K)]
+        sgl.moe_permute(cfg, T, idx, *out, ws)
+        torch.cuda.synchronize()
+        assert sgl.moe_read_error(cfg, T, ws) == 0
+        outs.append(out)
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("T", [40, 400])
+def test_permute_bad_id_sets_error_word(T):
+    cfg = workloads.CONFIGS["prefill"]
     idx = torch.randint(0, cfg.E, (T, cfg.K), dtype=torch.int32)
     idx[3, 2] = cfg.E + 5
     idx[9, 0] = -1
