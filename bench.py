@@ -241,65 +241,32 @@ def roofline_entry(bytes_, flops, seconds, peaks, sustained=False, fp8_flops=0.0
             "frac": round(ach / pk, 4)}
 
 
-# DRAM traffic of moe_ffn per algorithmic byte (dram__bytes_read.sum +
-# dram__bytes_write.sum over the bytes of algorithmic_work), from full ncu
-# captures of the same kernel on the small cases named in profiles/
-# (moe_ffn_decode_e128_t32.md: BN=16; moe_ffn_prefill_e128_t1024.md: BN=128).
-# Weight bytes dominate and scale with the experts touched, so the ratio
-# scales the counters to a full launch. Valid only for the ffn.cu they were
-# taken on: any other source reports traffic null.
-FFN_TRAFFIC_SOURCE_SHA256 = "818ebd24c8f7c68dfaf7bd5aef21b8c5f3ce2a25f63a82994be6053fbb104ba0"
-FFN_TRAFFIC_RATIO = {16: (424.94 + 3.77) / 424.82, 128: (780.68 + 48.33) / 760.2}
+# DRAM bytes (dram__bytes_read.sum, dram__bytes_write.sum) of one expert-FFN
+# launch of each full-size workload, from one-pass ncu captures of the bench's
+# own command at the same token count (profiles/ffn_traffic_full_size.md).
+# Valid only for the FFN sources they were taken on: another source reports
+# traffic null.
+FFN_TRAFFIC_SOURCES_SHA256 = None   # sha256 of ffn.cu + ffn_mx.cu at the captures
+FFN_TRAFFIC = {}                     # workload name -> (read bytes, write bytes)
 
 
-def ffn_tile_n(cfg) -> int:
-    """Token-tile width the library picks for a batch (same rule as choose_bn)."""
-    avg = cfg.T * cfg.K / cfg.E
-    return 16 if avg <= 12 else 32 if avg <= 24 else 64 if avg <= 48 else 128
-
-
-def ffn_traffic(cfg, algorithmic_bytes: float):
+def ffn_sources_sha256() -> str:
     import hashlib
-    src = os.path.join(os.path.dirname(os.path.abspath(__file__)), "sigmoid_group_limited_b200",
-                       "csrc", "ffn.cu")
+    h = hashlib.sha256()
+    for name in ("ffn.cu", "ffn_mx.cu"):
+        with open(os.path.join(ROOT, "sigmoid_group_limited_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def ffn_traffic(cfg):
+    """(read, write) DRAM bytes of one FFN launch of `cfg`'s workload, or None."""
     try:
-        with open(src, "rb") as f:
-            digest = hashlib.sha256(f.read()).hexdigest()
+        if FFN_TRAFFIC_SOURCES_SHA256 is None or ffn_sources_sha256() != FFN_TRAFFIC_SOURCES_SHA256:
+            return None
     except OSError:
         return None
-    ratio = FFN_TRAFFIC_RATIO.get(ffn_tile_n(cfg))
-    if digest != FFN_TRAFFIC_SOURCE_SHA256 or ratio is None or cfg.wfmt != workloads.MOE_W_BF16:
-        return None
-    return round(ratio * algorithmic_bytes)
-
-
-def popularity_slope(cfg, counts) -> float:
-    """Slope of ln(mean expert count per within-group popularity rank) against
-    ln(rank) (a Zipf law p(r) ~ r^-s has slope -s); ranks with no slot are
-    left out of the fit."""
-    ranks = workloads.zipf_ranks(cfg)
-    per = cfg.experts_per_group
-    m = np.array([counts[ranks == r].mean() for r in range(1, per + 1)], dtype=np.float64)
-    ok = m > 0
-    return float(np.polyfit(np.log(np.arange(1, per + 1)[ok]), np.log(m[ok]), 1)[0])
-
-
-def front_prefetch_bytes(cfg, touched: int) -> int:
-    """Bytes of FFN weights the fused decode front asks L2 for before the FFN
-    starts (its rule: the shared expert's three matrices, then the gate and up
-    matrices of the first touched experts, as many whole experts as fit the
-    budget SGL_MOE_PREFETCH MiB, 32 when unset); 0 when the front is not used."""
-    if not fused_front(cfg):
-        return 0
-    v = os.environ.get("SGL_MOE_PREFETCH")
-    budget = (32 << 20) if not v else max(0, int(v)) << 20
-    if budget == 0:
-        return 0
-    shared = 3 * cfg.I_shared * cfg.H * 2
-    if cfg.wfmt != workloads.MOE_W_BF16:
-        return shared
-    gu = 2 * cfg.I * cfg.H * 2
-    return shared + min(touched, budget // gu, 33) * gu
+    return FFN_TRAFFIC.get(cfg.name)
 
 
 # ------------------------------------------------------------------ GPU arm
@@ -662,12 +629,18 @@ def run_native(args, rank, world, local):
         src = "HBM copy" if ent["bound"] == "hbm" else (
             f"cuBLAS bf16 burst; routed MXFP8 x MXFP4 flops at {ratios['fp8']:.3f} x that "
             f"({ratios['source']} kind::mxf8f6f4 / kind::f16 ratio)" if mx else "cuBLAS bf16 burst")
+        tr = ffn_traffic(cfg_)
         ent.update(kernel="moe_ffn_mx (block-scaled gate/up + down)" if mx else "moe_ffn (gate/up + down)",
-                   traffic=ffn_traffic(cfg_, b),
-                   traffic_unit="bytes per launch (ncu DRAM read+write, scaled from the "
-                                "small-case capture of the same kernel)",
+                   traffic=(tr[0] + tr[1]) if tr else None,
+                   traffic_unit="bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum, "
+                                "one-pass capture of this workload at full size)",
                    peak_source=f"{peaks['source']} ({src})",
                    units_per_launch=f"{cfg_.T} tokens, {mm['routing']['experts_touched']} routed experts + shared")
+        if tr:
+            ent["traffic_read"], ent["traffic_write"] = tr
+            ent["traffic_over_algorithmic"] = round((tr[0] + tr[1]) / b, 3)
+            # the fp32 slot rows every token writes once: (T*K + T) rows of H floats
+            ent["y_slot_bytes"] = (cfg_.T * cfg_.K + cfg_.T) * cfg_.H * 4
         if mx:
             ent["time"] = "FFN stage events: scale atoms and MXFP8 x included"
         if cfg_.wfmt != workloads.MOE_W_BF16:

@@ -53,8 +53,8 @@ WsLayout ws_layout(const moe_cfg& c, int T) {
     L.ffn = kFfnMx;
   } else {
     L.ffn = choose_ffn(T, c.K, c.E, &L.bn);
-    // MXFP4 weights are expanded by the one-CTA kernel only
-    if (c.wfmt == MOE_W_MXFP4 && L.ffn == kFfnPair) L.ffn = kFfnNarrow, L.bn = kTileN;
+    // MXFP4 weights are expanded by the one-CTA kernel, on tiles of up to 128 rows
+    if (c.wfmt == MOE_W_MXFP4 && (L.ffn == kFfnPair || L.bn > kTileN)) L.ffn = kFfnNarrow, L.bn = kTileN;
   }
   ffn_tiles(L.ffn, &L.gu_ft, &L.dn_ft);
   const int gu_ft = L.gu_ft, dn_ft = L.dn_ft;

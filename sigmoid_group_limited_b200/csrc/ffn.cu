@@ -1011,6 +1011,7 @@ cudaError_t launch_ffn(const GemmArgs& a, cudaStream_t s) {
     case 32: return launch_bn<32, false, false>(a, s);
     case 64: return launch_bn<64, false, false>(a, s);
     case 128: return tm ? launch_bn<128, true, false>(a, s) : launch_bn<128, false, false>(a, s);
+    case 256: return launch_bn<256, false, false>(a, s);
     default: return cudaErrorInvalidValue;
   }
 }

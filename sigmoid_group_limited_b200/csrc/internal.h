@@ -65,6 +65,7 @@ inline FfnKind choose_ffn(int T, int K, int E, int* bn) {
   if (avg <= 24.0) return *bn = 32, kFfnNarrow;
   if (avg <= 48.0) return *bn = 64, kFfnNarrow;
   if (ffn_env_is("pair")) return *bn = kPairTileN, kFfnPair;
+  if (ffn_env_is("wide")) return *bn = 256, kFfnNarrow;
   return *bn = 128, kFfnNarrow;
 }
 

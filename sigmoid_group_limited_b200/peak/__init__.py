@@ -73,15 +73,16 @@ def measure(kind: str, n: int = 256, chains: int = 1, iters: int = 40000, repeat
             "tflops": flops / t / 1e12, "ns_per_mma": t / (iters * chains) * 1e9, "seconds": t}
 
 
+# shapes every kind can run: the block-scaled kinds keep TMEM columns 384-399
+# for their scale atoms, so at most 384 accumulator columns
+COMMON_SHAPES = ((256, 1), (128, 2), (128, 3), (192, 2))
+
+
 def peaks(device=None) -> dict:
-    """Best instruction throughput per kind over a few shapes: N = 256 with one
-    and (bf16) two accumulators, N = 128 with two and three (and four), N = 192
-    with two."""
+    """Best instruction throughput per kind over the same shapes for every kind
+    (COMMON_SHAPES), so that the ratios between kinds compare like with like."""
     out = {}
     for kind in KINDS:
-        shapes = [(256, 1), (128, 2), (128, 3), (192, 2)]
-        if kind == "bf16":
-            shapes += [(256, 2), (128, 4)]
-        best = max((measure(kind, n, c, device=device) for n, c in shapes), key=lambda r: r["tflops"])
+        best = max((measure(kind, n, c, device=device) for n, c in COMMON_SHAPES), key=lambda r: r["tflops"])
         out[kind] = best
     return out
