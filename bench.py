@@ -269,6 +269,35 @@ def ffn_traffic(cfg):
     return FFN_TRAFFIC.get(cfg.name)
 
 
+def popularity_slope(cfg, counts) -> float:
+    """Slope of ln(mean expert count per within-group popularity rank) against
+    ln(rank) (a Zipf law p(r) ~ r^-s has slope -s); ranks with no slot are
+    left out of the fit."""
+    ranks = workloads.zipf_ranks(cfg)
+    per = cfg.experts_per_group
+    m = np.array([counts[ranks == r].mean() for r in range(1, per + 1)], dtype=np.float64)
+    ok = m > 0
+    return float(np.polyfit(np.log(np.arange(1, per + 1)[ok]), np.log(m[ok]), 1)[0])
+
+
+def front_prefetch_bytes(cfg, touched: int) -> int:
+    """Bytes of FFN weights the fused decode front asks L2 for before the FFN
+    starts (its rule: the shared expert's three matrices, then the gate and up
+    matrices of the first touched experts, as many whole experts as fit the
+    budget SGL_MOE_PREFETCH MiB, 32 when unset); 0 when the front is not used."""
+    if not fused_front(cfg):
+        return 0
+    v = os.environ.get("SGL_MOE_PREFETCH")
+    budget = (32 << 20) if not v else max(0, int(v)) << 20
+    if budget == 0:
+        return 0
+    shared = 3 * cfg.I_shared * cfg.H * 2
+    if cfg.wfmt != workloads.MOE_W_BF16:
+        return shared
+    gu = 2 * cfg.I * cfg.H * 2
+    return shared + min(touched, budget // gu, 33) * gu
+
+
 # ------------------------------------------------------------------ GPU arm
 
 STAGES = ("route", "permute", "gateup", "down", "combine")

@@ -82,3 +82,26 @@ def test_block_scaled_formats_in_bench_accounting():
         assert fmt in bench.DTYPES
     # decode batches take the fused front: front, FFN, combine
     assert bench.kernels_per_step(workloads.CONFIGS["decode"]) == 3
+
+
+def test_bench_helpers_used_by_the_gpu_arm():
+    """Host helpers the GPU arm calls: the Zipf popularity slope of a count
+    vector, the fused front's L2-prefetched bytes, the traffic lookup and the
+    tensor-peak ratios (exercised here so that a missing name fails on CPU)."""
+    import numpy as np
+    cfg = workloads.CONFIGS["zipf"]
+    ranks = workloads.zipf_ranks(cfg)
+    counts = np.round(4000.0 * ranks.astype(np.float64) ** -1.1).astype(np.int64)
+    assert abs(bench.popularity_slope(cfg, counts) + 1.1) < 0.01
+    dec = workloads.CONFIGS["decode"]
+    shared = 3 * 768 * 2560 * 2
+    assert bench.front_prefetch_bytes(dec, 58) == shared + 4 * (2 * 768 * 2560 * 2)
+    assert bench.front_prefetch_bytes(dec, 2) == shared + 2 * (2 * 768 * 2560 * 2)
+    assert bench.front_prefetch_bytes(workloads.CONFIGS["prefill"], 122) == 0     # no fused front
+    assert bench.ffn_traffic(dec) is None or len(bench.ffn_traffic(dec)) == 2
+    r = bench.tensor_ratios(None)
+    assert r["source"] == "nominal" and r["fp8"] == 2.0 and r["fp4"] == 4.0
+    probe = {"bf16": {"tflops": 1000.0}, "e2m1xe4m3": {"tflops": 2000.0}, "e2m1xe2m1": {"tflops": 4100.0}}
+    r = bench.tensor_ratios(probe)
+    assert r["fp8"] == 2.0 and abs(r["fp4"] - 4.1) < 1e-12
+    assert set(bench.WORKLOAD_NOTES) >= {"decode", "prefill", "prefill_bias0", "zipf", "mxfp4", "mxfp4_a8"}

@@ -72,6 +72,33 @@ def test_tiny_layer_pair_ffn(T, variant, monkeypatch):
     _full_check(cfg, d)
 
 
+@pytest.mark.parametrize("form", ["tokens_m", "wide"])
+@pytest.mark.parametrize("T,variant", [(600, {}), (600, dict(limit_routed=0.5, limit_shared=0.7)),
+                                       (600, dict(I_shared=0)), (600, dict(I=192, I_shared=320)),
+                                       (1500, dict(H=384))])
+def test_tiny_layer_ffn_options(form, T, variant, monkeypatch):
+    """The optional orientations of the expert FFN for large batches, selected
+    explicitly: token rows as the MMA's M with two partial accumulators
+    (tokens_m), and 256-token tiles (wide)."""
+    monkeypatch.setenv("SGL_MOE_FFN", form)
+    cfg = TINY.with_(**variant)
+    d = workloads.generate(cfg, DEV, T=T)
+    if cfg.I_shared == 0:
+        d.update(Wg_s=None, Wu_s=None, Wd_s=None)
+        g = run_layer(cfg, d)
+        h = host_inputs({**d, "Wg_s": torch.zeros(1, dtype=torch.bfloat16),
+                         "Wu_s": torch.zeros(1, dtype=torch.bfloat16),
+                         "Wd_s": torch.zeros(1, dtype=torch.bfloat16)})
+        z = np.zeros((64, cfg.H), np.uint16)
+        ref = oracle.layer_forward(cfg.with_(I_shared=64), h["x"], h["Wr"], h["bias"],
+                                   DeviceExperts(d), z, z, z.T.copy())
+        check_routing(ref, g["idx"].cpu().numpy(), g["w"].cpu().numpy())
+        keep = ~np.isin(np.arange(T), near_tie_tokens(ref))
+        check_y(bits(g["y"])[keep], ref["y_f32"][keep], ref["y"][keep])
+    else:
+        _full_check(cfg, d)
+
+
 @pytest.mark.slow
 def test_prefill_pair_ffn_all_tokens(monkeypatch):
     monkeypatch.setenv("SGL_MOE_FFN", "pair")
