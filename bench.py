@@ -246,8 +246,15 @@ def roofline_entry(bytes_, flops, seconds, peaks, sustained=False, fp8_flops=0.0
 # own command at the same token count (profiles/ffn_traffic_full_size.md).
 # Valid only for the FFN sources they were taken on: another source reports
 # traffic null.
-FFN_TRAFFIC_SOURCES_SHA256 = None   # sha256 of ffn.cu + ffn_mx.cu at the captures
-FFN_TRAFFIC = {}                     # workload name -> (read bytes, write bytes)
+FFN_TRAFFIC_SOURCES_SHA256 = "c2dcf21acb02a388b9c7592539556273c8214f857808b3908bf972fbe8221e42"
+FFN_TRAFFIC = {                      # workload name -> (read bytes, write bytes)
+    "decode": (696.27e6, 5.06e6),
+    "prefill": (1.65e9, 375.26e6),
+    "prefill_bias0": (6.20e9, 376.40e6),
+    "zipf": (7.65e9, 1.68e9),
+    "mxfp4": (919.93e6, 809.77e6),
+    "mxfp4_a8": (735.50e6, 762.32e6),
+}
 
 
 def ffn_sources_sha256() -> str:
@@ -260,11 +267,15 @@ def ffn_sources_sha256() -> str:
 
 
 def ffn_traffic(cfg):
-    """(read, write) DRAM bytes of one FFN launch of `cfg`'s workload, or None."""
+    """(read, write) DRAM bytes of one FFN launch of `cfg`'s workload, or None
+    (other FFN sources, or a workload shrunk by --tokens / --experts)."""
     try:
         if FFN_TRAFFIC_SOURCES_SHA256 is None or ffn_sources_sha256() != FFN_TRAFFIC_SOURCES_SHA256:
             return None
     except OSError:
+        return None
+    full = workloads.CONFIGS.get(cfg.name)
+    if full is None or (cfg.T, cfg.E) != (full.T, full.E):
         return None
     return FFN_TRAFFIC.get(cfg.name)
 

@@ -99,6 +99,9 @@ def test_bench_helpers_used_by_the_gpu_arm():
     assert bench.front_prefetch_bytes(dec, 2) == shared + 2 * (2 * 768 * 2560 * 2)
     assert bench.front_prefetch_bytes(workloads.CONFIGS["prefill"], 122) == 0     # no fused front
     assert bench.ffn_traffic(dec) is None or len(bench.ffn_traffic(dec)) == 2
+    # counters are tied to the full-size workload: a shrunk one reports none
+    assert bench.ffn_traffic(dec.with_(E=128)) is None
+    assert bench.ffn_traffic(workloads.CONFIGS["prefill"].with_(T=1024)) is None
     r = bench.tensor_ratios(None)
     assert r["source"] == "nominal" and r["fp8"] == 2.0 and r["fp4"] == 4.0
     probe = {"bf16": {"tflops": 1000.0}, "e2m1xe4m3": {"tflops": 2000.0}, "e2m1xe2m1": {"tflops": 4100.0}}
