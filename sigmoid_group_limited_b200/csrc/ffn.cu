@@ -88,7 +88,7 @@ constexpr int kCodeTile = 128 * 32;  // one weight tile's codes of one k-block (
 constexpr int kQueue = 4;                 // item queue entries
 constexpr int kLead = 4;                  // claim the next item this many k-blocks early
 constexpr long long kProgStride = 1024;   // producer progress = n * stride + k-blocks issued
-constexpr int kSmemBudget = 210 * 1024;   // pipeline stages
+constexpr int kSmemLimit = 227 * 1024;    // dynamic shared memory of one CTA
 
 template <int BN, bool TM = false, bool F4 = false>
 struct Cfg {
@@ -100,7 +100,14 @@ struct Cfg {
   // less depth
   static constexpr int STG = F4 ? 6 : 0;
   static constexpr int STG_BYTES = 2 * kCodeTile;
-  static constexpr int STAGES_RAW = (kSmemBudget - STG * STG_BYTES) / STAGE_BYTES;
+  static constexpr int CTRL_BYTES = 512;        // barriers, queue, flags
+  // everything but the stages: alignment slack, control block, row metadata,
+  // the epilogue warps' store tiles, and the per-slot item starts and row
+  // offsets of the largest E, (3E + 5) ints (added at launch for the real E)
+  static constexpr int FIXED_BYTES =
+      1024 + CTRL_BYTES + BN * 8 + kEpiWarps * kEpiTileWords * 4;
+  static constexpr int STAGES_RAW =
+      (kSmemLimit - STG * STG_BYTES - FIXED_BYTES - (3 * kMaxExpertsCfg + 5) * 4) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
   // weights as M: two fp32 accumulators (gate | up, or the two Wd halves) of
   // BN columns side by side; token rows as M: two partial sums of 256
@@ -112,13 +119,12 @@ struct Cfg {
   static constexpr int TMEM_COLS = NACC * ACC_COLS < 32 ? 32 : NACC * ACC_COLS;
   static constexpr int H_BOX = BN < 64 ? BN : 64;  // rows per TMA box of h
   static_assert((TMEM_COLS & (TMEM_COLS - 1)) == 0 && TMEM_COLS <= 512, "TMEM allocation");
-  static constexpr int CTRL_BYTES = 512;        // barriers, queue, flags
   // + the per-slot item starts and row offsets, (3E + 5) ints, added at launch
-  static constexpr int SMEM =
-      STAGES * STAGE_BYTES + STG * STG_BYTES + 1024 /*align*/ + CTRL_BYTES + BN * 8;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + STG * STG_BYTES + FIXED_BYTES;
   static_assert(8 * (2 * 8 + 2 * 2 + 2 * kQueue + 2 * 8) + 8 + 4 * (2 + kQueue) <= CTRL_BYTES,
                 "control block");
   static_assert(STG <= 8 && STAGES >= 2, "rings");
+  static_assert(SMEM + (3 * kMaxExpertsCfg + 5) * 4 <= kSmemLimit, "shared memory");
 };
 
 // ---------------------------------------------------------------------------
@@ -247,7 +253,8 @@ __global__ void __launch_bounds__(F4 ? kFfnThreadsF4 : kFfnThreads, 1)
   volatile int* qitem = abort_flag + 1;  // [kQueue]
   int* meta_j = reinterpret_cast<int*>(ctrl + C::CTRL_BYTES);
   float* meta_w = reinterpret_cast<float*>(meta_j + BN);
-  int* s_gu = reinterpret_cast<int*>(meta_w + BN);  // [E+2]
+  uint32_t* epi_tile = reinterpret_cast<uint32_t*>(meta_w + BN);       // [warps][kEpiTileWords]
+  int* s_gu = reinterpret_cast<int*>(epi_tile + kEpiWarps * kEpiTileWords);  // [E+2]
   int* s_dn = s_gu + (p.E + 2);                      // [E+2]
   int* s_off = s_dn + (p.E + 2);                     // [E+1]
 
@@ -830,50 +837,46 @@ __global__ void __launch_bounds__(F4 ? kFfnThreadsF4 : kFfnThreads, 1)
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * C::ACC_COLS;
+      uint32_t* tile = epi_tile + (warp - 2) * kEpiTileWords;
       if (gu) {
-        const int nfeat = it.ntile * kTileN + orow;
+        const int fbase = it.ntile * kTileN + q * 32;  // this warp's 32 features
         const int ncols = sh ? p.Is : p.I;
-        const bool ok = nfeat < ncols;
+        const bool ok = fbase < ncols;  // I and Is are multiples of 64: whole warps
         const float L = sh ? p.lim_s : p.lim_r;
         uint16_t* hout = sh ? p.h_s : p.h_r;
         const int ncol = mma_n(it);
         // the two warps of a lane quarter take alternate 16-column chunks
 #pragma unroll 1
-        for (int c0 = 16 * cpart; c0 < ncol; c0 += 32) {
+        for (int c0 = 16 * cpart; c0 < ncol && ok; c0 += 32) {
           float gv[16], uv[16];
           tmem_ld16(taddr + c0, gv);
           tmem_ld16(taddr + BN + c0, uv);
           tmem_ld_wait();
-          if (ok) {
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              const int r = c0 + c;
-              if (r < it.nrows)
-                hout[static_cast<size_t>(it.row0 + r) * ncols + nfeat] = f2bf(swiglu(gv[c], uv[c], L));
-            }
-          }
+          for (int c = 0; c < 16; ++c) gv[c] = swiglu(gv[c], uv[c], L);
+          store_h16(gv, tile, hout, ncols, it.row0 + c0, it.nrows - c0, fbase, lane);
         }
       } else {
         const int ncol = mma_n(it);
 #pragma unroll 1
         for (int half = 0; half < 2; ++half) {
-          const int nfeat = it.ntile * kDownTile + half * kTileN + orow;
-          const bool ok = nfeat < p.H;
+          const int fbase = it.ntile * kDownTile + half * kTileN + q * 32;  // this warp's features
+          const bool ok = fbase < p.H;  // H is a multiple of 64: whole warps
           // kCols columns per TMEM wait (the loads of one group are in flight
           // together); the two warps of a lane quarter take alternate groups
           constexpr int kCols = BN >= 32 ? 32 : 16;
 #pragma unroll 1
-          for (int c0 = kCols * cpart; c0 < ncol; c0 += 2 * kCols) {
+          for (int c0 = kCols * cpart; c0 < ncol && ok; c0 += 2 * kCols) {
             float ov[kCols];
 #pragma unroll
             for (int u = 0; u < kCols; u += 16) tmem_ld16(taddr + half * BN + c0 + u, ov + u);
             tmem_ld_wait();
-            if (ok) {
 #pragma unroll
-              for (int c = 0; c < kCols; ++c) {
-                const int j = meta_j[c0 + c];
-                if (j >= 0) p.y_slot[static_cast<size_t>(j) * p.H + nfeat] = meta_w[c0 + c] * ov[c];
-              }
+            for (int g8 = 0; g8 < kCols / 8; ++g8) {
+              float v[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) v[i] = meta_w[c0 + 8 * g8 + i] * ov[8 * g8 + i];
+              store_y8(v, meta_j + c0 + 8 * g8, tile, p.y_slot, p.H, fbase, lane);
             }
           }
         }

@@ -123,16 +123,79 @@ __device__ __forceinline__ void epi_bar() {
   asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory");
 }
 
-// silu(g) * u after the clamp, with the hardware exponential and a rounded
-// reciprocal (h is rounded to bf16 right after).
+// silu(g) * u after the clamp, with the hardware exponential and the
+// hardware's approximate reciprocal (h is rounded to bf16 right after, whose
+// half-ulp is far above either error).
 __device__ __forceinline__ float swiglu(float g, float u, float L) {
   const float gg = clampL(g, L), uu = clampL(u, L);
-  return gg * __frcp_rn(1.0f + __expf(-gg)) * uu;
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.0f + __expf(-gg)));
+  return gg * r * uu;
 }
 
 
 __device__ __forceinline__ uint16_t f2bf(float v) {
   return __bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// Epilogue stores through a per-warp shared-memory tile (kEpiTileWords
+// 32-bit words): a lane of an epilogue warp holds one output feature (its
+// TMEM lane) for consecutive token columns, while the outputs are token rows
+// of features. Going through the tile turns 32 single-value stores per row
+// group into 16-byte stores of row pieces.
+constexpr int kEpiTileWords = 256;
+
+// h (bf16) of 16 token columns: hv[c] is this lane's feature fbase + lane of
+// token row `row0 + c`; rows c >= nvalid are not stored. hout + row * ncols
+// + fbase must be 16-byte aligned for every row (ncols and fbase multiples
+// of 8).
+__device__ __forceinline__ void store_h16(const float* hv, uint32_t* tile, uint16_t* hout,
+                                          int ncols, int row0, int nvalid, int fbase, int lane) {
+  const bool odd = (lane & 1) != 0;
+  // token pair (2k, 2k+1): the even lane of a lane pair packs features
+  // (l, l+1) of token 2k, the odd lane those of token 2k+1
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float mine = odd ? hv[2 * k + 1] : hv[2 * k];
+    const float other = __shfl_xor_sync(0xffffffffu, odd ? hv[2 * k] : hv[2 * k + 1], 1);
+    tile[(2 * k + (odd ? 1 : 0)) * 16 + (lane >> 1)] =
+        odd ? pack_bf16x2(other, mine) : pack_bf16x2(mine, other);
+  }
+  __syncwarp();
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const int r = half * 8 + (lane >> 2);  // token row; the lane's 8 features at 8 * (lane & 3)
+    const uint4 v = *reinterpret_cast<const uint4*>(tile + r * 16 + 4 * (lane & 3));
+    if (r < nvalid)
+      *reinterpret_cast<uint4*>(hout + static_cast<size_t>(row0 + r) * ncols + fbase +
+                                8 * (lane & 3)) = v;
+  }
+  __syncwarp();
+}
+
+// fp32 rows of 8 token columns: v[i] (already weighted) is this lane's
+// feature fbase + lane of y_slot row j[i] (j < 0: not stored). y + j * H +
+// fbase must be 16-byte aligned (H and fbase multiples of 4).
+__device__ __forceinline__ void store_y8(const float* v, const int* j, uint32_t* tile, float* y,
+                                         int H, int fbase, int lane) {
+  float* t = reinterpret_cast<float*>(tile);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) t[i * 32 + lane] = v[i];
+  __syncwarp();
+#pragma unroll
+  for (int pass = 0; pass < 2; ++pass) {
+    const int i = pass * 4 + (lane >> 3);  // row; the lane's 4 features at 4 * (lane & 7)
+    const float4 q = *reinterpret_cast<const float4*>(t + i * 32 + 4 * (lane & 7));
+    const int jj = j[i];
+    if (jj >= 0)
+      *reinterpret_cast<float4*>(y + static_cast<size_t>(jj) * H + fbase + 4 * (lane & 7)) = q;
+  }
+  __syncwarp();
 }
 
 __device__ __forceinline__ void fence_proxy_async_global() {

@@ -5,20 +5,24 @@
 // (an expert is a gate / up / down SwiGLU FFN, hidden 2560, intermediate 768;
 // one shared expert sees every token) and sec. 4 (SwiGLU limits).
 //
-// Same items and scheduling as ffn.cu, but each item runs on a pair of CTAs
-// (a cluster of two) that issue one M = 256 MMA: each CTA holds 128 rows of A
-// and half of the item's N token rows of B, and gets its 128 rows of D in its
-// own TMEM. Per CTA and 64-wide k-block that is 16 KB of A and up to 16 KB of
-// B for up to 256 x 256 x 64 MACs of the pair: twice the flops per byte of
-// shared-memory fill of a single CTA with 128-token tiles, with the
-// accumulators still double-buffered (two 256-column buffers).
-//   gate/up item (slot, 256-token tile, 128 features f0..f0+127): CTA r holds
-//       gate rows f0 + 64r .. +63 over up rows f0 + 64r .. +63 (lanes 0-63 /
-//       64-127 of its D); the epilogue pairs lane l with lane l + 64 through
-//       shared memory. B = the item's token rows, copied from x by the
-//       gatherer warps of each CTA (16-byte cp.async into the swizzled tile).
+// Same scheduling as ffn.cu, but each item runs on a pair of CTAs (a cluster
+// of two) that issue M = 256 MMAs: each CTA holds 128 rows of A and half of
+// the item's N token rows of B, and gets its 128 rows of D in its own TMEM.
+// TMEM holds two 256-column accumulators (halves 0 and 1).
+//   gate/up item (slot, 256-token tile, 256 features f0..f0+255): CTA r holds
+//       gate rows f0 + 128r .. +127 and up rows f0 + 128r .. +127 as two A
+//       operands; gate accumulates in half 0 and up in half 1, two
+//       independent MMA chains issued alternately (an MMA waits for the
+//       previous one into the same accumulator, so one chain alone issues
+//       at about two thirds of the rate of two). B = the item's token rows,
+//       copied from x by the gatherer warps of each CTA (16-byte cp.async
+//       into the swizzled tile). Per CTA and 64-wide k-block: 32 KB of A and
+//       up to 16 KB of B for 2 x 128 x 256 x 64 MACs of this SM.
 //   down item (slot, 256-token tile, 256 hidden features): CTA r holds Wd rows
-//       256 n + 128 r .. +127; B = h rows.
+//       256 n + 128 r .. +127; B = h rows; one accumulator, the halves taken
+//       in turn, so a down item's epilogue overlaps the next down item.
+// A gate/up item holds both halves, so its epilogue does not overlap the
+// next item's MMAs; eight epilogue warps keep that drain short.
 // A and the h rows of down items arrive by TMA (no multicast): each CTA loads
 // its own halves and the byte counts complete on the leader CTA's full
 // barrier, where the gatherer warps of both CTAs also arrive; the leader's
@@ -60,18 +64,18 @@ constexpr int kPThreads = 32 * (kPSchedWarp + 1);
 constexpr int kPQueue = 4;
 constexpr int kPLead = 4;                  // claim the next item this many k-blocks early
 constexpr long long kPProgStride = 1024;
-constexpr int kPStages = 6;
-constexpr int kPA = 128 * 128;             // A half: 128 rows x 64 bf16
+constexpr int kPStages = 4;
+constexpr int kPA = 128 * 128;             // one A operand: this CTA's 128 rows x 64 bf16
 constexpr int kPB = kPairTileN / 2 * 128;  // B half: up to 128 rows x 64 bf16
-constexpr int kPStage = kPA + kPB;
+constexpr int kPStage = 2 * kPA + kPB;     // gate A, up A (down: Wd rows only), B
 constexpr int kPBox = 32;                  // token rows per B box
-constexpr int kPAccCols = kPairTileN;      // fp32 columns of one accumulator
-constexpr int kPTmemCols = 2 * kPAccCols;  // two buffers
+constexpr int kPAccCols = kPairTileN;      // fp32 columns of one accumulator (a TMEM half)
+constexpr int kPTmemCols = 2 * kPAccCols;  // halves 0 and 1
 constexpr int kPCtrl = 512;
-constexpr int kPXchRow = 9;                // 8 floats + 1 (bank spread)
-constexpr int kPXchFloats = 2 * 2 * 64 * kPXchRow;  // [column part][gate/up][feature][8]
-constexpr int kPSmem = kPStages * kPStage + 1024 + kPCtrl + kPXchFloats * 4 + kPairTileN * 8;
+constexpr int kPSmem =
+    kPStages * kPStage + 1024 + kPCtrl + kPairTileN * 8 + kPEpiWarps * kEpiTileWords * 4;
 static_assert(kPTmemCols <= 512, "TMEM");
+static_assert(kPSmem + (3 * kMaxExpertsCfg + 5) * 4 <= 227 * 1024, "shared memory");
 // consumers of a queue entry, counted on the leader's qempty: leader producer,
 // MMA, epilogue and gatherer warps; peer producer, epilogue and gatherer warps
 constexpr int kPQueueConsumers = 1 + 1 + kPEpiWarps + kPGatherWarps + 1 + kPEpiWarps + kPGatherWarps;
@@ -83,7 +87,7 @@ __device__ __forceinline__ int pair_n(const WorkItem& it) {
 }
 
 struct PairMaps {
-  CUtensorMap wg, wu, wgs, wus;  // gate / up rows, 64-row boxes
+  CUtensorMap wg, wu, wgs, wus;  // gate / up rows, 128-row boxes
   CUtensorMap wd, wds;           // down rows, 128-row boxes
   CUtensorMap h, hs;             // h rows, 32-row boxes
 };
@@ -104,10 +108,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(const_cast<long long*>(prog) + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* qitem = abort_flag + 1;  // [kPQueue]
-  float* xch = reinterpret_cast<float*>(ctrl + kPCtrl);             // [kPXchFloats]
-  int* meta_j = reinterpret_cast<int*>(xch + kPXchFloats);          // [kPairTileN]
+  int* meta_j = reinterpret_cast<int*>(ctrl + kPCtrl);              // [kPairTileN]
   float* meta_w = reinterpret_cast<float*>(meta_j + kPairTileN);    // [kPairTileN]
-  int* s_gu = reinterpret_cast<int*>(meta_w + kPairTileN);          // [E+2]
+  uint32_t* epi_stage = reinterpret_cast<uint32_t*>(meta_w + kPairTileN);  // [warps][kEpiTileWords]
+  int* s_gu = reinterpret_cast<int*>(epi_stage + kPEpiWarps * kEpiTileWords);  // [E+2]
   int* s_dn = s_gu + (p.E + 2);                                      // [E+2]
   int* s_off = s_dn + (p.E + 2);                                     // [E+1]
   static_assert(8 * (2 * kPStages + 4 + 2 * kPQueue) + 8 + 4 * (2 + kPQueue) <= kPCtrl, "ctrl");
@@ -123,7 +127,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
       mbar_init(&full[s], 1 + 2 * kPGatherWarps);
       mbar_init(&empty[s], 1);  // the leader's multicast commit
     }
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < 2; ++a) {  // one pair per TMEM half
       mbar_init(&tfull[a], 1);   // multicast commit
       mbar_init(&tempty[a], 2 * kPEpiWarps);  // the epilogue warps of both CTAs
     }
@@ -162,6 +166,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
     return gu ? decode_item(i, s_gu, s_off, nslots, p.E, p.T, kPairTileN)
               : decode_item(i - n_gu, s_dn, s_off, nslots, p.E, p.T, kPairTileN);
   };
+  auto valid = [&](const WorkItem& it, bool gu) {
+    return item_ok(p, it, gu, kPairTileN, kPairGuTile, kDownTile);
+  };
   const int KB_gu = p.H / 64, KB_dn_r = p.I / 64, KB_dn_s = p.Is / 64;
   auto nkb_of = [&](bool gu, bool sh) { return gu ? KB_gu : (sh ? KB_dn_s : KB_dn_r); };
   // the leader's copy of a barrier, as a cluster address
@@ -199,15 +206,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
         if (item >= 0) {
           bool gu;
           const WorkItem it = item_at(item, gu);
-          if (item_ok(p, it, gu, kPairTileN)) {
+          if (valid(it, gu)) {
             const bool sh = it.e == p.E;
             prev_nkb = nkb_of(gu, sh);
             if (!gu) {
               // both halves of every gate/up output tile of this (slot, row tile) are in h
               const int r0 = sh ? 0 : s_off[it.e];
               const int ridx = s_gu[it.e] + (it.row0 - r0) / kPairTileN;
-              if (!wait_count(p.ready + ridx, 2 * cdiv_dev(sh ? p.Is : p.I, kTileN), abort_flag,
-                              p.err))
+              if (!wait_count(p.ready + ridx, 2 * cdiv_dev(sh ? p.Is : p.I, kPairGuTile),
+                              abort_flag, p.err))
                 item = -1;
             }
           } else {
@@ -239,7 +246,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
         if (leader) *prog = n * kPProgStride;
         bool gu;
         const WorkItem it = item_at(item, gu);
-        if (!item_ok(p, it, gu, kPairTileN)) continue;
+        if (!valid(it, gu)) continue;
         const bool sh = it.e == p.E;
         // h rows of a down item were published by other CTAs (acquired by the
         // leader's scheduler, released to this CTA through the queue)
@@ -249,13 +256,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
         const int nhalf = pair_n(it) / 2;  // this CTA's B rows (a multiple of 32)
         const int brow = it.row0 + static_cast<int>(rank) * nhalf;
         const int nbox = gu ? 0 : nhalf / kPBox;
-        const uint32_t pair_bytes = 2u * (kPA + nbox * kPBox * 128);
-        int arow0, arow1 = 0;
+        const uint32_t pair_bytes = 2u * ((gu ? 2 : 1) * kPA + nbox * kPBox * 128);
+        int arow0;
         const CUtensorMap *ma0, *ma1 = nullptr;
         if (gu) {
-          const int f = it.ntile * kTileN + static_cast<int>(rank) * 64;
-          arow0 = (sh ? 0 : wblk * p.I) + f;
-          arow1 = arow0;
+          arow0 = (sh ? 0 : wblk * p.I) + it.ntile * kPairGuTile + static_cast<int>(rank) * 128;
           ma0 = sh ? &m.wgs : &m.wg;
           ma1 = sh ? &m.wus : &m.wu;
         } else {
@@ -268,12 +273,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
             break;
           }
           uint8_t* sA = smem + stage * kPStage;
-          uint8_t* sB = sA + kPA;
+          uint8_t* sB = sA + 2 * kPA;
           const uint32_t lbar = at_leader(&full[stage]);
           if (leader) mbar_arrive_expect_tx(&full[stage], pair_bytes);
           if (gu) {
-            tma_load_2d_pair(sA, ma0, lbar, kb * 64, arow0, pol_w);            // gate rows
-            tma_load_2d_pair(sA + kPA / 2, ma1, lbar, kb * 64, arow1, pol_w);  // up rows
+            tma_load_2d_pair(sA, ma0, lbar, kb * 64, arow0, pol_w);        // gate rows
+            tma_load_2d_pair(sA + kPA, ma1, lbar, kb * 64, arow0, pol_w);  // up rows
           } else {
             tma_load_2d_pair(sA, ma0, lbar, kb * 64, arow0, pol_w);
           }
@@ -301,21 +306,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader)
     if (leader && lane == 0) {
-      int stage = 0, acc = 0;
-      uint32_t phase = 0, acc_phase = 0;
+      int stage = 0, dn_half = 0;
+      uint32_t phase = 0;
+      uint32_t used0 = 0u, used1 = 0u;  // items that took TMEM half 0 / 1 so far
       bool live = true;
       for (int n = 0; live; ++n) {
         int item;
         if (!next_item(n, item, false)) break;
         bool gu;
         const WorkItem it = item_at(item, gu);
-        if (!item_ok(p, it, gu, kPairTileN)) continue;
+        if (!valid(it, gu)) continue;
         const int nkb = nkb_of(gu, it.e == p.E);
         const uint32_t idesc = idesc_bf16(2 * kTileN, pair_n(it));
-        if (!mbar_wait_cluster(&tempty[acc], acc_phase ^ 1, abort_flag, p.err, MOE_DEVERR_TIMEOUT))
+        // gate/up: both halves (gate in 0, up in 1); down: the next half in turn
+        const int h0 = gu ? 0 : dn_half, h1 = gu ? 1 : dn_half;
+        const uint32_t par0 = (h0 ? used1 : used0) & 1u, par1 = (h1 ? used1 : used0) & 1u;
+        if (!mbar_wait_cluster(&tempty[h0], par0 ^ 1u, abort_flag, p.err, MOE_DEVERR_TIMEOUT))
+          break;
+        if (gu && !mbar_wait_cluster(&tempty[h1], par1 ^ 1u, abort_flag, p.err, MOE_DEVERR_TIMEOUT))
           break;
         tc_fence_after();
-        const uint32_t d0 = tmem_base + acc * kPAccCols;
+        const uint32_t d0 = tmem_base + h0 * kPAccCols;
+        const uint32_t d1 = tmem_base + h1 * kPAccCols;
         for (int kb = 0; kb < nkb; ++kb) {
           // acquire at cluster scope: the peer's gatherers arrive from the other CTA
           if (!mbar_wait_cluster(&full[stage], phase, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) {
@@ -324,11 +336,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
           }
           tc_fence_after();
           const uint32_t a0 = smem_u32(smem + stage * kPStage);
-          const uint32_t b0 = a0 + kPA;
+          const uint32_t b0 = a0 + 2 * kPA;
+          if (gu) {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            umma_bf16_pair(d0, sdesc_k128(a0 + kk * 32), sdesc_k128(b0 + kk * 32), idesc,
-                           (kb | kk) != 0 ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
+              umma_bf16_pair(d0, sdesc_k128(a0 + kk * 32), sdesc_k128(b0 + kk * 32), idesc, acc);
+              umma_bf16_pair(d1, sdesc_k128(a0 + kPA + kk * 32), sdesc_k128(b0 + kk * 32), idesc,
+                             acc);
+            }
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_bf16_pair(d0, sdesc_k128(a0 + kk * 32), sdesc_k128(b0 + kk * 32), idesc,
+                             (kb | kk) != 0 ? 1u : 0u);
+          }
           umma_commit_pair_mc(&empty[stage], 0x3);  // frees the stage in both CTAs
           if (++stage == kPStages) {
             stage = 0;
@@ -336,9 +358,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
           }
         }
         if (!live) break;
-        umma_commit_pair_mc(&tfull[acc], 0x3);
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1;
+        umma_commit_pair_mc(&tfull[h0], 0x3);
+        if (gu) {
+          umma_commit_pair_mc(&tfull[h1], 0x3);
+          ++used0;
+          ++used1;
+        } else {
+          if (h0) ++used1;
+          else ++used0;
+          dn_half ^= 1;
+        }
       }
     }
     __syncwarp();
@@ -393,7 +422,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
       if (!next_item(n, item, true)) break;
       bool gu;
       const WorkItem it = item_at(item, gu);
-      if (!item_ok(p, it, gu, kPairTileN)) continue;
+      if (!valid(it, gu)) continue;
       const bool sh = it.e == p.E;
       const int nkb = nkb_of(gu, sh);
       const int nhalf = pair_n(it) / 2;  // this CTA's B rows
@@ -414,7 +443,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
           break;
         }
         if (gu) {
-          uint8_t* sB = smem + stage * kPStage + kPA;
+          uint8_t* sB = smem + stage * kPStage + 2 * kPA;
 #pragma unroll
           for (int i = 0; i < kRowsPerThread; ++i) {
             const int r = rbase + 16 * i;
@@ -449,14 +478,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
     const int orow = q * 32 + lane;    // row of this CTA's D
     const int et = tid - 64;           // epilogue thread 0..255
     const int cpart = et >> 7;         // column chunks of this warp: alternate ones
-    int acc = 0;
-    uint32_t acc_phase = 0;
+    int dn_half = 0;
+    uint32_t used0 = 0u, used1 = 0u;  // the MMA issuer's sequence of TMEM halves
     for (int n = 0;; ++n) {
       int item;
       if (!next_item(n, item, true)) break;
       bool gu;
       const WorkItem it = item_at(item, gu);
-      if (!item_ok(p, it, gu, kPairTileN)) continue;
+      if (!valid(it, gu)) continue;
       const bool sh = it.e == p.E;
       const int ncol = pair_n(it);
       if (!gu) {
@@ -485,69 +514,72 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
         }
         epi_bar<kPEpiThreads>();
       }
-      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) break;
+      const int h0 = gu ? 0 : dn_half, h1 = gu ? 1 : dn_half;
+      const uint32_t par0 = (h0 ? used1 : used0) & 1u, par1 = (h1 ? used1 : used0) & 1u;
+      if (!mbar_wait(&tfull[h0], par0, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) break;
+      if (gu && !mbar_wait(&tfull[h1], par1, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) break;
       tc_fence_after();
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kPAccCols;
+      const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+      const uint32_t taddr = tq + h0 * kPAccCols;
       if (gu) {
-        // lanes 0-63 hold gate rows, lanes 64-127 the up rows of the same features.
-        // Per 16-column chunk the gate warps finish columns 0-7 and the up warps
-        // columns 8-15, each taking the other operand through shared memory.
-        const bool is_gate = q < 2;
-        const int fq = q & 1;  // which 32 of the CTA's 64 features
-        const int nfeat = it.ntile * kTileN + static_cast<int>(rank) * 64 + fq * 32 + lane;
+        // lane = feature: gate in half 0, up in half 1 of the same lane. Per
+        // 16-token chunk the warp's 32 features x 16 tokens of h go through
+        // its shared-memory tile, so that each lane then stores 16-byte
+        // pieces of token rows (8 features) instead of single values.
+        const int fbase = it.ntile * kPairGuTile + static_cast<int>(rank) * 128 + q * 32;
         const int ncols = sh ? p.Is : p.I;
-        const bool ok = nfeat < ncols;
+        const bool ok = fbase < ncols;  // I and Is are multiples of 64: whole warps
         const float L = sh ? p.lim_s : p.lim_r;
         uint16_t* hout = sh ? p.h_s : p.h_r;
-        float* give = xch + ((cpart * 2 + (is_gate ? 0 : 1)) * 64 + fq * 32 + lane) * kPXchRow;
-        const float* take = xch + ((cpart * 2 + (is_gate ? 1 : 0)) * 64 + fq * 32 + lane) * kPXchRow;
+        uint32_t* tile = epi_stage + (warp - 2) * kEpiTileWords;
 #pragma unroll 1
-        for (int c0 = 16 * cpart; c0 < ncol; c0 += 32) {
-          float v[16];
-          tmem_ld16(taddr + c0, v);
+        for (int c0 = 16 * cpart; c0 < ncol && ok; c0 += 32) {
+          float g[16], u[16];
+          tmem_ld16(tq + c0, g);
+          tmem_ld16(tq + kPAccCols + c0, u);
           tmem_ld_wait();
 #pragma unroll
-          for (int c = 0; c < 8; ++c) give[c] = is_gate ? v[8 + c] : v[c];
-          epi_bar<kPEpiThreads>();
-          if (ok) {
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              const int r = c0 + (is_gate ? c : 8 + c);
-              const float g = is_gate ? v[c] : take[c];
-              const float u = is_gate ? take[c] : v[8 + c];
-              if (r < it.nrows)
-                hout[static_cast<size_t>(it.row0 + r) * ncols + nfeat] = f2bf(swiglu(g, u, L));
-            }
-          }
-          epi_bar<kPEpiThreads>();
+          for (int c = 0; c < 16; ++c) g[c] = swiglu(g[c], u[c], L);
+          store_h16(g, tile, hout, ncols, it.row0 + c0, it.nrows - c0, fbase, lane);
         }
       } else {
-        const int nfeat = it.ntile * kDownTile + static_cast<int>(rank) * kTileN + orow;
-        const bool ok = nfeat < p.H;
+        const int fbase = it.ntile * kDownTile + static_cast<int>(rank) * kTileN + q * 32;
+        const bool ok = fbase < p.H;  // H is a multiple of 64: whole warps
+        uint32_t* tile = epi_stage + (warp - 2) * kEpiTileWords;
         // 32 columns per TMEM wait (ncol is a multiple of 64), alternate groups per warp
 #pragma unroll 1
-        for (int c0 = 32 * cpart; c0 < ncol; c0 += 64) {
+        for (int c0 = 32 * cpart; c0 < ncol && ok; c0 += 64) {
           float ov[32];
           tmem_ld16(taddr + c0, ov);
           tmem_ld16(taddr + c0 + 16, ov + 16);
           tmem_ld_wait();
-          if (ok) {
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              const int j = meta_j[c0 + c];
-              if (j >= 0) p.y_slot[static_cast<size_t>(j) * p.H + nfeat] = meta_w[c0 + c] * ov[c];
-            }
+          for (int g8 = 0; g8 < 4; ++g8) {
+            float v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = meta_w[c0 + 8 * g8 + i] * ov[8 * g8 + i];
+            store_y8(v, meta_j + c0 + 8 * g8, tile, p.y_slot, p.H, fbase, lane);
           }
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        if (leader) mbar_arrive(&tempty[acc]);
-        else mbar_arrive_cluster(at_leader(&tempty[acc]));
+        if (leader) mbar_arrive(&tempty[h0]);
+        else mbar_arrive_cluster(at_leader(&tempty[h0]));
+        if (gu) {
+          if (leader) mbar_arrive(&tempty[h1]);
+          else mbar_arrive_cluster(at_leader(&tempty[h1]));
+        }
       }
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1;
+      if (gu) {
+        ++used0;
+        ++used1;
+      } else {
+        if (h0) ++used1;
+        else ++used0;
+        dn_half ^= 1;
+      }
       if (gu) {
         // publish this CTA's half of the output tile of h
         fence_proxy_async_global();
@@ -603,12 +635,12 @@ cudaError_t launch_ffn_pair(const GemmArgs& a, cudaStream_t s) {
   p.err = a.err;
   PairMaps m;
   const uint64_t wr = static_cast<uint64_t>(a.wrows);
-  bool ok = map_bf16(&m.wg, a.Wg, wr * c.I, c.H, 64) && map_bf16(&m.wu, a.Wu, wr * c.I, c.H, 64) &&
+  bool ok = map_bf16(&m.wg, a.Wg, wr * c.I, c.H, 128) && map_bf16(&m.wu, a.Wu, wr * c.I, c.H, 128) &&
             map_bf16(&m.wd, a.Wd, wr * c.H, c.I, kTileN) &&
             map_bf16(&m.h, a.h_r, TK, c.I, kPBox);
   if (p.has_shared) {
-    ok = ok && map_bf16(&m.wgs, a.W->Wg_s, c.I_shared, c.H, 64) &&
-         map_bf16(&m.wus, a.W->Wu_s, c.I_shared, c.H, 64) &&
+    ok = ok && map_bf16(&m.wgs, a.W->Wg_s, c.I_shared, c.H, 128) &&
+         map_bf16(&m.wus, a.W->Wu_s, c.I_shared, c.H, 128) &&
          map_bf16(&m.wds, a.W->Wd_s, c.H, c.I_shared, kTileN) &&
          map_bf16(&m.hs, a.h_s, T, c.I_shared, kPBox);
   } else {

@@ -30,6 +30,7 @@ constexpr int kPermTile = 2048;   // (token, slot) entries per permutation tile
 constexpr int kTileN = 128;       // output features per GEMM tile (MMA M)
 constexpr int kDownTile = 256;    // hidden features per down item (two MMA tiles)
 constexpr int kPairTileN = 256;   // token tile of the CTA-pair FFN (large batches)
+constexpr int kPairGuTile = 256;  // intermediate features per gate/up item of the CTA-pair FFN
 // Block-scaled FFN (MOE_W_MXFP4_A8): token tile (MMA N; two double-buffered
 // gate/up accumulators of this width and the scale columns fill the 512 TMEM
 // columns), intermediate features per gate/up item and hidden features per
@@ -73,6 +74,7 @@ inline FfnKind choose_ffn(int T, int K, int E, int* bn) {
 inline void ffn_tiles(int kind, int* gu_ft, int* dn_ft) {
   switch (kind) {
     case kFfnMx: *gu_ft = kMxGuTile, *dn_ft = kMxDnTile; break;
+    case kFfnPair: *gu_ft = kPairGuTile, *dn_ft = kDownTile; break;
     default: *gu_ft = kTileN, *dn_ft = kDownTile; break;
   }
 }
