@@ -62,7 +62,9 @@ constexpr int kXSfCol = 2 * kXAccCols;      // scale atoms after the two buffers
 constexpr int kXTmemCols = 512;
 constexpr int kXCtrl = 512;
 constexpr int kXHBox = 16;                  // h rows per TMA box
-constexpr int kXSmem = kXStages * kXStage + 1024 + kXCtrl + kMxTileN * 8;
+constexpr int kXSmem =
+    kXStages * kXStage + 1024 + kXCtrl + kMxTileN * 8 + kXEpiWarps * kEpiTileWords * 4;
+static_assert(kXSmem + (3 * kMaxExpertsCfg + 5) * 4 <= 227 * 1024, "shared memory");
 static_assert(kXSfCol + 12 <= kXTmemCols, "TMEM");
 static_assert(kMxTileN % 16 == 0 && kMxTileN <= 128, "token tile");
 
@@ -111,7 +113,8 @@ __global__ void __launch_bounds__(kXThreads, 1)
   volatile int* qitem = abort_flag + 1;  // [kXQueue]
   int* meta_j = reinterpret_cast<int*>(ctrl + kXCtrl);
   float* meta_w = reinterpret_cast<float*>(meta_j + kMxTileN);
-  int* s_gu = reinterpret_cast<int*>(meta_w + kMxTileN);  // [E+2]
+  uint32_t* epi_tile = reinterpret_cast<uint32_t*>(meta_w + kMxTileN);    // [warps][kEpiTileWords]
+  int* s_gu = reinterpret_cast<int*>(epi_tile + kXEpiWarps * kEpiTileWords);  // [E+2]
   int* s_dn = s_gu + (p.E + 2);                           // [E+2]
   int* s_off = s_dn + (p.E + 2);                          // [E+1]
   static_assert(8 * (2 * kXStages + 4 + 2 * kXQueue) + 8 + 4 * (2 + kXQueue) <= kXCtrl, "ctrl");
@@ -450,7 +453,6 @@ __global__ void __launch_bounds__(kXThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int qd = warp & 3;            // TMEM lane quarter
-    const int orow = qd * 32 + lane;    // output feature within a 128-row tile
     const int et = tid - 2 * 32;        // epilogue thread 0..255
     const int cpart = et >> 7;          // the two warps of a quarter: alternate column chunks
     int acc = 0;
@@ -491,14 +493,16 @@ __global__ void __launch_bounds__(kXThreads, 1)
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(qd * 32) << 16) + acc * kXAccCols;
       const int ncol = mma_n(it);
+      uint32_t* tile = epi_tile + (warp - 2) * kEpiTileWords;
       if (gu) {
-        const int nfeat = it.ntile * kMxGuTile + orow;
+        const int fbase = it.ntile * kMxGuTile + qd * 32;  // this warp's 32 features
         const int ncols = sh ? p.Is : p.I;
-        const bool ok = nfeat < ncols;
+        const bool ok = fbase < ncols;  // I and Is are multiples of 64: whole warps
         const float L = sh ? p.lim_s : p.lim_r;
         // routed: this warp's 32 features are one MXFP8 block, chunk qd of the
         // h scale atom of (row tile, k-block ntile)
         uint8_t* hsf = sh ? nullptr : q.h_sf + (static_cast<size_t>(row_tile(it)) * kbi + it.ntile) * 512;
+        uint8_t* tb = reinterpret_cast<uint8_t*>(tile);
 #pragma unroll 1
         for (int c0 = 16 * cpart; c0 < ncol; c0 += 32) {
           float gv[16], uv[16];
@@ -506,42 +510,50 @@ __global__ void __launch_bounds__(kXThreads, 1)
           tmem_ld16(taddr + kMxTileN + c0, uv);
           tmem_ld_wait();
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const int col = c0 + c;
-            const float h = ok ? swiglu(gv[c], uv[c], L) : 0.f;
-            if (sh) {
-              if (ok && col < it.nrows)
-                p.h_s[static_cast<size_t>(it.row0 + col) * p.Is + nfeat] = f2bf(h);
-            } else {
-              const uint32_t amax = __reduce_max_sync(0xffffffffu, __float_as_uint(h) & 0x7FFFFFFFu);
-              const int byte = min(max(static_cast<int>(amax >> 23) - 8, 0), 254);
-              const int ie = 254 - byte;  // 1 / scale = 2^(127 - byte)
-              const float inv = ie > 0 ? __uint_as_float(static_cast<uint32_t>(ie) << 23)
-                                       : __uint_as_float(0x00400000u);
-              if (col < it.nrows) {
-                if (ok) q.h_q[static_cast<size_t>(it.row0 + col) * p.I + nfeat] = to_e4m3(h * inv);
-                if (lane == 0) hsf[atom_off(col, qd)] = static_cast<uint8_t>(byte);
-              }
-            }
+          for (int c = 0; c < 16; ++c) gv[c] = ok ? swiglu(gv[c], uv[c], L) : 0.f;
+          if (sh) {
+            if (ok) store_h16(gv, tile, p.h_s, p.Is, it.row0 + c0, it.nrows - c0, fbase, lane);
+            continue;
           }
+          // e4m3 codes of the 16 token rows, byte (row c, feature lane) of the tile
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const float h = gv[c];
+            const uint32_t amax = __reduce_max_sync(0xffffffffu, __float_as_uint(h) & 0x7FFFFFFFu);
+            const int byte = min(max(static_cast<int>(amax >> 23) - 8, 0), 254);
+            const int ie = 254 - byte;  // 1 / scale = 2^(127 - byte)
+            const float inv = ie > 0 ? __uint_as_float(static_cast<uint32_t>(ie) << 23)
+                                     : __uint_as_float(0x00400000u);
+            tb[c * 32 + lane] = to_e4m3(h * inv);
+            if (lane == 0 && c0 + c < it.nrows) hsf[atom_off(c0 + c, qd)] = static_cast<uint8_t>(byte);
+          }
+          __syncwarp();
+          {  // lane: 16 codes of token row lane / 2
+            const int r = lane >> 1;
+            if (ok && c0 + r < it.nrows)
+              *reinterpret_cast<uint4*>(q.h_q + static_cast<size_t>(it.row0 + c0 + r) * p.I + fbase +
+                                        16 * (lane & 1)) =
+                  *reinterpret_cast<const uint4*>(tb + r * 32 + 16 * (lane & 1));
+          }
+          __syncwarp();
         }
       } else {
         const bool two = two_halves(it, gu);
 #pragma unroll 1
         for (int half = 0; half < (two ? 2 : 1); ++half) {
-          const int nfeat = it.ntile * kMxDnTile + half * 128 + orow;
-          const bool ok = nfeat < p.H;
+          const int fbase = it.ntile * kMxDnTile + half * 128 + qd * 32;  // this warp's features
+          const bool ok = fbase < p.H;  // H is a multiple of 64: whole warps
 #pragma unroll 1
-          for (int c0 = 16 * cpart; c0 < ncol; c0 += 32) {
+          for (int c0 = 16 * cpart; c0 < ncol && ok; c0 += 32) {
             float ov[16];
             tmem_ld16(taddr + half * kMxTileN + c0, ov);
             tmem_ld_wait();
-            if (ok) {
 #pragma unroll
-              for (int c = 0; c < 16; ++c) {
-                const int j = meta_j[c0 + c];
-                if (j >= 0) p.y_slot[static_cast<size_t>(j) * p.H + nfeat] = meta_w[c0 + c] * ov[c];
-              }
+            for (int g8 = 0; g8 < 2; ++g8) {
+              float v[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) v[i] = meta_w[c0 + 8 * g8 + i] * ov[8 * g8 + i];
+              store_y8(v, meta_j + c0 + 8 * g8, tile, p.y_slot, p.H, fbase, lane);
             }
           }
         }
