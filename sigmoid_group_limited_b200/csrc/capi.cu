@@ -59,9 +59,10 @@ WsLayout ws_layout(const moe_cfg& c, int T) {
   ffn_tiles(L.ffn, &L.gu_ft, &L.dn_ft);
   const int gu_ft = L.gu_ft, dn_ft = L.dn_ft;
   const int rt_gu = cdiv(c.I, gu_ft), st_gu = cdiv(c.I_shared, gu_ft), nt_dn = cdiv(c.H, dn_ft);
-  const long long mt_r = cdiv(static_cast<long long>(TK), L.bn) +
+  const int bn_items = ffn_adaptive(L) ? kTileN : L.bn;  // the smallest tile the FFN may pick
+  const long long mt_r = cdiv(static_cast<long long>(TK), bn_items) +
                          (static_cast<long long>(TK) < c.E ? static_cast<long long>(TK) : c.E);
-  const long long mt_s = c.I_shared > 0 ? cdiv(T, L.bn) : 0;
+  const long long mt_s = c.I_shared > 0 ? cdiv(T, bn_items) : 0;
   L.max_items_gu = static_cast<int>(mt_r * rt_gu + mt_s * st_gu);
   L.max_row_tiles = static_cast<int>(mt_r);
   L.max_items_dn = static_cast<int>((mt_r + mt_s) * nt_dn);

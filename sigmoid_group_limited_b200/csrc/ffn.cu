@@ -89,6 +89,7 @@ constexpr int kQueue = 4;                 // item queue entries
 constexpr int kLead = 4;                  // claim the next item this many k-blocks early
 constexpr long long kProgStride = 1024;   // producer progress = n * stride + k-blocks issued
 constexpr int kSmemLimit = 227 * 1024;    // dynamic shared memory of one CTA
+constexpr int kMaxStages = 8;             // full / empty barriers in the control block
 
 template <int BN, bool TM = false, bool F4 = false>
 struct Cfg {
@@ -108,7 +109,7 @@ struct Cfg {
       1024 + CTRL_BYTES + BN * 8 + kEpiWarps * kEpiTileWords * 4;
   static constexpr int STAGES_RAW =
       (kSmemLimit - STG * STG_BYTES - FIXED_BYTES - (3 * kMaxExpertsCfg + 5) * 4) / STAGE_BYTES;
-  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+  static constexpr int STAGES = STAGES_RAW > kMaxStages ? kMaxStages : STAGES_RAW;
   // weights as M: two fp32 accumulators (gate | up, or the two Wd halves) of
   // BN columns side by side; token rows as M: two partial sums of 256
   // columns each (even and odd k-steps: two independent MMA chains)
@@ -261,7 +262,7 @@ __global__ void __launch_bounds__(F4 ? kFfnThreadsF4 : kFfnThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   pdl_trigger();
   if (tid == 0) {
-    for (int s = 0; s < C::STAGES; ++s) {
+    for (int s = 0; s < kMaxStages; ++s) {  // the adaptive kernel may use more than C::STAGES
       // weight / h TMA + one arrival per gatherer thread (+ one per expander warp)
       mbar_init(&full[s], 1 + 32 * kGatherWarps + (F4 ? kExpWarps : 0));
       mbar_init(&empty[s], 1);
@@ -292,10 +293,17 @@ __global__ void __launch_bounds__(F4 ? kFfnThreadsF4 : kFfnThreads, 1)
     tmem_relinquish();
   }
   pdl_wait();  // the schedule, the routing and x come from earlier kernels
+  // Token tile and stage geometry. Fixed for every instantiation but the
+  // adaptive one (256-row tiles, weights as M, bf16), which picks 128 or 256
+  // from the expert loads and, at 128, splits the same stage ring into
+  // 128-row stages and double-buffers the accumulators.
+  constexpr bool kAdaptive = BN == 256 && !TM && !F4;
+  int bn = BN;
   int n_gu_all, n_dn_all;
-  if (p.sched_counts) {
+  if (kAdaptive || p.sched_counts) {
     __shared__ int wsum[33];
-    derive_schedule(p, s_gu, s_dn, s_off, wsum, &n_gu_all, &n_dn_all);
+    if (kAdaptive) bn = adaptive_bn(p, wsum);
+    derive_schedule(p, bn, s_gu, s_dn, s_off, wsum, &n_gu_all, &n_dn_all);
   } else {
     for (int i = tid; i < p.E + 2; i += blockDim.x) {
       s_gu[i] = p.gu_start[i];
@@ -309,14 +317,19 @@ __global__ void __launch_bounds__(F4 ? kFfnThreadsF4 : kFfnThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  const bool split = kAdaptive && bn < BN;
+  const int stage_bytes = split ? 2 * C::A_BYTES + kTileN * 128 : C::STAGE_BYTES;
+  const int nstages = split ? C::STAGES * C::STAGE_BYTES / stage_bytes : C::STAGES;
+  const int acc_cols = split ? 2 * kTileN : C::ACC_COLS;
+  const int nacc = split ? 2 : C::NACC;
   const int nslots = p.E + (p.has_shared ? 1 : 0);
   const int n_gu = min(n_gu_all, p.max_gu);
   const int n_dn = min(n_dn_all, p.max_dn);
   const int n_all = n_gu + n_dn;
   auto item_at = [&](int i, bool& gu) {
     gu = i < n_gu;
-    return gu ? decode_item(i, s_gu, s_off, nslots, p.E, p.T, BN)
-              : decode_item(i - n_gu, s_dn, s_off, nslots, p.E, p.T, BN);
+    return gu ? decode_item(i, s_gu, s_off, nslots, p.E, p.T, bn)
+              : decode_item(i - n_gu, s_dn, s_off, nslots, p.E, p.T, bn);
   };
   const int KB_gu = p.H / 64, KB_dn_r = p.I / 64, KB_dn_s = p.Is / 64;
   auto nkb_of = [&](bool gu, bool sh) { return gu ? KB_gu : (sh ? KB_dn_s : KB_dn_r); };
@@ -324,7 +337,7 @@ __global__ void __launch_bounds__(F4 ? kFfnThreadsF4 : kFfnThreads, 1)
   auto two_halves = [&](const WorkItem& it, bool gu) {
     return gu || it.ntile * kDownTile + kTileN < p.H;
   };
-  auto mma_n = [&](const WorkItem& it) { return (min(it.nrows, BN) + 15) & ~15; };
+  auto mma_n = [&](const WorkItem& it) { return (min(it.nrows, bn) + 15) & ~15; };
   // queue entry n: wait for it, read it, release it (one arrival per warp)
   auto next_item = [&](int n, int& item, bool whole_warp) -> bool {
     const int q = n % kQueue;
@@ -355,13 +368,13 @@ __global__ void __launch_bounds__(F4 ? kFfnThreadsF4 : kFfnThreads, 1)
         if (item >= 0) {
           bool gu;
           const WorkItem it = item_at(item, gu);
-          if (item_ok(p, it, gu, BN)) {
+          if (item_ok(p, it, gu, bn)) {
             const bool sh = it.e == p.E;
             prev_nkb = nkb_of(gu, sh);
             if (!gu) {
               // every gate/up output tile of this (slot, row tile) must be in h
               const int r0 = sh ? 0 : s_off[it.e];
-              const int ridx = s_gu[it.e] + (it.row0 - r0) / BN;
+              const int ridx = s_gu[it.e] + (it.row0 - r0) / bn;
               if (!wait_count(p.ready + ridx, cdiv_dev(sh ? p.Is : p.I, kTileN) + p.ready_extra,
                               abort_flag, p.err, p.wait_limit))
                 item = -1;
@@ -390,7 +403,7 @@ __global__ void __launch_bounds__(F4 ? kFfnThreadsF4 : kFfnThreads, 1)
         *prog = n * kProgStride;
         bool gu;
         const WorkItem it = item_at(item, gu);
-        if (!item_ok(p, it, gu, BN)) continue;
+        if (!item_ok(p, it, gu, bn)) continue;
         const bool sh = it.e == p.E;
         const bool two = two_halves(it, gu);
         // h rows of a down item were published by other CTAs (the scheduler
@@ -412,7 +425,7 @@ __global__ void __launch_bounds__(F4 ? kFfnThreadsF4 : kFfnThreads, 1)
             live = false;
             break;
           }
-          uint8_t* sA = smem + stage * C::STAGE_BYTES;
+          uint8_t* sA = smem + stage * stage_bytes;
           mbar_arrive_expect_tx(&full[stage], bytes);
           if (wtma) {
             tma_load_2d(sA, mA0, &full[stage], kb * 64, arow0, pol_w);
@@ -422,16 +435,16 @@ __global__ void __launch_bounds__(F4 ? kFfnThreadsF4 : kFfnThreads, 1)
             tma_load_2d(sA + 2 * C::A_BYTES + hb * C::H_BOX * 128, sh ? &tHs : &tH, &full[stage],
                         kb * 64, it.row0 + hb * C::H_BOX, pol_h);
           *prog = n * kProgStride + kb + 1;
-          if (++stage == C::STAGES) {
+          if (++stage == nstages) {
             stage = 0;
             phase ^= 1;
           }
         }
       }
       // every stage must be released by its MMA commit before teardown
-      for (int i = 0; i < C::STAGES && live; ++i) {
+      for (int i = 0; i < nstages && live; ++i) {
         if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) break;
-        if (++stage == C::STAGES) {
+        if (++stage == nstages) {
           stage = 0;
           phase ^= 1;
         }
@@ -449,7 +462,7 @@ __global__ void __launch_bounds__(F4 ? kFfnThreadsF4 : kFfnThreads, 1)
         if (!next_item(n, item, false)) break;
         bool gu;
         const WorkItem it = item_at(item, gu);
-        if (!item_ok(p, it, gu, BN)) continue;
+        if (!item_ok(p, it, gu, bn)) continue;
         const int nkb = nkb_of(gu, it.e == p.E);
         const bool two = two_halves(it, gu);
         // weights as M: MMA N = the item's rows rounded up to 16 (the B rows past
@@ -459,14 +472,14 @@ __global__ void __launch_bounds__(F4 ? kFfnThreadsF4 : kFfnThreads, 1)
             TM ? idesc_bf16(kTileN, two ? 2 * kTileN : kTileN) : idesc_bf16(kTileN, mma_n(it));
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) break;
         tc_fence_after();
-        const uint32_t d0 = tmem_base + acc * C::ACC_COLS;
+        const uint32_t d0 = tmem_base + acc * acc_cols;
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) {
             live = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t a0 = smem_u32(smem + stage * stage_bytes);
           const uint32_t b0 = a0 + 2 * C::A_BYTES;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
@@ -480,18 +493,18 @@ __global__ void __launch_bounds__(F4 ? kFfnThreadsF4 : kFfnThreads, 1)
                         (kb | (kk >> 1)) != 0 ? 1u : 0u);
             } else {
               umma_bf16(d0, sdesc_k128(a0 + kk * 32), bd, idesc, accum);
-              if (two) umma_bf16(d0 + BN, sdesc_k128(a0 + C::A_BYTES + kk * 32), bd, idesc, accum);
+              if (two) umma_bf16(d0 + bn, sdesc_k128(a0 + C::A_BYTES + kk * 32), bd, idesc, accum);
             }
           }
           umma_commit(&empty[stage]);
-          if (++stage == C::STAGES) {
+          if (++stage == nstages) {
             stage = 0;
             phase ^= 1;
           }
         }
         if (!live) break;
         umma_commit(&tfull[acc]);
-        if (++acc == C::NACC) {
+        if (++acc == nacc) {
           acc = 0;
           acc_phase ^= 1;
         }
@@ -513,7 +526,7 @@ __global__ void __launch_bounds__(F4 ? kFfnThreadsF4 : kFfnThreads, 1)
         if (!next_item(n, item, false)) break;
         bool gu;
         const WorkItem it = item_at(item, gu);
-        if (!item_ok(p, it, gu, BN) || it.e == p.E) continue;
+        if (!item_ok(p, it, gu, bn) || it.e == p.E) continue;
         const bool two = two_halves(it, gu);
         const int nkb = nkb_of(gu, false);
         const CUtensorMap* m0 = gu ? &tWg : &tWd;  // the code maps of this kernel
@@ -565,7 +578,7 @@ __global__ void __launch_bounds__(F4 ? kFfnThreadsF4 : kFfnThreads, 1)
       if (!next_item(n, item, true)) break;
       bool gu;
       const WorkItem it = item_at(item, gu);
-      if (!item_ok(p, it, gu, BN)) continue;
+      if (!item_ok(p, it, gu, bn)) continue;
       const bool sh = it.e == p.E;
       const bool two = two_halves(it, gu);
       const int nkb = nkb_of(gu, sh);
@@ -600,7 +613,7 @@ __global__ void __launch_bounds__(F4 ? kFfnThreadsF4 : kFfnThreads, 1)
           }
           if (!sh && (half == 0 || two)) {
             const uint4* src = reinterpret_cast<const uint4*>(stg + slot * C::STG_BYTES + half * kCodeTile + r * 32);
-            f4_store_row(smem + stage * C::STAGE_BYTES + half * C::A_BYTES, r, src[0], src[1], sc[d] & 0xFFu,
+            f4_store_row(smem + stage * stage_bytes + half * C::A_BYTES, r, src[0], src[1], sc[d] & 0xFFu,
                          sc[d] >> 8);
           }
           fetch(kb + kExpDepth, d);
@@ -610,7 +623,7 @@ __global__ void __launch_bounds__(F4 ? kFfnThreadsF4 : kFfnThreads, 1)
             mbar_arrive(&full[stage]);
             if (!sh) mbar_arrive(&sempty[slot]);
           }
-          if (++stage == C::STAGES) {
+          if (++stage == nstages) {
             stage = 0;
             phase ^= 1;
           }
@@ -642,7 +655,7 @@ __global__ void __launch_bounds__(F4 ? kFfnThreadsF4 : kFfnThreads, 1)
       if (!next_item(n, item, true)) break;
       bool gu;
       const WorkItem it = item_at(item, gu);
-      if (!item_ok(p, it, gu, BN)) continue;
+      if (!item_ok(p, it, gu, bn)) continue;
       const bool sh = it.e == p.E;
       const int nkb = nkb_of(gu, sh);
       const int nb = mma_n(it);  // B rows the MMA reads
@@ -661,7 +674,7 @@ __global__ void __launch_bounds__(F4 ? kFfnThreadsF4 : kFfnThreads, 1)
           break;
         }
         if (gu) {
-          uint8_t* sB = smem + stage * C::STAGE_BYTES + 2 * C::A_BYTES;
+          uint8_t* sB = smem + stage * stage_bytes + 2 * C::A_BYTES;
 #pragma unroll
           for (int i = 0; i < kRowsPerThread; ++i) {
             const int r = rbase + 16 * i;
@@ -669,7 +682,7 @@ __global__ void __launch_bounds__(F4 ? kFfnThreadsF4 : kFfnThreads, 1)
           }
         }
         cp_async_mbar_arrive_noinc(&full[stage]);
-        if (++stage == C::STAGES) {
+        if (++stage == nstages) {
           stage = 0;
           phase ^= 1;
         }
@@ -696,7 +709,7 @@ __global__ void __launch_bounds__(F4 ? kFfnThreadsF4 : kFfnThreads, 1)
       if (!next_item(n, item, true)) break;
       bool gu;
       const WorkItem it = item_at(item, gu);
-      if (!item_ok(p, it, gu, BN)) continue;
+      if (!item_ok(p, it, gu, bn)) continue;
       const bool sh = it.e == p.E;
       const bool live = r < it.nrows;
       // down items: the row's flat slot and routing weight, read while the
@@ -720,7 +733,7 @@ __global__ void __launch_bounds__(F4 ? kFfnThreadsF4 : kFfnThreads, 1)
       }
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) break;
       tc_fence_after();
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * C::ACC_COLS;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * acc_cols;
       if (gu) {
         const int ncols = sh ? p.Is : p.I;
         const float L = sh ? p.lim_s : p.lim_r;
@@ -776,7 +789,7 @@ __global__ void __launch_bounds__(F4 ? kFfnThreadsF4 : kFfnThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
-      if (++acc == C::NACC) {
+      if (++acc == nacc) {
         acc = 0;
         acc_phase ^= 1;
       }
@@ -787,7 +800,7 @@ __global__ void __launch_bounds__(F4 ? kFfnThreadsF4 : kFfnThreads, 1)
         if (warp == 2 && lane == 0) {
           __threadfence();
           const int r0 = sh ? 0 : s_off[it.e];
-          atomicAdd(p.ready + s_gu[it.e] + (it.row0 - r0) / BN, 1);
+          atomicAdd(p.ready + s_gu[it.e] + (it.row0 - r0) / bn, 1);
         }
       }
     }
@@ -805,7 +818,7 @@ __global__ void __launch_bounds__(F4 ? kFfnThreadsF4 : kFfnThreads, 1)
       if (!next_item(n, item, true)) break;
       bool gu;
       const WorkItem it = item_at(item, gu);
-      if (!item_ok(p, it, gu, BN)) continue;
+      if (!item_ok(p, it, gu, bn)) continue;
       const bool sh = it.e == p.E;
       if (!gu) {
         // destination slot and routing weight of every row, staged while the
@@ -836,7 +849,7 @@ __global__ void __launch_bounds__(F4 ? kFfnThreadsF4 : kFfnThreads, 1)
       }
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err, MOE_DEVERR_TIMEOUT)) break;
       tc_fence_after();
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * C::ACC_COLS;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * acc_cols;
       uint32_t* tile = epi_tile + (warp - 2) * kEpiTileWords;
       if (gu) {
         const int fbase = it.ntile * kTileN + q * 32;  // this warp's 32 features
@@ -850,7 +863,7 @@ __global__ void __launch_bounds__(F4 ? kFfnThreadsF4 : kFfnThreads, 1)
         for (int c0 = 16 * cpart; c0 < ncol && ok; c0 += 32) {
           float gv[16], uv[16];
           tmem_ld16(taddr + c0, gv);
-          tmem_ld16(taddr + BN + c0, uv);
+          tmem_ld16(taddr + bn + c0, uv);
           tmem_ld_wait();
 #pragma unroll
           for (int c = 0; c < 16; ++c) gv[c] = swiglu(gv[c], uv[c], L);
@@ -869,7 +882,7 @@ __global__ void __launch_bounds__(F4 ? kFfnThreadsF4 : kFfnThreads, 1)
           for (int c0 = kCols * cpart; c0 < ncol && ok; c0 += 2 * kCols) {
             float ov[kCols];
 #pragma unroll
-            for (int u = 0; u < kCols; u += 16) tmem_ld16(taddr + half * BN + c0 + u, ov + u);
+            for (int u = 0; u < kCols; u += 16) tmem_ld16(taddr + half * bn + c0 + u, ov + u);
             tmem_ld_wait();
 #pragma unroll
             for (int g8 = 0; g8 < kCols / 8; ++g8) {
@@ -884,7 +897,7 @@ __global__ void __launch_bounds__(F4 ? kFfnThreadsF4 : kFfnThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
-      if (++acc == C::NACC) {
+      if (++acc == nacc) {
         acc = 0;
         acc_phase ^= 1;
       }
@@ -895,7 +908,7 @@ __global__ void __launch_bounds__(F4 ? kFfnThreadsF4 : kFfnThreads, 1)
         if (warp == 2 && lane == 0) {
           __threadfence();
           const int r0 = sh ? 0 : s_off[it.e];
-          atomicAdd(p.ready + s_gu[it.e] + (it.row0 - r0) / BN, 1);
+          atomicAdd(p.ready + s_gu[it.e] + (it.row0 - r0) / bn, 1);
         }
       }
     }

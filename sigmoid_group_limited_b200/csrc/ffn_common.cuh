@@ -81,23 +81,28 @@ __device__ __forceinline__ void smem_exscan(int* a, int n, int* wsum) {
   __syncthreads();
 }
 
-// The FFN work lists from the expert counts, in shared memory: the row
-// offsets s_off[0..E] (exclusive scan of the counts) and the per-slot item
-// starts s_gu / s_dn [E+2] (slot E the shared expert, entry E+1 the total),
-// exactly as the schedule builder of the permutation writes them. Returns the
-// item totals.
-__device__ __forceinline__ void derive_schedule(const FfnParams& p, int* s_gu, int* s_dn, int* s_off,
-                                                int* wsum, int* n_gu, int* n_dn) {
+// Rows of expert e: from the counts, else from the row offsets.
+__device__ __forceinline__ int expert_rows(const FfnParams& p, int e) {
+  return max(0, p.sched_counts ? p.sched_counts[e] : p.offsets[e + 1] - p.offsets[e]);
+}
+
+// The FFN work lists from the expert loads, in shared memory: the row
+// offsets s_off[0..E] (exclusive scan of the loads) and the per-slot item
+// starts s_gu / s_dn [E+2] (slot E the shared expert, entry E+1 the total)
+// for token tiles of bn rows, as the schedule builder of the permutation
+// writes them for its tile. Returns the item totals.
+__device__ __forceinline__ void derive_schedule(const FfnParams& p, int bn, int* s_gu, int* s_dn,
+                                                int* s_off, int* wsum, int* n_gu, int* n_dn) {
   const int nslots = p.E + (p.has_shared ? 1 : 0);
   const int nt_gu_r = cdiv_dev(p.I, p.gu_ft), nt_gu_s = cdiv_dev(p.Is, p.gu_ft);
   const int nt_dn = cdiv_dev(p.H, p.dn_ft);
   for (int e = threadIdx.x; e < p.E + 2; e += blockDim.x) {
     int gu = 0, dn = 0, c = 0;
-    if (e < p.E) c = max(0, p.sched_counts[e]);
+    if (e < p.E) c = expert_rows(p, e);
     if (e < nslots) {
       const bool sh = e == p.E;
       const int rows = sh ? p.T : c;
-      const int nm = (rows + p.bn - 1) / p.bn;
+      const int nm = (rows + bn - 1) / bn;
       gu = nm * (sh ? nt_gu_s : nt_gu_r);
       dn = nm * nt_dn;
     }
@@ -111,6 +116,28 @@ __device__ __forceinline__ void derive_schedule(const FfnParams& p, int* s_gu, i
   smem_exscan(s_off, p.E + 1, wsum);
   *n_gu = s_gu[p.E + 1];
   *n_dn = s_dn[p.E + 1];
+}
+
+// Token tile of the adaptive kernel: an MMA costs about the same for any N,
+// so 256-row tiles pay when they cut the number of row tiles, which they do
+// only for experts with more than 128 rows; otherwise the 128-row geometry
+// (more pipeline stages, double-buffered accumulators) is faster. 256 when
+// the 256-row tiles number at most 4/5 of the 128-row ones. Every CTA reads
+// the same loads, so all take the same decision. tot: 2 ints of shared
+// memory. Ends with a CTA barrier.
+__device__ __forceinline__ int adaptive_bn(const FfnParams& p, int* tot) {
+  if (threadIdx.x < 2) tot[threadIdx.x] = 0;
+  __syncthreads();
+  int t128 = 0, t256 = 0;
+  for (int e = threadIdx.x; e <= p.E; e += blockDim.x) {
+    const int rows = e < p.E ? expert_rows(p, e) : (p.has_shared ? p.T : 0);
+    t128 += (rows + 127) / 128;
+    t256 += (rows + 255) / 256;
+  }
+  atomicAdd(&tot[0], t128);
+  atomicAdd(&tot[1], t256);
+  __syncthreads();
+  return 5 * tot[1] <= 4 * tot[0] ? 256 : 128;
 }
 
 __device__ __forceinline__ float clampL(float v, float L) {

@@ -50,24 +50,29 @@ enum FfnKind {
   kFfnMx = 2,      // moe_ffn_mx: block-scaled MXFP8 x MXFP4
 };
 
-// The expert-FFN kernel for large batches: one CTA per item (default), or a
-// CTA pair per item when the environment variable SGL_MOE_FFN is "pair".
-// Read at every call, so the workspace layout and the launch always agree.
+// The expert-FFN kernel for large batches: one CTA per item with 256-token
+// tiles (default); the environment variable SGL_MOE_FFN selects 128-token
+// tiles ("narrow"), token rows as the MMA's M ("tokens_m", 128-token tiles) or
+// a CTA pair per item ("pair"). Read at every call, so the workspace layout
+// and the launch always agree.
 inline bool ffn_env_is(const char* name) {
   const char* v = getenv("SGL_MOE_FFN");
   return v != nullptr && strcmp(v, name) == 0;
 }
 
 // Kernel and token-tile width (MMA N) for a batch: narrow tiles for decode,
-// wide ones for prefill. T*K/E is the mean load over all experts.
+// wide ones for prefill. T*K/E is the mean load over all experts. Above 48,
+// 256-token tiles: an MMA costs about the same for any N, so the widest tile
+// issues the fewest instructions, at the price of single-buffered
+// accumulators (two 256-column chains fill TMEM).
 inline FfnKind choose_ffn(int T, int K, int E, int* bn) {
   const double avg = static_cast<double>(T) * K / E;
   if (avg <= 12.0) return *bn = 16, kFfnNarrow;
   if (avg <= 24.0) return *bn = 32, kFfnNarrow;
   if (avg <= 48.0) return *bn = 64, kFfnNarrow;
   if (ffn_env_is("pair")) return *bn = kPairTileN, kFfnPair;
-  if (ffn_env_is("wide")) return *bn = 256, kFfnNarrow;
-  return *bn = 128, kFfnNarrow;
+  if (ffn_env_is("narrow") || ffn_env_is("tokens_m")) return *bn = 128, kFfnNarrow;
+  return *bn = 256, kFfnNarrow;
 }
 
 // Output features per gate/up item and per down item of each kernel.
@@ -107,6 +112,11 @@ struct WsLayout {
 };
 
 WsLayout ws_layout(const moe_cfg& c, int T);
+
+// The 256-token-tile FFN picks its token tile (128 or 256) from the expert
+// loads on the device and derives its own work lists; its workspace is sized
+// for the 128-row tiles (more items).
+inline bool ffn_adaptive(const WsLayout& L) { return L.ffn == kFfnNarrow && L.bn == 256; }
 
 // Launchers (return cudaGetLastError()).
 // Routing. unc [T] / unc_n: scratch list (and its count, zeroed by the

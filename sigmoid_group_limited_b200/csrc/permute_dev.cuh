@@ -86,6 +86,7 @@ struct SchedArgs {
   int32_t* gu_start;  // [E+2] first gate/up work item of slot e (e == E: shared expert)
   int32_t* dn_start;  // [E+2] first down work item of slot e
   int32_t* ready;     // nullable: [gate/up items] zeroed for the fused FFN's row-tile counters
+  int ready_len;      // > 0: zero ready[0, ready_len) whole (the FFN picks its own tile)
   int32_t* nitems;    // [2] totals
 };
 
@@ -122,7 +123,11 @@ __device__ void build_schedule(const SchedArgs& a, const int* cnt, int* scratch)
       a.dn_start[e] = real ? base_dn + (q ? ndn[0] : 0) : tot_dn;
     }
   }
-  if (a.ready) {
+  if (a.ready && a.ready_len > 0) {
+    // the FFN derives its work lists for a tile it picks itself: every
+    // counter it may use
+    for (int i = threadIdx.x; i < a.ready_len; i += blockDim.x) a.ready[i] = 0;
+  } else if (a.ready) {
     // one counter per (slot, row tile): the slot's first nm gate/up item indices
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
@@ -247,6 +252,7 @@ SchedArgs make_sched(const moe_cfg& c, int T, const WsLayout& L, int32_t* gu_sta
   a.gu_start = gu_start;
   a.dn_start = dn_start;
   a.ready = ready;
+  a.ready_len = ffn_adaptive(L) ? L.max_items_gu : 0;
   a.nitems = nitems;
   return a;
 }

@@ -72,14 +72,16 @@ def test_tiny_layer_pair_ffn(T, variant, monkeypatch):
     _full_check(cfg, d)
 
 
-@pytest.mark.parametrize("form", ["tokens_m", "wide"])
+@pytest.mark.parametrize("form", ["tokens_m", "narrow"])
 @pytest.mark.parametrize("T,variant", [(600, {}), (600, dict(limit_routed=0.5, limit_shared=0.7)),
                                        (600, dict(I_shared=0)), (600, dict(I=192, I_shared=320)),
                                        (1500, dict(H=384))])
 def test_tiny_layer_ffn_options(form, T, variant, monkeypatch):
-    """The optional orientations of the expert FFN for large batches, selected
+    """The optional forms of the expert FFN for large batches, selected
     explicitly: token rows as the MMA's M with two partial accumulators
-    (tokens_m), and 256-token tiles (wide)."""
+    (tokens_m), and 128-token tiles with double-buffered accumulators
+    (narrow). The default, 256-token tiles, runs in every other test of a
+    large batch."""
     monkeypatch.setenv("SGL_MOE_FFN", form)
     cfg = TINY.with_(**variant)
     d = workloads.generate(cfg, DEV, T=T)
@@ -100,8 +102,10 @@ def test_tiny_layer_ffn_options(form, T, variant, monkeypatch):
 
 
 @pytest.mark.slow
-def test_prefill_pair_ffn_all_tokens(monkeypatch):
-    monkeypatch.setenv("SGL_MOE_FFN", "pair")
+@pytest.mark.parametrize("form", ["pair", "narrow"])
+def test_prefill_ffn_forms_all_tokens(form, monkeypatch):
+    """The full prefill batch on the CTA-pair kernel and on 128-token tiles."""
+    monkeypatch.setenv("SGL_MOE_FFN", form)
     cfg = workloads.CONFIGS["prefill"]
     d = workloads.generate(cfg, DEV)
     _full_check(cfg, d)
