@@ -53,10 +53,11 @@ WsLayout ws_layout(const moe_cfg& c, int T) {
     L.ffn = kFfnMx;
   } else {
     L.ffn = choose_ffn(T, c.K, c.E, &L.bn);
-    // MXFP4 weights are expanded by the one-CTA kernel, on tiles of up to 128 rows
-    if (c.wfmt == MOE_W_MXFP4 && (L.ffn == kFfnPair || L.bn > kTileN)) L.ffn = kFfnNarrow, L.bn = kTileN;
+    // MXFP4 weights are expanded by the one-CTA kernel
+    if (c.wfmt == MOE_W_MXFP4 && L.ffn == kFfnPair) L.ffn = kFfnNarrow, L.bn = 256;
   }
   ffn_tiles(L.ffn, &L.gu_ft, &L.dn_ft);
+  L.adaptive = L.ffn == kFfnNarrow && L.bn == 256 && c.wfmt == MOE_W_BF16 ? 1 : 0;
   const int gu_ft = L.gu_ft, dn_ft = L.dn_ft;
   const int rt_gu = cdiv(c.I, gu_ft), st_gu = cdiv(c.I_shared, gu_ft), nt_dn = cdiv(c.H, dn_ft);
   const int bn_items = ffn_adaptive(L) ? kTileN : L.bn;  // the smallest tile the FFN may pick

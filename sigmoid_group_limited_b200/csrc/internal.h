@@ -109,14 +109,15 @@ struct WsLayout {
   int max_touched;
   int n_ptiles, bn, max_items_gu, max_items_dn;
   int ffn, gu_ft, dn_ft;  // FfnKind and its output features per gate/up and down item
+  int adaptive;           // the FFN picks its token tile on the device (see ffn_adaptive)
 };
 
 WsLayout ws_layout(const moe_cfg& c, int T);
 
-// The 256-token-tile FFN picks its token tile (128 or 256) from the expert
-// loads on the device and derives its own work lists; its workspace is sized
-// for the 128-row tiles (more items).
-inline bool ffn_adaptive(const WsLayout& L) { return L.ffn == kFfnNarrow && L.bn == 256; }
+// The 256-token-tile FFN with bf16 weights picks its token tile (128 or 256)
+// from the expert loads on the device and derives its own work lists; its
+// workspace is sized for the 128-row tiles (more items).
+inline bool ffn_adaptive(const WsLayout& L) { return L.adaptive != 0; }
 
 // Launchers (return cudaGetLastError()).
 // Routing. unc [T] / unc_n: scratch list (and its count, zeroed by the

@@ -417,6 +417,29 @@ def test_tiny_mxfp4(T, variant):
     _full_check(cfg, d)
 
 
+def _tile_rule(counts, T):
+    """The token tile the large-batch FFN picks from the expert loads: 256
+    when 256-row tiles number at most 4/5 of the 128-row ones (the shared
+    expert's T rows included), else 128."""
+    rows = np.append(counts, T)
+    t128 = int(np.sum((rows + 127) // 128))
+    t256 = int(np.sum((rows + 255) // 256))
+    return 256 if 5 * t256 <= 4 * t128 else 128
+
+
+@pytest.mark.parametrize("wfmt", [workloads.MOE_W_BF16, workloads.MOE_W_MXFP4])
+@pytest.mark.parametrize("T,bias_kind,tile", [(600, "zero", 128), (2000, "normal", 256)])
+def test_tiny_adaptive_tile(wfmt, T, bias_kind, tile):
+    """Batches above 48 rows per expert, with near-uniform loads and with one
+    expert taking most rows: the bf16 FFN picks its token tile from the loads
+    on the device (one case per tile); the MXFP4 one runs 256-row tiles on
+    both. Each is checked against the oracle."""
+    cfg = TINY.with_(wfmt=wfmt, bias_kind=bias_kind)
+    d = workloads.generate(cfg, DEV, T=T)
+    g, ref, near = _full_check(cfg, d)
+    assert _tile_rule(g["counts"].cpu().numpy(), T) == tile
+
+
 # ------------------------------------------------------------------ block-scaled MXFP8 x MXFP4
 
 TINY_A8 = workloads.CONFIGS["tiny_a8"]
