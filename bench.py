@@ -244,23 +244,23 @@ def roofline_entry(bytes_, flops, seconds, peaks, sustained=False, fp8_flops=0.0
 # DRAM bytes (dram__bytes_read.sum, dram__bytes_write.sum) of one expert-FFN
 # launch of each full-size workload, from one-pass ncu captures of the bench's
 # own command at the same token count (profiles/ffn_traffic_full_size.md).
-# Valid only for the FFN sources they were taken on: another source reports
-# traffic null.
-FFN_TRAFFIC_SOURCES_SHA256 = "c2dcf21acb02a388b9c7592539556273c8214f857808b3908bf972fbe8221e42"
+# Valid only for the FFN sources they were taken on (ffn.cu, ffn_mx.cu and
+# ffn_common.cuh): another source reports traffic null.
+FFN_TRAFFIC_SOURCES_SHA256 = "7cbaa6b3231673557d8c4dca5e4c259cc2ebed313273c28f71f0f90f755d8304"
 FFN_TRAFFIC = {                      # workload name -> (read bytes, write bytes)
-    "decode": (696.27e6, 5.06e6),
-    "prefill": (1.65e9, 375.26e6),
-    "prefill_bias0": (6.20e9, 376.40e6),
-    "zipf": (7.65e9, 1.68e9),
-    "mxfp4": (919.93e6, 809.77e6),
-    "mxfp4_a8": (735.50e6, 762.32e6),
+    "decode": (696.27e6, 5.08e6),
+    "prefill": (1.72e9, 377.69e6),
+    "prefill_bias0": (6.19e9, 376.59e6),
+    "zipf": (7.97e9, 1.68e9),
+    "mxfp4": (919.87e6, 809.59e6),
+    "mxfp4_a8": (669.30e6, 761.82e6),
 }
 
 
 def ffn_sources_sha256() -> str:
     import hashlib
     h = hashlib.sha256()
-    for name in ("ffn.cu", "ffn_mx.cu"):
+    for name in ("ffn.cu", "ffn_mx.cu", "ffn_common.cuh"):
         with open(os.path.join(ROOT, "sigmoid_group_limited_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
