@@ -91,7 +91,7 @@ WsLayout ws_layout(const moe_cfg& c, int T) {
   L.h_s = take(static_cast<size_t>(T) * (c.I_shared > 0 ? c.I_shared : 0) * 2);
   L.y_slot = take((TK + T) * c.H * 4);
   L.wr_split = T > 32 ? take(static_cast<size_t>(3) * c.E * c.H * 2) : 0;
-  L.zp = T <= 32 ? take(static_cast<size_t>(8) * 32 * c.E * 4) : 0;
+  L.zp = T <= kFrontMaxT ? take(static_cast<size_t>(8) * kFrontMaxT * c.E * 4) : 0;
   if (mx) {
     // h_r holds the e4m3 h codes; the rest is scales
     L.max_touched = static_cast<int>(TK < static_cast<size_t>(c.E) ? TK : c.E);

@@ -1,4 +1,4 @@
-// front.cu - the decode front of the layer in one launch (batches of up to 32
+// front.cu - the decode front of the layer in one launch (batches of up to 64
 // tokens): router logits, certified group-limited top-k with the exact
 // re-derivation of close calls, permutation and FFN work lists. The separate
 // kernels for these stages are latency-bound at this size; one cooperative
@@ -44,8 +44,8 @@ namespace {
 constexpr int kFrontThreads = 512;
 constexpr int kFrontChunks = 8;   // hidden chunks per expert block
 constexpr int kFrontExperts = 32;  // experts per block
-constexpr int kFrontRed = 8 * 4 * kSmallT;  // floats: the second K half's partials
-constexpr int kFrontSmem = kFrontExperts * kMaxChunk * 4 + kSmallT * kXRow * 2 + kFrontRed * 4;
+constexpr int kFrontRed = 8 * 4 * kFrontMaxT;  // floats: the second K half's partials
+constexpr int kFrontSmem = kFrontExperts * kMaxChunk * 4 + kFrontMaxT * kXRow * 2 + kFrontRed * 4;
 
 struct FrontParams {
   int T, H, E, n_group, topk_group, K, renorm;
@@ -53,7 +53,7 @@ struct FrontParams {
   const uint16_t* x;
   const float* Wr;
   const float* bias;
-  float* zp;          // [8][32][E] partial logits
+  float* zp;          // [8][kFrontMaxT][E] partial logits
   float* z;           // [T][E] logits
   int32_t* idx;
   float* w;
@@ -100,7 +100,7 @@ __global__ void __launch_bounds__(kFrontThreads, 1) decode_front(const __grid_co
   // ---- phase 1: partial logits
   {
     float* ws = reinterpret_cast<float*>(fsm);                            // [32][kMaxChunk]
-    uint16_t* xs = reinterpret_cast<uint16_t*>(ws + kFrontExperts * kMaxChunk);  // [32][kXRow]
+    uint16_t* xs = reinterpret_cast<uint16_t*>(ws + kFrontExperts * kMaxChunk);  // [kFrontMaxT][kXRow]
     const int eb = blockIdx.x / kFrontChunks, r = blockIdx.x % kFrontChunks;
     const int e0 = eb * kFrontExperts;
     const int chunk = ((H / 64 + kFrontChunks - 1) / kFrontChunks) * 64;
@@ -116,7 +116,7 @@ __global__ void __launch_bounds__(kFrontThreads, 1) decode_front(const __grid_co
         *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     const uint64_t pol_x = policy_evict_last();
-    for (int i = tid; i < kSmallT * (kMaxChunk / 8); i += blockDim.x) {
+    for (int i = tid; i < kFrontMaxT * (kMaxChunk / 8); i += blockDim.x) {
       const int row = i / (kMaxChunk / 8), c = 8 * (i % (kMaxChunk / 8));
       uint16_t* dst = xs + row * kXRow + c;
       if (row < T && c < kn)
@@ -130,45 +130,52 @@ __global__ void __launch_bounds__(kFrontThreads, 1) decode_front(const __grid_co
       prefetch_range(p.pf_shared[tid], p.pf_shared_bytes, blockIdx.x, gridDim.x);
     cp_async_wait<0>();
     __syncthreads();
-    // warp w: experts 4 (w % 8) .. +3 over K half w / 8; lane = token
+    // warp w: experts 4 (w % 8) .. +3 over K half w / 8; lane = token, in
+    // passes of 32 tokens (token 32 tp + lane)
     constexpr int EW = 4;
-    float* red = reinterpret_cast<float*>(xs + kSmallT * kXRow);  // [8 warps][4][32 tokens]
+    float* red = reinterpret_cast<float*>(xs + kFrontMaxT * kXRow);  // [8 warps][4][kFrontMaxT tokens]
     const int wq = warp & 7, kh = warp >> 3;
     const int nk8 = kn / 8, half = nk8 / 2;  // kn is a multiple of 64: nk8 even
-    float acc[EW];
+    const int ntp = (T + 31) / 32;
+    for (int tp = 0; tp < ntp; ++tp) {
+      const int tok = 32 * tp + lane;
+      float acc[EW];
 #pragma unroll
-    for (int q = 0; q < EW; ++q) acc[q] = 0.f;
+      for (int q = 0; q < EW; ++q) acc[q] = 0.f;
 #pragma unroll 4
-    for (int i = kh * half; i < (kh + 1) * half; ++i) {
-      const uint4 xv8 = *reinterpret_cast<const uint4*>(xs + lane * kXRow + 8 * i);
-      const uint32_t pk[4] = {xv8.x, xv8.y, xv8.z, xv8.w};
+      for (int i = kh * half; i < (kh + 1) * half; ++i) {
+        const uint4 xv8 = *reinterpret_cast<const uint4*>(xs + tok * kXRow + 8 * i);
+        const uint32_t pk[4] = {xv8.x, xv8.y, xv8.z, xv8.w};
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const float xv0 = __uint_as_float(pk[2 * h] << 16);
-        const float xv1 = __uint_as_float(pk[2 * h] & 0xFFFF0000u);
-        const float xv2 = __uint_as_float(pk[2 * h + 1] << 16);
-        const float xv3 = __uint_as_float(pk[2 * h + 1] & 0xFFFF0000u);
+        for (int h = 0; h < 2; ++h) {
+          const float xv0 = __uint_as_float(pk[2 * h] << 16);
+          const float xv1 = __uint_as_float(pk[2 * h] & 0xFFFF0000u);
+          const float xv2 = __uint_as_float(pk[2 * h + 1] << 16);
+          const float xv3 = __uint_as_float(pk[2 * h + 1] & 0xFFFF0000u);
 #pragma unroll
-        for (int q = 0; q < EW; ++q) {
-          const float4 wv = *reinterpret_cast<const float4*>(ws + (wq * EW + q) * kMaxChunk + 8 * i + 4 * h);
-          acc[q] = fmaf(xv0, wv.x, acc[q]);
-          acc[q] = fmaf(xv1, wv.y, acc[q]);
-          acc[q] = fmaf(xv2, wv.z, acc[q]);
-          acc[q] = fmaf(xv3, wv.w, acc[q]);
+          for (int q = 0; q < EW; ++q) {
+            const float4 wv = *reinterpret_cast<const float4*>(ws + (wq * EW + q) * kMaxChunk + 8 * i + 4 * h);
+            acc[q] = fmaf(xv0, wv.x, acc[q]);
+            acc[q] = fmaf(xv1, wv.y, acc[q]);
+            acc[q] = fmaf(xv2, wv.z, acc[q]);
+            acc[q] = fmaf(xv3, wv.w, acc[q]);
+          }
         }
       }
-    }
-    if (kh == 1) {
+      if (kh == 1) {
 #pragma unroll
-      for (int q = 0; q < EW; ++q) red[(wq * EW + q) * kSmallT + lane] = acc[q];
-    }
-    __syncthreads();
-    if (kh == 0 && lane < T) {
+        for (int q = 0; q < EW; ++q) red[(wq * EW + q) * kFrontMaxT + tok] = acc[q];
+      }
+      __syncthreads();
+      if (kh == 0 && tok < T) {
 #pragma unroll
-      for (int q = 0; q < EW; ++q) {
-        const int e = e0 + wq * EW + q;
-        // the two K halves in a fixed order
-        if (e < E) p.zp[(static_cast<size_t>(r) * kSmallT + lane) * E + e] = acc[q] + red[(wq * EW + q) * kSmallT + lane];
+        for (int q = 0; q < EW; ++q) {
+          const int e = e0 + wq * EW + q;
+          // the two K halves in a fixed order
+          if (e < E)
+            p.zp[(static_cast<size_t>(r) * kFrontMaxT + tok) * E + e] =
+                acc[q] + red[(wq * EW + q) * kFrontMaxT + tok];
+        }
       }
     }
   }
@@ -195,7 +202,7 @@ __global__ void __launch_bounds__(kFrontThreads, 1) decode_front(const __grid_co
     for (int e = tid; e < E; e += blockDim.x) {
       float sum = 0.f;
 #pragma unroll
-      for (int q = 0; q < kFrontChunks; ++q) sum += p.zp[(static_cast<size_t>(q) * kSmallT + t) * E + e];
+      for (int q = 0; q < kFrontChunks; ++q) sum += p.zp[(static_cast<size_t>(q) * kFrontMaxT + t) * E + e];
       zs[e] = sum;
       zr[e] = sum;
       bs[e] = p.bias ? p.bias[e] : 0.f;
@@ -295,7 +302,9 @@ __global__ void __launch_bounds__(kFrontThreads, 1) decode_front(const __grid_co
 
 bool decode_front_ok(const moe_cfg& c, int T) {
   const int per = c.E / c.n_group;
-  return T <= kSmallT && (c.E == 128 || c.E == 256 || c.E == 512) && (per == 32 || per == 64) &&
+  // phase 2 takes one CTA per token: T <= the grid (32 CTAs for E = 128)
+  return T <= kFrontMaxT && T <= kFrontChunks * c.E / kFrontExperts &&
+         (c.E == 128 || c.E == 256 || c.E == 512) && (per == 32 || per == 64) &&
          c.n_group <= kSelMaxGroups && c.K + 1 <= kSelMaxCand && c.topk_group * (c.K + 1) <= 64 &&
          c.H <= kRowRegs * 128 && T * c.K <= kPermTile && 2 * kFrontThreads >= c.E + 2;
 }

@@ -27,6 +27,7 @@ struct WorkItem {
 };
 
 constexpr int kPermTile = 2048;   // (token, slot) entries per permutation tile
+constexpr int kFrontMaxT = 64;    // largest batch of the fused decode front
 constexpr int kTileN = 128;       // output features per GEMM tile (MMA M)
 constexpr int kDownTile = 256;    // hidden features per down item (two MMA tiles)
 constexpr int kPairTileN = 256;   // token tile of the CTA-pair FFN (large batches)
@@ -105,7 +106,7 @@ struct WsLayout {
   size_t x_q, x_sf, h_sf, sf_g, sf_u, sf_d;
   int max_row_tiles;
   size_t wr_split;  // router matrix as three bf16 terms (batches above 32 tokens)
-  size_t zp;        // partial router logits [8][32][E] of the fused decode front (T <= 32)
+  size_t zp;        // partial router logits [8][kFrontMaxT][E] of the fused decode front
   int max_touched;
   int n_ptiles, bn, max_items_gu, max_items_dn;
   int ffn, gu_ft, dn_ft;  // FfnKind and its output features per gate/up and down item
@@ -128,7 +129,7 @@ cudaError_t launch_router(const moe_cfg& c, int T, const uint16_t* x, const floa
                           const float* bias, float* z, int32_t* idx, float* w, int32_t* unc,
                           int32_t* unc_n, int32_t* err, uint16_t* wr_split, cudaStream_t s);
 
-// The decode front in one cooperative launch (T <= 32, see front.cu):
+// The decode front in one cooperative launch (T <= kFrontMaxT, see front.cu):
 // routing (logits via zp, certified selection, exact re-derivation of close
 // calls), then the permutation and the FFN work lists. bar: a zeroed grid
 // barrier counter. decode_front_ok: whether a configuration qualifies.
